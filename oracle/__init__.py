@@ -1,0 +1,178 @@
+"""CPU oracle for the expert-parallel dispatch/combine path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The product path
+(``combine_ep_get_08_b200``) never does: it has no CPU fallback.
+
+The arithmetic lives in ``ep_oracle.c`` (plain C, single-threaded, built with
+gcc without fast-math and without FP contraction).  This module only compiles
+it and marshals numpy arrays through ctypes.  Each wrapper names the passage
+it follows in the docstring of the C function it calls.
+
+Parity status: every function here is pinned by ``tests/test_oracle_*.py``
+(worked example from the lesson14_deepep practice task, brute force against a
+sort-based definition, exhaustive E4M3 checks, round-trip and dense-reference
+invariants).  None is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ep_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+OK, BAD_EXPERT, BAD_ARG = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile ep_oracle.c into liboracle.so next to it (no-op if up to date)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+           "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64 = ctypes.c_int32, ctypes.c_int64
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_encode_array.argtypes = [i64, P, P]
+        lib.oracle_e4m3_encode_array.restype = None
+        lib.oracle_capacity_rows.argtypes = [i32, i32, i32, i32]
+        lib.oracle_capacity_rows.restype = i64
+        lib.oracle_layout.argtypes = [i32, i32, i32, i32, i32] + [P] * 11
+        lib.oracle_layout.restype = ctypes.c_int
+        lib.oracle_dispatch_bf16.argtypes = [i32, i32, i32, P, P, P, P]
+        lib.oracle_dispatch_bf16.restype = ctypes.c_int
+        lib.oracle_dispatch_fp8.argtypes = [i32, i32, i32, P, P, P, P, P]
+        lib.oracle_dispatch_fp8.restype = ctypes.c_int
+        lib.oracle_combine.argtypes = [i32, i32, i32, i32, P, P, P, i32, P, P]
+        lib.oracle_combine.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """fp32 values -> OCP E4M3 codes (round to nearest even, saturate at 448)."""
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _load().oracle_e4m3_encode_array(v.size, _ptr(v), _ptr(out))
+    return out
+
+
+def capacity_rows(T: int, E: int, K: int, A: int) -> int:
+    return int(_load().oracle_capacity_rows(T, E, K, A))
+
+
+class Layout:
+    """Result of :func:`layout` (numpy arrays; rows = expert_offsets[-1])."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def layout(topk_idx, num_experts: int, num_ranks: int, expert_alignment: int = 1,
+           topk_weights=None) -> Layout:
+    """Counts, offsets and the stable (token, k) -> row permutation."""
+    idx = _c(topk_idx, np.int64)
+    T, K = idx.shape
+    E, R, A = num_experts, num_ranks, expert_alignment
+    cap = max(capacity_rows(T, E, K, A), 0)
+    w = None if topk_weights is None else _c(topk_weights, np.float32)
+    out = Layout(
+        num_tokens_per_expert=np.zeros(E, np.int32),
+        num_tokens_per_rank=np.zeros(R, np.int32),
+        is_token_in_rank=np.zeros((T, R), np.uint8),
+        expert_offsets=np.zeros(E + 1, np.int32),
+        rank_offsets=np.zeros(R + 1, np.int32),
+        pos=np.zeros((T, K), np.int32),
+        row_src=np.full(cap, -7, np.int32),
+        row_slot=np.full(cap, -7, np.int32),
+        row_weight=np.zeros(cap, np.float32),
+    )
+    rc = _load().oracle_layout(
+        T, E, R, K, A, _ptr(idx), _ptr(w), _ptr(out.num_tokens_per_expert),
+        _ptr(out.num_tokens_per_rank), _ptr(out.is_token_in_rank),
+        _ptr(out.expert_offsets), _ptr(out.rank_offsets), _ptr(out.pos),
+        _ptr(out.row_src), _ptr(out.row_slot), _ptr(out.row_weight))
+    out.status = rc
+    if rc == OK:
+        rows = int(out.expert_offsets[-1])
+        out.rows = rows
+        out.row_src = out.row_src[:rows]
+        out.row_slot = out.row_slot[:rows]
+        out.row_weight = out.row_weight[:rows]
+    out.capacity = cap
+    return out
+
+
+def dispatch_bf16(x_bits, row_src, sel_rows=None) -> np.ndarray:
+    """Received bf16 rows (as uint16 bit patterns) for all or selected rows."""
+    x = _c(x_bits, np.uint16)
+    T, H = x.shape
+    src = _c(row_src, np.int32)
+    sel = None if sel_rows is None else _c(sel_rows, np.int32)
+    n = src.shape[0] if sel is None else sel.shape[0]
+    out = np.empty((n, H), np.uint16)
+    rc = _load().oracle_dispatch_bf16(T, H, n, _ptr(sel), _ptr(src), _ptr(x), _ptr(out))
+    if rc != OK:
+        raise ValueError(f"oracle_dispatch_bf16 failed ({rc})")
+    return out
+
+
+def dispatch_fp8(x_bits, row_src, sel_rows=None):
+    """Received E4M3 codes [n, H] and fp32 scales [n, H/128]."""
+    x = _c(x_bits, np.uint16)
+    T, H = x.shape
+    src = _c(row_src, np.int32)
+    sel = None if sel_rows is None else _c(sel_rows, np.int32)
+    n = src.shape[0] if sel is None else sel.shape[0]
+    q = np.empty((n, H), np.uint8)
+    s = np.empty((n, H // 128), np.float32)
+    rc = _load().oracle_dispatch_fp8(T, H, n, _ptr(sel), _ptr(src), _ptr(x), _ptr(q), _ptr(s))
+    if rc != OK:
+        raise ValueError(f"oracle_dispatch_fp8 failed ({rc})")
+    return q, s
+
+
+def combine(y_bits, pos, topk_weights, sel_tokens=None) -> np.ndarray:
+    """fp64 weighted sum over k of the received rows, per (selected) token."""
+    y = _c(y_bits, np.uint16)
+    rows, H = y.shape
+    p = _c(pos, np.int32)
+    T, K = p.shape
+    w = _c(topk_weights, np.float32)
+    sel = None if sel_tokens is None else _c(sel_tokens, np.int32)
+    n = T if sel is None else sel.shape[0]
+    out = np.empty((n, H), np.float64)
+    rc = _load().oracle_combine(T, H, K, rows, _ptr(p), _ptr(y), _ptr(w), n, _ptr(sel), _ptr(out))
+    if rc != OK:
+        raise ValueError(f"oracle_combine failed ({rc})")
+    return out
