@@ -1,0 +1,418 @@
+// ep_api.cu -- host side of the C ABI declared in include/ep.h.
+//
+// Validates arguments, owns the handle's device arrays, chooses launch
+// shapes once per handle and enqueues kernels.  No host synchronisation,
+// allocation or copy on the layout/dispatch/combine calls.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "ep_internal.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+std::atomic<uint64_t> g_launches{0};
+
+int cuda_fail(cudaError_t e, const char *what) {
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s", what, cudaGetErrorString(e));
+    return EP_ERR_CUDA;
+}
+
+#define EP_CUDA(call)                                               \
+    do {                                                            \
+        cudaError_t _e = (call);                                    \
+        if (_e != cudaSuccess) return cuda_fail(_e, #call);         \
+    } while (0)
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Makes the handle's device current for the duration of a call.
+struct DeviceGuard {
+    int prev = -1;
+    cudaError_t err = cudaSuccess;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) err = cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+int check_handle(const ep_handle *h, bool need_layout) {
+    if (!h) return EP_ERR_ARG;
+    if (need_layout && !h->has_layout) return EP_ERR_STATE;
+    return EP_OK;
+}
+
+// Persistent grid for a kernel: SMs x resident blocks, capped by the units.
+int persistent_grid(const void *kernel, int threads, int num_sms) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    return per_sm * num_sms;
+}
+
+}  // namespace
+
+extern "C" {
+
+EP_API int ep_validate_config(const ep_config *c) {
+    if (!c) return EP_ERR_ARG;
+    if (c->num_tokens < 0 || c->hidden < 8 || c->hidden % 8 != 0) return EP_ERR_ARG;
+    if (c->num_experts < 1 || c->num_ranks < 1 || c->num_ranks > c->num_experts) return EP_ERR_ARG;
+    if (c->num_experts % c->num_ranks != 0) return EP_ERR_ARG;
+    if (c->num_topk < 1 || c->expert_alignment < 1) return EP_ERR_ARG;
+    if (c->num_experts > ep::kMaxExperts || c->num_topk > ep::kMaxTopk || c->expert_alignment > 65536)
+        return EP_ERR_UNSUPPORTED;
+    const int64_t cap = (int64_t)c->num_tokens * c->num_topk +
+                        (int64_t)c->num_experts * (c->expert_alignment - 1);
+    if (cap >= (int64_t(1) << 31)) return EP_ERR_UNSUPPORTED;
+    return EP_OK;
+}
+
+EP_API int64_t ep_capacity_rows(const ep_config *c) {
+    const int rc = ep_validate_config(c);
+    if (rc != EP_OK) return rc;
+    return (int64_t)c->num_tokens * c->num_topk + (int64_t)c->num_experts * (c->expert_alignment - 1);
+}
+
+EP_API int32_t ep_scales_per_row(const ep_config *c) {
+    const int rc = ep_validate_config(c);
+    if (rc != EP_OK) return rc;
+    return c->hidden / 128;
+}
+
+EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
+    if (!out) return EP_ERR_ARG;
+    *out = nullptr;
+    int rc = ep_validate_config(cfg);
+    if (rc != EP_OK) return rc;
+
+    ep_handle *h = new (std::nothrow) ep_handle();
+    if (!h) return EP_ERR_ARG;
+    h->cfg = *cfg;
+    h->cap = ep_capacity_rows(cfg);
+    h->wait_limit_ns = ep::kDefaultWaitLimitNs;
+    h->barrier_extra = 0;
+    h->has_layout = false;
+
+    auto fail = [&](int code) {
+        delete h;
+        return code;
+    };
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaGetDevice"));
+    e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaDeviceGetAttribute"));
+
+    const int T = cfg->num_tokens, E = cfg->num_experts, R = cfg->num_ranks, K = cfg->num_topk;
+
+    // layout: one chunk of >= kMinTokensPerChunk tokens per CTA, all CTAs resident
+    h->layout_smem = ep::layout_smem_bytes(E, R);
+    // the attribute is per kernel, not per handle: allow the largest supported size
+    e = cudaFuncSetAttribute(ep::layout_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)ep::layout_smem_bytes(ep::kMaxExperts, ep::kMaxExperts));
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaFuncSetAttribute(layout)"));
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ep::layout_kernel_ptr(),
+                                                      ep::kLayoutThreads, h->layout_smem);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor"));
+    if (per_sm < 1) return fail(EP_ERR_UNSUPPORTED);
+    const int g_max = h->num_sms;   // one CTA per SM keeps the grid-wide waits short
+    int G = (T + ep::kMinTokensPerChunk - 1) / ep::kMinTokensPerChunk;
+    G = G < 1 ? 1 : (G > g_max ? g_max : G);
+    int tpc = T > 0 ? (T + G - 1) / G : 1;
+    G = T > 0 ? (T + tpc - 1) / tpc : 1;
+    h->G = G;
+    h->tokens_per_chunk = tpc;
+
+    h->dispatch_grid = persistent_grid(ep::dispatch_bf16_kernel_ptr(), ep::dispatch_threads(), h->num_sms);
+    h->dispatch_fp8_grid = persistent_grid(ep::dispatch_fp8_kernel_ptr(), ep::dispatch_threads(), h->num_sms);
+    h->combine_grid = persistent_grid(ep::combine_kernel_ptr(K), ep::combine_threads(), h->num_sms);
+
+    // carve one allocation
+    const size_t A256 = 256;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = round_up(off + (bytes ? bytes : 1), A256);
+        return o;
+    };
+    const size_t o_pos = take(sizeof(int32_t) * (size_t)T * K);
+    const size_t o_src = take(sizeof(int32_t) * (size_t)h->cap);
+    const size_t o_slot = take(sizeof(int32_t) * (size_t)h->cap);
+    const size_t o_w = take(sizeof(float) * (size_t)h->cap);
+    const size_t o_cnt = take(sizeof(int32_t) * E);
+    const size_t o_rtok = take(sizeof(int32_t) * R);
+    const size_t o_eoff = take(sizeof(int32_t) * (E + 1));
+    const size_t o_roff = take(sizeof(int32_t) * (R + 1));
+    const size_t o_chunk = take(sizeof(int32_t) * (size_t)G * (E + R));
+    const size_t o_ctot = take(sizeof(int32_t) * (E + R));
+    const size_t o_bar = take(sizeof(ep::GridBarrier));
+    const size_t o_stat = take(sizeof(unsigned int));
+    h->block_bytes = off;
+    e = cudaMalloc(&h->block, h->block_bytes);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaMalloc(handle)"));
+    e = cudaMemset(h->block, 0, h->block_bytes);
+    if (e != cudaSuccess) {
+        cudaFree(h->block);
+        return fail(cuda_fail(e, "cudaMemset(handle)"));
+    }
+    char *b = static_cast<char *>(h->block);
+    h->pos = reinterpret_cast<int32_t *>(b + o_pos);
+    h->row_src = reinterpret_cast<int32_t *>(b + o_src);
+    h->row_slot = reinterpret_cast<int32_t *>(b + o_slot);
+    h->row_weight = reinterpret_cast<float *>(b + o_w);
+    h->cnt = reinterpret_cast<int32_t *>(b + o_cnt);
+    h->rank_tok = reinterpret_cast<int32_t *>(b + o_rtok);
+    h->eoff = reinterpret_cast<int32_t *>(b + o_eoff);
+    h->roff = reinterpret_cast<int32_t *>(b + o_roff);
+    h->chunk_counts = reinterpret_cast<int32_t *>(b + o_chunk);
+    h->col_total = reinterpret_cast<int32_t *>(b + o_ctot);
+    h->barrier = reinterpret_cast<ep::GridBarrier *>(b + o_bar);
+    h->status = reinterpret_cast<unsigned int *>(b + o_stat);
+    *out = h;
+    return EP_OK;
+}
+
+EP_API int ep_handle_destroy(ep_handle *h) {
+    if (!h) return EP_ERR_ARG;
+    int rc = EP_OK;
+    {
+        DeviceGuard g(h->device);
+        if (g.err != cudaSuccess) rc = cuda_fail(g.err, "cudaSetDevice");
+        cudaError_t e = cudaDeviceSynchronize();
+        if (e != cudaSuccess && rc == EP_OK) rc = cuda_fail(e, "cudaDeviceSynchronize");
+        e = cudaFree(h->block);
+        if (e != cudaSuccess && rc == EP_OK) rc = cuda_fail(e, "cudaFree(handle)");
+    }
+    delete h;
+    return rc;
+}
+
+EP_API int ep_handle_get_view(const ep_handle *h, ep_handle_view *v) {
+    if (!h || !v) return EP_ERR_ARG;
+    v->pos = h->pos;
+    v->row_src = h->row_src;
+    v->row_slot = h->row_slot;
+    v->row_weight = h->row_weight;
+    v->num_tokens_per_expert = h->cnt;
+    v->num_tokens_per_rank = h->rank_tok;
+    v->expert_offsets = h->eoff;
+    v->rank_offsets = h->roff;
+    v->status = h->status;
+    v->capacity = h->cap;
+    return EP_OK;
+}
+
+EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *topk_weights,
+                         int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+                         uint8_t *is_token_in_rank, int32_t *expert_offsets, int32_t *rank_offsets,
+                         ep_stream_t stream) {
+    int rc = check_handle(h, false);
+    if (rc != EP_OK) return rc;
+    const ep_config &c = h->cfg;
+    if (c.num_tokens > 0 && !topk_idx) return EP_ERR_ARG;
+    if (!aligned(topk_idx, 8) || !aligned(topk_weights, 4) || !aligned(num_tokens_per_expert, 4) ||
+        !aligned(num_tokens_per_rank, 4) || !aligned(expert_offsets, 4) || !aligned(rank_offsets, 4))
+        return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+
+    ep::LayoutParams p{};
+    p.topk_idx = topk_idx;
+    p.topk_weights = topk_weights;
+    p.T = c.num_tokens;
+    p.K = c.num_topk;
+    p.E = c.num_experts;
+    p.R = c.num_ranks;
+    p.L = c.num_experts / c.num_ranks;
+    p.A = c.expert_alignment;
+    p.G = h->G;
+    p.tokens_per_chunk = h->tokens_per_chunk;
+    p.pos = h->pos;
+    p.row_src = h->row_src;
+    p.row_slot = h->row_slot;
+    p.row_weight = h->row_weight;
+    p.cnt = h->cnt;
+    p.rank_tok = h->rank_tok;
+    p.eoff = h->eoff;
+    p.roff = h->roff;
+    p.u_cnt = num_tokens_per_expert;
+    p.u_rank_tok = num_tokens_per_rank;
+    p.u_eoff = expert_offsets;
+    p.u_roff = rank_offsets;
+    p.u_in_rank = is_token_in_rank;
+    p.chunk_counts = h->chunk_counts;
+    p.col_total = h->col_total;
+    p.barrier = h->barrier;
+    p.status = h->status;
+    p.wait_limit_ns = h->wait_limit_ns;
+    p.barrier_extra = h->barrier_extra;
+    cudaError_t e = ep::launch_layout(p, h->layout_smem, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launch(layout)");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    h->has_layout = true;
+    return EP_OK;
+}
+
+static int dispatch_common(const ep_handle *h, const void *x, void *recv, float *scales, bool fp8,
+                           ep_stream_t stream) {
+    int rc = check_handle(h, true);
+    if (rc != EP_OK) return rc;
+    const ep_config &c = h->cfg;
+    if (fp8 && c.hidden % 128 != 0) return EP_ERR_ARG;
+    if (c.num_tokens == 0) return EP_OK;   // nothing to write: rows == 0
+    if (!x || !recv || (fp8 && !scales)) return EP_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(recv, 16) || !aligned(scales, 4)) return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+
+    ep::DispatchParams p{};
+    p.x = x;
+    p.recv = recv;
+    p.recv_scale = scales;
+    p.pos = h->pos;
+    p.row_src = h->row_src;
+    p.eoff = h->eoff;
+    p.T = c.num_tokens;
+    p.K = c.num_topk;
+    p.E = c.num_experts;
+    p.H = c.hidden;
+    p.splits = 1;
+    p.n_token_units = p.T * p.splits;
+    p.n_zero_units = c.expert_alignment > 1
+                         ? (int)((h->cap + ep::kZeroRowsPerUnit - 1) / ep::kZeroRowsPerUnit)
+                         : 0;
+    const int units = p.n_token_units + p.n_zero_units;
+    int grid = fp8 ? h->dispatch_fp8_grid : h->dispatch_grid;
+    if (grid > units) grid = units;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = fp8 ? ep::launch_dispatch_fp8(p, grid, s) : ep::launch_dispatch_bf16(p, grid, s);
+    if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(dispatch_fp8)" : "launch(dispatch)");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return EP_OK;
+}
+
+EP_API int ep_dispatch(const ep_handle *h, const void *x, void *recv_x, ep_stream_t stream) {
+    return dispatch_common(h, x, recv_x, nullptr, false, stream);
+}
+
+EP_API int ep_dispatch_fp8(const ep_handle *h, const void *x, void *recv_q, float *recv_scales,
+                           ep_stream_t stream) {
+    return dispatch_common(h, x, recv_q, recv_scales, true, stream);
+}
+
+EP_API int ep_combine(const ep_handle *h, const void *y, const float *topk_weights, void *out,
+                      ep_stream_t stream) {
+    int rc = check_handle(h, true);
+    if (rc != EP_OK) return rc;
+    const ep_config &c = h->cfg;
+    if (c.num_tokens == 0) return EP_OK;
+    if (!y || !topk_weights || !out) return EP_ERR_ARG;
+    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(topk_weights, 4)) return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+
+    ep::CombineParams p{};
+    p.y = y;
+    p.w = topk_weights;
+    p.out = out;
+    p.pos = h->pos;
+    p.T = c.num_tokens;
+    p.K = c.num_topk;
+    p.H = c.hidden;
+    p.splits = 1;
+    p.n_units = p.T * p.splits;
+    int grid = h->combine_grid;
+    if (grid > p.n_units) grid = p.n_units;
+    cudaError_t e = ep::launch_combine(p, grid, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launch(combine)");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return EP_OK;
+}
+
+EP_API int ep_copy_routing(const ep_handle *h, int32_t *pos, int32_t *row_src, int32_t *row_slot,
+                           float *row_weight, ep_stream_t stream) {
+    int rc = check_handle(h, true);
+    if (rc != EP_OK) return rc;
+    if (!aligned(pos, 4) || !aligned(row_src, 4) || !aligned(row_slot, 4) || !aligned(row_weight, 4))
+        return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t npairs = (size_t)h->cfg.num_tokens * h->cfg.num_topk, ncap = (size_t)h->cap;
+    const cudaMemcpyKind d2d = cudaMemcpyDeviceToDevice;
+    if (pos && npairs) EP_CUDA(cudaMemcpyAsync(pos, h->pos, sizeof(int32_t) * npairs, d2d, s));
+    if (row_src && ncap) EP_CUDA(cudaMemcpyAsync(row_src, h->row_src, sizeof(int32_t) * ncap, d2d, s));
+    if (row_slot && ncap) EP_CUDA(cudaMemcpyAsync(row_slot, h->row_slot, sizeof(int32_t) * ncap, d2d, s));
+    if (row_weight && ncap) EP_CUDA(cudaMemcpyAsync(row_weight, h->row_weight, sizeof(float) * ncap, d2d, s));
+    return EP_OK;
+}
+
+EP_API int ep_get_num_rows(const ep_handle *h, int32_t *rows, ep_stream_t stream) {
+    int rc = check_handle(h, true);
+    if (rc != EP_OK) return rc;
+    if (!rows) return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    EP_CUDA(cudaMemcpyAsync(rows, h->eoff + h->cfg.num_experts, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+    EP_CUDA(cudaStreamSynchronize(s));
+    return EP_OK;
+}
+
+EP_API int ep_get_status(const ep_handle *h, uint32_t *bits, ep_stream_t stream) {
+    int rc = check_handle(h, false);
+    if (rc != EP_OK) return rc;
+    if (!bits) return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    EP_CUDA(cudaMemcpyAsync(bits, h->status, sizeof(uint32_t), cudaMemcpyDeviceToHost, s));
+    EP_CUDA(cudaStreamSynchronize(s));
+    return *bits ? EP_ERR_DEVICE : EP_OK;
+}
+
+EP_API int ep_clear_status(ep_handle *h, ep_stream_t stream) {
+    int rc = check_handle(h, false);
+    if (rc != EP_OK) return rc;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    EP_CUDA(cudaMemsetAsync(h->status, 0, sizeof(unsigned int), s));
+    EP_CUDA(cudaMemsetAsync(h->barrier, 0, sizeof(ep::GridBarrier), s));
+    return EP_OK;
+}
+
+EP_API int ep_set_wait_limit(ep_handle *h, uint64_t limit_ns, int32_t extra_arrivals) {
+    if (!h || limit_ns == 0 || extra_arrivals < 0) return EP_ERR_ARG;
+    h->wait_limit_ns = limit_ns;
+    h->barrier_extra = extra_arrivals;
+    return EP_OK;
+}
+
+EP_API const char *ep_status_string(int code) {
+    switch (code) {
+        case EP_OK: return "ok";
+        case EP_ERR_ARG: return "invalid argument (null pointer, size, alignment or E % R != 0)";
+        case EP_ERR_CUDA: return "CUDA runtime error (see ep_last_error)";
+        case EP_ERR_UNSUPPORTED: return "sizes beyond this build's limits";
+        case EP_ERR_STATE: return "handle has no layout yet";
+        case EP_ERR_DEVICE: return "device reported an error (bad expert id or wait timeout)";
+        default: return "unknown status";
+    }
+}
+
+EP_API const char *ep_last_error(void) { return g_last_error; }
+
+EP_API uint64_t ep_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,230 @@
+/*
+ * ep.h -- C ABI of the single-GPU expert-parallel dispatch/combine path
+ * (sm_100a).  Plain pointers and sizes only; no C++ or framework types.
+ *
+ * What it computes (the DeepEP-style dispatch/combine pair):
+ *   layout    counts, offsets and the stable (token, k) -> received-row
+ *             permutation from the router's top-k expert ids;
+ *   dispatch  copies (bf16) or quantises (FP8 E4M3, one fp32 scale per
+ *             1x128 block) each token row into the expert-contiguous
+ *             received buffer, once per selected expert;
+ *   combine   gathers the K expert-output rows of every token back and
+ *             returns their top-k weighted sum in token order.
+ * Sources: "bowenzhou.top/repos/deepep/01-overview" section 1.1 (EPBuffer
+ * dispatch arguments: expert_alignment, do_expand, do_zero_padding, handle),
+ * section 1.3 (golden path: dispatch returns data and a handle, combine(x,
+ * handle) reverses it), section 1.4 (V1 layout tensors num_tokens_per_rank,
+ * is_token_in_rank, num_tokens_per_expert); "lesson14_deepep" section 3 and
+ * its practice task (dispatch queues per expert, combine weighted sum);
+ * "2kiu.com/news/5702702" section 2.3 (FP8 transport); "blog.hotdry.top ...
+ * deepep-expert-parallel-alltoall" buffer section (num_experts divisible by
+ * the number of ranks).
+ *
+ * Notation: T tokens, H hidden size, E experts, R logical ranks, K top-k,
+ * A expert_alignment, L = E/R experts per rank.  Expert e belongs to rank
+ * e / L.  Received rows are expert-major (so rank-major), and inside an
+ * expert in (token, k) order; each expert segment is padded with zero rows
+ * to a multiple of A.  rows = sum_e ceil(cnt_e / A) * A <= capacity =
+ * T*K + E*(A-1).
+ *
+ * Conventions for every entry point:
+ *   - return EP_OK (0) or a negative ep_error code; nothing throws;
+ *   - every device pointer is a CUDA device allocation owned by the caller
+ *     (except the arrays a handle owns), contiguous, row-major, 16-byte
+ *     aligned unless stated; argument errors are found on the host before
+ *     any launch and leave all outputs untouched;
+ *   - work is enqueued on `stream` (NULL = legacy default stream) and is
+ *     asynchronous: no host synchronisation, allocation or copy happens in
+ *     ep_get_layout, ep_dispatch, ep_dispatch_fp8 or ep_combine;
+ *   - errors found on the device (an expert id outside [0, E), a bounded
+ *     in-kernel wait that gave up) set sticky bits in the handle's status
+ *     word, read with ep_get_status; outputs of that call are unspecified
+ *     but no out-of-bounds access is made;
+ *   - a handle may be used from one stream at a time; calls on one handle
+ *     from two streams that overlap on the GPU race.
+ */
+#ifndef EP_B200_EP_H
+#define EP_B200_EP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define EP_API __attribute__((visibility("default")))
+#else
+#define EP_API
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st *ep_stream_t;
+
+/* Host-side return codes. */
+enum ep_error {
+    EP_OK = 0,
+    EP_ERR_ARG = -1,         /* null pointer, bad size, misalignment, E % R != 0 ... */
+    EP_ERR_CUDA = -2,        /* a CUDA runtime call failed (see ep_last_error) */
+    EP_ERR_UNSUPPORTED = -3, /* sizes beyond this build's limits (see ep_config) */
+    EP_ERR_STATE = -4,       /* handle used before ep_get_layout, or on another device */
+    EP_ERR_DEVICE = -5       /* ep_get_status found device-side error bits */
+};
+
+/* Device status bits (sticky until ep_clear_status). */
+#define EP_DEV_BAD_EXPERT 0x1u   /* some topk_idx entry is outside [0, E) */
+#define EP_DEV_WAIT_TIMEOUT 0x2u /* a bounded in-kernel wait gave up */
+
+/*
+ * Problem sizes, fixed for the life of a handle.
+ *   num_tokens        T >= 0 (T = 0 is an empty batch)
+ *   hidden            H >= 8, H % 8 == 0; H % 128 == 0 for FP8 dispatch
+ *   num_experts       1 <= E <= 1024
+ *   num_ranks         1 <= R <= E, E % R == 0
+ *   num_topk          1 <= K <= 64 (repeated experts in a row are allowed:
+ *                     every (token, k) pair still gets its own row)
+ *   expert_alignment  1 <= A <= 65536
+ *   T*K + E*(A-1) must stay below 2^31.
+ */
+typedef struct {
+    int32_t num_tokens;
+    int32_t hidden;
+    int32_t num_experts;
+    int32_t num_ranks;
+    int32_t num_topk;
+    int32_t expert_alignment;
+} ep_config;
+
+/* Device arrays owned by a handle (valid until ep_handle_destroy). */
+typedef struct {
+    const int32_t *pos;                   /* [T, K]  received row of pair (t, k), -1 if its id was invalid */
+    const int32_t *row_src;               /* [capacity] token of row r, -1 for padding (rows < rows only) */
+    const int32_t *row_slot;              /* [capacity] k of row r, -1 for padding */
+    const float *row_weight;              /* [capacity] topk weight of row r, 0 for padding
+                                             (written only if ep_get_layout had topk_weights) */
+    const int32_t *num_tokens_per_expert; /* [E] */
+    const int32_t *num_tokens_per_rank;   /* [R] distinct tokens with >= 1 expert on rank r */
+    const int32_t *expert_offsets;        /* [E+1] padded exclusive prefix; [E] = rows */
+    const int32_t *rank_offsets;          /* [R+1] = expert_offsets[r * L] */
+    const uint32_t *status;               /* device status word (EP_DEV_* bits) */
+    int64_t capacity;                     /* T*K + E*(A-1) */
+} ep_handle_view;
+
+typedef struct ep_handle ep_handle;
+
+/* Checks cfg against the limits above.  Host only, no CUDA call. */
+EP_API int ep_validate_config(const ep_config *cfg);
+
+/* Worst-case received rows T*K + E*(A-1) (size recv buffers with it);
+ * a negative ep_error if cfg is invalid.  Host only. */
+EP_API int64_t ep_capacity_rows(const ep_config *cfg);
+
+/* Number of scale floats per received row for FP8 dispatch: H / 128. */
+EP_API int32_t ep_scales_per_row(const ep_config *cfg);
+
+/*
+ * Creates a handle on the current CUDA device: validates cfg and allocates
+ * (cudaMalloc, once) the routing arrays of ep_handle_view plus a small
+ * scratch area.  The only allocating call of this library.
+ */
+EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out);
+
+/* Frees the handle's device memory.  Synchronises the device first. */
+EP_API int ep_handle_destroy(ep_handle *h);
+
+/* Device pointers of the arrays the handle owns (see ep_handle_view). */
+EP_API int ep_handle_get_view(const ep_handle *h, ep_handle_view *out);
+
+/*
+ * Layout: from topk_idx [T, K] int64 (and optional topk_weights [T, K]
+ * fp32) fills the handle's routing arrays and, for each non-NULL pointer,
+ * the caller's copy:
+ *   num_tokens_per_expert [E] int32, num_tokens_per_rank [R] int32,
+ *   is_token_in_rank [T, R] uint8 (0/1), expert_offsets [E+1] int32,
+ *   rank_offsets [R+1] int32.
+ * topk_idx/topk_weights need 8/4-byte alignment only.  One cooperative
+ * kernel launch; its grid-wide waits are bounded (EP_DEV_WAIT_TIMEOUT).
+ * An id outside [0, E) sets EP_DEV_BAD_EXPERT; that pair gets pos = -1 and
+ * no row.
+ */
+EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *topk_weights,
+                         int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+                         uint8_t *is_token_in_rank, int32_t *expert_offsets,
+                         int32_t *rank_offsets, ep_stream_t stream);
+
+/*
+ * bf16 dispatch: recv_x[pos[t,k], :] = x[t, :] for every pair, and zero
+ * rows for the padding of each expert segment.  x is [T, H] bf16, recv_x is
+ * [capacity, H] bf16; rows at or beyond `rows` are not written.  Uses the
+ * layout last computed in h (a layout may serve any number of dispatches).
+ */
+EP_API int ep_dispatch(const ep_handle *h, const void *x, void *recv_x, ep_stream_t stream);
+
+/*
+ * FP8 dispatch: per token and 128-column block b, amax = max|x|,
+ * a = max(amax, 1e-4), codes = e4m3_rn_satfinite(x * (448 / a)) (IEEE fp32
+ * divide and multiply), recv_scales[row, b] = a / 448 (the dequantisation
+ * factor: x ~ code * scale).  All K copies of a token are identical;
+ * padding rows are code 0x00 with scale 0.  recv_q is [capacity, H] bytes
+ * (16-byte aligned), recv_scales is [capacity, H/128] fp32 (4-byte
+ * aligned).  Needs H % 128 == 0.
+ */
+EP_API int ep_dispatch_fp8(const ep_handle *h, const void *x, void *recv_q, float *recv_scales,
+                           ep_stream_t stream);
+
+/*
+ * Combine: out[t, :] = bf16_rn( sum_{k=0..K-1} topk_weights[t,k] *
+ * y[pos[t,k], :] ), accumulated in fp32 with fused multiply-adds in k order
+ * starting from 0.  y is [capacity, H] bf16 in the received-row layout of h
+ * (expert outputs), topk_weights [T, K] fp32 (4-byte aligned), out [T, H]
+ * bf16.  Padding rows are never read; pairs with pos = -1 add nothing.
+ */
+EP_API int ep_combine(const ep_handle *h, const void *y, const float *topk_weights, void *out,
+                      ep_stream_t stream);
+
+/*
+ * Copies the handle's routing arrays into caller device buffers (any
+ * pointer may be NULL to skip it), stream-ordered: pos [T, K] int32,
+ * row_src / row_slot [capacity] int32, row_weight [capacity] fp32.  The
+ * analogue of EPBuffer.dispatch's do_handle_copy (bowenzhou.top
+ * "deepep/01-overview" section 1.1): the copy outlives later layouts.
+ */
+EP_API int ep_copy_routing(const ep_handle *h, int32_t *pos, int32_t *row_src, int32_t *row_slot,
+                           float *row_weight, ep_stream_t stream);
+
+/* Synchronises `stream` and returns rows (= expert_offsets[E]) on the host. */
+EP_API int ep_get_num_rows(const ep_handle *h, int32_t *rows, ep_stream_t stream);
+
+/*
+ * Synchronises `stream` and returns the device status bits; EP_OK if they
+ * are zero, EP_ERR_DEVICE otherwise.
+ */
+EP_API int ep_get_status(const ep_handle *h, uint32_t *bits, ep_stream_t stream);
+
+/* Clears the status word and the in-kernel wait state (stream-ordered). */
+EP_API int ep_clear_status(ep_handle *h, ep_stream_t stream);
+
+/*
+ * Limit for each bounded in-kernel wait, in nanoseconds of %globaltimer
+ * (default 1e9).  `extra_arrivals` > 0 makes the layout's grid-wide wait
+ * expect that many CTAs that never arrive: a test hook that exercises the
+ * timeout path without hanging (the wait gives up after limit_ns and sets
+ * EP_DEV_WAIT_TIMEOUT).  Use 0 in normal operation.
+ */
+EP_API int ep_set_wait_limit(ep_handle *h, uint64_t limit_ns, int32_t extra_arrivals);
+
+/* Static description of a return code. */
+EP_API const char *ep_status_string(int code);
+
+/* Text of the last CUDA error seen by this library on the calling thread. */
+EP_API const char *ep_last_error(void);
+
+/* Number of kernels this library has launched in this process. */
+EP_API uint64_t ep_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_EP_H */

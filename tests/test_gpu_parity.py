@@ -1,0 +1,254 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bit-exact: layout (counts, membership, offsets, pos, row_src/row_slot,
+row_weight), bf16 received rows, FP8 codes and scales.  Combine within
+rtol 1e-2 / atol 1e-3 of the oracle's fp64 weighted sum.
+"""
+import numpy as np
+import pytest
+import torch
+
+import combine_ep_get_08_b200 as ep
+import oracle
+import workloads
+from ep_harness import (assert_layout_equal, combine_close, expert_outputs, gpu_layout)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from combine_ep_get_08_b200 import build_lib
+    build_lib.build()
+    oracle.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def run_full(wl, fp8: bool, y_seed=99, check_rows=None, check_tokens=None):
+    """Layout + dispatch + combine on the GPU, compared with the oracle.
+
+    check_rows / check_tokens: compare only these received rows / tokens
+    (indexing happens on the device); None compares everything."""
+    dev = torch.device("cuda")
+    idx, w = wl.topk_idx.numpy(), wl.topk_weights.numpy()
+    o = oracle.layout(idx, wl.E, wl.R, wl.A, topk_weights=w)
+    assert o.status == 0
+    g = gpu_layout(wl)
+    try:
+        assert_layout_equal(g, o)
+        x_d = wl.x.to(dev)
+        xb = workloads.bf16_bits(wl.x)
+        cap = g.cap
+        sel = np.arange(g.rows, dtype=np.int32) if check_rows is None else np.asarray(check_rows, np.int32)
+        sel_d = torch.from_numpy(sel).long().to(dev)
+        if fp8:
+            q = torch.full((max(cap, 1), wl.H), 0x5A, dtype=torch.uint8, device=dev)
+            s = torch.full((max(cap, 1), wl.H // 128), -3.0, dtype=torch.float32, device=dev)
+            ep.ep_dispatch_fp8(g.handle, x_d, q, s)
+            q_h = q[sel_d].cpu().numpy()
+            s_h = s[sel_d].cpu().numpy()
+            oq, osc = oracle.dispatch_fp8(xb, o.row_src, sel)
+            np.testing.assert_array_equal(q_h, oq, err_msg="fp8 codes")
+            np.testing.assert_array_equal(s_h.view(np.uint32), osc.view(np.uint32), err_msg="fp8 scales")
+            if cap > g.rows:                      # rows beyond `rows` are untouched
+                assert bool((q[g.rows:cap] == 0x5A).all())
+            del q, s
+        else:
+            recv = torch.full((max(cap, 1), wl.H), 12345, dtype=torch.int16, device=dev).view(torch.bfloat16)
+            ep.ep_dispatch(g.handle, x_d, recv)
+            r_h = workloads.bf16_bits(recv[sel_d])
+            np.testing.assert_array_equal(r_h, oracle.dispatch_bf16(xb, o.row_src, sel), err_msg="bf16 rows")
+            if cap > g.rows:
+                assert bool((recv[g.rows:cap].view(torch.int16) == 12345).all())
+            del recv
+        # combine of stand-in expert outputs y [cap, H] (seeded N(0,1), made on the device)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(y_seed)
+        y_d = torch.randn((max(cap, 1), wl.H), generator=gen, device=dev).to(torch.bfloat16)
+        w_d = wl.topk_weights.to(dev)
+        out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+        ep.ep_combine(g.handle, y_d, w_d, out)
+        tsel = np.arange(wl.T, dtype=np.int32) if check_tokens is None else np.asarray(check_tokens, np.int32)
+        if len(tsel):
+            need = o.pos[tsel]                     # [n, K] rows those tokens read
+            uniq, inv = np.unique(need, return_inverse=True)
+            y_small = workloads.bf16_bits(y_d[torch.from_numpy(uniq).long().to(dev)])
+            ref = oracle.combine(y_small, inv.reshape(need.shape).astype(np.int32), w[tsel])
+            combine_close(out[torch.from_numpy(tsel).long().to(dev)], ref)
+        assert ep.ep_get_status(g.handle) == 0
+    finally:
+        ep.ep_handle_destroy(g.handle)
+
+
+SMALL = [
+    dict(name="tiny"),
+    dict(T=1000, H=7168, E=64, R=4, K=6, A=3, router="topk", seed=21),
+    dict(T=777, H=200, E=32, R=8, K=4, A=1, router="uniform", seed=22),      # ragged row (25 vectors)
+    dict(T=513, H=384, E=256, R=32, K=8, A=16, router="group", seed=23),
+    dict(T=33, H=128, E=1024, R=128, K=64, A=2, router="topk", seed=24),      # max E, max K, R > 64
+    dict(T=1, H=8, E=1, R=1, K=1, A=1, router="topk", seed=25),
+    dict(T=300, H=1024, E=8, R=2, K=8, A=300, router="topk", seed=26),      # A > T*K/E
+]
+
+
+def _wl(spec):
+    spec = dict(spec)
+    name = spec.pop("name", None)
+    return workloads.generate(name, **spec)
+
+
+@pytest.mark.parametrize("spec", SMALL, ids=lambda s: s.get("name") or f"T{s['T']}H{s['H']}E{s['E']}K{s['K']}A{s['A']}")
+@pytest.mark.parametrize("fp8", [False, True])
+def test_small_parity(spec, fp8):
+    wl = _wl(spec)
+    if fp8 and wl.H % 128:
+        pytest.skip("FP8 needs H % 128 == 0")
+    run_full(wl, fp8)
+
+
+@pytest.mark.parametrize("name", ["dsv3", "decode", "skew", "large"])
+def test_full_size_parity(name):
+    """Full-size workloads in the launch configuration the bench uses:
+    full layout bit-exact, sampled received rows and tokens."""
+    wl = workloads.generate(name)
+    rng = np.random.default_rng(5)
+    cap = wl.T * wl.K + wl.E * (wl.A - 1)
+    o = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A)
+    rows = o.rows
+    sel_rows = np.unique(np.concatenate([[0, rows - 1], rng.integers(0, rows, 1500),
+                                         np.flatnonzero(o.row_src < 0)[:200]]))
+    sel_tok = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 300)]))
+    run_full(wl, wl.fp8, check_rows=sel_rows, check_tokens=sel_tok)
+    if name == "dsv3":
+        # bench's dsv3 step is bf16; also check the FP8 variant on the same routing
+        run_full(wl, True, check_rows=sel_rows, check_tokens=sel_tok)
+
+
+def test_identity_round_trip_bf16():
+    """combine(dispatch(x)) with identity experts returns x * sum_k w."""
+    dev = torch.device("cuda")
+    wl = workloads.generate(None, T=2048, H=7168, E=256, R=8, K=8, A=1, router="group", seed=31)
+    g = gpu_layout(wl)
+    try:
+        x_d = wl.x.to(dev)
+        recv = torch.empty((g.cap, wl.H), dtype=torch.bfloat16, device=dev)
+        ep.ep_dispatch(g.handle, x_d, recv)
+        out = torch.empty_like(x_d)
+        ep.ep_combine(g.handle, recv, wl.topk_weights.to(dev), out)
+        ref = wl.x.double().numpy() * wl.topk_weights.double().numpy().sum(1, keepdims=True)
+        combine_close(out, ref)
+    finally:
+        ep.ep_handle_destroy(g.handle)
+
+
+def test_handle_reuse_and_determinism():
+    dev = torch.device("cuda")
+    wl = workloads.generate(None, T=600, H=1024, E=64, R=8, K=8, A=4, router="topk", seed=41)
+    g = gpu_layout(wl)
+    try:
+        g2 = gpu_layout(wl, handle=g.handle)      # same handle, second layout: identical bytes
+        for key in ("pos", "row_src", "row_slot", "expert_offsets"):
+            np.testing.assert_array_equal(getattr(g, key), getattr(g2, key))
+        o = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A)
+        for seed in (1, 2, 3):                     # three dispatches on one layout
+            x = workloads.bf16_normal(np.random.default_rng(seed), wl.T, wl.H)
+            recv = torch.empty((g.cap, wl.H), dtype=torch.bfloat16, device=dev)
+            ep.ep_dispatch(g.handle, x.to(dev), recv)
+            np.testing.assert_array_equal(workloads.bf16_bits(recv[:g.rows]),
+                                          oracle.dispatch_bf16(workloads.bf16_bits(x), o.row_src))
+    finally:
+        ep.ep_handle_destroy(g.handle)
+
+
+def test_empty_batch():
+    dev = torch.device("cuda")
+    wl = workloads.generate(None, T=0, H=256, E=16, R=4, K=2, A=8, router="topk", seed=1)
+    g = gpu_layout(wl)
+    try:
+        assert g.rows == 0 and g.status == 0
+        assert (g.expert_offsets == 0).all() and (g.num_tokens_per_expert == 0).all()
+        x = torch.empty((0, wl.H), dtype=torch.bfloat16, device=dev)
+        ep.ep_dispatch(g.handle, x, x)
+        ep.ep_combine(g.handle, x, torch.empty((0, 2), device=dev), x)
+    finally:
+        ep.ep_handle_destroy(g.handle)
+
+
+def test_repeated_experts_in_a_row():
+    wl = workloads.generate(None, T=100, H=256, E=8, R=2, K=4, A=2, router="topk", seed=3)
+    idx = wl.topk_idx.clone()
+    idx[:, 1] = idx[:, 0]                         # every token names its first expert twice
+    wl.topk_idx = idx
+    run_full(wl, False)
+    run_full(wl, True)
+
+
+def test_invalid_expert_id_sets_status():
+    dev = torch.device("cuda")
+    wl = workloads.generate(None, T=50, H=256, E=16, R=4, K=2, A=1, router="uniform", seed=4)
+    idx = wl.topk_idx.clone()
+    idx[7, 1] = 16
+    idx[9, 0] = -1
+    g = gpu_layout(wl, idx_d=idx.to(dev))
+    try:
+        assert g.status & ep.EP_DEV_BAD_EXPERT
+        assert g.pos[7, 1] == -1 and g.pos[9, 0] == -1
+        assert int(g.num_tokens_per_expert.sum()) == 50 * 2 - 2
+        # dispatch/combine skip the invalid pairs and stay in bounds
+        x_d = wl.x.to(dev)
+        recv = torch.zeros((g.cap, wl.H), dtype=torch.bfloat16, device=dev)
+        ep.ep_dispatch(g.handle, x_d, recv)
+        out = torch.empty_like(x_d)
+        ep.ep_combine(g.handle, recv, wl.topk_weights.to(dev), out)
+        torch.cuda.synchronize()
+        ep.ep_clear_status(g.handle)
+        assert ep.ep_get_status(g.handle) == 0
+    finally:
+        ep.ep_handle_destroy(g.handle)
+
+
+def test_bounded_wait_gives_up():
+    """A grid-wide wait that can never complete ends after its limit with
+    EP_DEV_WAIT_TIMEOUT; after ep_clear_status the handle works again."""
+    dev = torch.device("cuda")
+    wl = workloads.generate(None, T=4096, H=256, E=256, R=8, K=8, A=1, router="topk", seed=5)
+    cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
+    h = ep.ep_handle_create(cfg)
+    try:
+        ep.ep_set_wait_limit(h, 20_000_000, 1)     # 20 ms, one CTA that never arrives
+        idx_d = wl.topk_idx.to(dev)
+        ep.ep_get_layout(h, idx_d)
+        assert ep.ep_get_status(h) & ep.EP_DEV_WAIT_TIMEOUT
+        ep.ep_set_wait_limit(h, 1_000_000_000, 0)
+        ep.ep_clear_status(h)
+        g = gpu_layout(wl, handle=h, with_weights=False)
+        assert g.status == 0
+        o = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A)
+        assert_layout_equal(g, o, with_weights=False)
+    finally:
+        ep.ep_handle_destroy(h)
+
+
+def test_host_argument_errors():
+    dev = torch.device("cuda")
+    cfg = ep.make_config(16, 256, 8, 2, 2, 1)
+    h = ep.ep_handle_create(cfg)
+    try:
+        x = torch.zeros((16, 256), dtype=torch.bfloat16, device=dev)
+        with pytest.raises(ep.EpError) as ei:
+            ep.ep_dispatch(h, x, x)               # no layout yet
+        assert ei.value.code == ep.EP_ERR_STATE
+        idx = torch.zeros((16, 2), dtype=torch.int64, device=dev)
+        ep.ep_get_layout(h, idx)
+        recv = torch.zeros((40, 256), dtype=torch.bfloat16, device=dev)
+        with pytest.raises(ep.EpError) as ei:
+            ep.ep_dispatch(h, x.data_ptr() + 2, recv)   # misaligned
+        assert ei.value.code == ep.EP_ERR_ARG
+        with pytest.raises(ep.EpError) as ei:
+            ep.ep_dispatch_fp8(h, x, recv, None)  # FP8 without a scale buffer
+        assert ei.value.code == ep.EP_ERR_ARG
+    finally:
+        ep.ep_handle_destroy(h)
+    with pytest.raises(ep.EpError):
+        ep.ep_handle_create(ep.make_config(16, 256, 9, 2, 2, 1))   # E % R != 0
