@@ -1,0 +1,527 @@
+#!/usr/bin/env python
+"""Benchmark of the dispatch/combine hot path on B200.
+
+One step = layout (ep_get_layout) + dispatch (ep_dispatch, or
+ep_dispatch_fp8) + combine (ep_combine) over one batch of the named
+workload, through the C ABI.  Default workload: the DeepSeek-V3 prefill
+shape (4096 tokens x hidden 7168 bf16, 256 experts over 8 logical ranks,
+group-limited top-8), bf16 dispatch + combine, identity experts (combine
+reads the dispatched rows).
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and torch.cuda.synchronize() on both sides.  Every kernel is timed with CUDA
+events on the stream it is launched on.  The 126 MB L2 is flushed (256 MiB
+write, outside the events) before each step and between dispatch and
+combine, where the expert GEMMs would run (a 256 MiB read: it leaves no dirty
+lines for the timed kernel to write back).  value = algorithmic bytes of
+dispatch + combine per step / device time of the step (layout + dispatch +
+combine), summed over ranks and divided by the max over ranks.
+
+--impl reference times the CPU oracle (single thread) on a bounded sample of
+the same workload instead.  Multi-GPU (torchrun): every rank runs its own
+replica on its own GPU (independent batches, no collective on the data
+path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine µs/call and effective HBM GB/s (% of B200 peak) at 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------
+# byte model (algorithmic bytes, metadata excluded)
+# ----------------------------------------------------------------------------
+def row_bytes(H: int, fp8: bool) -> int:
+    return H + 4 * (H // 128) if fp8 else 2 * H
+
+
+def dispatch_bytes(T, H, K, rows, fp8) -> int:
+    """read x once + write every received row (padding rows included)."""
+    return 2 * T * H + rows * row_bytes(H, fp8)
+
+
+def combine_bytes(T, H, K) -> int:
+    """read the T*K expert-output rows (bf16) + write out (bf16)."""
+    return 2 * T * K * H + 2 * T * H
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (host logic; tested with gloo on CPU)
+# ----------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# clocks (NVML reads only; no setting is changed)
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {  # NVML clocks-event reason bits
+        0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+        0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._nvml = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# roofline inputs
+# ----------------------------------------------------------------------------
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "combine_ep_get_08_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            data = json.load(f)
+    except Exception:  # noqa: BLE001
+        return None
+    if data.get("source_digest") != kernel_source_digest():
+        return None
+    entry = data.get("kernels", {}).get(workload, {}).get(kernel)
+    return None if entry is None else entry.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle arm
+# ----------------------------------------------------------------------------
+def oracle_sample(wl, budget_s: float, min_steps: int = 1):
+    """Time the oracle on full steps of the workload until budget_s elapsed.
+    Returns (GB/s, steps, seconds, bytes_per_step)."""
+    import numpy as np
+
+    import oracle
+    import workloads
+    oracle.build()
+    idx, w = wl.topk_idx.numpy(), wl.topk_weights.numpy()
+    xb = workloads.bf16_bits(wl.x)
+    n, t0 = 0, time.perf_counter()
+    bytes_step = None
+    while True:
+        lay = oracle.layout(idx, wl.E, wl.R, wl.A, topk_weights=w)
+        if wl.fp8:
+            oracle.dispatch_fp8(xb, lay.row_src)
+            y = np.zeros((lay.rows, wl.H), np.uint16)
+        else:
+            y = oracle.dispatch_bf16(xb, lay.row_src)
+        oracle.combine(y, lay.pos, w)
+        n += 1
+        bytes_step = dispatch_bytes(wl.T, wl.H, wl.K, lay.rows, wl.fp8) + combine_bytes(wl.T, wl.H, wl.K)
+        el = time.perf_counter() - t0
+        if n >= min_steps and el >= budget_s:
+            break
+    return bytes_step * n / el / 1e9, n, el, bytes_step
+
+
+def run_reference(args, world, rank):
+    import workloads
+    if rank != 0:
+        return 0
+    wl = workloads.generate(args.config)
+    _, _, _, bytes_step = oracle_sample(wl, 0.0)              # one untimed call
+    # warm-up steps (untimed), then K timed steps; a step is one oracle pass
+    # over a token sample of the batch, scaled to GB/s by the bytes it covers
+    sample_T = min(wl.T, args.ref_tokens)
+    sub = workloads.generate(args.config) if sample_T == wl.T else _subsample(wl, sample_T)
+    for _ in range(args.warmup):
+        oracle_sample(sub, 0.0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        gbs, _, _, bstep = oracle_sample(sub, 0.0)
+    el = time.perf_counter() - t0
+    value = bstep * args.steps / el / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workloads.DESCRIPTIONS[args.config], "sample_tokens": sample_T},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: oracle layout + dispatch + combine over the first "
+                                   f"{sample_T} of {wl.T} tokens of the workload (single thread)"},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _subsample(wl, T):
+    import copy
+    sub = copy.copy(wl)
+    sub.T = T
+    sub.topk_idx = wl.topk_idx[:T].contiguous()
+    sub.topk_weights = wl.topk_weights[:T].contiguous()
+    sub.x = wl.x[:T].contiguous()
+    return sub
+
+
+# ----------------------------------------------------------------------------
+# CUDA arm
+# ----------------------------------------------------------------------------
+class Path:
+    """Device buffers and one handle for a workload; step() enqueues one pass."""
+
+    def __init__(self, wl, dev):
+        import torch
+
+        import combine_ep_get_08_b200 as ep
+        self.ep, self.torch, self.wl, self.dev = ep, torch, wl, dev
+        cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
+        self.cap = ep.ep_capacity_rows(cfg)
+        self.h = ep.ep_handle_create(cfg)
+        self.idx = wl.topk_idx.to(dev)
+        self.w = wl.topk_weights.to(dev)
+        self.x = wl.x.to(dev)
+        if wl.fp8:
+            self.recv = torch.empty((self.cap, wl.H), dtype=torch.uint8, device=dev)
+            self.scales = torch.empty((self.cap, wl.H // 128), dtype=torch.float32, device=dev)
+            g = torch.Generator(device=dev)
+            g.manual_seed(7)
+            self.y = torch.randn((self.cap, wl.H), generator=g, device=dev).to(torch.bfloat16)
+        else:
+            self.recv = torch.empty((self.cap, wl.H), dtype=torch.bfloat16, device=dev)
+            self.scales = None
+            self.y = self.recv                     # identity experts
+        self.out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+        # fp32 so that the reduction reads it in place (an int32 sum would first
+        # widen it to an int64 copy: 512 MB of writes)
+        self.flush_buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.flush_sink = None
+
+    def flush_l2(self):
+        # read 256 MiB (2x the L2): evicts every line without leaving dirty
+        # lines behind for the next timed kernel to write back
+        self.flush_sink = self.flush_buf.sum()
+
+    def layout(self, stream):
+        self.ep.ep_get_layout(self.h, self.idx, self.w, stream=stream)
+
+    def dispatch(self, stream, x=None):
+        x = self.x if x is None else x
+        if self.wl.fp8:
+            self.ep.ep_dispatch_fp8(self.h, x, self.recv, self.scales, stream=stream)
+        else:
+            self.ep.ep_dispatch(self.h, x, self.recv, stream=stream)
+
+    def combine(self, stream, out=None):
+        self.ep.ep_combine(self.h, self.y, self.w, self.out if out is None else out, stream=stream)
+
+    def close(self):
+        self.ep.ep_handle_destroy(self.h)
+
+
+def run_cuda(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import combine_ep_get_08_b200 as ep
+    import workloads
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}), flush=True)
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    from combine_ep_get_08_b200 import build_lib
+    if rank == 0:
+        build_lib.build()
+    barrier(world)
+    ep.library()
+
+    base = workloads.CONFIGS[args.config]
+    wl = workloads.generate(args.config, seed=base["seed"] + 1000 * rank)
+    reuse = base["reuse"] if args.reuse is None else args.reuse
+    path = Path(wl, dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+
+    def one_step(ev=None):
+        path.flush_l2()
+        if ev is not None:
+            ev[0].record(stream)
+        path.layout(sptr)
+        if ev is not None:
+            ev[1].record(stream)
+        for r in range(reuse):
+            path.dispatch(sptr)
+            if ev is not None and r == 0:
+                ev[2].record(stream)
+            path.flush_l2()
+            if ev is not None and r == 0:
+                ev[3].record(stream)
+            path.combine(sptr)
+            if ev is not None and r == 0:
+                ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    rows = ep.ep_get_num_rows(path.h)
+    status = ep.ep_get_status(path.h)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    bracket = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    launches0 = ep.ep_launch_count()
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        bracket[0].record(stream)
+        for i in range(args.steps):
+            one_step(evs[i])
+        bracket[1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    launches = ep.ep_launch_count() - launches0
+
+    lay_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dis_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    com_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    # with reuse > 1 only the first dispatch/combine pair of a step carries events;
+    # the step's device time counts every call at that per-call time
+    step_ms = [l + reuse * (d + c) for l, d, c in zip(lay_ms, dis_ms, com_ms)]
+    total_ms = sum(step_ms)
+    bracket_ms = bracket[0].elapsed_time(bracket[1])
+
+    b_dis = dispatch_bytes(wl.T, wl.H, wl.K, rows, wl.fp8)
+    b_com = combine_bytes(wl.T, wl.H, wl.K)
+    bytes_step = reuse * (b_dis + b_com)
+    my_bytes = bytes_step * args.steps
+    all_bytes = sum_over_ranks(my_bytes, world, dev)
+    max_total_ms = max_over_ranks(total_ms, world, dev)
+    value = all_bytes / (max_total_ms * 1e-3) / 1e9
+
+    # e2e: same step through the public API with pinned host buffers
+    e2e = run_e2e(path, args, stream, reuse, world, dev, bytes_step)
+
+    lay_us, dis_us, com_us = (statistics.mean(v) * 1e3 for v in (lay_ms, dis_ms, com_ms))
+    peak, peak_src = measured_peak()
+    kern = {"layout": lay_us, "dispatch": dis_us, "combine": com_us}
+    dom = "dispatch" if dis_us >= com_us else "combine"
+    dom_bytes = b_dis if dom == "dispatch" else b_com
+    achieved = dom_bytes / (kern[dom] * 1e-6) / 1e9
+    kname = {"dispatch": "dispatch_fp8_kernel" if wl.fp8 else "dispatch_bf16_kernel",
+             "combine": "combine_kernel"}[dom]
+    clocks = sampler.summary()
+    status_end = ep.ep_get_status(path.h)
+    path.close()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(max_total_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": workloads.DESCRIPTIONS[args.config], "name": args.config,
+                "rows": rows, "reuse": reuse,
+                "parallelism": f"replicas x{world} (independent batches, no data-path collective)",
+                "l2": "flushed (256 MiB read, outside the timed events) before each step and "
+                      "between dispatch and combine",
+            },
+            "us_per_call": {k: round(v, 2) for k, v in kern.items()},
+            "bytes_per_call": {"dispatch": b_dis, "combine": b_com},
+            "gbs_per_call": {"dispatch": round(b_dis / dis_us / 1e3, 1),
+                             "combine": round(b_com / com_us / 1e3, 1)},
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
+                         "peak": peak, "peak_source": peak_src, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4),
+                         "traffic": ncu_traffic(kname, args.config)},
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+            "bracket_ms": round(bracket_ms, 3),
+            "device_status": int(status | status_end),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            gbs, n, el, _ = oracle_sample(wl, args.cpu_budget)
+            line["cpu_baseline"] = {
+                "value": round(gbs, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                "sample": f"{n} full step(s) of the same workload (layout + dispatch + combine, "
+                          f"{el:.1f} s, single thread)"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(path, args, stream, reuse, world, dev, bytes_step):
+    """Host buffers in, host result out, through the same C-ABI calls."""
+    import torch
+    wl = path.wl
+    x_h = wl.x.pin_memory()
+    idx_h = wl.topk_idx.pin_memory()
+    w_h = wl.topk_weights.pin_memory()
+    out_h = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(path.x)
+    sptr = stream.cuda_stream
+    n = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        path.idx.copy_(idx_h, non_blocking=True)
+        path.w.copy_(w_h, non_blocking=True)
+        path.layout(sptr)
+        for _ in range(reuse):
+            path.dispatch(sptr, x=x_d)
+            path.combine(sptr)
+        out_h.copy_(path.out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    t = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(world)
+    t[0].record(stream)
+    for _ in range(n):
+        e2e_step()
+    t[1].record(stream)
+    torch.cuda.synchronize()
+    ms = t[0].elapsed_time(t[1]) / n
+    ms = max_over_ranks(ms, world, dev)
+    total = sum_over_ranks(bytes_step, world, dev)
+    h2d = x_h.numel() * 2 + idx_h.numel() * 8 + w_h.numel() * 4
+    d2h = out_h.numel() * 2
+    return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--config", default="dsv3", choices=["tiny", "dsv3", "decode", "skew", "large"])
+    ap.add_argument("--reuse", type=int, default=None, help="dispatch+combine calls per layout")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds for the oracle baseline")
+    ap.add_argument("--ref-tokens", type=int, default=4096, help="tokens per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 must be launched with torchrun (one process per GPU)")
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_cuda(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -26,13 +26,31 @@ __device__ __forceinline__ unsigned int pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const unsigned int *>(&v);
 }
 
+// NW = bf16x2 words per vector (4: 16-byte loads; a 32-byte variant needs
+// ~100 registers, halves occupancy and measured slower).
+template <int NW>
+struct CVec;
+template <>
+struct CVec<4> {
+    static __device__ __forceinline__ void load(const void *p, unsigned int (&w)[4]) {
+        const uint4 v = ld_stream_v4(p);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    }
+    static __device__ __forceinline__ void store(void *p, const unsigned int (&w)[4]) {
+        st_v4(p, make_uint4(w[0], w[1], w[2], w[3]));
+    }
+};
+
+template <int NW>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
+    constexpr int VB = NW * 4;               // bytes per vector
     __shared__ int32_t s_src[kMaxTopk];
     __shared__ float s_w[kMaxTopk];
-    const int V = p.H / 8;
+    const int row_bytes = p.H * 2;
+    const int V = row_bytes / VB;
     const int vps = (V + p.splits - 1) / p.splits;
-    const uint4 *y = static_cast<const uint4 *>(p.y);
-    uint4 *out = static_cast<uint4 *>(p.out);
+    const uint8_t *y = static_cast<const uint8_t *>(p.y);
+    uint8_t *out = static_cast<uint8_t *>(p.out);
     for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
         const int t = u / p.splits, s = u - t * p.splits;
         if (threadIdx.x < p.K) {
@@ -42,38 +60,38 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
         __syncthreads();
         const int v0 = s * vps, v1 = min(V, v0 + vps);
         for (int v = v0 + threadIdx.x; v < v1; v += kThreads) {
-            float acc[8];
+            float acc[2 * NW];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 2 * NW; ++i) acc[i] = 0.0f;
             for (int k0 = 0; k0 < p.K; k0 += kLoadsInFlight) {
-                uint4 yv[kLoadsInFlight];
+                unsigned int yv[kLoadsInFlight][NW];
 #pragma unroll
                 for (int j = 0; j < kLoadsInFlight; ++j) {
                     const int k = k0 + j;
                     const int src = k < p.K ? s_src[k] : -1;
-                    yv[j] = src >= 0 ? ld_stream_v4(y + (int64_t)src * V + v) : make_uint4(0, 0, 0, 0);
+                    if (src >= 0) {
+                        CVec<NW>::load(y + (int64_t)src * row_bytes + (int64_t)v * VB, yv[j]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < NW; ++i) yv[j][i] = 0;
+                    }
                 }
 #pragma unroll
                 for (int j = 0; j < kLoadsInFlight; ++j) {
                     const int k = k0 + j;
                     if (k >= p.K || s_src[k] < 0) continue;
                     const float wk = s_w[k];
-                    acc[0] = fmaf(wk, bf16_lo(yv[j].x), acc[0]);
-                    acc[1] = fmaf(wk, bf16_hi(yv[j].x), acc[1]);
-                    acc[2] = fmaf(wk, bf16_lo(yv[j].y), acc[2]);
-                    acc[3] = fmaf(wk, bf16_hi(yv[j].y), acc[3]);
-                    acc[4] = fmaf(wk, bf16_lo(yv[j].z), acc[4]);
-                    acc[5] = fmaf(wk, bf16_hi(yv[j].z), acc[5]);
-                    acc[6] = fmaf(wk, bf16_lo(yv[j].w), acc[6]);
-                    acc[7] = fmaf(wk, bf16_hi(yv[j].w), acc[7]);
+#pragma unroll
+                    for (int i = 0; i < NW; ++i) {
+                        acc[2 * i] = fmaf(wk, bf16_lo(yv[j][i]), acc[2 * i]);
+                        acc[2 * i + 1] = fmaf(wk, bf16_hi(yv[j][i]), acc[2 * i + 1]);
+                    }
                 }
             }
-            uint4 o;
-            o.x = pack_bf16x2(acc[0], acc[1]);
-            o.y = pack_bf16x2(acc[2], acc[3]);
-            o.z = pack_bf16x2(acc[4], acc[5]);
-            o.w = pack_bf16x2(acc[6], acc[7]);
-            st_v4(out + (int64_t)t * V + v, o);
+            unsigned int o[NW];
+#pragma unroll
+            for (int i = 0; i < NW; ++i) o[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+            CVec<NW>::store(out + (int64_t)t * row_bytes + (int64_t)v * VB, o);
         }
         __syncthreads();
     }
@@ -81,11 +99,11 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
 
 }  // namespace
 
-int combine_threads() { return kThreads; }
-const void *combine_kernel_ptr(int) { return reinterpret_cast<const void *>(&combine_kernel); }
-
-cudaError_t launch_combine(const CombineParams &p, int grid, cudaStream_t s) {
-    combine_kernel<<<grid, kThreads, 0, s>>>(p);
+cudaError_t launch_combine(const CombineParams &p, int num_sms, cudaStream_t s) {
+    static int occ = 0;
+    const void *k = reinterpret_cast<const void *>(&combine_kernel<4>);
+    const int grid = persistent_grid(p.n_units, blocks_per_sm(k, kThreads, 0, &occ), num_sms);
+    combine_kernel<4><<<grid, kThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -50,15 +50,6 @@ int check_handle(const ep_handle *h, bool need_layout) {
     return EP_OK;
 }
 
-// Persistent grid for a kernel: SMs x resident blocks, capped by the units.
-int persistent_grid(const void *kernel, int threads, int num_sms) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
-    return per_sm * num_sms;
-}
-
 }  // namespace
 
 extern "C" {
@@ -102,6 +93,7 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->wait_limit_ns = ep::kDefaultWaitLimitNs;
     h->barrier_extra = 0;
     h->has_layout = false;
+    h->layout_epoch = 0;
 
     auto fail = [&](int code) {
         delete h;
@@ -114,7 +106,7 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
 
     const int T = cfg->num_tokens, E = cfg->num_experts, R = cfg->num_ranks, K = cfg->num_topk;
 
-    // layout: one chunk of >= kMinTokensPerChunk tokens per CTA, all CTAs resident
+    // layout: about kLayoutPairsPerCta (token, k) pairs per CTA, all CTAs resident
     h->layout_smem = ep::layout_smem_bytes(E, R);
     // the attribute is per kernel, not per handle: allow the largest supported size
     e = cudaFuncSetAttribute(ep::layout_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -125,17 +117,14 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
                                                       ep::kLayoutThreads, h->layout_smem);
     if (e != cudaSuccess) return fail(cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor"));
     if (per_sm < 1) return fail(EP_ERR_UNSUPPORTED);
-    const int g_max = h->num_sms;   // one CTA per SM keeps the grid-wide waits short
-    int G = (T + ep::kMinTokensPerChunk - 1) / ep::kMinTokensPerChunk;
-    G = G < 1 ? 1 : (G > g_max ? g_max : G);
-    int tpc = T > 0 ? (T + G - 1) / G : 1;
+    const int64_t pairs = (int64_t)T * K;
+    int64_t G = (pairs + ep::kLayoutPairsPerCta - 1) / ep::kLayoutPairsPerCta;
+    G = G < 1 ? 1 : (G > h->num_sms ? h->num_sms : G);   // one CTA per SM at most
+    int tpc = T > 0 ? (int)((T + G - 1) / G) : 1;
     G = T > 0 ? (T + tpc - 1) / tpc : 1;
-    h->G = G;
+    h->G = (int)G;
     h->tokens_per_chunk = tpc;
 
-    h->dispatch_grid = persistent_grid(ep::dispatch_bf16_kernel_ptr(), ep::dispatch_threads(), h->num_sms);
-    h->dispatch_fp8_grid = persistent_grid(ep::dispatch_fp8_kernel_ptr(), ep::dispatch_threads(), h->num_sms);
-    h->combine_grid = persistent_grid(ep::combine_kernel_ptr(K), ep::combine_threads(), h->num_sms);
 
     // carve one allocation
     const size_t A256 = 256;
@@ -153,8 +142,7 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     const size_t o_rtok = take(sizeof(int32_t) * R);
     const size_t o_eoff = take(sizeof(int32_t) * (E + 1));
     const size_t o_roff = take(sizeof(int32_t) * (R + 1));
-    const size_t o_chunk = take(sizeof(int32_t) * (size_t)G * (E + R));
-    const size_t o_ctot = take(sizeof(int32_t) * (E + R));
+    const size_t o_chunk = take(sizeof(int32_t) * (size_t)((G + 3) / 4 * 4) * (E + R));
     const size_t o_bar = take(sizeof(ep::GridBarrier));
     const size_t o_stat = take(sizeof(unsigned int));
     h->block_bytes = off;
@@ -175,7 +163,6 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->eoff = reinterpret_cast<int32_t *>(b + o_eoff);
     h->roff = reinterpret_cast<int32_t *>(b + o_roff);
     h->chunk_counts = reinterpret_cast<int32_t *>(b + o_chunk);
-    h->col_total = reinterpret_cast<int32_t *>(b + o_ctot);
     h->barrier = reinterpret_cast<ep::GridBarrier *>(b + o_bar);
     h->status = reinterpret_cast<unsigned int *>(b + o_stat);
     *out = h;
@@ -235,8 +222,12 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
     p.R = c.num_ranks;
     p.L = c.num_experts / c.num_ranks;
     p.A = c.expert_alignment;
+    p.id_bits = 0;
+    while ((1 << p.id_bits) < c.num_experts) ++p.id_bits;
     p.G = h->G;
+    p.G_stride = (h->G + 3) / 4 * 4;
     p.tokens_per_chunk = h->tokens_per_chunk;
+    p.epoch = ++h->layout_epoch;
     p.pos = h->pos;
     p.row_src = h->row_src;
     p.row_slot = h->row_slot;
@@ -251,7 +242,6 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
     p.u_roff = rank_offsets;
     p.u_in_rank = is_token_in_rank;
     p.chunk_counts = h->chunk_counts;
-    p.col_total = h->col_total;
     p.barrier = h->barrier;
     p.status = h->status;
     p.wait_limit_ns = h->wait_limit_ns;
@@ -286,16 +276,15 @@ static int dispatch_common(const ep_handle *h, const void *x, void *recv, float 
     p.K = c.num_topk;
     p.E = c.num_experts;
     p.H = c.hidden;
+    p.status = h->status;
+    p.wait_limit_ns = h->wait_limit_ns;
     p.splits = 1;
     p.n_token_units = p.T * p.splits;
     p.n_zero_units = c.expert_alignment > 1
                          ? (int)((h->cap + ep::kZeroRowsPerUnit - 1) / ep::kZeroRowsPerUnit)
                          : 0;
-    const int units = p.n_token_units + p.n_zero_units;
-    int grid = fp8 ? h->dispatch_fp8_grid : h->dispatch_grid;
-    if (grid > units) grid = units;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = fp8 ? ep::launch_dispatch_fp8(p, grid, s) : ep::launch_dispatch_bf16(p, grid, s);
+    cudaError_t e = fp8 ? ep::launch_dispatch_fp8(p, h->num_sms, s) : ep::launch_dispatch_bf16(p, h->num_sms, s);
     if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(dispatch_fp8)" : "launch(dispatch)");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return EP_OK;
@@ -331,9 +320,7 @@ EP_API int ep_combine(const ep_handle *h, const void *y, const float *topk_weigh
     p.H = c.hidden;
     p.splits = 1;
     p.n_units = p.T * p.splits;
-    int grid = h->combine_grid;
-    if (grid > p.n_units) grid = p.n_units;
-    cudaError_t e = ep::launch_combine(p, grid, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = ep::launch_combine(p, h->num_sms, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launch(combine)");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return EP_OK;
@@ -389,6 +376,7 @@ EP_API int ep_clear_status(ep_handle *h, ep_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     EP_CUDA(cudaMemsetAsync(h->status, 0, sizeof(unsigned int), s));
     EP_CUDA(cudaMemsetAsync(h->barrier, 0, sizeof(ep::GridBarrier), s));
+    h->layout_epoch = 0;
     return EP_OK;
 }
 

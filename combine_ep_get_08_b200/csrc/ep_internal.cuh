@@ -13,15 +13,15 @@ namespace ep {
 // ---------------------------------------------------------------------------
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopk = 64;
-constexpr int kLayoutThreads = 512;
+constexpr int kLayoutThreads = 1024;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
-constexpr int kMinTokensPerChunk = 16;
+constexpr int kLayoutPairsPerCta = 1024;   // target (token, k) pairs per layout CTA
 constexpr int kZeroRowsPerUnit = 8;    // padding rows zero-filled per work unit
 constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;
 
 struct GridBarrier {
-    unsigned int count;
-    unsigned int gen;
+    unsigned int count;          // arrivals so far (grows by G per layout launch)
+    unsigned int pad;
 };
 
 // ---------------------------------------------------------------------------
@@ -31,8 +31,11 @@ struct LayoutParams {
     const int64_t *topk_idx;
     const float *topk_weights;   // may be null
     int T, K, E, R, L, A;
+    int id_bits;                 // bits needed for an expert id: ceil(log2(E))
     int G;                       // CTAs == chunks
+    int G_stride;                // row stride of chunk_counts: G rounded up to 4
     int tokens_per_chunk;
+    unsigned int epoch;          // launch number on this handle (grid-wait target)
     // handle arrays
     int32_t *pos, *row_src, *row_slot;
     float *row_weight;
@@ -41,8 +44,7 @@ struct LayoutParams {
     int32_t *u_cnt, *u_rank_tok, *u_eoff, *u_roff;
     uint8_t *u_in_rank;
     // scratch
-    int32_t *chunk_counts;       // [G][E+R]
-    int32_t *col_total;          // [E+R]
+    int32_t *chunk_counts;       // [E+R][G_stride] (one row per expert / rank column)
     GridBarrier *barrier;
     unsigned int *status;
     unsigned long long wait_limit_ns;
@@ -56,6 +58,8 @@ struct DispatchParams {
     const int32_t *pos;          // [T, K]
     const int32_t *row_src;      // [cap]
     const int32_t *eoff;         // [E+1]
+    unsigned int *status;
+    unsigned long long wait_limit_ns;
     int T, K, E, H;
     int splits;                  // column splits per token
     int n_token_units;           // T * splits
@@ -76,14 +80,25 @@ struct CombineParams {
 cudaError_t launch_layout(const LayoutParams &p, size_t smem, cudaStream_t s);
 size_t layout_smem_bytes(int E, int R);
 const void *layout_kernel_ptr();
-cudaError_t launch_dispatch_bf16(const DispatchParams &p, int grid, cudaStream_t s);
-cudaError_t launch_dispatch_fp8(const DispatchParams &p, int grid, cudaStream_t s);
-cudaError_t launch_combine(const CombineParams &p, int grid, cudaStream_t s);
-int dispatch_threads();
-int combine_threads();
-const void *dispatch_bf16_kernel_ptr();
-const void *dispatch_fp8_kernel_ptr();
-const void *combine_kernel_ptr(int K);
+// Launchers size their persistent grid from the occupancy of the kernel
+// instance they pick: min(units, resident blocks per SM x num_sms).
+cudaError_t launch_dispatch_bf16(const DispatchParams &p, int num_sms, cudaStream_t s);
+cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams &p, int num_sms, cudaStream_t s);
+
+// Resident blocks per SM of `kernel` at `threads` threads and `smem` dynamic
+// shared memory, cached in *slot (0 = not yet known).
+inline int blocks_per_sm(const void *kernel, int threads, size_t smem, int *slot) {
+    int v = __atomic_load_n(slot, __ATOMIC_RELAXED);
+    if (v > 0) return v;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, threads, smem) != cudaSuccess || v < 1) v = 1;
+    __atomic_store_n(slot, v, __ATOMIC_RELAXED);
+    return v;
+}
+inline int persistent_grid(int units, int per_sm, int num_sms) {
+    const int g = per_sm * num_sms;
+    return units < g ? units : g;
+}
 
 // ---------------------------------------------------------------------------
 // Device helpers (inline PTX for cache hints, ordering and the timer)
@@ -126,6 +141,99 @@ __device__ __forceinline__ unsigned int lanemask_lt() {
     return m;
 }
 
+// 32-byte load / store (sm_100 256-bit vector access); address 32-byte aligned.
+struct alignas(32) u32x8 {
+    unsigned int v[8];
+};
+
+__device__ __forceinline__ u32x8 ld_stream_v8(const void *p) {
+    u32x8 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r.v[0]), "=r"(r.v[1]), "=r"(r.v[2]), "=r"(r.v[3]), "=r"(r.v[4]), "=r"(r.v[5]),
+                   "=r"(r.v[6]), "=r"(r.v[7])
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_v8(void *p, const u32x8 &r) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :
+                 : "l"(p), "r"(r.v[0]), "r"(r.v[1]), "r"(r.v[2]), "r"(r.v[3]), "r"(r.v[4]), "r"(r.v[5]),
+                   "r"(r.v[6]), "r"(r.v[7])
+                 : "memory");
+}
+
+// ---- shared-memory barriers and bulk (non-tensor) async copies ------------
+// Only CTA-local forms are used: no cluster multicast anywhere.
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" : : "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :
+                 : "r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete, at most limit_ns.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    return true;
+}
+
+// global -> shared bulk copy completing on an mbarrier (16-byte aligned, size % 16 == 0)
+__device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :
+        : "r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// shared -> global bulk copy in the current bulk group
+__device__ __forceinline__ void bulk_s2g(void *gdst, const void *smem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 :
+                 : "l"(gdst), "r"(smem_u32(smem_src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" : : : "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" : : "n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" : : : "memory"); }
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (bulk copy) reads of them.
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" : : : "memory");
+}
+
 // bf16 pair in a 32-bit word -> two floats (exact)
 __device__ __forceinline__ float bf16_lo(unsigned int u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(unsigned int u) { return __uint_as_float(u & 0xffff0000u); }
@@ -142,20 +250,17 @@ struct ep_handle {
     int G;
     int tokens_per_chunk;
     size_t layout_smem;
-    // persistent grids
-    int dispatch_grid;
-    int dispatch_fp8_grid;
-    int combine_grid;
     // one device allocation, carved
     void *block;
     size_t block_bytes;
     int32_t *pos, *row_src, *row_slot;
     float *row_weight;
     int32_t *cnt, *rank_tok, *eoff, *roff;
-    int32_t *chunk_counts, *col_total;
+    int32_t *chunk_counts;
     ep::GridBarrier *barrier;
     unsigned int *status;
     bool has_layout;
+    unsigned int layout_epoch;      // layout launches since creation / ep_clear_status
     unsigned long long wait_limit_ns;
     int barrier_extra;
 };

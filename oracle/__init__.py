@@ -45,30 +45,69 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def _bind(lib):
+    P = ctypes.c_void_p
+    i32, i64 = ctypes.c_int32, ctypes.c_int64
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_e4m3_encode_array.argtypes = [i64, P, P]
+    lib.oracle_e4m3_encode_array.restype = None
+    lib.oracle_capacity_rows.argtypes = [i32, i32, i32, i32]
+    lib.oracle_capacity_rows.restype = i64
+    lib.oracle_layout.argtypes = [i32, i32, i32, i32, i32] + [P] * 11
+    lib.oracle_layout.restype = ctypes.c_int
+    lib.oracle_dispatch_bf16.argtypes = [i32, i32, i32, P, P, P, P]
+    lib.oracle_dispatch_bf16.restype = ctypes.c_int
+    lib.oracle_dispatch_fp8.argtypes = [i32, i32, i32, P, P, P, P, P]
+    lib.oracle_dispatch_fp8.restype = ctypes.c_int
+    lib.oracle_combine.argtypes = [i32, i32, i32, i32, P, P, P, i32, P, P]
+    lib.oracle_combine.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
-        if _lib is not None:
-            return _lib
-        lib = ctypes.CDLL(build())
-        P = ctypes.c_void_p
-        i32, i64 = ctypes.c_int32, ctypes.c_int64
-        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
-        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
-        lib.oracle_e4m3_encode_array.argtypes = [i64, P, P]
-        lib.oracle_e4m3_encode_array.restype = None
-        lib.oracle_capacity_rows.argtypes = [i32, i32, i32, i32]
-        lib.oracle_capacity_rows.restype = i64
-        lib.oracle_layout.argtypes = [i32, i32, i32, i32, i32] + [P] * 11
-        lib.oracle_layout.restype = ctypes.c_int
-        lib.oracle_dispatch_bf16.argtypes = [i32, i32, i32, P, P, P, P]
-        lib.oracle_dispatch_bf16.restype = ctypes.c_int
-        lib.oracle_dispatch_fp8.argtypes = [i32, i32, i32, P, P, P, P, P]
-        lib.oracle_dispatch_fp8.restype = ctypes.c_int
-        lib.oracle_combine.argtypes = [i32, i32, i32, i32, P, P, P, i32, P, P]
-        lib.oracle_combine.restype = ctypes.c_int
-        _lib = lib
-        return lib
+        if _lib is None:
+            _lib = _bind(ctypes.CDLL(build()))
+        return _lib
+
+
+class use_library:
+    """Context manager that points this module at another build of the
+    oracle's C source (the mutation tests compile deliberately broken copies
+    to show that the pins catch them)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self._saved = _load()
+        with _lock:
+            _lib = _bind(ctypes.CDLL(self.path))
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        with _lock:
+            _lib = self._saved
+
+
+def compile_source(src_text: str, out_path: str) -> str:
+    """Compile a variant of ep_oracle.c (given as text) to a shared library."""
+    c_path = out_path + ".c"
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    cmd = ["gcc", "-O1", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+           "-fPIC", "-shared", "-o", out_path, c_path, "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True)
+    return out_path
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
 
 
 def _ptr(a):
@@ -105,6 +144,9 @@ def layout(topk_idx, num_experts: int, num_ranks: int, expert_alignment: int = 1
     T, K = idx.shape
     E, R, A = num_experts, num_ranks, expert_alignment
     cap = max(capacity_rows(T, E, K, A), 0)
+    # slack rows past the capacity: a layout that overruns it is reported as
+    # an error (BAD_ARG) instead of writing outside the buffer
+    room = cap + E + 16
     w = None if topk_weights is None else _c(topk_weights, np.float32)
     out = Layout(
         num_tokens_per_expert=np.zeros(E, np.int32),
@@ -113,9 +155,9 @@ def layout(topk_idx, num_experts: int, num_ranks: int, expert_alignment: int = 1
         expert_offsets=np.zeros(E + 1, np.int32),
         rank_offsets=np.zeros(R + 1, np.int32),
         pos=np.zeros((T, K), np.int32),
-        row_src=np.full(cap, -7, np.int32),
-        row_slot=np.full(cap, -7, np.int32),
-        row_weight=np.zeros(cap, np.float32),
+        row_src=np.full(room, -7, np.int32),
+        row_slot=np.full(room, -7, np.int32),
+        row_weight=np.zeros(room, np.float32),
     )
     rc = _load().oracle_layout(
         T, E, R, K, A, _ptr(idx), _ptr(w), _ptr(out.num_tokens_per_expert),
@@ -123,7 +165,9 @@ def layout(topk_idx, num_experts: int, num_ranks: int, expert_alignment: int = 1
         _ptr(out.expert_offsets), _ptr(out.rank_offsets), _ptr(out.pos),
         _ptr(out.row_src), _ptr(out.row_slot), _ptr(out.row_weight))
     out.status = rc
-    if rc == OK:
+    if rc == OK and int(out.expert_offsets[-1]) > cap:
+        out.status = BAD_ARG
+    if out.status == OK:
         rows = int(out.expert_offsets[-1])
         out.rows = rows
         out.row_src = out.row_src[:rows]

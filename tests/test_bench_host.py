@@ -1,0 +1,81 @@
+"""Host-side logic of bench.py on CPU: the multi-rank reductions (world size
+2 over gloo), the byte model, and the reference arm's JSON line."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_path):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    bench.init_dist(world, "gloo")
+    w, r, _ = bench.dist_env()
+    bench.barrier(w)
+    mx = bench.max_over_ranks(10.0 + r, w)
+    sm = bench.sum_over_ranks(1.5 * (r + 1), w)
+    with open(f"{out_path}.{r}", "w") as f:
+        json.dump({"max": mx, "sum": sm, "world": w}, f)
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_two_rank_reductions(tmp_path):
+    port = _free_port()
+    out = str(tmp_path / "res")
+    mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
+    for r in range(2):
+        d = json.load(open(f"{out}.{r}"))
+        assert d == {"max": 11.0, "sum": 4.5, "world": 2}
+
+
+def test_single_rank_is_identity():
+    assert bench.max_over_ranks(3.25, 1) == 3.25
+    assert bench.sum_over_ranks(3.25, 1) == 3.25
+
+
+def test_byte_model():
+    # DeepSeek-V3 shape: 528.5 MB each way
+    assert bench.dispatch_bytes(4096, 7168, 8, 32768, False) == 528482304
+    assert bench.combine_bytes(4096, 7168, 8) == 528482304
+    assert bench.row_bytes(7168, True) == 7168 + 56 * 4
+
+
+def test_reference_arm_line():
+    env = dict(os.environ)
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3",
+                        "--config", "tiny"], cwd=ROOT, capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
+
+
+def test_reference_arm_other_ranks_are_silent():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
+                        "--warmup", "3", "--config", "tiny"], cwd=ROOT, capture_output=True, text=True,
+                       env=env, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_warmup_floor():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])

@@ -1,0 +1,113 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the oracle's C source (a dropped
+term, a wrong index or sign, a transposed operand, a wrong rounding or
+order), compiles it, points the oracle module at the mutant and runs the pin
+battery of tests/test_oracle_*.py on it: at least one pin must fail.
+Mistakes are planted only in the oracle, on the CPU.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import test_oracle_dispatch_combine as tdc
+import test_oracle_fp8 as tf8
+import test_oracle_layout as tlay
+
+MUTANTS = {
+    "padding rounds up a full segment": (
+        "int32_t padded = ((c + A - 1) / A) * A;", "int32_t padded = (c / A + 1) * A;"),
+    "offsets not accumulated": (
+        "expert_offsets[e + 1] = expert_offsets[e] + padded;", "expert_offsets[e + 1] = padded;"),
+    "rank of an expert by modulo": (
+        "if (topk_idx[(int64_t)t * K + k] / L == r) in = 1;",
+        "if (topk_idx[(int64_t)t * K + k] % R == r) in = 1;"),
+    "tokens appended in reverse order": (
+        "    for (int32_t t = 0; t < T; ++t) {\n        for (int32_t k = 0; k < K; ++k) {\n            int64_t i",
+        "    for (int32_t t = T - 1; t >= 0; --t) {\n        for (int32_t k = 0; k < K; ++k) {\n            int64_t i"),
+    "slot recorded as token": ("row_slot[r] = k;", "row_slot[r] = t;"),
+    "ties rounded away from zero": ("if (d > 0.5f) return n + 1;", "if (d >= 0.5f) return n + 1;"),
+    "no saturation (NaN code)": (
+        "if (a >= 448.0f) return (uint8_t)(sign | 0x7E);", "if (a >= 448.0f) return (uint8_t)(sign | 0x7F);"),
+    "subnormal step 2^-8": ("round_half_even_u(a * 512.0f)", "round_half_even_u(a * 256.0f)"),
+    "exponent bias off by one": ("((uint32_t)(e + 7) << 3) | m", "((uint32_t)(e + 8) << 3) | m"),
+    "amax without abs": (
+        "amax = fmaxf(amax, fabsf(bf16_bits_to_float(xb[j])));",
+        "amax = fmaxf(amax, bf16_bits_to_float(xb[j]));"),
+    "scale stored inverted": ("scale[b] = amax_floor / 448.0f;", "scale[b] = 448.0f / amax_floor;"),
+    "quantised with the dequant scale": (
+        "float v = bf16_bits_to_float(xb[j]) * inv;", "float v = bf16_bits_to_float(xb[j]) * (amax_floor / 448.0f);"),
+    "combine uses weight of k=0": (
+        "double wk = (double)w[(int64_t)t * K + k];", "double wk = (double)w[(int64_t)t * K];"),
+    "combine reads row of k=0": (
+        "int32_t r = pos[(int64_t)t * K + k];", "int32_t r = pos[(int64_t)t * K];"),
+    "combine drops the last k": ("for (int32_t k = 0; k < K; ++k) {\n            int32_t r = pos",
+                                 "for (int32_t k = 0; k < K - 1; ++k) {\n            int32_t r = pos"),
+    "dispatch copies the previous token": (
+        "memcpy(dst, x + (int64_t)t * H, sizeof(uint16_t) * (size_t)H);",
+        "memcpy(dst, x + (int64_t)(t > 0 ? t - 1 : 0) * H, sizeof(uint16_t) * (size_t)H);"),
+    "padding row not zeroed": (
+        "            memset(dst, 0, sizeof(uint16_t) * (size_t)H);\n",
+        "            memset(dst, 0, sizeof(uint16_t) * (size_t)(H / 2));\n"),
+}
+
+
+def small_bruteforce(lib):
+    for T in range(0, 3):
+        for E in (1, 2, 4):
+            for K in (1, 2):
+                for flat in np.ndindex(*([E] * (T * K))) if T * K else [()]:
+                    idx = np.array(flat, dtype=np.int64).reshape(T, K)
+                    for R in [d for d in range(1, E + 1) if E % d == 0]:
+                        for A in (1, 3):
+                            L = lib.layout(idx, E, R, A)
+                            ref = tlay.naive_layout(idx, E, R, A)
+                            assert L.status == 0
+                            for key, val in ref.items():
+                                np.testing.assert_array_equal(
+                                    getattr(L, key), np.asarray(val).reshape(getattr(L, key).shape))
+
+
+PINS = [
+    ("worked example", lambda lib: tlay.test_worked_example(lib)),
+    ("brute force", small_bruteforce),
+    ("invariants tiny", lambda lib: tlay.test_invariants_on_workloads(lib, "tiny")),
+    ("invariants skew", lambda lib: tlay.test_invariants_on_workloads(lib, "skew")),
+    ("e4m3 known codes", lambda lib: tf8.test_known_codes(lib)),
+    ("e4m3 round trip", lambda lib: tf8.test_representable_values_round_trip(lib)),
+    ("e4m3 brute force", lambda lib: tf8.test_brute_force_all_bf16(lib)),
+    ("e4m3 ties", lambda lib: tf8.test_ties_and_neighbours(lib)),
+    ("identity round trip", lambda lib: tdc.test_identity_round_trip(lib, 4)),
+    ("one-hot", lambda lib: tdc.test_one_hot_selects_expert_row(lib)),
+    ("lesson exercise", lambda lib: tdc.test_lesson_exercise_restated(lib)),
+    ("fp8 properties", lambda lib: tdc.test_fp8_dispatch_properties(lib, 5)),
+]
+
+
+def run_pins(lib):
+    failed = []
+    for name, fn in PINS:
+        try:
+            fn(lib)
+        except Exception:  # noqa: BLE001 - any failure of a pin counts
+            failed.append(name)
+    return failed
+
+
+def test_unmutated_source_passes_battery(tmp_path):
+    so = oracle.compile_source(oracle.source_text(), str(tmp_path / "orig.so"))
+    with oracle.use_library(so):
+        assert run_pins(oracle) == []
+
+
+@pytest.mark.parametrize("name", list(MUTANTS))
+def test_mutant_is_caught(tmp_path, name):
+    old, new = MUTANTS[name]
+    src = oracle.source_text()
+    assert src.count(old) == 1, f"mutation anchor not unique: {name}"
+    so = oracle.compile_source(src.replace(old, new), str(tmp_path / "mutant.so"))
+    with oracle.use_library(so):
+        failed = run_pins(oracle)
+    assert failed, f"no pin caught the mutant '{name}'"
