@@ -67,6 +67,7 @@ def _load():
             "ep_handle_destroy": ([P], ctypes.c_int),
             "ep_handle_get_view": ([P, ctypes.POINTER(ep_handle_view)], ctypes.c_int),
             "ep_get_layout": ([P] + [P] * 7 + [P], ctypes.c_int),
+            "ep_get_layout_noalloc": ([CFG] + [P] * 13, ctypes.c_int),
             "ep_dispatch": ([P, P, P, P], ctypes.c_int),
             "ep_dispatch_fp8": ([P, P, P, P, P], ctypes.c_int),
             "ep_combine": ([P, P, P, P, P], ctypes.c_int),
@@ -101,7 +102,7 @@ def status_text(code: int) -> str:
 
 def _check(fn: str, rc: int) -> int:
     if rc < 0:
-        detail = _load().ep_last_error().decode() if rc == EP_ERR_CUDA else ""
+        detail = _load().ep_last_error().decode() if rc in (EP_ERR_CUDA, EP_ERR_UNSUPPORTED) else ""
         raise EpError(fn, rc, detail)
     return rc
 
@@ -164,6 +165,16 @@ def ep_get_layout(h: int, topk_idx, topk_weights=None, num_tokens_per_expert=Non
         h, _ptr(topk_idx), _ptr(topk_weights), _ptr(num_tokens_per_expert),
         _ptr(num_tokens_per_rank), _ptr(is_token_in_rank), _ptr(expert_offsets),
         _ptr(rank_offsets), _stream(stream)))
+
+
+def ep_get_layout_noalloc(cfg: ep_config, topk_idx, topk_weights, pos, row_src, row_slot, row_weight,
+                          num_tokens_per_expert, num_tokens_per_rank, is_token_in_rank, expert_offsets,
+                          rank_offsets, status, stream=None) -> None:
+    """Layout into caller buffers without any allocation (see include/ep.h)."""
+    _check("ep_get_layout_noalloc", _load().ep_get_layout_noalloc(
+        ctypes.byref(cfg), _ptr(topk_idx), _ptr(topk_weights), _ptr(pos), _ptr(row_src), _ptr(row_slot),
+        _ptr(row_weight), _ptr(num_tokens_per_expert), _ptr(num_tokens_per_rank), _ptr(is_token_in_rank),
+        _ptr(expert_offsets), _ptr(rank_offsets), _ptr(status), _stream(stream)))
 
 
 def ep_dispatch(h: int, x, recv_x, stream=None) -> None:

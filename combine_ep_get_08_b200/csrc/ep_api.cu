@@ -52,6 +52,12 @@ int check_handle(const ep_handle *h, bool need_layout) {
 
 }  // namespace
 
+namespace ep {
+void record_error(const char *msg) { snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+int record_cuda_error(cudaError_t e, const char *what) { return cuda_fail(e, what); }
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace ep
+
 extern "C" {
 
 EP_API int ep_validate_config(const ep_config *c) {

@@ -86,6 +86,11 @@ cudaError_t launch_dispatch_bf16(const DispatchParams &p, int num_sms, cudaStrea
 cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams &p, int num_sms, cudaStream_t s);
 
+// Error text for ep_last_error and the library's launch counter (ep_api.cu).
+void record_error(const char *msg);
+int record_cuda_error(cudaError_t e, const char *what);   // returns EP_ERR_CUDA
+void count_launch();
+
 // Resident blocks per SM of `kernel` at `threads` threads and `smem` dynamic
 // shared memory, cached in *slot (0 = not yet known).
 inline int blocks_per_sm(const void *kernel, int threads, size_t smem, int *slot) {

@@ -193,6 +193,38 @@ EP_API int ep_combine(const ep_handle *h, const void *y, const float *topk_weigh
 EP_API int ep_copy_routing(const ep_handle *h, int32_t *pos, int32_t *row_src, int32_t *row_slot,
                            float *row_weight, ep_stream_t stream);
 
+/*
+ * Layout without any allocation.  This entry point has no counterpart on the
+ * pages: it exists for callers that cannot call cudaMalloc where they route
+ * tokens -- code that must not trigger a device allocation (it can
+ * synchronise the device or fail under memory pressure), runtimes that hand
+ * out device memory only from their own pools, or callers with nowhere to
+ * keep a handle.  It computes exactly what ep_get_layout computes, but every
+ * output comes from the caller:
+ *   pos [T, K], row_src / row_slot [capacity] int32, row_weight [capacity]
+ *   fp32 (required iff topk_weights is non-NULL), num_tokens_per_expert [E],
+ *   num_tokens_per_rank [R], expert_offsets [E+1], rank_offsets [R+1]
+ *   (all required, 4-byte aligned); is_token_in_rank [T, R] (optional);
+ *   status: one device uint32, set to 0 and then to the EP_DEV_* bits of this
+ *   call (read it after the stream has reached it).
+ * The kernel's scratch lives in a fixed 256 KiB array in the library's
+ * device code, held on every GPU that loads the library until exit.  A
+ * problem whose layout needs more (E + R columns of ceil(G/4)*4 int32, G
+ * layout CTAs ~ T*K/1024 up to the SM count, plus 256 bytes) is rejected with
+ * EP_ERR_UNSUPPORTED and a message in ep_last_error.
+ * The first call on a device does a one-time set-up on the host (it looks up
+ * the array's device address and sets a kernel attribute): make that first
+ * call before any stream capture.  Every call shares the one array and
+ * clears the part it uses (stream-ordered memset), so calls that overlap on
+ * the GPU -- on two streams, or from two threads -- race and must not be
+ * issued.  No cudaMalloc, cudaFree or other allocating call is made.
+ */
+EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, const float *topk_weights,
+                                 int32_t *pos, int32_t *row_src, int32_t *row_slot, float *row_weight,
+                                 int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+                                 uint8_t *is_token_in_rank, int32_t *expert_offsets, int32_t *rank_offsets,
+                                 uint32_t *status, ep_stream_t stream);
+
 /* Synchronises `stream` and returns rows (= expert_offsets[E]) on the host. */
 EP_API int ep_get_num_rows(const ep_handle *h, int32_t *rows, ep_stream_t stream);
 
