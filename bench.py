@@ -179,19 +179,22 @@ def kernel_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+def ncu_traffic(role: str, workload: str):
+    """(kernel name, DRAM bytes per launch) of a role ("layout", "dispatch",
+    "combine") from the committed ncu summary, if it was taken on the current
+    kernel sources; else (None, None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             data = json.load(f)
     except Exception:  # noqa: BLE001
-        return None
+        return None, None
     if data.get("source_digest") != kernel_source_digest():
-        return None
-    entry = data.get("kernels", {}).get(workload, {}).get(kernel)
-    return None if entry is None else entry.get("dram_bytes_per_launch")
+        return None, None
+    entry = data.get("roles", {}).get(workload, {}).get(role)
+    if entry is None:
+        return None, None
+    return entry.get("kernel"), entry.get("dram_bytes_per_launch")
 
 
 # ----------------------------------------------------------------------------
@@ -413,8 +416,7 @@ def run_cuda(args, world, rank, local):
     dom = "dispatch" if dis_us >= com_us else "combine"
     dom_bytes = b_dis if dom == "dispatch" else b_com
     achieved = dom_bytes / (kern[dom] * 1e-6) / 1e9
-    kname = {"dispatch": "dispatch_fp8_kernel" if wl.fp8 else "dispatch_bf16_kernel",
-             "combine": "combine_kernel"}[dom]
+    kname, traffic = ncu_traffic(dom, args.config)
     clocks = sampler.summary()
     status_end = ep.ep_get_status(path.h)
     path.close()
@@ -436,10 +438,9 @@ def run_cuda(args, world, rank, local):
             "bytes_per_call": {"dispatch": b_dis, "combine": b_com},
             "gbs_per_call": {"dispatch": round(b_dis / dis_us / 1e3, 1),
                              "combine": round(b_com / com_us / 1e3, 1)},
-            "roofline": {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
-                         "peak": peak, "peak_source": peak_src, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4),
-                         "traffic": ncu_traffic(kname, args.config)},
+            "roofline": {"bound": "hbm", "kernel": dom if kname is None else f"{dom}: {kname}",
+                         "achieved": round(achieved, 1), "peak": peak, "peak_source": peak_src,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic},
             "e2e": e2e,
             "gpu_launches": int(launches),
             "clocks": clocks,

@@ -132,6 +132,9 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->tokens_per_chunk = tpc;
 
 
+    e = ep::dispatch_prepare();
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaFuncSetAttribute(dispatch)"));
+
     // carve one allocation
     const size_t A256 = 256;
     size_t off = 0;
@@ -285,6 +288,7 @@ static int dispatch_common(const ep_handle *h, const void *x, void *recv, float 
     p.status = h->status;
     p.wait_limit_ns = h->wait_limit_ns;
     p.splits = 1;
+    p.stages = 0;
     p.n_token_units = p.T * p.splits;
     p.n_zero_units = c.expert_alignment > 1
                          ? (int)((h->cap + ep::kZeroRowsPerUnit - 1) / ep::kZeroRowsPerUnit)

@@ -64,6 +64,8 @@ struct DispatchParams {
     int splits;                  // column splits per token
     int n_token_units;           // T * splits
     int n_zero_units;            // ceil(cap / kZeroRowsPerUnit) when A > 1, else 0
+    int stages;                  // shared-memory ring depth (staged kernel)
+    int groups;                  // consumer groups (staged kernel)
 };
 
 struct CombineParams {
@@ -84,6 +86,9 @@ const void *layout_kernel_ptr();
 // instance they pick: min(units, resident blocks per SM x num_sms).
 cudaError_t launch_dispatch_bf16(const DispatchParams &p, int num_sms, cudaStream_t s);
 cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream_t s);
+// Per device, before the first dispatch launch: kernel attributes (dynamic
+// shared memory of the staged kernel).
+cudaError_t dispatch_prepare();
 cudaError_t launch_combine(const CombineParams &p, int num_sms, cudaStream_t s);
 
 // Error text for ep_last_error and the library's launch counter (ep_api.cu).
@@ -185,6 +190,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" : : "r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -221,6 +230,42 @@ __device__ __forceinline__ void bulk_s2g(void *gdst, const void *smem_src, uint3
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
                  :
                  : "l"(gdst), "r"(smem_u32(smem_src)), "r"(bytes)
+                 : "memory");
+}
+
+// L2 cache policies (fraction 1.0) for the .L2::cache_hint operand
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// Bulk prefetch of global memory into L2 (16-byte aligned, size % 16 == 0)
+// with an eviction-priority policy.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gsrc, uint32_t bytes, uint64_t pol) {
+    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;"
+                 :
+                 : "l"(gsrc), "r"(bytes), "l"(pol)
+                 : "memory");
+}
+
+// 32-byte store with an L2 eviction-priority policy.
+__device__ __forceinline__ void st_v8_policy(void *p, const u32x8 &r, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8}, %9;"
+                 :
+                 : "l"(p), "r"(r.v[0]), "r"(r.v[1]), "r"(r.v[2]), "r"(r.v[3]), "r"(r.v[4]), "r"(r.v[5]),
+                   "r"(r.v[6]), "r"(r.v[7]), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_v4_policy(void *p, uint4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;"
+                 :
+                 : "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
                  : "memory");
 }
 
