@@ -348,6 +348,8 @@ def run_cuda(args, world, rank, local):
     wl = workloads.generate(args.config, seed=base["seed"] + 1000 * rank)
     reuse = base["reuse"] if args.reuse is None else args.reuse
     path = Path(wl, dev)
+    if args.sm_limit:
+        ep.ep_set_sm_limit(path.h, args.sm_limit)
     stream = torch.cuda.current_stream(dev)
     sptr = stream.cuda_stream
 
@@ -431,6 +433,7 @@ def run_cuda(args, world, rank, local):
                 "workload": workloads.DESCRIPTIONS[args.config], "name": args.config,
                 "rows": rows, "reuse": reuse,
                 "parallelism": f"replicas x{world} (independent batches, no data-path collective)",
+                "sm_limit": args.sm_limit or None,
                 "l2": "flushed (256 MiB read, outside the timed events) before each step and "
                       "between dispatch and combine",
             },
@@ -512,6 +515,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds for the oracle baseline")
     ap.add_argument("--ref-tokens", type=int, default=4096, help="tokens per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sm-limit", type=int, default=0, help="SMs dispatch/combine may occupy (0: all)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -18,6 +18,7 @@ LIB_PATH = os.environ.get("EP_B200_LIB", os.path.join(_HERE, "libep_b200.so"))
 
 EP_OK, EP_ERR_ARG, EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EP_ERR_STATE, EP_ERR_DEVICE = 0, -1, -2, -3, -4, -5
 EP_DEV_BAD_EXPERT, EP_DEV_WAIT_TIMEOUT = 0x1, 0x2
+EP_SCALES_ROW_MAJOR, EP_SCALES_COL_MAJOR_TMA = 0, 1
 
 
 class EpError(RuntimeError):
@@ -63,6 +64,8 @@ def _load():
             "ep_validate_config": ([CFG], ctypes.c_int),
             "ep_capacity_rows": ([CFG], I64),
             "ep_scales_per_row": ([CFG], I32),
+            "ep_scale_buffer_floats": ([CFG, I32], I64),
+            "ep_set_scale_layout": ([P, I32], ctypes.c_int),
             "ep_handle_create": ([CFG, ctypes.POINTER(P)], ctypes.c_int),
             "ep_handle_destroy": ([P], ctypes.c_int),
             "ep_handle_get_view": ([P, ctypes.POINTER(ep_handle_view)], ctypes.c_int),
@@ -76,6 +79,7 @@ def _load():
             "ep_get_status": ([P, ctypes.POINTER(ctypes.c_uint32), P], ctypes.c_int),
             "ep_clear_status": ([P, P], ctypes.c_int),
             "ep_set_wait_limit": ([P, U64, I32], ctypes.c_int),
+            "ep_set_sm_limit": ([P, I32], ctypes.c_int),
             "ep_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "ep_last_error": ([], ctypes.c_char_p),
             "ep_launch_count": ([], U64),
@@ -140,6 +144,14 @@ def ep_capacity_rows(cfg: ep_config) -> int:
 
 def ep_scales_per_row(cfg: ep_config) -> int:
     return _check("ep_scales_per_row", _load().ep_scales_per_row(ctypes.byref(cfg)))
+
+
+def ep_scale_buffer_floats(cfg: ep_config, layout: int = EP_SCALES_ROW_MAJOR) -> int:
+    return _check("ep_scale_buffer_floats", _load().ep_scale_buffer_floats(ctypes.byref(cfg), layout))
+
+
+def ep_set_scale_layout(h: int, layout: int) -> None:
+    _check("ep_set_scale_layout", _load().ep_set_scale_layout(h, layout))
 
 
 def ep_handle_create(cfg: ep_config) -> int:
@@ -212,6 +224,10 @@ def ep_get_status(h: int, stream=None) -> int:
 
 def ep_clear_status(h: int, stream=None) -> None:
     _check("ep_clear_status", _load().ep_clear_status(h, _stream(stream)))
+
+
+def ep_set_sm_limit(h: int, num_sms: int) -> None:
+    _check("ep_set_sm_limit", _load().ep_set_sm_limit(h, num_sms))
 
 
 def ep_set_wait_limit(h: int, limit_ns: int, extra_arrivals: int = 0) -> None:

@@ -342,6 +342,11 @@ __device__ __forceinline__ unsigned int e4m3x2(float a, float b) {
 // EPT bf16 elements per thread (16: 16-byte accesses, 32: 32-byte accesses);
 // TPB = 128 / EPT consecutive lanes share one 1x128 block and reduce its
 // amax with shuffles.  Each thread stores EPT code bytes per received row.
+// Index of the scale of received row `row`, block b, in either layout.
+__device__ __forceinline__ int64_t scale_index(const DispatchParams &p, int row, int b, int NB) {
+    return p.scale_ld > 0 ? (int64_t)b * p.scale_ld + row : (int64_t)row * NB + b;
+}
+
 template <int EPT>
 struct Fp8Io;
 template <>
@@ -420,7 +425,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p
                         const int dst = s_dst[k];
                         if (dst < 0) continue;
                         Fp8Io<EPT>::store(recv + (int64_t)dst * p.H + (int64_t)g * EPT, q);
-                        if (lead) p.recv_scale[(int64_t)dst * NB + b] = scale;
+                        if (lead) p.recv_scale[scale_index(p, dst, b, NB)] = scale;
                     }
                 }
             }
@@ -433,7 +438,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p
                 if (__ldg(&p.row_src[r]) >= 0) continue;
                 uint8_t *o = recv + (int64_t)r * p.H;
                 for (int v = threadIdx.x; v < p.H / 16; v += kThreads) st_v4(o + v * 16, make_uint4(0, 0, 0, 0));
-                for (int b = threadIdx.x; b < NB; b += kThreads) p.recv_scale[(int64_t)r * NB + b] = 0.0f;
+                for (int b = threadIdx.x; b < NB; b += kThreads) p.recv_scale[scale_index(p, r, b, NB)] = 0.0f;
             }
         }
     }

@@ -86,6 +86,16 @@ EP_API int32_t ep_scales_per_row(const ep_config *c) {
     return c->hidden / 128;
 }
 
+EP_API int64_t ep_scale_buffer_floats(const ep_config *c, int32_t layout) {
+    const int64_t cap = ep_capacity_rows(c);
+    if (cap < 0) return cap;
+    if (c->hidden % 128 != 0) return EP_ERR_ARG;
+    const int64_t nb = c->hidden / 128;
+    if (layout == EP_SCALES_ROW_MAJOR) return cap * nb;
+    if (layout == EP_SCALES_COL_MAJOR_TMA) return nb * ((cap + 3) / 4 * 4);
+    return EP_ERR_ARG;
+}
+
 EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     if (!out) return EP_ERR_ARG;
     *out = nullptr;
@@ -99,6 +109,8 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->wait_limit_ns = ep::kDefaultWaitLimitNs;
     h->barrier_extra = 0;
     h->has_layout = false;
+    h->sm_limit = 0;
+    h->scale_layout = EP_SCALES_ROW_MAJOR;
     h->layout_epoch = 0;
 
     auto fail = [&](int code) {
@@ -278,6 +290,7 @@ static int dispatch_common(const ep_handle *h, const void *x, void *recv, float 
     p.x = x;
     p.recv = recv;
     p.recv_scale = scales;
+    p.scale_ld = h->scale_layout == EP_SCALES_COL_MAJOR_TMA ? (int)((h->cap + 3) / 4 * 4) : 0;
     p.pos = h->pos;
     p.row_src = h->row_src;
     p.eoff = h->eoff;
@@ -294,7 +307,8 @@ static int dispatch_common(const ep_handle *h, const void *x, void *recv, float 
                          ? (int)((h->cap + ep::kZeroRowsPerUnit - 1) / ep::kZeroRowsPerUnit)
                          : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = fp8 ? ep::launch_dispatch_fp8(p, h->num_sms, s) : ep::launch_dispatch_bf16(p, h->num_sms, s);
+    const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
+    cudaError_t e = fp8 ? ep::launch_dispatch_fp8(p, sms, s) : ep::launch_dispatch_bf16(p, sms, s);
     if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(dispatch_fp8)" : "launch(dispatch)");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return EP_OK;
@@ -328,9 +342,13 @@ EP_API int ep_combine(const ep_handle *h, const void *y, const float *topk_weigh
     p.T = c.num_tokens;
     p.K = c.num_topk;
     p.H = c.hidden;
+    p.status = h->status;
+    p.wait_limit_ns = h->wait_limit_ns;
     p.splits = 1;
+    p.stages = 0;
     p.n_units = p.T * p.splits;
-    cudaError_t e = ep::launch_combine(p, h->num_sms, reinterpret_cast<cudaStream_t>(stream));
+    const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
+    cudaError_t e = ep::launch_combine(p, sms, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launch(combine)");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return EP_OK;
@@ -387,6 +405,18 @@ EP_API int ep_clear_status(ep_handle *h, ep_stream_t stream) {
     EP_CUDA(cudaMemsetAsync(h->status, 0, sizeof(unsigned int), s));
     EP_CUDA(cudaMemsetAsync(h->barrier, 0, sizeof(ep::GridBarrier), s));
     h->layout_epoch = 0;
+    return EP_OK;
+}
+
+EP_API int ep_set_scale_layout(ep_handle *h, int32_t layout) {
+    if (!h || (layout != EP_SCALES_ROW_MAJOR && layout != EP_SCALES_COL_MAJOR_TMA)) return EP_ERR_ARG;
+    h->scale_layout = layout;
+    return EP_OK;
+}
+
+EP_API int ep_set_sm_limit(ep_handle *h, int32_t num_sms) {
+    if (!h || num_sms < 0) return EP_ERR_ARG;
+    h->sm_limit = num_sms;
     return EP_OK;
 }
 

@@ -54,7 +54,8 @@ struct LayoutParams {
 struct DispatchParams {
     const void *x;               // [T, H] bf16
     void *recv;                  // [cap, H] bf16 or e4m3
-    float *recv_scale;           // [cap, H/128] (FP8 only)
+    float *recv_scale;           // FP8 only: [cap, H/128], or [H/128][scale_ld] when scale_ld > 0
+    int scale_ld;                // 0: row-major scales; > 0: column-major leading dimension
     const int32_t *pos;          // [T, K]
     const int32_t *row_src;      // [cap]
     const int32_t *eoff;         // [E+1]
@@ -73,9 +74,12 @@ struct CombineParams {
     const float *w;              // [T, K]
     void *out;                   // [T, H] bf16
     const int32_t *pos;          // [T, K]
+    unsigned int *status;
+    unsigned long long wait_limit_ns;
     int T, K, H;
     int splits;
     int n_units;
+    int stages;                  // shared-memory ring depth (staged kernel)
 };
 
 // launchers (return cudaError_t of the launch)
@@ -310,6 +314,8 @@ struct ep_handle {
     ep::GridBarrier *barrier;
     unsigned int *status;
     bool has_layout;
+    int sm_limit;                   // SMs dispatch / combine may occupy (0: all)
+    int scale_layout;               // EP_SCALES_*
     unsigned int layout_epoch;      // layout launches since creation / ep_clear_status
     unsigned long long wait_limit_ns;
     int barrier_extra;

@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutParams 
         const int64_t v = __ldg(p.topk_idx + p_begin + tid);
         my_e = valid_expert(v, E) ? (int)v : -1;
         if (p.topk_weights) my_w = __ldg(p.topk_weights + p_begin + tid);
-        if (my_e < 0) atomicOr(p.status, EP_DEV_BAD_EXPERT);
+        if (my_e < 0 && v != -1) atomicOr(p.status, EP_DEV_BAD_EXPERT);   // -1: masked slot
         s_ids[tid] = my_e;
     }
     __syncthreads();
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutParams 
             const int64_t e = __ldg(p.topk_idx + q);
             if (valid_expert(e, E))
                 atomicAdd(&s_hist[e], 1);
-            else
+            else if (e != -1)
                 atomicOr(p.status, EP_DEV_BAD_EXPERT);
         }
     }

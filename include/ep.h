@@ -73,7 +73,7 @@ enum ep_error {
 };
 
 /* Device status bits (sticky until ep_clear_status). */
-#define EP_DEV_BAD_EXPERT 0x1u   /* some topk_idx entry is outside [0, E) */
+#define EP_DEV_BAD_EXPERT 0x1u   /* some topk_idx entry is outside [0, E) and not -1 */
 #define EP_DEV_WAIT_TIMEOUT 0x2u /* a bounded in-kernel wait gave up */
 
 /*
@@ -123,6 +123,17 @@ EP_API int64_t ep_capacity_rows(const ep_config *cfg);
 /* Number of scale floats per received row for FP8 dispatch: H / 128. */
 EP_API int32_t ep_scales_per_row(const ep_config *cfg);
 
+/* FP8 scale-factor layouts (ep_set_scale_layout). */
+#define EP_SCALES_ROW_MAJOR 0     /* scales[row * (H/128) + b] (default) */
+#define EP_SCALES_COL_MAJOR_TMA 1 /* scales[b * ld + row], ld = capacity rounded up to 4 */
+
+/*
+ * Floats a recv_scales buffer needs for `layout`: capacity * H/128 for
+ * EP_SCALES_ROW_MAJOR, (H/128) * round_up(capacity, 4) for
+ * EP_SCALES_COL_MAJOR_TMA; a negative ep_error for a bad cfg or layout.
+ */
+EP_API int64_t ep_scale_buffer_floats(const ep_config *cfg, int32_t layout);
+
 /*
  * Creates a handle on the current CUDA device: validates cfg and allocates
  * (cudaMalloc, once) the routing arrays of ep_handle_view plus a small
@@ -145,8 +156,10 @@ EP_API int ep_handle_get_view(const ep_handle *h, ep_handle_view *out);
  *   rank_offsets [R+1] int32.
  * topk_idx/topk_weights need 8/4-byte alignment only.  One cooperative
  * kernel launch; its grid-wide waits are bounded (EP_DEV_WAIT_TIMEOUT).
- * An id outside [0, E) sets EP_DEV_BAD_EXPERT; that pair gets pos = -1 and
- * no row.
+ * An id of -1 marks an unused top-k slot (the token selects fewer than K
+ * experts): that pair gets pos = -1, no row, is not counted and adds
+ * nothing in combine.  Any other id outside [0, E) also gets pos = -1 and
+ * sets EP_DEV_BAD_EXPERT.
  */
 EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *topk_weights,
                          int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
@@ -164,11 +177,12 @@ EP_API int ep_dispatch(const ep_handle *h, const void *x, void *recv_x, ep_strea
 /*
  * FP8 dispatch: per token and 128-column block b, amax = max|x|,
  * a = max(amax, 1e-4), codes = e4m3_rn_satfinite(x * (448 / a)) (IEEE fp32
- * divide and multiply), recv_scales[row, b] = a / 448 (the dequantisation
+ * divide and multiply), scale[row, b] = a / 448 (the dequantisation
  * factor: x ~ code * scale).  All K copies of a token are identical;
  * padding rows are code 0x00 with scale 0.  recv_q is [capacity, H] bytes
- * (16-byte aligned), recv_scales is [capacity, H/128] fp32 (4-byte
- * aligned).  Needs H % 128 == 0.
+ * (16-byte aligned); recv_scales is fp32, 4-byte aligned, in the handle's
+ * scale layout (ep_set_scale_layout; default [capacity, H/128] row-major).
+ * Needs H % 128 == 0.
  */
 EP_API int ep_dispatch_fp8(const ep_handle *h, const void *x, void *recv_q, float *recv_scales,
                            ep_stream_t stream);
@@ -236,6 +250,30 @@ EP_API int ep_get_status(const ep_handle *h, uint32_t *bits, ep_stream_t stream)
 
 /* Clears the status word and the in-kernel wait state (stream-ordered). */
 EP_API int ep_clear_status(ep_handle *h, ep_stream_t stream);
+
+/*
+ * Layout of the scales ep_dispatch_fp8 writes on this handle (default
+ * EP_SCALES_ROW_MAJOR).  EP_SCALES_COL_MAJOR_TMA stores them column-major
+ * with the row dimension padded to a multiple of 4 floats, so every 1x128
+ * block column starts 16-byte aligned -- the layout a grouped FP8 GEMM reads
+ * with TMA (the use_tma_aligned_col_major_sf option of EPBuffer.dispatch,
+ * bowenzhou.top "deepep/01-overview" section 1.1).  Values are identical in
+ * both layouts; size the buffer with ep_scale_buffer_floats.
+ */
+EP_API int ep_set_scale_layout(ep_handle *h, int32_t layout);
+
+/*
+ * Caps the SMs that ep_dispatch, ep_dispatch_fp8 and ep_combine occupy on
+ * this handle (0 = all, the default; values above the device's count mean
+ * all).  Their persistent grids are sized to at most `num_sms` SMs, so the
+ * rest of the GPU stays free for work that overlaps them -- the role of
+ * DeepEP's num_sms argument (bowenzhou.top "deepep/01-overview" section 1.1;
+ * "blog.hotdry.top ... deepep-expert-parallel-alltoall": 24 SMs by default;
+ * "lesson14_deepep" section 1(2): 20 communication SMs beside 110 compute
+ * SMs).  The layout kernel is not capped (it uses at most one CTA per 1024
+ * pairs).  Results do not depend on the cap.
+ */
+EP_API int ep_set_sm_limit(ep_handle *h, int32_t num_sms);
 
 /*
  * Limit for each bounded in-kernel wait, in nanoseconds of %globaltimer

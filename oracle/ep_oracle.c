@@ -30,7 +30,8 @@
  * num_tokens_per_rank counts distinct tokens; FP8 is OCP E4M3 with one fp32
  * scale per 1x128 block of a token row, amax floored at 1e-4, quantised as
  * e4m3_rne_satfinite(x * (448/amax)) with the dequantisation scale amax/448
- * stored; combine is the exact weighted sum (computed here in fp64).
+ * stored; combine is the exact weighted sum (computed here in fp64); an id
+ * of -1 marks a masked top-k slot (no row, no contribution).
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fPIC -shared (no fast-math).
  */
@@ -119,7 +120,9 @@ int64_t oracle_capacity_rows(int32_t T, int32_t E, int32_t K, int32_t A)
  * rank_offsets [R+1], pos [T,K], and for every received row r < rows:
  * row_src[r] (token or -1 for padding), row_slot[r] (k or -1),
  * row_weight[r] (topk weight or 0; untouched if topk_weights is NULL).
- * Returns ORACLE_BAD_EXPERT if some id is outside [0, E).
+ * An id of -1 marks an unused top-k slot: it gets pos = -1 and no row and
+ * is not counted.  Returns ORACLE_BAD_EXPERT if some other id is outside
+ * [0, E).
  */
 int oracle_layout(int32_t T, int32_t E, int32_t R, int32_t K, int32_t A,
                   const int64_t *topk_idx, const float *topk_weights,
@@ -132,22 +135,28 @@ int oracle_layout(int32_t T, int32_t E, int32_t R, int32_t K, int32_t A,
         return ORACLE_BAD_ARG;
     const int32_t L = E / R; /* local experts per rank */
 
+    /* -1 marks an unused top-k slot (masked: no expert, no row); any other id
+       outside [0, E) is an error */
     for (int64_t i = 0; i < (int64_t)T * K; ++i)
-        if (topk_idx[i] < 0 || topk_idx[i] >= E) return ORACLE_BAD_EXPERT;
+        if (topk_idx[i] != -1 && (topk_idx[i] < 0 || topk_idx[i] >= E)) return ORACLE_BAD_EXPERT;
 
-    /* counts per expert: each (token, k) pair is one received row */
+    /* counts per expert: each selected (token, k) pair is one received row */
     for (int32_t e = 0; e < E; ++e) num_tokens_per_expert[e] = 0;
     for (int32_t t = 0; t < T; ++t)
-        for (int32_t k = 0; k < K; ++k)
-            num_tokens_per_expert[topk_idx[(int64_t)t * K + k]] += 1;
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t e = topk_idx[(int64_t)t * K + k];
+            if (e >= 0) num_tokens_per_expert[e] += 1;
+        }
 
     /* token membership per rank, and distinct tokens per rank */
     for (int32_t r = 0; r < R; ++r) num_tokens_per_rank[r] = 0;
     for (int32_t t = 0; t < T; ++t) {
         for (int32_t r = 0; r < R; ++r) {
             uint8_t in = 0;
-            for (int32_t k = 0; k < K; ++k)
-                if (topk_idx[(int64_t)t * K + k] / L == r) in = 1;
+            for (int32_t k = 0; k < K; ++k) {
+                int64_t e = topk_idx[(int64_t)t * K + k];
+                if (e >= 0 && e / L == r) in = 1;
+            }
             is_token_in_rank[(int64_t)t * R + r] = in;
             num_tokens_per_rank[r] += in;
         }
@@ -170,6 +179,7 @@ int oracle_layout(int32_t T, int32_t E, int32_t R, int32_t K, int32_t A,
         for (int32_t k = 0; k < K; ++k) {
             int64_t i = (int64_t)t * K + k;
             int32_t e = (int32_t)topk_idx[i];
+            if (e < 0) { pos[i] = -1; continue; }   /* masked slot */
             int32_t r = cursor[e]++;
             pos[i] = r;
             row_src[r] = t;
@@ -263,7 +273,8 @@ int oracle_dispatch_fp8(int32_t T, int32_t H, int32_t n_sel, const int32_t *sel_
 /*
  * out[i, :] = sum_{k=0..K-1} w[t,k] * y[pos[t,k], :]  for t = sel_tokens[i]
  * (sel_tokens == NULL: t = i).  y is [rows, H] bf16, w is [T,K] fp32, the
- * sum is taken in fp64 in k order and returned unrounded.
+ * sum is taken in fp64 in k order and returned unrounded.  Masked slots
+ * (pos = -1) add nothing.
  */
 int oracle_combine(int32_t T, int32_t H, int32_t K, int32_t rows, const int32_t *pos,
                    const uint16_t *y, const float *w, int32_t n_sel,
@@ -276,6 +287,7 @@ int oracle_combine(int32_t T, int32_t H, int32_t K, int32_t rows, const int32_t 
         for (int32_t h = 0; h < H; ++h) o[h] = 0.0;
         for (int32_t k = 0; k < K; ++k) {
             int32_t r = pos[(int64_t)t * K + k];
+            if (r == -1) continue;                    /* masked slot adds nothing */
             if (r < 0 || r >= rows) return ORACLE_BAD_ARG;
             double wk = (double)w[(int64_t)t * K + k];
             const uint16_t *yr = y + (int64_t)r * H;

@@ -71,10 +71,13 @@ def run_full(wl, fp8: bool, y_seed=99, check_rows=None, check_tokens=None):
         ep.ep_combine(g.handle, y_d, w_d, out)
         tsel = np.arange(wl.T, dtype=np.int32) if check_tokens is None else np.asarray(check_tokens, np.int32)
         if len(tsel):
-            need = o.pos[tsel]                     # [n, K] rows those tokens read
-            uniq, inv = np.unique(need, return_inverse=True)
-            y_small = workloads.bf16_bits(y_d[torch.from_numpy(uniq).long().to(dev)])
-            ref = oracle.combine(y_small, inv.reshape(need.shape).astype(np.int32), w[tsel])
+            need = o.pos[tsel]                     # [n, K] rows those tokens read (-1: masked slot)
+            uniq, inv = np.unique(need[need >= 0], return_inverse=True)
+            small_pos = np.full(need.shape, -1, np.int32)
+            small_pos[need >= 0] = inv
+            y_small = workloads.bf16_bits(y_d[torch.from_numpy(uniq).long().to(dev)]) if len(uniq) \
+                else np.zeros((1, wl.H), np.uint16)
+            ref = oracle.combine(y_small, small_pos, w[tsel])
             combine_close(out[torch.from_numpy(tsel).long().to(dev)], ref)
         assert ep.ep_get_status(g.handle) == 0
     finally:
@@ -252,3 +255,70 @@ def test_host_argument_errors():
         ep.ep_handle_destroy(h)
     with pytest.raises(ep.EpError):
         ep.ep_handle_create(ep.make_config(16, 256, 9, 2, 2, 1))   # E % R != 0
+
+
+@pytest.mark.parametrize("sms", [1, 7, 24])
+def test_sm_limit_same_results(sms):
+    """Capping dispatch/combine to a few SMs changes the launch, not the results."""
+    dev = torch.device("cuda")
+    wl = workloads.generate(None, T=1200, H=2048, E=64, R=8, K=8, A=4, router="topk", seed=61)
+    outs = []
+    for limit in (0, sms):
+        g = gpu_layout(wl)
+        try:
+            ep.ep_set_sm_limit(g.handle, limit)
+            x = wl.x.to(dev)
+            recv = torch.zeros((g.cap, wl.H), dtype=torch.bfloat16, device=dev)
+            ep.ep_dispatch(g.handle, x, recv)
+            q = torch.zeros((g.cap, wl.H), dtype=torch.uint8, device=dev)
+            sc = torch.zeros((g.cap, wl.H // 128), dtype=torch.float32, device=dev)
+            ep.ep_dispatch_fp8(g.handle, x, q, sc)
+            out = torch.empty_like(x)
+            ep.ep_combine(g.handle, recv, wl.topk_weights.to(dev), out)
+            torch.cuda.synchronize()
+            outs.append([t.cpu() for t in (recv[:g.rows], q[:g.rows], sc[:g.rows], out)])
+        finally:
+            ep.ep_handle_destroy(g.handle)
+    for a, b in zip(*outs):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+
+
+def test_masked_slots_parity():
+    """-1 slots (tokens that select fewer than K experts): no row, nothing in combine."""
+    wl = workloads.generate(None, T=900, H=1024, E=64, R=8, K=8, A=4, router="topk", seed=71)
+    idx = wl.topk_idx.clone()
+    g = torch.Generator().manual_seed(5)
+    idx[torch.rand(idx.shape, generator=g) < 0.25] = -1
+    idx[3, :] = -1                                 # one token with no expert at all
+    wl.topk_idx = idx
+    run_full(wl, False)
+    run_full(wl, True)
+
+
+def test_col_major_tma_scales():
+    """The column-major, 4-float-aligned scale layout holds the same values."""
+    dev = torch.device("cuda")
+    wl = workloads.generate(None, T=333, H=1024, E=32, R=4, K=6, A=8, router="topk", seed=81)
+    g = gpu_layout(wl)
+    try:
+        cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
+        nb = wl.H // 128
+        ld = (g.cap + 3) // 4 * 4
+        assert ep.ep_scale_buffer_floats(cfg, ep.EP_SCALES_COL_MAJOR_TMA) == nb * ld
+        x = wl.x.to(dev)
+        q_r = torch.zeros((g.cap, wl.H), dtype=torch.uint8, device=dev)
+        s_r = torch.zeros((g.cap, nb), dtype=torch.float32, device=dev)
+        ep.ep_dispatch_fp8(g.handle, x, q_r, s_r)
+        ep.ep_set_scale_layout(g.handle, ep.EP_SCALES_COL_MAJOR_TMA)
+        q_c = torch.zeros((g.cap, wl.H), dtype=torch.uint8, device=dev)
+        s_c = torch.full((nb, ld), -1.0, dtype=torch.float32, device=dev)
+        ep.ep_dispatch_fp8(g.handle, x, q_c, s_c)
+        torch.cuda.synchronize()
+        assert torch.equal(q_r[:g.rows], q_c[:g.rows])
+        assert torch.equal(s_r[:g.rows].t().contiguous().view(torch.int32), s_c[:, :g.rows].contiguous().view(torch.int32))
+        assert (s_c.data_ptr() % 16 == 0) and (ld * 4) % 16 == 0     # every block column 16-byte aligned
+        o = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A)
+        oq, osc = oracle.dispatch_fp8(workloads.bf16_bits(wl.x), o.row_src)
+        np.testing.assert_array_equal(s_c[:, :g.rows].t().cpu().numpy().view(np.uint32), osc.view(np.uint32))
+    finally:
+        ep.ep_handle_destroy(g.handle)

@@ -139,3 +139,19 @@ def test_selected_rows_and_tokens(oracle_lib):
     out = oracle_lib.combine(full, L.pos, w)
     tsel = np.array([7, 0, 29], np.int32)
     np.testing.assert_array_equal(oracle_lib.combine(full, L.pos, w, tsel), out[tsel])
+
+
+def test_masked_slots_round_trip(oracle_lib):
+    """Identity experts with some slots masked (-1): out = x * sum of the unmasked weights."""
+    wl, idx, w, xb = _setup(T=40, H=256, E=8, R=2, K=4, A=3, seed=17)
+    rng = np.random.default_rng(3)
+    idx = idx.copy()
+    idx[rng.random(idx.shape) < 0.3] = -1
+    L = oracle_lib.layout(idx, wl.E, wl.R, wl.A, topk_weights=w)
+    assert L.status == 0
+    assert int(L.num_tokens_per_expert.sum()) == int((idx >= 0).sum())
+    assert (L.pos[idx < 0] == -1).all()
+    recv = oracle_lib.dispatch_bf16(xb, L.row_src)
+    out = oracle_lib.combine(recv, L.pos, w)
+    wsum = np.where(idx >= 0, w.astype(np.float64), 0.0).sum(1, keepdims=True)
+    np.testing.assert_allclose(out, _to_f64(xb) * wsum, rtol=1e-13, atol=1e-13)

@@ -41,7 +41,8 @@ def naive_layout(idx, E, R, A):
     """Second definition: sort the (expert, token, k) triples, pad each segment."""
     T, K = idx.shape
     Lr = E // R
-    triples = sorted((int(idx[t, k]), t, k) for t in range(T) for k in range(K))
+    # -1 marks an unused slot: no row, pos = -1
+    triples = sorted((int(idx[t, k]), t, k) for t in range(T) for k in range(K) if idx[t, k] != -1)
     rows, offsets, pos = [], [0], {}
     for e in range(E):
         seg = [(t, k) for (ee, t, k) in triples if ee == e]
@@ -51,14 +52,14 @@ def naive_layout(idx, E, R, A):
         rows.extend([None] * ((-len(seg)) % A))
         offsets.append(len(rows))
     counts = [sum(1 for tr in triples if tr[0] == e) for e in range(E)]
-    ranks_of = [set(int(idx[t, k]) // Lr for k in range(K)) for t in range(T)]
+    ranks_of = [set(int(idx[t, k]) // Lr for k in range(K) if idx[t, k] != -1) for t in range(T)]
     in_rank = [[1 if r in ranks_of[t] else 0 for r in range(R)] for t in range(T)]
     per_rank = [sum(in_rank[t][r] for t in range(T)) for r in range(R)]
     return dict(
         num_tokens_per_expert=counts, num_tokens_per_rank=per_rank,
         is_token_in_rank=np.array(in_rank, dtype=np.uint8).reshape(T, R),
         expert_offsets=offsets, rank_offsets=[offsets[r * Lr] for r in range(R + 1)],
-        pos=np.array([[pos[(t, k)] for k in range(K)] for t in range(T)], dtype=np.int32).reshape(T, K),
+        pos=np.array([[pos.get((t, k), -1) for k in range(K)] for t in range(T)], dtype=np.int32).reshape(T, K),
         row_src=[-1 if x is None else x[0] for x in rows],
         row_slot=[-1 if x is None else x[1] for x in rows])
 
@@ -74,7 +75,7 @@ def test_bruteforce_tiny(oracle_lib):
             for K in (1, 2):
                 if T * K > 6:
                     continue
-                tables = itertools.product(range(E), repeat=T * K)
+                tables = itertools.product(range(-1 if E <= 3 else 0, E), repeat=T * K)
                 for flat in tables:
                     idx = np.array(flat, dtype=np.int64).reshape(T, K)
                     for R in _divisors(E):
@@ -94,7 +95,7 @@ def check_layout_invariants(L, idx, E, R, A, w=None):
     T, K = idx.shape
     Lr = E // R
     cnt = L.num_tokens_per_expert
-    assert int(cnt.sum()) == T * K                       # conservation
+    assert int(cnt.sum()) == T * K                       # conservation (no masked slots here)
     np.testing.assert_array_equal(cnt, np.bincount(idx.ravel(), minlength=E))
     pad = -(-cnt // A) * A
     np.testing.assert_array_equal(np.diff(L.expert_offsets), pad)
@@ -152,9 +153,22 @@ def test_workload_shapes():
 def test_invalid_expert_ids(oracle_lib):
     idx = np.array([[0, 1], [2, 4]], dtype=np.int64)
     assert oracle_lib.layout(idx, 4, 2, 1).status == oracle_lib.BAD_EXPERT
-    idx = np.array([[0, -1]], dtype=np.int64)
+    idx = np.array([[0, -2]], dtype=np.int64)
     assert oracle_lib.layout(idx, 4, 2, 1).status == oracle_lib.BAD_EXPERT
     assert oracle_lib.layout(np.zeros((1, 1), np.int64), 4, 3, 1).status == oracle_lib.BAD_ARG
+
+
+def test_masked_slots(oracle_lib):
+    """-1 marks an unused top-k slot: no row, not counted, pos = -1."""
+    idx = np.array([[0, -1], [-1, -1], [3, 0]], dtype=np.int64)
+    L = oracle_lib.layout(idx, 4, 2, 2)
+    assert L.status == 0
+    assert list(L.num_tokens_per_expert) == [2, 0, 0, 1]
+    assert L.pos.tolist() == [[0, -1], [-1, -1], [2, 1]]
+    assert list(L.expert_offsets) == [0, 2, 2, 2, 4]
+    assert list(L.row_src) == [0, 2, 2, -1]
+    assert L.is_token_in_rank.tolist() == [[1, 0], [0, 0], [1, 1]]
+    assert list(L.num_tokens_per_rank) == [2, 1]
 
 
 def test_empty_and_degenerate(oracle_lib):

@@ -21,9 +21,9 @@ MUTANTS = {
         "int32_t padded = ((c + A - 1) / A) * A;", "int32_t padded = (c / A + 1) * A;"),
     "offsets not accumulated": (
         "expert_offsets[e + 1] = expert_offsets[e] + padded;", "expert_offsets[e + 1] = padded;"),
-    "rank of an expert by modulo": (
-        "if (topk_idx[(int64_t)t * K + k] / L == r) in = 1;",
-        "if (topk_idx[(int64_t)t * K + k] % R == r) in = 1;"),
+    "rank of an expert by modulo": ("if (e >= 0 && e / L == r) in = 1;", "if (e >= 0 && e % R == r) in = 1;"),
+    "masked slot counted": ("            if (e >= 0) num_tokens_per_expert[e] += 1;",
+                            "            num_tokens_per_expert[e < 0 ? 0 : e] += 1;"),
     "tokens appended in reverse order": (
         "    for (int32_t t = 0; t < T; ++t) {\n        for (int32_t k = 0; k < K; ++k) {\n            int64_t i",
         "    for (int32_t t = T - 1; t >= 0; --t) {\n        for (int32_t k = 0; k < K; ++k) {\n            int64_t i"),
@@ -80,6 +80,8 @@ PINS = [
     ("e4m3 brute force", lambda lib: tf8.test_brute_force_all_bf16(lib)),
     ("e4m3 ties", lambda lib: tf8.test_ties_and_neighbours(lib)),
     ("identity round trip", lambda lib: tdc.test_identity_round_trip(lib, 4)),
+    ("masked slots", lambda lib: tlay.test_masked_slots(lib)),
+    ("masked round trip", lambda lib: tdc.test_masked_slots_round_trip(lib)),
     ("one-hot", lambda lib: tdc.test_one_hot_selects_expert_row(lib)),
     ("lesson exercise", lambda lib: tdc.test_lesson_exercise_restated(lib)),
     ("fp8 properties", lambda lib: tdc.test_fp8_dispatch_properties(lib, 5)),
