@@ -29,7 +29,7 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-OK, BAD_EXPERT, BAD_ARG = 0, 1, 2
+OK, BAD_EXPERT, BAD_ARG, SLOT_OVERFLOW = 0, 1, 2, 3
 
 
 def build(force: bool = False) -> str:
@@ -56,6 +56,8 @@ def _bind(lib):
     lib.oracle_capacity_rows.restype = i64
     lib.oracle_layout.argtypes = [i32, i32, i32, i32, i32] + [P] * 11
     lib.oracle_layout.restype = ctypes.c_int
+    lib.oracle_ll_layout.argtypes = [i32, i32, i32, i32, P, P, P]
+    lib.oracle_ll_layout.restype = ctypes.c_int
     lib.oracle_dispatch_bf16.argtypes = [i32, i32, i32, P, P, P, P]
     lib.oracle_dispatch_bf16.restype = ctypes.c_int
     lib.oracle_dispatch_fp8.argtypes = [i32, i32, i32, P, P, P, P, P]
@@ -174,6 +176,25 @@ def layout(topk_idx, num_experts: int, num_ranks: int, expert_alignment: int = 1
         out.row_slot = out.row_slot[:rows]
         out.row_weight = out.row_weight[:rows]
     out.capacity = cap
+    return out
+
+
+def ll_layout(topk_idx, num_experts: int, max_tokens: int) -> Layout:
+    """Low-latency static layout: M = max_tokens slots per expert.
+
+    Fields: status (OK, BAD_EXPERT or SLOT_OVERFLOW), recv_count [E],
+    pos [T, K] (e*M + slot, or -1), capacity = E*M, and row_src [E*M]
+    (token of each used slot, -1 elsewhere) for the dispatch functions."""
+    idx = _c(topk_idx, np.int64)
+    T, K = idx.shape
+    E, M = num_experts, max_tokens
+    out = Layout(recv_count=np.zeros(E, np.int32), pos=np.zeros((T, K), np.int32), capacity=E * M)
+    out.status = _load().oracle_ll_layout(T, E, K, M, _ptr(idx), _ptr(out.recv_count), _ptr(out.pos))
+    if out.status in (OK, SLOT_OVERFLOW):
+        src = np.full(E * M, -1, np.int32)
+        used = out.pos >= 0
+        src[out.pos[used]] = np.nonzero(used)[0].astype(np.int32)
+        out.row_src = src
     return out
 
 

@@ -43,6 +43,7 @@
 #define ORACLE_OK 0
 #define ORACLE_BAD_EXPERT 1
 #define ORACLE_BAD_ARG 2
+#define ORACLE_SLOT_OVERFLOW 3
 
 /* ------------------------------------------------------------------ */
 /* Number formats                                                       */
@@ -197,6 +198,42 @@ int oracle_layout(int32_t T, int32_t E, int32_t R, int32_t K, int32_t A,
     }
     free(cursor);
     return ORACLE_OK;
+}
+
+/*
+ * Low-latency (static, masked) layout: every expert e owns M fixed slots,
+ * received rows e*M .. e*M+M-1, and the per-expert count is the mask a
+ * masked grouped GEMM reads ("lesson14_deepep" section 2(1): decode mode is
+ * static for CUDA graphs, with pre-allocated buffers and mask marks; section
+ * 3: low_latency_dispatch feeds m_grouped_fp8_gemm_nt_masked with a mask).
+ * Slots are filled in the same order as the normal layout: tokens, then k.
+ *
+ * Outputs: recv_count [E] = slots used by expert e (at most M), pos [T,K]
+ * = e*M + slot, or -1 for a masked id (-1) or a pair past an expert's M-th.
+ * Returns ORACLE_BAD_EXPERT if an id other than -1 is outside [0, E)
+ * (outputs unspecified), ORACLE_SLOT_OVERFLOW if some expert was offered
+ * more than M pairs (outputs as described), else ORACLE_OK.
+ */
+int oracle_ll_layout(int32_t T, int32_t E, int32_t K, int32_t M, const int64_t *topk_idx,
+                     int32_t *recv_count, int32_t *pos)
+{
+    if (T < 0 || E <= 0 || K <= 0 || M <= 0) return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < (int64_t)T * K; ++i)
+        if (topk_idx[i] != -1 && (topk_idx[i] < 0 || topk_idx[i] >= E)) return ORACLE_BAD_EXPERT;
+
+    int overflow = 0;
+    for (int32_t e = 0; e < E; ++e) recv_count[e] = 0;
+    for (int32_t t = 0; t < T; ++t) {
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t i = (int64_t)t * K + k;
+            int32_t e = (int32_t)topk_idx[i];
+            if (e < 0) { pos[i] = -1; continue; }              /* masked slot */
+            if (recv_count[e] >= M) { pos[i] = -1; overflow = 1; continue; }
+            pos[i] = (int32_t)((int64_t)e * M + recv_count[e]);
+            recv_count[e] += 1;
+        }
+    }
+    return overflow ? ORACLE_SLOT_OVERFLOW : ORACLE_OK;
 }
 
 /* ------------------------------------------------------------------ */

@@ -15,6 +15,7 @@ import oracle
 import test_oracle_dispatch_combine as tdc
 import test_oracle_fp8 as tf8
 import test_oracle_layout as tlay
+import test_oracle_ll as tll
 
 MUTANTS = {
     "padding rounds up a full segment": (
@@ -25,8 +26,8 @@ MUTANTS = {
     "masked slot counted": ("            if (e >= 0) num_tokens_per_expert[e] += 1;",
                             "            num_tokens_per_expert[e < 0 ? 0 : e] += 1;"),
     "tokens appended in reverse order": (
-        "    for (int32_t t = 0; t < T; ++t) {\n        for (int32_t k = 0; k < K; ++k) {\n            int64_t i",
-        "    for (int32_t t = T - 1; t >= 0; --t) {\n        for (int32_t k = 0; k < K; ++k) {\n            int64_t i"),
+        "cursor[e] = expert_offsets[e];\n    for (int32_t t = 0; t < T; ++t) {",
+        "cursor[e] = expert_offsets[e];\n    for (int32_t t = T - 1; t >= 0; --t) {"),
     "slot recorded as token": ("row_slot[r] = k;", "row_slot[r] = t;"),
     "ties rounded away from zero": ("if (d > 0.5f) return n + 1;", "if (d >= 0.5f) return n + 1;"),
     "no saturation (NaN code)": (
@@ -48,6 +49,13 @@ MUTANTS = {
     "dispatch copies the previous token": (
         "memcpy(dst, x + (int64_t)t * H, sizeof(uint16_t) * (size_t)H);",
         "memcpy(dst, x + (int64_t)(t > 0 ? t - 1 : 0) * H, sizeof(uint16_t) * (size_t)H);"),
+    "low-latency slot not advanced": ("            recv_count[e] += 1;\n", "\n"),
+    "low-latency overflow off by one": ("if (recv_count[e] >= M)", "if (recv_count[e] > M)"),
+    "low-latency expert stride": ("pos[i] = (int32_t)((int64_t)e * M + recv_count[e]);",
+                                  "pos[i] = (int32_t)((int64_t)e * (M - 1) + recv_count[e]);"),
+    "low-latency masked slot counted": (
+        "if (e < 0) { pos[i] = -1; continue; }              /* masked slot */",
+        "if (e < 0) { pos[i] = -1; recv_count[0] += 1; continue; }"),
     "padding row not zeroed": (
         "            memset(dst, 0, sizeof(uint16_t) * (size_t)H);\n",
         "            memset(dst, 0, sizeof(uint16_t) * (size_t)(H / 2));\n"),
@@ -85,6 +93,9 @@ PINS = [
     ("one-hot", lambda lib: tdc.test_one_hot_selects_expert_row(lib)),
     ("lesson exercise", lambda lib: tdc.test_lesson_exercise_restated(lib)),
     ("fp8 properties", lambda lib: tdc.test_fp8_dispatch_properties(lib, 5)),
+    ("ll worked example", lambda lib: tll.test_ll_worked_example(lib)),
+    ("ll brute force", lambda lib: tll.test_ll_bruteforce_tiny(lib)),
+    ("ll round trip", lambda lib: tll.test_ll_round_trip(lib)),
 ]
 
 
