@@ -325,6 +325,51 @@ class Path:
         self.ep.ep_handle_destroy(self.h)
 
 
+class LLPath(Path):
+    """The low-latency static layout: M fixed slots per expert, layout fused
+    into the dispatch launch (ep_ll_dispatch), no padding rows."""
+
+    def __init__(self, wl, dev, M):
+        import torch
+
+        import combine_ep_get_08_b200 as ep
+        self.ep, self.torch, self.wl, self.dev = ep, torch, wl, dev
+        cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, 1)
+        self.M = M
+        self.cap = ep.ep_ll_capacity_rows(cfg, M)
+        self.h = ep.ep_ll_handle_create(cfg, M)
+        self.idx = wl.topk_idx.to(dev)
+        self.w = wl.topk_weights.to(dev)
+        self.x = wl.x.to(dev)
+        self.cnt = torch.zeros((wl.E,), dtype=torch.int32, device=dev)
+        if wl.fp8:
+            self.recv = torch.empty((self.cap, wl.H), dtype=torch.uint8, device=dev)
+            self.scales = torch.empty((ep.ep_ll_scale_buffer_floats(cfg, M),), dtype=torch.float32, device=dev)
+            g = torch.Generator(device=dev)
+            g.manual_seed(7)
+            self.y = torch.randn((self.cap, wl.H), generator=g, device=dev).to(torch.bfloat16)
+        else:
+            self.recv = torch.empty((self.cap, wl.H), dtype=torch.bfloat16, device=dev)
+            self.scales = None
+            self.y = self.recv
+        self.out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+        self.flush_buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.flush_sink = None
+
+    def layout(self, stream):
+        pass                                   # fused into the dispatch launch
+
+    def dispatch(self, stream, x=None):
+        x = self.x if x is None else x
+        if self.wl.fp8:
+            self.ep.ep_ll_dispatch_fp8(self.h, self.idx, x, self.recv, self.scales, self.cnt, stream=stream)
+        else:
+            self.ep.ep_ll_dispatch(self.h, self.idx, x, self.recv, self.cnt, stream=stream)
+
+    def combine(self, stream, out=None):
+        self.ep.ep_ll_combine(self.h, self.y, self.w, self.out if out is None else out, stream=stream)
+
+
 def run_cuda(args, world, rank, local):
     import numpy as np
     import torch
@@ -347,7 +392,8 @@ def run_cuda(args, world, rank, local):
     base = workloads.CONFIGS[args.config]
     wl = workloads.generate(args.config, seed=base["seed"] + 1000 * rank)
     reuse = base["reuse"] if args.reuse is None else args.reuse
-    path = Path(wl, dev)
+    ll = args.mode == "ll"
+    path = LLPath(wl, dev, args.ll_slots or max(wl.T, 1)) if ll else Path(wl, dev)
     if args.sm_limit:
         ep.ep_set_sm_limit(path.h, args.sm_limit)
     stream = torch.cuda.current_stream(dev)
@@ -374,7 +420,7 @@ def run_cuda(args, world, rank, local):
     for _ in range(args.warmup):
         one_step()
     torch.cuda.synchronize()
-    rows = ep.ep_get_num_rows(path.h)
+    rows = int(path.cnt.sum()) if ll else ep.ep_get_num_rows(path.h)
     status = ep.ep_get_status(path.h)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
@@ -418,7 +464,7 @@ def run_cuda(args, world, rank, local):
     dom = "dispatch" if dis_us >= com_us else "combine"
     dom_bytes = b_dis if dom == "dispatch" else b_com
     achieved = dom_bytes / (kern[dom] * 1e-6) / 1e9
-    kname, traffic = ncu_traffic(dom, args.config)
+    kname, traffic = ncu_traffic(dom, args.config + ("-ll" if ll else ""))
     clocks = sampler.summary()
     status_end = ep.ep_get_status(path.h)
     path.close()
@@ -432,6 +478,8 @@ def run_cuda(args, world, rank, local):
             "config": {
                 "workload": workloads.DESCRIPTIONS[args.config], "name": args.config,
                 "rows": rows, "reuse": reuse,
+                "layout_mode": (f"low-latency static: {path.M} slots per expert, layout fused into "
+                                "the dispatch launch" if ll else "normal: padded expert-major rows"),
                 "parallelism": f"replicas x{world} (independent batches, no data-path collective)",
                 "sm_limit": args.sm_limit or None,
                 "l2": "flushed (256 MiB read, outside the timed events) before each step and "
@@ -516,6 +564,9 @@ def main(argv=None):
     ap.add_argument("--ref-tokens", type=int, default=4096, help="tokens per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sm-limit", type=int, default=0, help="SMs dispatch/combine may occupy (0: all)")
+    ap.add_argument("--mode", choices=["normal", "ll"], default="normal",
+                    help="layout: normal (padded, ep_get_layout) or low-latency static slots (ep_ll_*)")
+    ap.add_argument("--ll-slots", type=int, default=0, help="slots per expert in --mode ll (0: T)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("EP_B200_LIB", os.path.join(_HERE, "libep_b200.so"))
 
 EP_OK, EP_ERR_ARG, EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EP_ERR_STATE, EP_ERR_DEVICE = 0, -1, -2, -3, -4, -5
-EP_DEV_BAD_EXPERT, EP_DEV_WAIT_TIMEOUT = 0x1, 0x2
+EP_DEV_BAD_EXPERT, EP_DEV_WAIT_TIMEOUT, EP_DEV_SLOT_OVERFLOW = 0x1, 0x2, 0x4
 EP_SCALES_ROW_MAJOR, EP_SCALES_COL_MAJOR_TMA = 0, 1
 
 
@@ -80,6 +80,12 @@ def _load():
             "ep_clear_status": ([P, P], ctypes.c_int),
             "ep_set_wait_limit": ([P, U64, I32], ctypes.c_int),
             "ep_set_sm_limit": ([P, I32], ctypes.c_int),
+            "ep_ll_capacity_rows": ([CFG, I32], I64),
+            "ep_ll_scale_buffer_floats": ([CFG, I32, I32], I64),
+            "ep_ll_handle_create": ([CFG, I32, ctypes.POINTER(P)], ctypes.c_int),
+            "ep_ll_dispatch": ([P] * 6, ctypes.c_int),
+            "ep_ll_dispatch_fp8": ([P] * 7, ctypes.c_int),
+            "ep_ll_combine": ([P] * 5, ctypes.c_int),
             "ep_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "ep_last_error": ([], ctypes.c_char_p),
             "ep_launch_count": ([], U64),
@@ -232,6 +238,37 @@ def ep_set_sm_limit(h: int, num_sms: int) -> None:
 
 def ep_set_wait_limit(h: int, limit_ns: int, extra_arrivals: int = 0) -> None:
     _check("ep_set_wait_limit", _load().ep_set_wait_limit(h, limit_ns, extra_arrivals))
+
+
+def ep_ll_capacity_rows(cfg: ep_config, num_max_dispatch_tokens: int) -> int:
+    return _check("ep_ll_capacity_rows", _load().ep_ll_capacity_rows(ctypes.byref(cfg), num_max_dispatch_tokens))
+
+
+def ep_ll_scale_buffer_floats(cfg: ep_config, num_max_dispatch_tokens: int,
+                              layout: int = EP_SCALES_ROW_MAJOR) -> int:
+    return _check("ep_ll_scale_buffer_floats",
+                  _load().ep_ll_scale_buffer_floats(ctypes.byref(cfg), num_max_dispatch_tokens, layout))
+
+
+def ep_ll_handle_create(cfg: ep_config, num_max_dispatch_tokens: int) -> int:
+    out = ctypes.c_void_p()
+    _check("ep_ll_handle_create",
+           _load().ep_ll_handle_create(ctypes.byref(cfg), num_max_dispatch_tokens, ctypes.byref(out)))
+    return out.value
+
+
+def ep_ll_dispatch(h: int, topk_idx, x, recv_x, recv_count=None, stream=None) -> None:
+    _check("ep_ll_dispatch", _load().ep_ll_dispatch(
+        h, _ptr(topk_idx), _ptr(x), _ptr(recv_x), _ptr(recv_count), _stream(stream)))
+
+
+def ep_ll_dispatch_fp8(h: int, topk_idx, x, recv_q, recv_scales, recv_count=None, stream=None) -> None:
+    _check("ep_ll_dispatch_fp8", _load().ep_ll_dispatch_fp8(
+        h, _ptr(topk_idx), _ptr(x), _ptr(recv_q), _ptr(recv_scales), _ptr(recv_count), _stream(stream)))
+
+
+def ep_ll_combine(h: int, y, topk_weights, out, stream=None) -> None:
+    _check("ep_ll_combine", _load().ep_ll_combine(h, _ptr(y), _ptr(topk_weights), _ptr(out), _stream(stream)))
 
 
 def ep_status_string(code: int) -> str:

@@ -78,7 +78,74 @@ __device__ __forceinline__ void zero_fill_unit(const DispatchParams &p, int z, i
     }
 }
 
-template <int VB>
+// ---------------------------------------------------------------------------
+// Low-latency static layout (lesson14_deepep section 2(1): decode buffers are
+// pre-allocated per expert and the per-expert count is the mask).  Expert e
+// owns rows e*M .. e*M+M-1, filled in (token, k) order, so the slot of pair
+// (t, k) is the number of earlier pairs with the same expert.  Every CTA
+// walks its tokens in increasing order and keeps a shared-memory histogram
+// of the pairs of all tokens before the current one (each CTA re-reads the
+// ids it has not counted yet: T*K ids at most, an L2 hit), so no CTA waits
+// on another and layout and copy are one launch.  The grid's last CTA only
+// counts all pairs and writes recv_count.
+// ---------------------------------------------------------------------------
+struct LlState {
+    int32_t *hist;   // [E] pairs per expert among tokens [0, upto)
+    int32_t *ids;    // [kMaxTopk] this token's ids (-1 masked, -2 invalid)
+    int upto;
+};
+
+__device__ __forceinline__ void ll_init(const DispatchParams &p, LlState &st) {
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) st.hist[e] = 0;
+    st.upto = 0;
+    __syncthreads();
+}
+
+__device__ __forceinline__ void ll_advance(const DispatchParams &p, LlState &st, int t) {
+    for (int64_t i = (int64_t)st.upto * p.K + threadIdx.x; i < (int64_t)t * p.K; i += blockDim.x) {
+        const int64_t e = __ldg(&p.topk_idx[i]);
+        if (e >= 0 && e < p.E) atomicAdd(&st.hist[e], 1);
+    }
+    st.upto = t;
+}
+
+// Destinations of token t's K pairs into s_dst (split 0 also writes pos);
+// ends with a block barrier.
+__device__ __forceinline__ void ll_destinations(const DispatchParams &p, LlState &st, int t, bool write_pos,
+                                                int32_t *s_dst) {
+    if (t > st.upto) ll_advance(p, st, t);
+    if (threadIdx.x < p.K) {
+        const int64_t e = __ldg(&p.topk_idx[(int64_t)t * p.K + threadIdx.x]);
+        st.ids[threadIdx.x] = (e >= 0 && e < p.E) ? (int)e : (e == -1 ? -1 : -2);
+    }
+    __syncthreads();
+    if (threadIdx.x < p.K) {
+        const int k = threadIdx.x, e = st.ids[k];
+        int dst = -1;
+        if (e >= 0) {
+            int slot = st.hist[e];
+            for (int j = 0; j < k; ++j) slot += st.ids[j] == e;
+            if (slot < p.ll_M)
+                dst = e * p.ll_M + slot;
+            else if (write_pos)
+                atomicOr(p.status, EP_DEV_SLOT_OVERFLOW);
+        } else if (e == -2 && write_pos) {
+            atomicOr(p.status, EP_DEV_BAD_EXPERT);
+        }
+        s_dst[k] = dst;
+        if (write_pos) p.pos_out[(int64_t)t * p.K + k] = dst;
+    }
+    __syncthreads();
+}
+
+// The count CTA: recv_count[e] = min(pairs of expert e, M).
+__device__ __forceinline__ void ll_count(const DispatchParams &p, LlState &st) {
+    ll_advance(p, st, p.T);
+    __syncthreads();
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) p.recv_count[e] = min(st.hist[e], p.ll_M);
+}
+
+template <int VB, bool LL>
 __global__ void __launch_bounds__(kThreads, EP_LSU_MINB) dispatch_bf16_kernel(DispatchParams p) {
     using V = Vec<VB>;
     using VT = typename V::T;
@@ -90,11 +157,30 @@ __global__ void __launch_bounds__(kThreads, EP_LSU_MINB) dispatch_bf16_kernel(Di
     const uint8_t *x = static_cast<const uint8_t *>(p.x);
     uint8_t *recv = static_cast<uint8_t *>(p.recv);
     int rows = -1;
-    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+    LlState st;
+    int nblk = gridDim.x;
+    if constexpr (LL) {
+        extern __shared__ int32_t ll_smem[];
+        st.ids = ll_smem;
+        st.hist = ll_smem + kMaxTopk;
+        ll_init(p, st);
+        if (p.recv_count) {
+            nblk = gridDim.x - 1;
+            if (blockIdx.x == nblk) {
+                ll_count(p, st);
+                return;
+            }
+        }
+    }
+    for (int u = blockIdx.x; u < total; u += nblk) {
         if (u < p.n_token_units) {
             const int t = u / p.splits, s = u - t * p.splits;
-            if (threadIdx.x < p.K) s_dst[threadIdx.x] = __ldg(&p.pos[(int64_t)t * p.K + threadIdx.x]);
-            __syncthreads();
+            if constexpr (LL) {
+                ll_destinations(p, st, t, s == 0, s_dst);
+            } else {
+                if (threadIdx.x < p.K) s_dst[threadIdx.x] = __ldg(&p.pos[(int64_t)t * p.K + threadIdx.x]);
+                __syncthreads();
+            }
             const int v0 = s * vps, v1 = min(nv, v0 + vps);
             const uint8_t *xr = x + (int64_t)t * row_bytes;
             for (int v = v0 + threadIdx.x; v < v1; v += kThreads * kUnroll) {
@@ -343,8 +429,12 @@ __device__ __forceinline__ unsigned int e4m3x2(float a, float b) {
 // TPB = 128 / EPT consecutive lanes share one 1x128 block and reduce its
 // amax with shuffles.  Each thread stores EPT code bytes per received row.
 // Index of the scale of received row `row`, block b, in either layout.
+// Column-major scales come in groups of scale_group_rows rows (the whole
+// buffer, or one expert's M slots), each group [H/128][scale_ld].
 __device__ __forceinline__ int64_t scale_index(const DispatchParams &p, int row, int b, int NB) {
-    return p.scale_ld > 0 ? (int64_t)b * p.scale_ld + row : (int64_t)row * NB + b;
+    if (p.scale_ld == 0) return (int64_t)row * NB + b;
+    const int g = row / p.scale_group_rows;
+    return ((int64_t)g * NB + b) * p.scale_ld + (row - g * p.scale_group_rows);
 }
 
 template <int EPT>
@@ -378,7 +468,7 @@ struct Fp8Io<32> {
     }
 };
 
-template <int EPT>
+template <int EPT, bool LL>
 __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p) {
     constexpr int TPB = 128 / EPT;
     constexpr int NW = EPT / 2;              // bf16x2 words loaded per thread
@@ -389,11 +479,30 @@ __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p
     const uint8_t *x = static_cast<const uint8_t *>(p.x);
     uint8_t *recv = static_cast<uint8_t *>(p.recv);
     int rows = -1;
-    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+    LlState st;
+    int nblk = gridDim.x;
+    if constexpr (LL) {
+        extern __shared__ int32_t ll_smem[];
+        st.ids = ll_smem;
+        st.hist = ll_smem + kMaxTopk;
+        ll_init(p, st);
+        if (p.recv_count) {
+            nblk = gridDim.x - 1;
+            if (blockIdx.x == nblk) {
+                ll_count(p, st);
+                return;
+            }
+        }
+    }
+    for (int u = blockIdx.x; u < total; u += nblk) {
         if (u < p.n_token_units) {
             const int t = u;
-            if (threadIdx.x < p.K) s_dst[threadIdx.x] = __ldg(&p.pos[(int64_t)t * p.K + threadIdx.x]);
-            __syncthreads();
+            if constexpr (LL) {
+                ll_destinations(p, st, t, true, s_dst);
+            } else {
+                if (threadIdx.x < p.K) s_dst[threadIdx.x] = __ldg(&p.pos[(int64_t)t * p.K + threadIdx.x]);
+                __syncthreads();
+            }
             const uint8_t *xr = x + (int64_t)t * p.H * 2;
             for (int g0 = 0; g0 < nthr_row; g0 += kThreads) {
                 const int g = g0 + threadIdx.x;
@@ -493,15 +602,52 @@ cudaError_t launch_dispatch_bf16(const DispatchParams &p_in, int num_sms, cudaSt
     }
     const int units = p.n_token_units + p.n_zero_units;
     if (v32) {
-        const void *k = reinterpret_cast<const void *>(&dispatch_bf16_kernel<32>);
+        const void *k = reinterpret_cast<const void *>(&dispatch_bf16_kernel<32, false>);
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ32), num_sms);
-        dispatch_bf16_kernel<32><<<grid, kThreads, 0, s>>>(p);
+        dispatch_bf16_kernel<32, false><<<grid, kThreads, 0, s>>>(p);
     } else {
-        const void *k = reinterpret_cast<const void *>(&dispatch_bf16_kernel<16>);
+        const void *k = reinterpret_cast<const void *>(&dispatch_bf16_kernel<16, false>);
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ16), num_sms);
-        dispatch_bf16_kernel<16><<<grid, kThreads, 0, s>>>(p);
+        dispatch_bf16_kernel<16, false><<<grid, kThreads, 0, s>>>(p);
     }
     return cudaGetLastError();
+}
+
+// Low-latency launches: the register kernels with in-kernel destinations.
+// The copy CTAs come from the occupancy-sized persistent grid; one more CTA
+// counts all pairs into recv_count.
+static size_t ll_smem_bytes(int E) { return sizeof(int32_t) * (size_t)(kMaxTopk + E); }
+
+cudaError_t launch_ll_dispatch(const DispatchParams &p_in, bool fp8, int num_sms, cudaStream_t s) {
+    static int occ[4] = {0, 0, 0, 0};
+    DispatchParams p = p_in;
+    p.n_zero_units = 0;
+    const size_t smem = ll_smem_bytes(p.E);
+    const size_t smem_max = ll_smem_bytes(kMaxExperts);
+    const bool v32 = (fp8 || p.H % 16 == 0) &&
+                     ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
+    const void *k;
+    int *slot;
+    if (fp8) {
+        p.splits = 1;
+        k = v32 ? reinterpret_cast<const void *>(&dispatch_fp8_kernel<32, true>)
+                : reinterpret_cast<const void *>(&dispatch_fp8_kernel<16, true>);
+        slot = &occ[v32 ? 0 : 1];
+    } else {
+        // split rows so that a small batch still spreads over the SMs
+        const int nv = p.H * 2 / (v32 ? 32 : 16);
+        int sp = 1;
+        while (sp < 8 && p.T * sp < 2 * num_sms && nv / (sp * 2) >= kThreads / 2) sp *= 2;
+        p.splits = sp;
+        k = v32 ? reinterpret_cast<const void *>(&dispatch_bf16_kernel<32, true>)
+                : reinterpret_cast<const void *>(&dispatch_bf16_kernel<16, true>);
+        slot = &occ[v32 ? 2 : 3];
+    }
+    p.n_token_units = p.T * p.splits;
+    const int grid = persistent_grid(p.n_token_units, blocks_per_sm(k, kThreads, smem_max, slot), num_sms) +
+                     (p.recv_count ? 1 : 0);
+    void *args[] = {&p};
+    return cudaLaunchKernel(k, dim3(grid), dim3(kThreads), args, smem, s);
 }
 
 // FP8 uses the register kernel: quantising from a staged ring with one
@@ -512,13 +658,13 @@ cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream
     const int units = p.n_token_units + p.n_zero_units;
     const bool v32 = ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
     if (v32) {
-        const void *k = reinterpret_cast<const void *>(&dispatch_fp8_kernel<32>);
+        const void *k = reinterpret_cast<const void *>(&dispatch_fp8_kernel<32, false>);
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ32), num_sms);
-        dispatch_fp8_kernel<32><<<grid, kThreads, 0, s>>>(p);
+        dispatch_fp8_kernel<32, false><<<grid, kThreads, 0, s>>>(p);
     } else {
-        const void *k = reinterpret_cast<const void *>(&dispatch_fp8_kernel<16>);
+        const void *k = reinterpret_cast<const void *>(&dispatch_fp8_kernel<16, false>);
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ16), num_sms);
-        dispatch_fp8_kernel<16><<<grid, kThreads, 0, s>>>(p);
+        dispatch_fp8_kernel<16, false><<<grid, kThreads, 0, s>>>(p);
     }
     return cudaGetLastError();
 }

@@ -50,6 +50,14 @@ int check_handle(const ep_handle *h, bool need_layout) {
     return EP_OK;
 }
 
+// Calls of one layout mode on a handle of the other return EP_ERR_STATE.
+int check_mode(const ep_handle *h, bool ll, bool need_layout) {
+    int rc = check_handle(h, false);
+    if (rc != EP_OK) return rc;
+    if ((h->ll_M > 0) != ll) return EP_ERR_STATE;
+    return check_handle(h, need_layout);
+}
+
 }  // namespace
 
 namespace ep {
@@ -111,6 +119,7 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->has_layout = false;
     h->sm_limit = 0;
     h->scale_layout = EP_SCALES_ROW_MAJOR;
+    h->ll_M = 0;
     h->layout_epoch = 0;
 
     auto fail = [&](int code) {
@@ -224,7 +233,7 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
                          int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
                          uint8_t *is_token_in_rank, int32_t *expert_offsets, int32_t *rank_offsets,
                          ep_stream_t stream) {
-    int rc = check_handle(h, false);
+    int rc = check_mode(h, false, false);
     if (rc != EP_OK) return rc;
     const ep_config &c = h->cfg;
     if (c.num_tokens > 0 && !topk_idx) return EP_ERR_ARG;
@@ -276,7 +285,7 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
 
 static int dispatch_common(const ep_handle *h, const void *x, void *recv, float *scales, bool fp8,
                            ep_stream_t stream) {
-    int rc = check_handle(h, true);
+    int rc = check_mode(h, false, true);
     if (rc != EP_OK) return rc;
     const ep_config &c = h->cfg;
     if (fp8 && c.hidden % 128 != 0) return EP_ERR_ARG;
@@ -291,6 +300,7 @@ static int dispatch_common(const ep_handle *h, const void *x, void *recv, float 
     p.recv = recv;
     p.recv_scale = scales;
     p.scale_ld = h->scale_layout == EP_SCALES_COL_MAJOR_TMA ? (int)((h->cap + 3) / 4 * 4) : 0;
+    p.scale_group_rows = (int)h->cap;
     p.pos = h->pos;
     p.row_src = h->row_src;
     p.eoff = h->eoff;
@@ -323,9 +333,9 @@ EP_API int ep_dispatch_fp8(const ep_handle *h, const void *x, void *recv_q, floa
     return dispatch_common(h, x, recv_q, recv_scales, true, stream);
 }
 
-EP_API int ep_combine(const ep_handle *h, const void *y, const float *topk_weights, void *out,
-                      ep_stream_t stream) {
-    int rc = check_handle(h, true);
+static int combine_common(const ep_handle *h, const void *y, const float *topk_weights, void *out,
+                          bool ll, ep_stream_t stream) {
+    int rc = check_mode(h, ll, true);
     if (rc != EP_OK) return rc;
     const ep_config &c = h->cfg;
     if (c.num_tokens == 0) return EP_OK;
@@ -354,12 +364,135 @@ EP_API int ep_combine(const ep_handle *h, const void *y, const float *topk_weigh
     return EP_OK;
 }
 
+EP_API int ep_combine(const ep_handle *h, const void *y, const float *topk_weights, void *out,
+                      ep_stream_t stream) {
+    return combine_common(h, y, topk_weights, out, false, stream);
+}
+
+EP_API int ep_ll_combine(const ep_handle *h, const void *y, const float *topk_weights, void *out,
+                         ep_stream_t stream) {
+    return combine_common(h, y, topk_weights, out, true, stream);
+}
+
+// ---- low-latency (static, masked) layout ----
+
+EP_API int64_t ep_ll_capacity_rows(const ep_config *c, int32_t M) {
+    int rc = ep_validate_config(c);
+    if (rc != EP_OK) return rc;
+    if (M < 1 || M < c->num_tokens) return EP_ERR_ARG;
+    const int64_t cap = (int64_t)c->num_experts * M;
+    if (cap > INT32_MAX) return EP_ERR_UNSUPPORTED;
+    return cap;
+}
+
+EP_API int64_t ep_ll_scale_buffer_floats(const ep_config *c, int32_t M, int32_t layout) {
+    const int64_t cap = ep_ll_capacity_rows(c, M);
+    if (cap < 0) return cap;
+    if (c->hidden % 128 != 0) return EP_ERR_ARG;
+    const int64_t nb = c->hidden / 128;
+    if (layout == EP_SCALES_ROW_MAJOR) return cap * nb;
+    if (layout == EP_SCALES_COL_MAJOR_TMA) return (int64_t)c->num_experts * nb * ((M + 3) / 4 * 4);
+    return EP_ERR_ARG;
+}
+
+EP_API int ep_ll_handle_create(const ep_config *cfg, int32_t M, ep_handle **out) {
+    if (!out) return EP_ERR_ARG;
+    *out = nullptr;
+    const int64_t cap = ep_ll_capacity_rows(cfg, M);
+    if (cap < 0) return (int)cap;
+    ep_handle *h = new (std::nothrow) ep_handle();
+    if (!h) return EP_ERR_ARG;
+    h->cfg = *cfg;
+    h->cap = cap;
+    h->ll_M = M;
+    h->wait_limit_ns = ep::kDefaultWaitLimitNs;
+    h->scale_layout = EP_SCALES_ROW_MAJOR;
+    auto fail = [&](int code) {
+        delete h;
+        return code;
+    };
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaGetDevice"));
+    e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaDeviceGetAttribute"));
+    const size_t o_stat = round_up(sizeof(int32_t) * (size_t)cfg->num_tokens * cfg->num_topk + 1, 256);
+    const size_t o_bar = o_stat + 256;
+    h->block_bytes = o_bar + round_up(sizeof(ep::GridBarrier), 256);
+    e = cudaMalloc(&h->block, h->block_bytes);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaMalloc(handle)"));
+    e = cudaMemset(h->block, 0, h->block_bytes);
+    if (e != cudaSuccess) {
+        cudaFree(h->block);
+        return fail(cuda_fail(e, "cudaMemset(handle)"));
+    }
+    char *b = static_cast<char *>(h->block);
+    h->pos = reinterpret_cast<int32_t *>(b);
+    h->status = reinterpret_cast<unsigned int *>(b + o_stat);
+    h->barrier = reinterpret_cast<ep::GridBarrier *>(b + o_bar);
+    *out = h;
+    return EP_OK;
+}
+
+static int ll_dispatch_common(ep_handle *h, const int64_t *topk_idx, const void *x, void *recv,
+                              float *scales, int32_t *recv_count, bool fp8, ep_stream_t stream) {
+    int rc = check_mode(h, true, false);
+    if (rc != EP_OK) return rc;
+    const ep_config &c = h->cfg;
+    if (fp8 && c.hidden % 128 != 0) return EP_ERR_ARG;
+    if (!aligned(recv_count, 4)) return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (c.num_tokens == 0) {   // no pairs: every expert's count is 0
+        if (recv_count) EP_CUDA(cudaMemsetAsync(recv_count, 0, sizeof(int32_t) * c.num_experts, s));
+        h->has_layout = true;
+        return EP_OK;
+    }
+    if (!topk_idx || !x || !recv || (fp8 && !scales)) return EP_ERR_ARG;
+    if (!aligned(topk_idx, 8) || !aligned(x, 16) || !aligned(recv, 16) || !aligned(scales, 4))
+        return EP_ERR_ARG;
+
+    ep::DispatchParams p{};
+    p.x = x;
+    p.recv = recv;
+    p.recv_scale = scales;
+    p.scale_ld = h->scale_layout == EP_SCALES_COL_MAJOR_TMA ? (h->ll_M + 3) / 4 * 4 : 0;
+    p.scale_group_rows = h->ll_M;
+    p.T = c.num_tokens;
+    p.K = c.num_topk;
+    p.E = c.num_experts;
+    p.H = c.hidden;
+    p.status = h->status;
+    p.wait_limit_ns = h->wait_limit_ns;
+    p.ll_M = h->ll_M;
+    p.topk_idx = topk_idx;
+    p.pos_out = h->pos;
+    p.recv_count = recv_count;
+    const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
+    cudaError_t e = ep::launch_ll_dispatch(p, fp8, sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(ll_dispatch_fp8)" : "launch(ll_dispatch)");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    h->has_layout = true;
+    return EP_OK;
+}
+
+EP_API int ep_ll_dispatch(ep_handle *h, const int64_t *topk_idx, const void *x, void *recv_x,
+                          int32_t *recv_count, ep_stream_t stream) {
+    return ll_dispatch_common(h, topk_idx, x, recv_x, nullptr, recv_count, false, stream);
+}
+
+EP_API int ep_ll_dispatch_fp8(ep_handle *h, const int64_t *topk_idx, const void *x, void *recv_q,
+                              float *recv_scales, int32_t *recv_count, ep_stream_t stream) {
+    return ll_dispatch_common(h, topk_idx, x, recv_q, recv_scales, recv_count, true, stream);
+}
+
 EP_API int ep_copy_routing(const ep_handle *h, int32_t *pos, int32_t *row_src, int32_t *row_slot,
                            float *row_weight, ep_stream_t stream) {
     int rc = check_handle(h, true);
     if (rc != EP_OK) return rc;
     if (!aligned(pos, 4) || !aligned(row_src, 4) || !aligned(row_slot, 4) || !aligned(row_weight, 4))
         return EP_ERR_ARG;
+    if (h->ll_M > 0 && (row_src || row_slot || row_weight)) return EP_ERR_ARG;   // pos only
     DeviceGuard g(h->device);
     if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -373,7 +506,7 @@ EP_API int ep_copy_routing(const ep_handle *h, int32_t *pos, int32_t *row_src, i
 }
 
 EP_API int ep_get_num_rows(const ep_handle *h, int32_t *rows, ep_stream_t stream) {
-    int rc = check_handle(h, true);
+    int rc = check_mode(h, false, true);
     if (rc != EP_OK) return rc;
     if (!rows) return EP_ERR_ARG;
     DeviceGuard g(h->device);
@@ -433,8 +566,8 @@ EP_API const char *ep_status_string(int code) {
         case EP_ERR_ARG: return "invalid argument (null pointer, size, alignment or E % R != 0)";
         case EP_ERR_CUDA: return "CUDA runtime error (see ep_last_error)";
         case EP_ERR_UNSUPPORTED: return "sizes beyond this build's limits";
-        case EP_ERR_STATE: return "handle has no layout yet";
-        case EP_ERR_DEVICE: return "device reported an error (bad expert id or wait timeout)";
+        case EP_ERR_STATE: return "handle has no layout yet, or is of the other layout mode";
+        case EP_ERR_DEVICE: return "device reported an error (bad expert id, wait timeout or slot overflow)";
         default: return "unknown status";
     }
 }

@@ -67,6 +67,13 @@ struct DispatchParams {
     int n_zero_units;            // ceil(cap / kZeroRowsPerUnit) when A > 1, else 0
     int stages;                  // shared-memory ring depth (staged kernel)
     int groups;                  // consumer groups (staged kernel)
+    int scale_group_rows;        // column-major scales: rows per [H/128][scale_ld] group
+    // low-latency static layout (ll_M > 0): destinations computed in-kernel
+    // from topk_idx, e*ll_M + slot; no padding rows, no zero fill
+    int ll_M;                    // fixed slots per expert
+    const int64_t *topk_idx;     // [T, K]
+    int32_t *pos_out;            // [T, K] destination of every pair (-1: none)
+    int32_t *recv_count;         // [E] slots used per expert (NULL: not written)
 };
 
 struct CombineParams {
@@ -90,6 +97,8 @@ const void *layout_kernel_ptr();
 // instance they pick: min(units, resident blocks per SM x num_sms).
 cudaError_t launch_dispatch_bf16(const DispatchParams &p, int num_sms, cudaStream_t s);
 cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream_t s);
+// Low-latency static layout + copy in one launch (p.ll_M > 0).
+cudaError_t launch_ll_dispatch(const DispatchParams &p, bool fp8, int num_sms, cudaStream_t s);
 // Per device, before the first dispatch launch: kernel attributes (dynamic
 // shared memory of the staged kernel).
 cudaError_t dispatch_prepare();
@@ -316,6 +325,7 @@ struct ep_handle {
     bool has_layout;
     int sm_limit;                   // SMs dispatch / combine may occupy (0: all)
     int scale_layout;               // EP_SCALES_*
+    int ll_M;                       // > 0: low-latency handle with ll_M slots per expert
     unsigned int layout_epoch;      // layout launches since creation / ep_clear_status
     unsigned long long wait_limit_ns;
     int barrier_extra;

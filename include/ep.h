@@ -75,6 +75,7 @@ enum ep_error {
 /* Device status bits (sticky until ep_clear_status). */
 #define EP_DEV_BAD_EXPERT 0x1u   /* some topk_idx entry is outside [0, E) and not -1 */
 #define EP_DEV_WAIT_TIMEOUT 0x2u /* a bounded in-kernel wait gave up */
+#define EP_DEV_SLOT_OVERFLOW 0x4u /* low-latency: an expert was offered more pairs than its slots */
 
 /*
  * Problem sizes, fixed for the life of a handle.
@@ -238,6 +239,76 @@ EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, 
                                  int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
                                  uint8_t *is_token_in_rank, int32_t *expert_offsets, int32_t *rank_offsets,
                                  uint32_t *status, ep_stream_t stream);
+
+/*
+ * ---- Low-latency (static, masked) layout ----
+ * The decode-time mode of lesson14_deepep (hsthanb4.github.io) section 2(1)
+ * -- pre-allocated static buffers and a per-expert mask, no host
+ * involvement, CUDA-graph compatible -- and its section 3 listing
+ * (low_latency_dispatch returns received rows per expert plus counts that a
+ * masked grouped GEMM takes as its mask; low_latency_combine takes the expert
+ * outputs with topk_idx and topk_weights).  blog.hotdry.top (buffer
+ * section) advises num_max_dispatch_tokens_per_rank below 256.
+ *
+ * Every expert e owns M = num_max_dispatch_tokens fixed received rows
+ * e*M .. e*M+M-1 (capacity E*M rows).  Pair (t, k) with e = topk_idx[t,k]
+ * takes slot s = #{(t', k') before (t, k) in (token, k) order with the
+ * same expert}, i.e. row e*M + s, the same order as the normal layout.
+ * recv_count[e] = min(pairs of e, M) is the mask: slots at or past it are
+ * not written (no padding, no zero fill).  A pair past an expert's M-th
+ * slot is dropped (pos = -1) and sets EP_DEV_SLOT_OVERFLOW; with distinct
+ * experts per token and T <= M that cannot happen.  -1 ids are masked
+ * slots; other ids outside [0, E) set EP_DEV_BAD_EXPERT.  Layout and copy
+ * are one kernel launch with no grid-wide wait.
+ */
+
+/* E * M received rows for M slots per expert; negative ep_error if invalid. */
+EP_API int64_t ep_ll_capacity_rows(const ep_config *cfg, int32_t num_max_dispatch_tokens);
+
+/*
+ * Floats a low-latency recv_scales buffer needs: E*M*(H/128) for
+ * EP_SCALES_ROW_MAJOR; for EP_SCALES_COL_MAJOR_TMA each expert's scales are
+ * [H/128][round_up(M, 4)] (one TMA-aligned block per expert), E of them.
+ */
+EP_API int64_t ep_ll_scale_buffer_floats(const ep_config *cfg, int32_t num_max_dispatch_tokens, int32_t layout);
+
+/*
+ * Creates a low-latency handle: T = cfg->num_tokens tokens per call with
+ * T <= num_max_dispatch_tokens (else EP_ERR_ARG); cfg->expert_alignment is
+ * not used.  Owns pos [T, K] and the status word (one cudaMalloc).  Works
+ * with ep_ll_dispatch, ep_ll_dispatch_fp8, ep_ll_combine, ep_copy_routing
+ * (pos only), ep_get_status, ep_clear_status, ep_set_sm_limit,
+ * ep_set_scale_layout and ep_handle_get_view (pos, status, capacity); the
+ * normal-layout calls return EP_ERR_STATE on it, and ep_ll_* calls on a
+ * normal handle return EP_ERR_STATE.
+ */
+EP_API int ep_ll_handle_create(const ep_config *cfg, int32_t num_max_dispatch_tokens, ep_handle **out);
+
+/*
+ * Low-latency bf16 dispatch: slots from topk_idx [T, K] int64 as above,
+ * recv_x[e*M + s, :] = x[t, :]; recv_count [E] int32 (NULL: skip).  x is
+ * [T, H] bf16, recv_x [E*M, H] bf16 (16-byte aligned).  Also records pos in
+ * the handle for ep_ll_combine.  One kernel launch.
+ */
+EP_API int ep_ll_dispatch(ep_handle *h, const int64_t *topk_idx, const void *x, void *recv_x,
+                          int32_t *recv_count, ep_stream_t stream);
+
+/*
+ * Low-latency FP8 dispatch: the slots of ep_ll_dispatch with the
+ * quantisation of ep_dispatch_fp8.  recv_q [E*M, H] bytes; recv_scales in
+ * the handle's scale layout (ep_ll_scale_buffer_floats).  Needs H % 128 == 0.
+ */
+EP_API int ep_ll_dispatch_fp8(ep_handle *h, const int64_t *topk_idx, const void *x, void *recv_q,
+                              float *recv_scales, int32_t *recv_count, ep_stream_t stream);
+
+/*
+ * Low-latency combine: out[t, :] = bf16_rn(fp32 fma chain over k of
+ * topk_weights[t,k] * y[pos[t,k], :]) with the pos of the last
+ * ep_ll_dispatch on h; y is [E*M, H] bf16 (expert outputs in the slots),
+ * out [T, H] bf16.  Dropped and masked pairs add nothing.
+ */
+EP_API int ep_ll_combine(const ep_handle *h, const void *y, const float *topk_weights, void *out,
+                         ep_stream_t stream);
 
 /* Synchronises `stream` and returns rows (= expert_offsets[E]) on the host. */
 EP_API int ep_get_num_rows(const ep_handle *h, int32_t *rows, ep_stream_t stream);
