@@ -103,8 +103,16 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
 // ring, one consumer group per SM) measured slower (123 vs 80.7 us at the
 // DeepSeek-V3 shape): the fp32 accumulation needs the register kernel's
 // four resident blocks per SM.
-cudaError_t launch_combine(const CombineParams &p, int num_sms, cudaStream_t s) {
+cudaError_t launch_combine(const CombineParams &p_in, int num_sms, cudaStream_t s) {
     static int occ = 0;
+    CombineParams p = p_in;
+    // a small batch splits each row over several CTAs (at least half a
+    // block of vectors each) so that it still spreads over the SMs
+    const int nv = p.H * 2 / 16;
+    int sp = 1;
+    while (sp < 8 && p.T * sp < 2 * num_sms && nv / (sp * 2) >= kThreads / 2) sp *= 2;
+    p.splits = sp;
+    p.n_units = p.T * sp;
     const void *k = reinterpret_cast<const void *>(&combine_kernel<4>);
     const int grid = persistent_grid(p.n_units, blocks_per_sm(k, kThreads, 0, &occ), num_sms);
     combine_kernel<4><<<grid, kThreads, 0, s>>>(p);

@@ -175,19 +175,27 @@ __global__ void __launch_bounds__(kThreads, EP_LSU_MINB) dispatch_bf16_kernel(Di
     for (int u = blockIdx.x; u < total; u += nblk) {
         if (u < p.n_token_units) {
             const int t = u / p.splits, s = u - t * p.splits;
+            const int v0 = s * vps, v1 = min(nv, v0 + vps);
+            const uint8_t *xr = x + (int64_t)t * row_bytes;
+            // the first vectors of the row are loaded before the destinations
+            // are known, so the two memory round trips overlap
+            VT buf[kUnroll];
+            const int vfirst = v0 + threadIdx.x;
+#pragma unroll
+            for (int j = 0; j < kUnroll; ++j)
+                if (vfirst + j * kThreads < v1) buf[j] = V::load(xr + (int64_t)(vfirst + j * kThreads) * VB);
             if constexpr (LL) {
                 ll_destinations(p, st, t, s == 0, s_dst);
             } else {
                 if (threadIdx.x < p.K) s_dst[threadIdx.x] = __ldg(&p.pos[(int64_t)t * p.K + threadIdx.x]);
                 __syncthreads();
             }
-            const int v0 = s * vps, v1 = min(nv, v0 + vps);
-            const uint8_t *xr = x + (int64_t)t * row_bytes;
-            for (int v = v0 + threadIdx.x; v < v1; v += kThreads * kUnroll) {
-                VT buf[kUnroll];
+            for (int v = vfirst; v < v1; v += kThreads * kUnroll) {
+                if (v != vfirst) {
 #pragma unroll
-                for (int j = 0; j < kUnroll; ++j)
-                    if (v + j * kThreads < v1) buf[j] = V::load(xr + (int64_t)(v + j * kThreads) * VB);
+                    for (int j = 0; j < kUnroll; ++j)
+                        if (v + j * kThreads < v1) buf[j] = V::load(xr + (int64_t)(v + j * kThreads) * VB);
+                }
                 for (int k = 0; k < p.K; ++k) {
                     const int dst = s_dst[k];
                     if (dst < 0) continue;
@@ -497,22 +505,32 @@ __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p
     for (int u = blockIdx.x; u < total; u += nblk) {
         if (u < p.n_token_units) {
             const int t = u;
+            const uint8_t *xr = x + (int64_t)t * p.H * 2;
+            // the first part of the row is loaded before the destinations are
+            // known, so the two memory round trips overlap
+            unsigned int w[NW];
+            if (threadIdx.x < nthr_row) {
+                Fp8Io<EPT>::load(xr + (int64_t)threadIdx.x * EPT * 2, w);
+            } else {
+#pragma unroll
+                for (int i = 0; i < NW; ++i) w[i] = 0;
+            }
             if constexpr (LL) {
                 ll_destinations(p, st, t, true, s_dst);
             } else {
                 if (threadIdx.x < p.K) s_dst[threadIdx.x] = __ldg(&p.pos[(int64_t)t * p.K + threadIdx.x]);
                 __syncthreads();
             }
-            const uint8_t *xr = x + (int64_t)t * p.H * 2;
             for (int g0 = 0; g0 < nthr_row; g0 += kThreads) {
                 const int g = g0 + threadIdx.x;
                 const bool act = g < nthr_row;
-                unsigned int w[NW];
-                if (act) {
-                    Fp8Io<EPT>::load(xr + (int64_t)g * EPT * 2, w);
-                } else {
+                if (g0 > 0) {
+                    if (act) {
+                        Fp8Io<EPT>::load(xr + (int64_t)g * EPT * 2, w);
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < NW; ++i) w[i] = 0;
+                        for (int i = 0; i < NW; ++i) w[i] = 0;
+                    }
                 }
                 float amax = 0.0f;
 #pragma unroll

@@ -133,25 +133,20 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
 
     const int T = cfg->num_tokens, E = cfg->num_experts, R = cfg->num_ranks, K = cfg->num_topk;
 
-    // layout: about kLayoutPairsPerCta (token, k) pairs per CTA, all CTAs resident
-    h->layout_smem = ep::layout_smem_bytes(E, R);
-    // the attribute is per kernel, not per handle: allow the largest supported size
-    e = cudaFuncSetAttribute(ep::layout_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)ep::layout_smem_bytes(ep::kMaxExperts, ep::kMaxExperts));
-    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaFuncSetAttribute(layout)"));
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ep::layout_kernel_ptr(),
-                                                      ep::kLayoutThreads, h->layout_smem);
-    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor"));
-    if (per_sm < 1) return fail(EP_ERR_UNSUPPORTED);
-    const int64_t pairs = (int64_t)T * K;
-    int64_t G = (pairs + ep::kLayoutPairsPerCta - 1) / ep::kLayoutPairsPerCta;
-    G = G < 1 ? 1 : (G > h->num_sms ? h->num_sms : G);   // one CTA per SM at most
-    int tpc = T > 0 ? (int)((T + G - 1) / G) : 1;
-    G = T > 0 ? (T + tpc - 1) / tpc : 1;
-    h->G = (int)G;
-    h->tokens_per_chunk = tpc;
-
+    // layout launch shape (cluster kernel, or the cooperative fallback)
+    e = ep::layout_prepare(h->device);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "layout set-up"));
+    h->plan = ep::plan_layout(h->device, T, E, R, K, h->num_sms);
+    if (!h->plan.cluster) {
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ep::layout_kernel_ptr(), ep::kLayoutThreads,
+                                                          h->plan.smem);
+        if (e != cudaSuccess) return fail(cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor"));
+        if (per_sm < 1) return fail(EP_ERR_UNSUPPORTED);
+    }
+    const int64_t G = h->plan.G;
+    h->G = h->plan.G;
+    h->tokens_per_chunk = h->plan.tokens_per_chunk;
 
     e = ep::dispatch_prepare();
     if (e != cudaSuccess) return fail(cuda_fail(e, "cudaFuncSetAttribute(dispatch)"));
@@ -172,7 +167,8 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     const size_t o_rtok = take(sizeof(int32_t) * R);
     const size_t o_eoff = take(sizeof(int32_t) * (E + 1));
     const size_t o_roff = take(sizeof(int32_t) * (R + 1));
-    const size_t o_chunk = take(sizeof(int32_t) * (size_t)((G + 3) / 4 * 4) * (E + R));
+    // chunk histograms of the cooperative kernel (the cluster kernel needs none)
+    const size_t o_chunk = take(h->plan.cluster ? 0 : sizeof(int32_t) * (size_t)((G + 3) / 4 * 4) * (E + R));
     const size_t o_bar = take(sizeof(ep::GridBarrier));
     const size_t o_stat = take(sizeof(unsigned int));
     h->block_bytes = off;
@@ -276,7 +272,7 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
     p.status = h->status;
     p.wait_limit_ns = h->wait_limit_ns;
     p.barrier_extra = h->barrier_extra;
-    cudaError_t e = ep::launch_layout(p, h->layout_smem, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = ep::launch_layout(p, h->plan, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launch(layout)");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     h->has_layout = true;

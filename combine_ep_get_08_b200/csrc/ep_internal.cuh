@@ -89,8 +89,24 @@ struct CombineParams {
     int stages;                  // shared-memory ring depth (staged kernel)
 };
 
+// Layout launch shape: the cluster kernel (G CTAs in one thread-block
+// cluster, exchange through distributed shared memory) when a CTA can hold
+// its share of the pairs, else the cooperative kernel (G CTAs, one grid-wide
+// wait, chunk histograms in global scratch).
+struct LayoutPlan {
+    bool cluster;
+    int G;
+    int tokens_per_chunk;
+    size_t smem;
+};
+constexpr int kClusterPairsTarget = 2048;   // target (token, k) pairs per cluster CTA
+// Per device, before the first layout launch (kernel attributes, the
+// largest co-schedulable cluster).
+cudaError_t layout_prepare(int device);
+LayoutPlan plan_layout(int device, int T, int E, int R, int K, int num_sms);
+
 // launchers (return cudaError_t of the launch)
-cudaError_t launch_layout(const LayoutParams &p, size_t smem, cudaStream_t s);
+cudaError_t launch_layout(const LayoutParams &p, const LayoutPlan &plan, cudaStream_t s);
 size_t layout_smem_bytes(int E, int R);
 const void *layout_kernel_ptr();
 // Launchers size their persistent grid from the occupancy of the kernel
@@ -310,9 +326,9 @@ struct ep_handle {
     int num_sms;
     int64_t cap;
     // layout launch shape
+    ep::LayoutPlan plan;
     int G;
     int tokens_per_chunk;
-    size_t layout_smem;
     // one device allocation, carved
     void *block;
     size_t block_bytes;

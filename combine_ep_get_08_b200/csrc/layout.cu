@@ -12,6 +12,14 @@
 // (EPBuffer.dispatch arguments expert_alignment / do_zero_padding,
 // bowenzhou.top "deepep/01-overview" section 1.1).
 //
+// Two kernels compute the same result.  layout_cluster_kernel, used
+// whenever a CTA can hold its share (at most 8192 pairs per CTA, 16 CTAs),
+// is one thread-block cluster: every warp ranks a contiguous range of pairs
+// while it loads them, and the CTAs exchange their histograms through
+// distributed shared memory, so there is no global scratch and no polled
+// barrier.  layout_kernel, the fallback for larger batches, is a cooperative
+// grid:
+//
 // Phases, separated by one bounded grid-wide wait (none when G == 1):
 //   1. chunk histogram of experts (shared-memory atomics decide counts only)
 //      and of distinct tokens per rank; is_token_in_rank rows.  The
@@ -24,6 +32,8 @@
 //      with the same expert from ballots over the id bits, and a per-warp
 //      prefix table in shared memory orders the warps, so no atomic ever
 //      decides a position.
+#include <cooperative_groups.h>
+
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -99,6 +109,10 @@ __device__ bool grid_wait(const LayoutParams &p, int *s_flag) {
 }
 
 __device__ __forceinline__ bool valid_expert(int64_t e, int E) { return e >= 0 && e < E; }
+
+// Brings the line holding *p (an in-bounds address) into L2; no register result.
+__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" : : "l"(p)); }
+
 
 // Loads up to 8 consecutive expert ids of one token (all loads issued
 // before any is used); missing entries read as -1.
@@ -365,6 +379,315 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutParams 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Cluster layout.  CTA c of the cluster takes tokens
+// [c*tokens_per_chunk, (c+1)*tokens_per_chunk); inside it, warp w takes a
+// contiguous range of ppw pairs (a multiple of 32, at most
+// kClusterMaxSteps*32) and walks it 32 pairs at a time in (token, k) order.
+// Per step, each lane finds the lanes with the same expert from ballots over
+// the id bits; its rank inside the warp's range is the warp's running count
+// of that expert (a private shared-memory row) plus the peers below it.
+// The rows of counts then become exclusive prefixes over the warps, the CTA
+// histograms are read across the cluster (distributed shared memory) for
+// the totals and the pairs of earlier CTAs, and a pair's row is
+// offset + earlier CTAs + earlier warps + rank in warp.  A CTA's rows of one
+// expert are consecutive, so the row-indexed outputs are staged in shared
+// memory in the CTA's own row order and written out segment by segment:
+// the stores coalesce instead of scattering one sector per pair.
+// ---------------------------------------------------------------------------
+constexpr int kClusterMaxSteps = 4;
+constexpr int kClusterMaxPairs = kLayoutThreads * kClusterMaxSteps;   // pairs per CTA
+
+// Exclusive scans of a[0..n) and b[0..n) in shared memory, in place, in one
+// pass; returns both totals.  Caller must have synchronised after writing.
+__device__ int2 block_exclusive_scan2(int32_t *a, int32_t *b, int n, int32_t *s_tmp /*[2*(kLayoutWarps+1)]*/) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (n + kLayoutThreads - 1) / kLayoutThreads;
+    const int lo = min(n, tid * per), hi = min(n, lo + per);
+    int sa = 0, sb = 0;
+    for (int i = lo; i < hi; ++i) {
+        sa += a[i];
+        sb += b[i];
+    }
+    int ia = sa, ib = sb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int va = __shfl_up_sync(0xffffffffu, ia, o), vb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+            ia += va;
+            ib += vb;
+        }
+    }
+    int32_t *ta = s_tmp, *tb = s_tmp + (kLayoutWarps + 1);
+    if (lane == 31) {
+        ta[warp] = ia;
+        tb[warp] = ib;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int va = lane < kLayoutWarps ? ta[lane] : 0, vb = lane < kLayoutWarps ? tb[lane] : 0;
+        int xa = va, xb = vb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int ua = __shfl_up_sync(0xffffffffu, xa, o), ub = __shfl_up_sync(0xffffffffu, xb, o);
+            if (lane >= o) {
+                xa += ua;
+                xb += ub;
+            }
+        }
+        if (lane < kLayoutWarps) {
+            ta[lane] = xa - va;
+            tb[lane] = xb - vb;
+        }
+        if (lane == 31) {
+            ta[kLayoutWarps] = xa;
+            tb[kLayoutWarps] = xb;
+        }
+    }
+    __syncthreads();
+    int ra = ta[warp] + ia - sa, rb = tb[warp] + ib - sb;
+    for (int i = lo; i < hi; ++i) {
+        const int va = a[i], vb = b[i];
+        a[i] = ra;
+        b[i] = rb;
+        ra += va;
+        rb += vb;
+    }
+    const int2 tot = make_int2(ta[kLayoutWarps], tb[kLayoutWarps]);
+    __syncthreads();
+    return tot;
+}
+
+// Expert (low 16 bits, -1: none) of a pair's packed shared-memory entry.
+__device__ __forceinline__ int cl_expert(int er) { return (int)(short)(er & 0xffff); }
+
+__global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(LayoutParams p) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = (int)cluster.num_blocks();
+    const int c = (int)cluster.block_rank();
+    extern __shared__ int32_t smem[];
+    const int E = p.E, R = p.R, K = p.K, L = p.L;
+    const int ncols = E + R, ES = E + 1;            // ES: padded row stride (no bank conflicts)
+    int32_t *s_cnt = smem;                          // [kLayoutWarps][ES] per-warp counts, then prefixes
+    int32_t *s_hist = s_cnt + kLayoutWarps * ES;    // [E+R] this CTA's counts (read by the cluster)
+    int32_t *s_tot = s_hist + ncols;                // [E+R] cluster totals
+    int32_t *s_before = s_tot + ncols;              // [E]   pairs of expert e in earlier CTAs
+    int32_t *s_eoff = s_before + E;                 // [E+1] padded expert offsets
+    int32_t *s_loff = s_eoff + (E + 1);             // [E+1] this CTA's rows: exclusive offsets per expert
+    int32_t *s_er = s_loff + (E + 1);               // [steps][kLayoutThreads] pair: expert | rank << 16
+    int32_t *s_qe = s_er + kClusterMaxPairs;        // [pairs] in this CTA's row order: pair | expert << 16
+    __shared__ int32_t s_tmp[2 * (kLayoutWarps + 1)];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t_begin = min(p.T, c * p.tokens_per_chunk);
+    const int t_end = min(p.T, t_begin + p.tokens_per_chunk);
+    const int64_t p_begin = (int64_t)t_begin * K;
+    const int npairs = (int)((int64_t)t_end * K - p_begin);
+    const int ppw = (npairs + kLayoutThreads - 1) / kLayoutThreads * 32;   // pairs per warp
+    const int steps = ppw / 32;
+    const int w_lo = warp * ppw, w_hi = min(npairs, w_lo + ppw);          // this warp's local pairs
+
+    for (int i = tid; i < kLayoutWarps * ES; i += kLayoutThreads) s_cnt[i] = 0;
+    for (int i = tid; i < ncols; i += kLayoutThreads) s_hist[i] = 0;
+    // the weights are read in row order at the end: bring them into L2 now
+    if (p.topk_weights && tid * 32 < npairs) prefetch_l2(p.topk_weights + p_begin + tid * 32);
+    // every id of this warp's range is requested before any is used
+#pragma unroll
+    for (int j = 0; j < kClusterMaxSteps; ++j) {
+        if (j < steps) {
+            const int i = w_lo + j * 32 + lane;
+            int e = -1;
+            if (i < w_hi) {
+                const int64_t v = __ldg(p.topk_idx + p_begin + i);
+                e = valid_expert(v, E) ? (int)v : -1;
+                if (e < 0 && v != -1) atomicOr(p.status, EP_DEV_BAD_EXPERT);   // -1: masked slot
+            }
+            s_er[j * kLayoutThreads + tid] = e & 0xffff;
+        }
+    }
+    __syncthreads();
+    int32_t *wrow = s_cnt + warp * ES;
+#pragma unroll 1
+    for (int j = 0; j < steps; ++j) {
+        const int er = s_er[j * kLayoutThreads + tid];
+        const int e = cl_expert(er);
+        unsigned int peers = __ballot_sync(0xffffffffu, e >= 0);
+        if (e < 0) peers = ~peers;
+        for (int b = 0; b < p.id_bits; ++b) {
+            const int bit = (e >> b) & 1;
+            const unsigned int bal = __ballot_sync(0xffffffffu, bit);
+            peers &= bit ? bal : ~bal;
+        }
+        const int lrank = __popc(peers & lanemask_lt());
+        const int base = e >= 0 ? wrow[e] : 0;
+        __syncwarp();
+        if (e >= 0 && lrank == 0) wrow[e] = base + __popc(peers);
+        __syncwarp();
+        s_er[j * kLayoutThreads + tid] = er | ((base + lrank) << 16);
+    }
+    __syncthreads();
+
+    // exclusive prefix of each expert's counts over the warps; P lanes share
+    // one expert, each summing 32/P rows, with a shuffle scan across them
+    {
+        int P = 1;
+        while (P < 32 && 2 * P * E <= kLayoutThreads) P <<= 1;
+        const int e = tid / P, part = tid % P, rows = kLayoutWarps / P;
+        const bool act = e < E;
+        int local = 0;
+        if (act)
+            for (int w = part * rows; w < (part + 1) * rows; ++w) local += s_cnt[w * ES + e];
+        int incl = local;
+        for (int o = 1; o < P; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o, P);
+            if (part >= o) incl += v;
+        }
+        if (act) {
+            int run = incl - local;
+            for (int w = part * rows; w < (part + 1) * rows; ++w) {
+                const int v = s_cnt[w * ES + e];
+                s_cnt[w * ES + e] = run;
+                run += v;
+            }
+            if (part == P - 1) s_hist[e] = run;
+        }
+    }
+    // distinct tokens per rank and is_token_in_rank rows, from the staged ids
+    for (int t = t_begin + tid; t < t_end; t += kLayoutThreads) {
+        const int i0 = (t - t_begin) * K;
+        if (R <= 64) {
+            unsigned long long mask = 0;
+            for (int k = 0; k < K; ++k) {
+                const int i = i0 + k, w = i / ppw, r = i - w * ppw;
+                const int e = cl_expert(s_er[(r >> 5) * kLayoutThreads + w * 32 + (r & 31)]);
+                if (e >= 0) mask |= 1ull << (e / L);
+            }
+            for (unsigned long long m = mask; m; m &= m - 1) atomicAdd(&s_hist[E + __ffsll((long long)m) - 1], 1);
+            if (p.u_in_rank) {
+                uint8_t *dst = p.u_in_rank + (int64_t)t * R;
+                if ((R & 3) == 0 && ((reinterpret_cast<uintptr_t>(dst) & 3) == 0)) {
+                    for (int r = 0; r < R; r += 4) {
+                        const unsigned int bits = (unsigned int)(mask >> r) & 0xfu;
+                        const unsigned int word = (bits & 1u) | ((bits >> 1) & 1u) << 8 |
+                                                  ((bits >> 2) & 1u) << 16 | ((bits >> 3) & 1u) << 24;
+                        *reinterpret_cast<unsigned int *>(dst + r) = word;
+                    }
+                } else {
+                    for (int r = 0; r < R; ++r) dst[r] = (uint8_t)((mask >> r) & 1ull);
+                }
+            }
+        } else {
+            // more than 64 ranks: distinct ranks by pairwise comparison
+            uint8_t *dst = p.u_in_rank ? p.u_in_rank + (int64_t)t * R : nullptr;
+            if (dst)
+                for (int r = 0; r < R; ++r) dst[r] = 0;
+            for (int k = 0; k < K; ++k) {
+                const int i = i0 + k, w = i / ppw, rr = i - w * ppw;
+                const int e = cl_expert(s_er[(rr >> 5) * kLayoutThreads + w * 32 + (rr & 31)]);
+                if (e < 0) continue;
+                const int r = e / L;
+                bool dup = false;
+                for (int k2 = 0; k2 < k; ++k2) {
+                    const int i2 = i0 + k2, w2 = i2 / ppw, r2 = i2 - w2 * ppw;
+                    const int e2 = cl_expert(s_er[(r2 >> 5) * kLayoutThreads + w2 * 32 + (r2 & 31)]);
+                    if (e2 >= 0 && e2 / L == r) dup = true;
+                }
+                if (!dup) atomicAdd(&s_hist[E + r], 1);
+                if (dst) dst[r] = 1;
+            }
+        }
+    }
+    // every CTA's histogram complete and visible to the cluster
+    cluster.sync();
+    for (int j = tid; j < ncols; j += kLayoutThreads) {
+        int tot = 0, before = 0;
+        for (int cc = 0; cc < C; ++cc) {
+            const int v = *cluster.map_shared_rank(s_hist + j, cc);
+            tot += v;
+            before += cc < c ? v : 0;
+        }
+        s_tot[j] = tot;
+        if (j < E) s_before[j] = before;
+    }
+    // this CTA is done reading the others' shared memory; it must not exit
+    // before they are done reading its own (waited for at the end)
+    cluster.barrier_arrive();
+    __syncthreads();
+    for (int e = tid; e < E; e += kLayoutThreads) {
+        s_eoff[e] = (s_tot[e] + p.A - 1) / p.A * p.A;
+        s_loff[e] = s_hist[e];
+    }
+    __syncthreads();
+    const int2 totals = block_exclusive_scan2(s_eoff, s_loff, E, s_tmp);
+    if (tid == 0) {
+        s_eoff[E] = totals.x;
+        s_loff[E] = totals.y;
+    }
+    __syncthreads();
+
+    // pos in pair order; each pair's entry staged at its row in this CTA's order
+#pragma unroll 1
+    for (int j = 0; j < steps; ++j) {
+        const int i = w_lo + j * 32 + lane;
+        if (i < w_hi) {
+            const int er = s_er[j * kLayoutThreads + tid];
+            const int e = cl_expert(er);
+            if (e >= 0) {
+                const int within = wrow[e] + (er >> 16);   // rank among this CTA's pairs of e
+                p.pos[p_begin + i] = s_eoff[e] + s_before[e] + within;
+                s_qe[s_loff[e] + within] = i | (e << 16);
+            } else {
+                p.pos[p_begin + i] = -1;
+            }
+        }
+    }
+    __syncthreads();
+    for (int lr = tid; lr < s_loff[E]; lr += kLayoutThreads) {
+        const int qe = s_qe[lr];
+        const int i = qe & 0xffff, e = qe >> 16;
+        const int dst = s_eoff[e] + s_before[e] + (lr - s_loff[e]);
+        const int64_t q = p_begin + i;
+        const int t = (int)(q / K);
+        p.row_src[dst] = t;
+        p.row_slot[dst] = (int)(q - (int64_t)t * K);
+        if (p.topk_weights) p.row_weight[dst] = __ldg(p.topk_weights + q);
+    }
+    if (c == 0) {
+        for (int e = tid; e < E; e += kLayoutThreads) {
+            p.cnt[e] = s_tot[e];
+            if (p.u_cnt) p.u_cnt[e] = s_tot[e];
+        }
+        for (int r = tid; r < R; r += kLayoutThreads) {
+            p.rank_tok[r] = s_tot[E + r];
+            if (p.u_rank_tok) p.u_rank_tok[r] = s_tot[E + r];
+        }
+        for (int e = tid; e <= E; e += kLayoutThreads) {
+            p.eoff[e] = s_eoff[e];
+            if (p.u_eoff) p.u_eoff[e] = s_eoff[e];
+        }
+        for (int r = tid; r <= R; r += kLayoutThreads) {
+            p.roff[r] = s_eoff[r * L];
+            if (p.u_roff) p.u_roff[r] = s_eoff[r * L];
+        }
+    }
+    // padding rows of experts c, c+C, ..., one expert per thread
+    for (int e = c + C * tid; e < E; e += C * kLayoutThreads) {
+        const int r0 = s_eoff[e] + s_tot[e], r1 = s_eoff[e + 1];
+        for (int r = r0; r < r1; ++r) {
+            p.row_src[r] = -1;
+            p.row_slot[r] = -1;
+            if (p.topk_weights) p.row_weight[r] = 0.0f;
+        }
+    }
+    cluster.barrier_wait();
+}
+
+size_t cluster_smem_bytes(int E, int R) {
+    return sizeof(int32_t) * ((size_t)kLayoutWarps * (E + 1) + 2 * (size_t)(E + R) + E + 2 * (size_t)(E + 1) +
+                              2 * (size_t)kClusterMaxPairs);
+}
+
 }  // namespace
 
 size_t layout_smem_bytes(int E, int R) {
@@ -373,15 +696,103 @@ size_t layout_smem_bytes(int E, int R) {
 
 const void *layout_kernel_ptr() { return reinterpret_cast<const void *>(&layout_kernel); }
 
-cudaError_t launch_layout(const LayoutParams &p, size_t smem, cudaStream_t s) {
+// Per device, once: kernel attributes (dynamic shared memory for the
+// largest supported E and R, clusters of 16) and the largest cluster size
+// that can be resident with one 1024-thread CTA per SM.
+static int g_max_cluster[64];
+
+cudaError_t layout_prepare(int device) {
+    if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+    if (__atomic_load_n(&g_max_cluster[device], __ATOMIC_ACQUIRE) > 0) return cudaSuccess;
+    const void *coop = reinterpret_cast<const void *>(&layout_kernel);
+    const void *clus = reinterpret_cast<const void *>(&layout_cluster_kernel);
+    cudaError_t e = cudaFuncSetAttribute(coop, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)layout_smem_bytes(kMaxExperts, kMaxExperts));
+    if (e != cudaSuccess) return e;
+    const size_t csmem = cluster_smem_bytes(kMaxExperts, kMaxExperts);
+    e = cudaFuncSetAttribute(clus, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);
+    if (e != cudaSuccess) return e;
+    int best = 1;
+    if (cudaFuncSetAttribute(clus, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+        for (int cs = 16; cs >= 2 && best == 1; cs /= 2) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(cs);
+            cfg.blockDim = dim3(kLayoutThreads);
+            cfg.dynamicSmemBytes = csmem;
+            cudaLaunchAttribute attr;
+            attr.id = cudaLaunchAttributeClusterDimension;
+            attr.val.clusterDim.x = cs;
+            attr.val.clusterDim.y = 1;
+            attr.val.clusterDim.z = 1;
+            cfg.attrs = &attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, clus, &cfg) == cudaSuccess && n >= 1) best = cs;
+        }
+    }
+    cudaGetLastError();   // a refused size query leaves no sticky error behind
+    __atomic_store_n(&g_max_cluster[device], best, __ATOMIC_RELEASE);
+    return cudaSuccess;
+}
+
+LayoutPlan plan_layout(int device, int T, int E, int R, int K, int num_sms) {
+    LayoutPlan pl{};
+    const int64_t pairs = (int64_t)T * K;
+    const int cmax = (device >= 0 && device < 64) ? __atomic_load_n(&g_max_cluster[device], __ATOMIC_ACQUIRE) : 0;
+    if (cmax >= 1) {
+        // about kClusterPairsTarget pairs per CTA, at most kClusterMaxPairs
+        int C = (int)((pairs + kClusterPairsTarget - 1) / kClusterPairsTarget);
+        C = C < 1 ? 1 : C;
+        while (C < cmax && (int64_t)((T + C - 1) / C) * K > kClusterMaxPairs) ++C;
+        if (C > cmax) C = cmax;
+        // cluster sizes that are powers of two schedule best; round up
+        int Cp = 1;
+        while (Cp < C) Cp <<= 1;
+        if (Cp <= cmax) C = Cp;
+        const int tpc = T > 0 ? (T + C - 1) / C : 1;
+        if ((int64_t)tpc * K <= kClusterMaxPairs) {
+            pl.cluster = true;
+            pl.G = C;
+            pl.tokens_per_chunk = tpc;
+            pl.smem = cluster_smem_bytes(E, R);
+            return pl;
+        }
+    }
+    int64_t G = (pairs + kLayoutPairsPerCta - 1) / kLayoutPairsPerCta;
+    G = G < 1 ? 1 : (G > num_sms ? num_sms : G);   // one CTA per SM at most
+    const int tpc = T > 0 ? (int)((T + G - 1) / G) : 1;
+    G = T > 0 ? (T + tpc - 1) / tpc : 1;
+    pl.cluster = false;
+    pl.G = (int)G;
+    pl.tokens_per_chunk = tpc;
+    pl.smem = layout_smem_bytes(E, R);
+    return pl;
+}
+
+cudaError_t launch_layout(const LayoutParams &p, const LayoutPlan &pl, cudaStream_t s) {
+    if (pl.cluster) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(pl.G);
+        cfg.blockDim = dim3(kLayoutThreads);
+        cfg.dynamicSmemBytes = pl.smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = pl.G;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, layout_cluster_kernel, p);
+    }
     if (p.G == 1) {   // a single CTA never waits on another: plain launch
-        layout_kernel<<<1, kLayoutThreads, smem, s>>>(p);
+        layout_kernel<<<1, kLayoutThreads, pl.smem, s>>>(p);
         return cudaGetLastError();
     }
     LayoutParams args = p;
     void *kargs[] = {&args};
     return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(&layout_kernel), dim3(p.G),
-                                       dim3(kLayoutThreads), kargs, smem, s);
+                                       dim3(kLayoutThreads), kargs, pl.smem, s);
 }
 
 }  // namespace ep

@@ -45,8 +45,7 @@ int setup_device(int dev, DeviceSetup *out) {
         void *ptr = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&ptr, g_layout_scratch);
         if (e != cudaSuccess) return ep::record_cuda_error(e, "cudaGetSymbolAddress(layout scratch)");
-        e = cudaFuncSetAttribute(ep::layout_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)ep::layout_smem_bytes(ep::kMaxExperts, ep::kMaxExperts));
+        e = ep::layout_prepare(dev);
         if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return ep::record_cuda_error(e, "layout set-up");
         s.scratch = static_cast<unsigned char *>(ptr);
@@ -90,14 +89,13 @@ EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, 
     rc = setup_device(dev, &s);
     if (rc != EP_OK) return rc;
 
-    // same launch shape as a handle's layout: ~1024 pairs per CTA, at most one CTA per SM
-    const int64_t pairs = (int64_t)T * K;
-    int64_t G = (pairs + ep::kLayoutPairsPerCta - 1) / ep::kLayoutPairsPerCta;
-    G = G < 1 ? 1 : (G > s.num_sms ? s.num_sms : G);
-    const int tpc = T > 0 ? (int)((T + G - 1) / G) : 1;
-    G = T > 0 ? (T + tpc - 1) / tpc : 1;
+    // same launch shape as a handle's layout; only the cooperative fallback
+    // uses the scratch array
+    const ep::LayoutPlan plan = ep::plan_layout(dev, T, E, R, K, s.num_sms);
+    const int64_t G = plan.G;
+    const int tpc = plan.tokens_per_chunk;
     const int G_stride = (int)((G + 3) / 4 * 4);
-    const size_t need = kCountsOffset + sizeof(int32_t) * (size_t)G_stride * (E + R);
+    const size_t need = plan.cluster ? 0 : kCountsOffset + sizeof(int32_t) * (size_t)G_stride * (E + R);
     if (need > kScratchBytes) {
         char msg[160];
         snprintf(msg, sizeof msg, "ep_get_layout_noalloc: %zu bytes of scratch needed, the fixed array holds %zu",
@@ -109,7 +107,7 @@ EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // the array keeps the previous call's contents: the arrival counter and
     // the histogram rows (whose tail past G is read as zeros) start at zero
-    e = cudaMemsetAsync(s.scratch, 0, need, st);
+    e = need ? cudaMemsetAsync(s.scratch, 0, need, st) : cudaSuccess;
     if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, sizeof(uint32_t), st);
     if (e != cudaSuccess) return ep::record_cuda_error(e, "cudaMemsetAsync(layout scratch)");
 
@@ -142,7 +140,7 @@ EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, 
     p.status = status;
     p.wait_limit_ns = ep::kDefaultWaitLimitNs;
     p.barrier_extra = 0;
-    e = ep::launch_layout(p, ep::layout_smem_bytes(E, R), st);
+    e = ep::launch_layout(p, plan, st);
     if (e != cudaSuccess) return ep::record_cuda_error(e, "launch(layout)");
     ep::count_launch();
     return EP_OK;

@@ -155,8 +155,11 @@ EP_API int ep_handle_get_view(const ep_handle *h, ep_handle_view *out);
  *   num_tokens_per_expert [E] int32, num_tokens_per_rank [R] int32,
  *   is_token_in_rank [T, R] uint8 (0/1), expert_offsets [E+1] int32,
  *   rank_offsets [R+1] int32.
- * topk_idx/topk_weights need 8/4-byte alignment only.  One cooperative
- * kernel launch; its grid-wide waits are bounded (EP_DEV_WAIT_TIMEOUT).
+ * topk_idx/topk_weights need 8/4-byte alignment only.  One kernel launch:
+ * a thread-block cluster of up to 16 CTAs (at most 8192 pairs each) that
+ * exchanges its histograms in distributed shared memory, or, for larger
+ * batches, a cooperative grid whose one grid-wide wait is bounded
+ * (EP_DEV_WAIT_TIMEOUT).
  * An id of -1 marks an unused top-k slot (the token selects fewer than K
  * experts): that pair gets pos = -1, no row, is not counted and adds
  * nothing in combine.  Any other id outside [0, E) also gets pos = -1 and
@@ -222,11 +225,12 @@ EP_API int ep_copy_routing(const ep_handle *h, int32_t *pos, int32_t *row_src, i
  *   (all required, 4-byte aligned); is_token_in_rank [T, R] (optional);
  *   status: one device uint32, set to 0 and then to the EP_DEV_* bits of this
  *   call (read it after the stream has reached it).
- * The kernel's scratch lives in a fixed 256 KiB array in the library's
- * device code, held on every GPU that loads the library until exit.  A
- * problem whose layout needs more (E + R columns of ceil(G/4)*4 int32, G
- * layout CTAs ~ T*K/1024 up to the SM count, plus 256 bytes) is rejected with
- * EP_ERR_UNSUPPORTED and a message in ep_last_error.
+ * A batch that fits one thread-block cluster (see ep_get_layout) needs no
+ * scratch.  A larger one runs the cooperative kernel, whose scratch lives in
+ * a fixed 256 KiB array in the library's device code, held on every GPU that
+ * loads the library until exit; one that needs more (E + R columns of
+ * ceil(G/4)*4 int32, G layout CTAs ~ T*K/1024 up to the SM count, plus 256
+ * bytes) is rejected with EP_ERR_UNSUPPORTED and a message in ep_last_error.
  * The first call on a device does a one-time set-up on the host (it looks up
  * the array's device address and sets a kernel attribute): make that first
  * call before any stream capture.  Every call shares the one array and
@@ -341,8 +345,8 @@ EP_API int ep_set_scale_layout(ep_handle *h, int32_t layout);
  * DeepEP's num_sms argument (bowenzhou.top "deepep/01-overview" section 1.1;
  * "blog.hotdry.top ... deepep-expert-parallel-alltoall": 24 SMs by default;
  * "lesson14_deepep" section 1(2): 20 communication SMs beside 110 compute
- * SMs).  The layout kernel is not capped (it uses at most one CTA per 1024
- * pairs).  Results do not depend on the cap.
+ * SMs).  The layout kernel is not capped (it uses at most 16 CTAs, or one
+ * CTA per 1024 pairs beyond that).  Results do not depend on the cap.
  */
 EP_API int ep_set_sm_limit(ep_handle *h, int32_t num_sms);
 

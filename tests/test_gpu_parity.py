@@ -92,6 +92,8 @@ SMALL = [
     dict(T=33, H=128, E=1024, R=128, K=64, A=2, router="topk", seed=24),      # max E, max K, R > 64
     dict(T=1, H=8, E=1, R=1, K=1, A=1, router="topk", seed=25),
     dict(T=300, H=1024, E=8, R=2, K=8, A=300, router="topk", seed=26),      # A > T*K/E
+    dict(T=20000, H=64, E=64, R=8, K=8, A=4, router="topk", seed=27),        # beyond one cluster: cooperative
+    dict(T=16384, H=64, E=256, R=64, K=8, A=2, router="group", seed=28),     # 16-CTA cluster, 8192 pairs each
 ]
 
 
@@ -213,9 +215,11 @@ def test_invalid_expert_id_sets_status():
 
 def test_bounded_wait_gives_up():
     """A grid-wide wait that can never complete ends after its limit with
-    EP_DEV_WAIT_TIMEOUT; after ep_clear_status the handle works again."""
+    EP_DEV_WAIT_TIMEOUT; after ep_clear_status the handle works again.
+    160 000 pairs exceed one cluster (16 CTAs x 8192 pairs), so the layout
+    takes the cooperative kernel, the one with a grid-wide wait."""
     dev = torch.device("cuda")
-    wl = workloads.generate(None, T=4096, H=256, E=256, R=8, K=8, A=1, router="topk", seed=5)
+    wl = workloads.generate(None, T=20000, H=64, E=64, R=8, K=8, A=1, router="topk", seed=5)
     cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
     h = ep.ep_handle_create(cfg)
     try:

@@ -86,9 +86,11 @@ def assert_same(na, g):
 
 def test_matches_handle_layout_calls_in_a_row():
     shapes = [
-        workloads.generate("dsv3", with_x=False),                       # 32 layout CTAs
-        workloads.generate(None, T=700, H=256, E=64, R=8, K=6, A=5,     # 5 CTAs: histogram rows padded
+        workloads.generate("dsv3", with_x=False),                       # an 8-CTA cluster
+        workloads.generate(None, T=700, H=256, E=64, R=8, K=6, A=5,
                            router="topk", seed=77, with_x=False),
+        workloads.generate(None, T=20000, H=64, E=64, R=8, K=8, A=3,    # beyond one cluster: the
+                           router="topk", seed=78, with_x=False),       # cooperative kernel and its scratch
         workloads.generate("skew", with_x=False),                        # expert_alignment 128
         workloads.generate("decode", with_x=False),                      # one CTA, no grid-wide wait
         workloads.generate("dsv3", seed=11, with_x=False),               # back to the first shape
@@ -108,9 +110,10 @@ def test_same_call_twice():
 
 def test_rejects_sizes_beyond_the_array():
     dev = torch.device("cuda")
-    cfg = ep.make_config(16384, 256, 1024, 1024, 8, 1)     # 2048 columns x 128 CTAs: about 1 MiB
-    idx = torch.zeros((16384, 8), dtype=torch.int64, device=dev)
-    t = torch.zeros(16384 * 8 + 4096, dtype=torch.int32, device=dev)
+    # 160 000 pairs need the cooperative kernel: 2048 columns x 148 CTAs, about 1.2 MiB of scratch
+    cfg = ep.make_config(20000, 256, 1024, 1024, 8, 1)
+    idx = torch.zeros((20000, 8), dtype=torch.int64, device=dev)
+    t = torch.zeros(20000 * 8 + 4096, dtype=torch.int32, device=dev)
     with pytest.raises(ep.EpError) as ei:
         ep.ep_get_layout_noalloc(cfg, idx, None, t, t, t, None, t, t, None, t, t, t)
     assert ei.value.code == ep.EP_ERR_UNSUPPORTED
