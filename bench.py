@@ -438,7 +438,9 @@ def run_cuda(args, world, rank, local):
     barrier(world)
     launches = ep.ep_launch_count() - launches0
 
-    lay_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    # the low-latency mode has no layout launch (it is fused into the dispatch):
+    # the empty event pair around it would only add the events' own overhead
+    lay_ms = [0.0 if ll else e[0].elapsed_time(e[1]) for e in evs]
     dis_ms = [e[1].elapsed_time(e[2]) for e in evs]
     com_ms = [e[3].elapsed_time(e[4]) for e in evs]
     # with reuse > 1 only the first dispatch/combine pair of a step carries events;
@@ -552,6 +554,61 @@ def run_e2e(path, args, stream, reuse, world, dev, bytes_step):
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+def ncu_ingest(rep: str, workload: str) -> int:
+    """Record DRAM bytes per launch of the layout / dispatch / combine kernels
+    from an ncu report (``ncu -i REP --page raw --csv``; per kernel the mean
+    over its captured launches) into profiles/ncu_traffic.json under
+    `workload`, stamped with the digest of the current kernel sources.
+    Entries taken on other sources are dropped."""
+    import csv
+    import io
+    import subprocess
+
+    raw = subprocess.run(["ncu", "-i", rep, "--page", "raw", "--csv"], check=True,
+                         capture_output=True, text=True).stdout
+    rows = list(csv.reader(io.StringIO(raw)))
+    hdr = rows[0]
+    col = {k: hdr.index(k) for k in ("Kernel Name", "dram__bytes_read.sum", "dram__bytes_write.sum")}
+    unit = rows[1]
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    per_role = {}
+    for r in rows[2:]:
+        name = r[col["Kernel Name"]]
+        role = ("layout" if "layout" in name else "dispatch" if "dispatch" in name
+                else "combine" if "combine" in name else None)
+        if role is None:
+            continue
+        rd = float(r[col["dram__bytes_read.sum"]].replace(",", "")) * scale[unit[col["dram__bytes_read.sum"]]]
+        wr = float(r[col["dram__bytes_write.sum"]].replace(",", "")) * scale[unit[col["dram__bytes_write.sum"]]]
+        short = name.split("(")[0].replace("void ", "").split("::")[-1]
+        per_role.setdefault(role, {"kernel": short, "n": 0, "rd": 0.0, "wr": 0.0})
+        e = per_role[role]
+        e["n"] += 1
+        e["rd"] += rd
+        e["wr"] += wr
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    digest = kernel_source_digest()
+    try:
+        with open(path) as f:
+            data = json.load(f)
+    except Exception:  # noqa: BLE001
+        data = {}
+    if data.get("source_digest") != digest:
+        data = {"source_digest": digest, "roles": {}}
+    data["how"] = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none on the "
+                   "bench command; caches are flushed between replays; mean over the captured launches")
+    data.setdefault("roles", {})[workload] = {
+        role: {"kernel": e["kernel"], "launches": e["n"], "dram_bytes_read": round(e["rd"] / e["n"]),
+               "dram_bytes_write": round(e["wr"] / e["n"]),
+               "dram_bytes_per_launch": round((e["rd"] + e["wr"]) / e["n"])}
+        for role, e in per_role.items()}
+    with open(path, "w") as f:
+        json.dump(data, f, indent=1)
+        f.write("\n")
+    print(json.dumps(data["roles"][workload], indent=1))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -567,7 +624,10 @@ def main(argv=None):
     ap.add_argument("--mode", choices=["normal", "ll"], default="normal",
                     help="layout: normal (padded, ep_get_layout) or low-latency static slots (ep_ll_*)")
     ap.add_argument("--ll-slots", type=int, default=0, help="slots per expert in --mode ll (0: T)")
+    ap.add_argument("--ncu-ingest", metavar="REP", help="record DRAM traffic from an ncu report and exit")
     args = ap.parse_args(argv)
+    if args.ncu_ingest:
+        return ncu_ingest(args.ncu_ingest, args.config + ("-ll" if args.mode == "ll" else ""))
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_env()

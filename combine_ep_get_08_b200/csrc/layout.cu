@@ -313,10 +313,11 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutParams 
             if (p.u_roff) p.u_roff[r] = s_eoff[r * L];
         }
     }
-    // padding rows of experts c, c+G, ..., one expert per thread
-    for (int e = c + G * tid; e < E; e += G * kLayoutThreads) {
+    // padding rows of experts c, c+G, ...: one warp per expert, its lanes
+    // over consecutive rows
+    for (int e = c + G * warp; e < E; e += G * kLayoutWarps) {
         const int r0 = s_eoff[e] + s_hist[e], r1 = s_eoff[e + 1];
-        for (int r = r0; r < r1; ++r) {
+        for (int r = r0 + (tid & 31); r < r1; r += 32) {
             p.row_src[r] = -1;
             p.row_slot[r] = -1;
             if (p.topk_weights) p.row_weight[r] = 0.0f;
@@ -671,10 +672,11 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
             if (p.u_roff) p.u_roff[r] = s_eoff[r * L];
         }
     }
-    // padding rows of experts c, c+C, ..., one expert per thread
-    for (int e = c + C * tid; e < E; e += C * kLayoutThreads) {
+    // padding rows of experts c, c+C, ...: one warp per expert, its lanes
+    // over consecutive rows
+    for (int e = c + C * warp; e < E; e += C * kLayoutWarps) {
         const int r0 = s_eoff[e] + s_tot[e], r1 = s_eoff[e + 1];
-        for (int r = r0; r < r1; ++r) {
+        for (int r = r0 + lane; r < r1; r += 32) {
             p.row_src[r] = -1;
             p.row_slot[r] = -1;
             if (p.topk_weights) p.row_weight[r] = 0.0f;
