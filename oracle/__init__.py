@@ -62,6 +62,8 @@ def _bind(lib):
     lib.oracle_dispatch_bf16.restype = ctypes.c_int
     lib.oracle_dispatch_fp8.argtypes = [i32, i32, i32, P, P, P, P, P]
     lib.oracle_dispatch_fp8.restype = ctypes.c_int
+    lib.oracle_expert_combine.argtypes = [i32] * 6 + [P] * 5 + [i32, P, P]
+    lib.oracle_expert_combine.restype = ctypes.c_int
     lib.oracle_combine.argtypes = [i32, i32, i32, i32, P, P, P, i32, P, P]
     lib.oracle_combine.restype = ctypes.c_int
     return lib
@@ -241,3 +243,25 @@ def combine(y_bits, pos, topk_weights, sel_tokens=None) -> np.ndarray:
     if rc != OK:
         raise ValueError(f"oracle_combine failed ({rc})")
     return out
+
+
+def expert_combine(act_bits, w_bits, topk_idx, pos, topk_weights, sel_tokens=None) -> np.ndarray:
+    """fp64 out[t] = sum_k w[t,k] * act[pos[t,k]] @ W[topk_idx[t,k]]^T (see ep_oracle.c)."""
+    act = _c(act_bits, np.uint16)
+    rows, I = act.shape
+    w = _c(w_bits, np.uint16)
+    E, N, I2 = w.shape
+    assert I2 == I
+    idx = _c(topk_idx, np.int64)
+    p = _c(pos, np.int32)
+    T, K = p.shape
+    tw = _c(topk_weights, np.float32)
+    sel = None if sel_tokens is None else _c(sel_tokens, np.int32)
+    n = T if sel is None else sel.shape[0]
+    out = np.empty((n, N), np.float64)
+    rc = _load().oracle_expert_combine(T, K, I, N, E, rows, _ptr(idx), _ptr(p), _ptr(act), _ptr(w), _ptr(tw),
+                                       n, _ptr(sel), _ptr(out))
+    if rc != OK:
+        raise ValueError(f"oracle_expert_combine failed ({rc})")
+    return out
+

@@ -333,3 +333,51 @@ int oracle_combine(int32_t T, int32_t H, int32_t K, int32_t rows, const int32_t 
     }
     return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* Expert GEMM followed by combine                                      */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The expert computation that sits between dispatch and combine, for a
+ * linear expert map, with combine applied to its output ("lesson14_deepep"
+ * practice task: each expert transforms the rows it received, then
+ * moe_combine adds weight * expert_output back into the token's row).
+ *
+ * act [rows, I] bf16 bits: the expert inputs in the received-row layout
+ * (row pos[t,k] belongs to pair (t,k)); w [E, N, I] bf16 bits: expert e's
+ * matrix, row n holding the weights of output feature n; topk_w [T, K] fp32.
+ * For each selected token t (all if sel_tokens is NULL):
+ *   out[t, n] = sum_k topk_w[t,k] * sum_i act[pos[t,k], i] * w[e, n, i],
+ *   e = topk_idx[t,k], in fp64; pairs with e == -1 (or pos == -1) add nothing.
+ */
+int oracle_expert_combine(int32_t T, int32_t K, int32_t I, int32_t N, int32_t E, int32_t rows,
+                          const int64_t *topk_idx, const int32_t *pos, const uint16_t *act,
+                          const uint16_t *w, const float *topk_w, int32_t n_sel,
+                          const int32_t *sel_tokens, double *out)
+{
+    if (T < 0 || K <= 0 || I <= 0 || N <= 0 || E <= 0 || rows < 0) return ORACLE_BAD_ARG;
+    for (int32_t j = 0; j < n_sel; ++j) {
+        int32_t t = sel_tokens ? sel_tokens[j] : j;
+        if (t < 0 || t >= T) return ORACLE_BAD_ARG;
+        double *o = out + (int64_t)j * N;
+        for (int32_t n = 0; n < N; ++n) o[n] = 0.0;
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t e = topk_idx[(int64_t)t * K + k];
+            int32_t r = pos[(int64_t)t * K + k];
+            if (e == -1 || r == -1) continue;
+            if (e < 0 || e >= E || r < 0 || r >= rows) return ORACLE_BAD_ARG;
+            const uint16_t *a = act + (int64_t)r * I;
+            const uint16_t *we = w + (int64_t)e * N * I;
+            double wk = (double)topk_w[(int64_t)t * K + k];
+            for (int32_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int32_t i = 0; i < I; ++i)
+                    acc += (double)bf16_bits_to_float(a[i]) * (double)bf16_bits_to_float(we[(int64_t)n * I + i]);
+                o[n] += wk * acc;
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+

@@ -13,6 +13,7 @@ import pytest
 
 import oracle
 import test_oracle_dispatch_combine as tdc
+import test_oracle_expert_combine as tec
 import test_oracle_fp8 as tf8
 import test_oracle_layout as tlay
 import test_oracle_ll as tll
@@ -43,7 +44,8 @@ MUTANTS = {
     "combine uses weight of k=0": (
         "double wk = (double)w[(int64_t)t * K + k];", "double wk = (double)w[(int64_t)t * K];"),
     "combine reads row of k=0": (
-        "int32_t r = pos[(int64_t)t * K + k];", "int32_t r = pos[(int64_t)t * K];"),
+        "int32_t r = pos[(int64_t)t * K + k];\n            if (r == -1) continue;",
+        "int32_t r = pos[(int64_t)t * K];\n            if (r == -1) continue;"),
     "combine drops the last k": ("for (int32_t k = 0; k < K; ++k) {\n            int32_t r = pos",
                                  "for (int32_t k = 0; k < K - 1; ++k) {\n            int32_t r = pos"),
     "dispatch copies the previous token": (
@@ -56,6 +58,12 @@ MUTANTS = {
     "low-latency masked slot counted": (
         "if (e < 0) { pos[i] = -1; continue; }              /* masked slot */",
         "if (e < 0) { pos[i] = -1; recv_count[0] += 1; continue; }"),
+    "expert matrix transposed": ("* (double)bf16_bits_to_float(we[(int64_t)n * I + i]);",
+                                 "* (double)bf16_bits_to_float(we[(int64_t)i * N + n]);"),
+    "expert taken from k = 0": ("int64_t e = topk_idx[(int64_t)t * K + k];\n            int32_t r = pos[",
+                                "int64_t e = topk_idx[(int64_t)t * K];\n            int32_t r = pos["),
+    "gemm weight of the wrong slot": ("double wk = (double)topk_w[(int64_t)t * K + k];\n            for (int32_t n",
+                                      "double wk = (double)topk_w[(int64_t)t * K + (K - 1 - k)];\n            for (int32_t n"),
     "padding row not zeroed": (
         "            memset(dst, 0, sizeof(uint16_t) * (size_t)H);\n",
         "            memset(dst, 0, sizeof(uint16_t) * (size_t)(H / 2));\n"),
@@ -93,6 +101,9 @@ PINS = [
     ("one-hot", lambda lib: tdc.test_one_hot_selects_expert_row(lib)),
     ("lesson exercise", lambda lib: tdc.test_lesson_exercise_restated(lib)),
     ("fp8 properties", lambda lib: tdc.test_fp8_dispatch_properties(lib, 5)),
+    ("gemm scaled identity", lambda lib: tec.test_scaled_identity_experts(lib)),
+    ("gemm rank one", lambda lib: tec.test_rank_one_experts(lib)),
+    ("gemm masked", lambda lib: tec.test_masked_slots_and_selection(lib)),
     ("ll worked example", lambda lib: tll.test_ll_worked_example(lib)),
     ("ll brute force", lambda lib: tll.test_ll_bruteforce_tiny(lib)),
     ("ll round trip", lambda lib: tll.test_ll_round_trip(lib)),
