@@ -370,6 +370,45 @@ EP_API int ep_ll_combine(const ep_handle *h, const void *y, const float *topk_we
     return combine_common(h, y, topk_weights, out, true, stream);
 }
 
+EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner, const void *w, int32_t n_out,
+                             const float *topk_weights, float *out_acc, void *out, ep_stream_t stream) {
+    int rc = check_mode(h, false, true);
+    if (rc != EP_OK) return rc;
+    const ep_config &c = h->cfg;
+    if (c.expert_alignment % 128 != 0 || inner <= 0 || inner % 64 != 0 || n_out <= 0 || n_out % 256 != 0)
+        return EP_ERR_ARG;
+    if ((int64_t)c.num_experts * n_out > INT32_MAX || h->cap > INT32_MAX) return EP_ERR_UNSUPPORTED;
+    if (c.num_tokens == 0) return EP_OK;
+    if (!act || !w || !topk_weights || !out_acc || !out) return EP_ERR_ARG;
+    if (!aligned(act, 16) || !aligned(w, 16) || !aligned(out_acc, 16) || !aligned(out, 16) ||
+        !aligned(topk_weights, 4))
+        return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    ep::GemmCombineArgs a{};
+    a.p.eoff = h->eoff;
+    a.p.row_src = h->row_src;
+    a.p.row_slot = h->row_slot;
+    a.p.topk_w = topk_weights;
+    a.p.out_acc = out_acc;
+    a.p.status = h->status;
+    a.p.wait_limit_ns = h->wait_limit_ns;
+    a.p.E = c.num_experts;
+    a.p.K = c.num_topk;
+    a.p.N = n_out;
+    a.p.I = inner;
+    a.act = act;
+    a.w = w;
+    a.out = out;
+    a.cap = h->cap;
+    a.T = c.num_tokens;
+    const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
+    cudaError_t e = ep::launch_gemm_combine(a, sms, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launch(expert_combine)");
+    g_launches.fetch_add(2, std::memory_order_relaxed);
+    return EP_OK;
+}
+
 // ---- low-latency (static, masked) layout ----
 
 EP_API int64_t ep_ll_capacity_rows(const ep_config *c, int32_t M) {

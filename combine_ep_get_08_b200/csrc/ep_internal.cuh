@@ -89,6 +89,28 @@ struct CombineParams {
     int stages;                  // shared-memory ring depth (staged kernel)
 };
 
+// Expert GEMM with the combine fused into its epilogue.
+struct GemmCombineParams {
+    const int32_t *eoff;         // [E+1] padded expert offsets (row block -> expert)
+    const int32_t *row_src;      // [cap] token of a received row, -1 for padding
+    const int32_t *row_slot;     // [cap] k of a received row
+    const float *topk_w;         // [T, K]
+    float *out_acc;              // [T, N] fp32 accumulator (zeroed by the launcher)
+    unsigned int *status;
+    unsigned long long wait_limit_ns;
+    int E, K, N, I;              // N output features, I inner features
+};
+struct GemmCombineArgs {
+    GemmCombineParams p;
+    const void *act;             // [cap, I] bf16, received-row layout
+    const void *w;               // [E, N, I] bf16
+    void *out;                   // [T, N] bf16
+    int64_t cap;
+    int T;
+};
+// memset of the accumulator, the GEMM (one CTA per SM, num_sms CTAs) and the bf16 rounding
+cudaError_t launch_gemm_combine(const GemmCombineArgs &g, int num_sms, cudaStream_t s);
+
 // Layout launch shape: the cluster kernel (G CTAs in one thread-block
 // cluster, exchange through distributed shared memory) when a CTA can hold
 // its share of the pairs, else the cooperative kernel (G CTAs, one grid-wide

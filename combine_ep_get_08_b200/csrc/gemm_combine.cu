@@ -1,0 +1,341 @@
+// gemm_combine.cu -- expert GEMM with the combine fused into its epilogue
+// (sm_100a, tcgen05 tensor cores).
+//
+//   out[t, :] = bf16_rn( sum_k w[t,k] * act[pos[t,k], :] @ W_e^T ),  e = expert of pair (t, k)
+//
+// The expert step between dispatch and combine ("lesson14_deepep" practice
+// task: each expert transforms the rows it received, combine adds
+// weight * expert output back into the token's row), for the linear map of
+// an expert's last projection.  The rows arrive in the handle's received-row
+// layout, whose expert segments are padded to expert_alignment -- with an
+// alignment that is a multiple of 128 (EPBuffer.dispatch's
+// expert_alignment, bowenzhou.top "deepep/01-overview" section 1.1) every
+// 128-row tile belongs to one expert, so the GEMM needs no per-row expert
+// lookup.
+//
+// Persistent grid, one CTA per SM, 192 threads:
+//   warp 0     TMA producer: 128x64 tiles of act and 256x64 tiles of W_e
+//              (128-byte swizzle) into a 4-stage shared-memory ring;
+//   warp 1     allocates 512 TMEM columns (two fp32 128x256 accumulators)
+//              and issues tcgen05.mma (M=128, N=256, K=16, bf16 in, fp32
+//              accumulate) from one thread; tcgen05.commit frees ring
+//              stages and hands finished accumulators to the epilogue;
+//   warps 2-5  epilogue: tcgen05.ld a row's columns from TMEM (warp w reads
+//              lanes 32*(w%4)...), scale them by the pair's top-k weight and
+//              add them into an fp32 [T, N] accumulator with 16-byte vector
+//              atomics -- the combine, fused.  Padding rows add nothing.
+// A second kernel rounds the fp32 accumulator to bf16.  Every wait on an
+// mbarrier is bounded; a timeout sets EP_DEV_WAIT_TIMEOUT, lets the copies
+// and MMAs in flight finish (bounded again), frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+
+namespace {
+
+constexpr int kGM = 128;                              // rows per tile
+constexpr int kGN = 256;                              // output columns per tile
+constexpr int kGK = 64;                               // inner elements per stage: one 128-byte row
+constexpr int kGStages = 4;
+constexpr uint32_t kGABytes = kGM * kGK * 2;          // 16 KB
+constexpr uint32_t kGBBytes = kGN * kGK * 2;          // 32 KB
+constexpr int kGThreads = 192;
+constexpr int kGAcc = 2;                              // TMEM accumulators
+constexpr uint32_t kGTmemCols = kGAcc * kGN;          // 512: all of an SM's TMEM
+constexpr size_t kGSmem = 1024 + kGStages * (size_t)(kGABytes + kGBBytes) + 256;
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
+// 4-5 = 1), bf16 A and B (bits 7-9, 10-12 = 1), both K-major (bits 15, 16 =
+// 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kGIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kGN >> 3) << 17) |
+                             ((uint32_t)(kGM >> 4) << 24);
+
+// Shared-memory matrix descriptor of a K-major tile with 128-byte swizzle:
+// rows of 128 bytes, 8-row atoms of 1024 bytes (stride byte offset), start
+// address >> 4 in bits 0-13, leading byte offset 1 (unused for this
+// layout), version 1 at bit 46, layout type 2 (128-byte swizzle) at 61-63.
+__device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :
+        : "r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        :
+        : "r"(tmem_d), "l"(a), "l"(b), "r"(kGIdesc), "r"(accumulate));
+}
+
+// Arrives once on `bar` when every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :
+                 : "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" : : : "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" : : : "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : : : "memory");
+}
+
+// Largest e with eoff[e] <= r: the expert whose segment holds row r.
+__device__ __forceinline__ int expert_of_row(const int32_t *eoff, int E, int r) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(&eoff[mid]) <= r)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(kGThreads, 1)
+    gemm_combine_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                        GemmCombineParams p) {
+    extern __shared__ uint8_t g_smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(g_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;
+    uint8_t *sB = base + kGStages * kGABytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sB + kGStages * kGBBytes);
+    uint64_t *empty = full + kGStages;
+    uint64_t *acc_full = empty + kGStages;
+    uint64_t *acc_empty = acc_full + kGAcc;
+    uint64_t *drain = acc_empty + kGAcc;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows = __ldg(&p.eoff[p.E]);
+    const int n_blocks = p.N / kGN;
+    const int tiles = (rows / kGM) * n_blocks;
+    const int k_blocks = p.I / kGK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < kGAcc; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);     // lane 0 of each epilogue warp
+        }
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_async_smem();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :
+                     : "r"(smem_u32(s_tmem)), "r"(kGTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" : : : "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 0) {
+        // ---- TMA producer ----
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
+                const int m = tile / n_blocks, n = tile - m * n_blocks;
+                const int e = expert_of_row(p.eoff, p.E, m * kGM);
+                for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+                    const int s = it % kGStages, use = it / kGStages;
+                    if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1, p.wait_limit_ns)) {
+                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *s_abort = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], kGABytes + kGBBytes);
+                    tma_load_2d(sA + s * kGABytes, &map_a, kb * kGK, m * kGM, &full[s]);
+                    tma_load_2d(sB + s * kGBBytes, &map_b, kb * kGK, e * p.N + n * kGN, &full[s]);
+                }
+            }
+            // on abort, let the loads already issued land before shared memory goes away
+            if (*s_abort)
+                for (int j = max(0, it - kGStages); j < it; ++j)
+                    mbar_wait_bounded(&full[j % kGStages], (j / kGStages) & 1, p.wait_limit_ns);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer ----
+        if (lane == 0) {
+            int it = 0, local = 0;
+            for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x, ++local) {
+                const int acc = local % kGAcc, ause = local / kGAcc;
+                if (ause > 0 && !mbar_wait_bounded(&acc_empty[acc], (ause - 1) & 1, p.wait_limit_ns)) {
+                    atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                    *s_abort = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(acc * kGN);
+                bool ok = true;
+                for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+                    const int s = it % kGStages;
+                    if (!mbar_wait_bounded(&full[s], (it / kGStages) & 1, p.wait_limit_ns)) {
+                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *s_abort = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a = umma_desc_k_sw128(smem_u32(sA + s * kGABytes));
+                    const uint64_t b = umma_desc_k_sw128(smem_u32(sB + s * kGBBytes));
+#pragma unroll
+                    for (int kk = 0; kk < kGK / 16; ++kk)   // 16 bf16 = 32 bytes = 2 descriptor units
+                        umma_bf16(d, a + 2 * kk, b + 2 * kk, (kb | kk) != 0);
+                    umma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[acc]);
+            }
+            // every MMA issued has completed before TMEM is freed
+            umma_commit(drain);
+            mbar_wait_bounded(drain, 0, p.wait_limit_ns);
+        }
+    } else {
+        // ---- epilogue: scale by the pair's weight, add into the token's row ----
+        const int q = warp & 3;                    // TMEM lanes 32q .. 32q+31
+        int local = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
+            const int acc = local % kGAcc, ause = local / kGAcc;
+            if (*s_abort || !mbar_wait_bounded(&acc_full[acc], ause & 1, p.wait_limit_ns)) {
+                if (!*s_abort) {
+                    atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                    *s_abort = 1;
+                }
+                break;
+            }
+            tc_fence_after();
+            const int m = tile / n_blocks, n = tile - m * n_blocks;
+            const int r = m * kGM + q * 32 + lane;
+            const int src = __ldg(&p.row_src[r]);
+            float wt = 0.0f;
+            if (src >= 0) wt = __ldg(&p.topk_w[(int64_t)src * p.K + __ldg(&p.row_slot[r])]);
+            float *orow = p.out_acc + (int64_t)(src >= 0 ? src : 0) * p.N + (int64_t)n * kGN;
+            for (int c = 0; c < kGN / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kGN + c * 32), v);
+                if (src >= 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        atomicAdd(reinterpret_cast<float4 *>(orow + c * 32 + j),
+                                  make_float4(wt * __uint_as_float(v[j]), wt * __uint_as_float(v[j + 1]),
+                                              wt * __uint_as_float(v[j + 2]), wt * __uint_as_float(v[j + 3])));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" : : "r"(tmem), "r"(kGTmemCols) : "memory");
+}
+
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// out = bf16_rn(acc), 8 elements per thread per step.
+__global__ void acc_to_bf16_kernel(const float *acc, void *out, int64_t n8) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = reinterpret_cast<const float4 *>(acc)[2 * i];
+        const float4 b = reinterpret_cast<const float4 *>(acc)[2 * i + 1];
+        reinterpret_cast<uint4 *>(out)[i] =
+            make_uint4(bf16x2_rn(a.x, a.y), bf16x2_rn(a.z, a.w), bf16x2_rn(b.x, b.y), bf16x2_rn(b.z, b.w));
+    }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// A [rows_total, inner] bf16 row-major matrix read in (box_rows x 64) tiles with 128-byte swizzle.
+bool make_map(CUtensorMap *map, const void *ptr, int64_t rows_total, int inner, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows_total};
+    const cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kGK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_combine(const GemmCombineArgs &g, int num_sms, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        const cudaError_t e = cudaFuncSetAttribute(gemm_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)kGSmem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    CUtensorMap map_a, map_b;
+    if (!make_map(&map_a, g.act, g.cap, g.p.I, kGM) || !make_map(&map_b, g.w, (int64_t)g.p.E * g.p.N, g.p.I, kGN))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(g.p.out_acc, 0, sizeof(float) * (size_t)g.T * g.p.N, s);
+    if (e != cudaSuccess) return e;
+    gemm_combine_kernel<<<num_sms, kGThreads, kGSmem, s>>>(map_a, map_b, g.p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t n8 = (int64_t)g.T * g.p.N / 8;
+    if (n8 > 0) {
+        const int grid = (int)((n8 + 255) / 256 < 4 * num_sms ? (n8 + 255) / 256 : 4 * num_sms);
+        acc_to_bf16_kernel<<<grid, 256, 0, s>>>(g.p.out_acc, g.out, n8);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace ep

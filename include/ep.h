@@ -314,6 +314,29 @@ EP_API int ep_ll_dispatch_fp8(ep_handle *h, const int64_t *topk_idx, const void 
 EP_API int ep_ll_combine(const ep_handle *h, const void *y, const float *topk_weights, void *out,
                          ep_stream_t stream);
 
+/*
+ * Expert GEMM with the combine fused into its epilogue (tcgen05 tensor
+ * cores): the last linear map of each expert applied to its received rows,
+ * each result row scaled by its pair's top-k weight and added into the
+ * token's output row -- the step between dispatch and combine of
+ * "lesson14_deepep" (practice task: experts transform the rows they
+ * received, moe_combine adds weight * expert output back per token), done
+ * without writing the expert outputs.
+ *   out[t, :] = bf16_rn( sum_k topk_weights[t,k] * act[pos[t,k], :] @ W_e^T ),
+ *   e = topk_idx[t,k]; masked (-1) pairs and padding rows add nothing.
+ * act [capacity, inner] bf16 in h's received-row layout; w [E, n_out, inner]
+ * bf16 (expert e's matrix, row n = output feature n); topk_weights [T, K]
+ * fp32; out_acc [T, n_out] fp32 workspace (zeroed by the call); out
+ * [T, n_out] bf16.  Needs expert_alignment % 128 == 0 (each 128-row tile
+ * belongs to one expert), inner % 64 == 0, n_out % 256 == 0 and 16-byte
+ * aligned act, w, out_acc and out; else EP_ERR_ARG.  The fp32 sums are
+ * formed with atomic adds, so their order (and the last bit of out) may
+ * vary between calls.  Launches the GEMM (one CTA per SM, capped by
+ * ep_set_sm_limit) and a rounding kernel.
+ */
+EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner, const void *w, int32_t n_out,
+                             const float *topk_weights, float *out_acc, void *out, ep_stream_t stream);
+
 /* Synchronises `stream` and returns rows (= expert_offsets[E]) on the host. */
 EP_API int ep_get_num_rows(const ep_handle *h, int32_t *rows, ep_stream_t stream);
 
