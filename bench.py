@@ -554,6 +554,118 @@ def run_e2e(path, args, stream, reuse, world, dev, bytes_step):
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+# ----------------------------------------------------------------------------
+# Expert GEMM with the fused combine (ep_expert_combine)
+# ----------------------------------------------------------------------------
+EGEMM = dict(T=4096, H=7168, E=32, R=8, K=8, A=128, router="topk", seed=5, I=2048)
+EGEMM_DESC = ("one expert-parallel rank of a DeepSeek-V3 layer: 32 local experts receiving 4096 tokens x "
+              "top-8 (32768 rows, 1024 per expert, align 128); expert down projection 2048 -> 7168 bf16 "
+              "with the top-k weighted combine in the epilogue")
+
+
+def run_expert_gemm(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import combine_ep_get_08_b200 as ep
+    import workloads
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    from combine_ep_get_08_b200 import build_lib
+    if rank == 0:
+        build_lib.build()
+    barrier(world)
+    c = dict(EGEMM)
+    I = c.pop("I")
+    seed = c.pop("seed") + 1000 * rank
+    wl = workloads.generate(None, seed=seed, with_x=False, **c)
+    N = wl.H
+    cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
+    h = ep.ep_handle_create(cfg)
+    if args.sm_limit:
+        ep.ep_set_sm_limit(h, args.sm_limit)
+    idx, tw = wl.topk_idx.to(dev), wl.topk_weights.to(dev)
+    ep.ep_get_layout(h, idx, tw)
+    rows = ep.ep_get_num_rows(h)
+    cap = ep.ep_capacity_rows(cfg)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    act = torch.randn((cap, I), generator=gen, device=dev).to(torch.bfloat16)
+    w = (torch.randn((wl.E, N, I), generator=gen, device=dev) / I ** 0.5).to(torch.bfloat16)
+    acc = torch.empty((wl.T, N), dtype=torch.float32, device=dev)
+    out = torch.empty((wl.T, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        ep.ep_expert_combine(h, act, I, w, N, tw, acc, out, stream=stream.cuda_stream)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = ep.ep_launch_count()
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        for e0, e1 in evs:
+            flush.sum()
+            e0.record(stream)
+            ep.ep_expert_combine(h, act, I, w, N, tw, acc, out, stream=stream.cuda_stream)
+            e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    launches = ep.ep_launch_count() - launches0
+    ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = max_over_ranks(sum(ms), world, dev)
+    pairs = int((wl.topk_idx >= 0).sum())
+    flops_call = 2.0 * pairs * N * I               # algorithmic: real rows only
+    all_flops = sum_over_ranks(flops_call * args.steps, world, dev)
+    tflops = all_flops / (total_ms * 1e-3) / 1e12
+    status = ep.ep_get_status(h)
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, peak_src = float(json.load(f)["bf16_tflops"]), "measured burst (MEASURED_PEAKS.json bf16_tflops)"
+    except Exception:  # noqa: BLE001
+        peak, peak_src = 1590.0, "fallback 1.59 PFLOP/s"
+    mean_ms = statistics.mean(ms)
+    if rank == 0:
+        line = {
+            "metric": "expert GEMM + fused combine TFLOP/s", "value": round(tflops, 1), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": EGEMM_DESC, "rows": rows, "padded_rows_computed": rows, "pairs": pairs,
+                       "inner": I, "n_out": N, "sm_limit": args.sm_limit or None,
+                       "l2": "flushed (256 MiB read, outside the timed events) before each call"},
+            "roofline": {"bound": "tensor", "kernel": "gemm_combine_kernel (+ memset and bf16 rounding)",
+                         "achieved": round(flops_call / (mean_ms * 1e-3) / 1e12, 1), "peak": peak,
+                         "peak_source": peak_src, "unit": "TFLOP/s",
+                         "frac": round(flops_call / (mean_ms * 1e-3) / 1e12 / peak, 4), "traffic": None},
+            "gpu_launches": int(launches), "clocks": sampler.summary(), "device_status": int(status),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            oracle.build()
+            o = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A)
+            act_b = workloads.bf16_bits(act[:rows])
+            w_b = workloads.bf16_bits(w)
+            n_tok, t0 = 0, time.perf_counter()
+            while time.perf_counter() - t0 < args.cpu_budget:
+                oracle.expert_combine(act_b, w_b, wl.topk_idx.numpy(), o.pos, wl.topk_weights.numpy(),
+                                      np.array([n_tok % wl.T], np.int32))
+                n_tok += 1
+            el = time.perf_counter() - t0
+            line["cpu_baseline"] = {
+                "value": round(2.0 * wl.K * N * I * n_tok / el / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+                "kind": "oracle", "sample": f"{n_tok} token(s) of the same workload ({el:.1f} s, single thread, fp64)"}
+        print(json.dumps(line), flush=True)
+    ep.ep_handle_destroy(h)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def ncu_ingest(rep: str, workload: str) -> int:
     """Record DRAM bytes per launch of the layout / dispatch / combine kernels
     from an ncu report (``ncu -i REP --page raw --csv``; per kernel the mean
@@ -625,6 +737,8 @@ def main(argv=None):
                     help="layout: normal (padded, ep_get_layout) or low-latency static slots (ep_ll_*)")
     ap.add_argument("--ll-slots", type=int, default=0, help="slots per expert in --mode ll (0: T)")
     ap.add_argument("--ncu-ingest", metavar="REP", help="record DRAM traffic from an ncu report and exit")
+    ap.add_argument("--expert-gemm", action="store_true",
+                    help="time ep_expert_combine (expert GEMM + fused combine) instead of the step")
     args = ap.parse_args(argv)
     if args.ncu_ingest:
         return ncu_ingest(args.ncu_ingest, args.config + ("-ll" if args.mode == "ll" else ""))
@@ -636,6 +750,8 @@ def main(argv=None):
             ap.error("--gpus N > 1 must be launched with torchrun (one process per GPU)")
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.expert_gemm:
+        return run_expert_gemm(args, world, rank, local)
     return run_cuda(args, world, rank, local)
 
 

@@ -20,10 +20,13 @@
 //              and issues tcgen05.mma (M=128, N=256, K=16, bf16 in, fp32
 //              accumulate) from one thread; tcgen05.commit frees ring
 //              stages and hands finished accumulators to the epilogue;
-//   warps 2-5  epilogue: tcgen05.ld a row's columns from TMEM (warp w reads
-//              lanes 32*(w%4)...), scale them by the pair's top-k weight and
-//              add them into an fp32 [T, N] accumulator with 16-byte vector
-//              atomics -- the combine, fused.  Padding rows add nothing.
+//   warps 2-5  epilogue, one warp per 32-lane quarter of TMEM (warp w reads
+//              lanes 32*(w%4)...): tcgen05.ld a row's columns, scale them
+//              by the pair's top-k weight,
+//              transpose each 32x32 chunk through shared memory and add it
+//              into an fp32 [T, N] accumulator with 16-byte vector atomics
+//              that cover 128 contiguous bytes per 8 lanes -- the combine,
+//              fused.  Padding rows add nothing.
 // A second kernel rounds the fp32 accumulator to bf16.  Every wait on an
 // mbarrier is bounded; a timeout sets EP_DEV_WAIT_TIMEOUT, lets the copies
 // and MMAs in flight finish (bounded again), frees TMEM and returns.
@@ -36,16 +39,36 @@ namespace ep {
 
 namespace {
 
+#ifndef EP_GEMM_ORDER
+#define EP_GEMM_ORDER 1      // 1: tiles expert by expert, column block, row block; 0: row block, column block
+#endif
+#ifndef EP_GEMM_NGROUP
+#define EP_GEMM_NGROUP 0     // column blocks per pass over the experts (0: all of them)
+#endif
+#ifndef EP_GEMM_EPI
+#define EP_GEMM_EPI 0        // 0: thread vector atomics over transposed chunks; 1: a bulk reduce-add
+                             // (TMA engine) per 128-byte row chunk, measured 1% slower
+#endif
+#ifndef EP_GEMM_POLICY
+#define EP_GEMM_POLICY 0     // L2 hints on the TMA loads: 0 none; 1 W evict_first, act evict_last; 2 W evict_first
+#endif
+
 constexpr int kGM = 128;                              // rows per tile
 constexpr int kGN = 256;                              // output columns per tile
 constexpr int kGK = 64;                               // inner elements per stage: one 128-byte row
 constexpr int kGStages = 4;
 constexpr uint32_t kGABytes = kGM * kGK * 2;          // 16 KB
 constexpr uint32_t kGBBytes = kGN * kGK * 2;          // 32 KB
-constexpr int kGThreads = 192;
+constexpr int kGEpiWarps = 4;                        // one per TMEM lane quarter (8 measured slower: the
+                                                      // atomic adds are bound by L2, not by issue)
+constexpr int kGThreads = 64 + 32 * kGEpiWarps;
 constexpr int kGAcc = 2;                              // TMEM accumulators
 constexpr uint32_t kGTmemCols = kGAcc * kGN;          // 512: all of an SM's TMEM
-constexpr size_t kGSmem = 1024 + kGStages * (size_t)(kGABytes + kGBBytes) + 256;
+// one epilogue warp's 32x32 fp32 staging tile: transposed and swizzled for
+// thread atomics, or rows padded to 36 floats (16-byte aligned, no bank
+// conflicts) for bulk reductions
+constexpr uint32_t kGStageT = 32 * 36 * 4;
+constexpr size_t kGSmem = 1024 + kGStages * (size_t)(kGABytes + kGBBytes) + kGEpiWarps * kGStageT + 256;
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
 // 4-5 = 1), bf16 A and B (bits 7-9, 10-12 = 1), both K-major (bits 15, 16 =
@@ -62,12 +85,15 @@ __device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t saddr) {
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int x, int y,
-                                            uint64_t *bar) {
+// 2-D tiled TMA load (no multicast) with an L2 eviction-priority policy.
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int x, int y, uint64_t *bar,
+                                            uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;"
         :
-        : "r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)),
+          "l"(policy)
         : "memory");
 }
 
@@ -77,6 +103,15 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t 
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
         :
         : "r"(tmem_d), "l"(a), "l"(b), "r"(kGIdesc), "r"(accumulate));
+}
+
+// out[0 .. bytes/4) += src[...] in fp32, performed by the TMA engine in L2
+// (16-byte aligned addresses, bytes % 16 == 0; joins this thread's bulk group).
+__device__ __forceinline__ void bulk_reduce_add_f32(float *gdst, const float *ssrc, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
+                 :
+                 : "l"(gdst), "r"(smem_u32(ssrc)), "r"(bytes)
+                 : "memory");
 }
 
 // Arrives once on `bar` when every tcgen05 operation this thread issued so far has completed.
@@ -103,17 +138,59 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" : : : "memory");
 }
 
-// Largest e with eoff[e] <= r: the expert whose segment holds row r.
-__device__ __forceinline__ int expert_of_row(const int32_t *eoff, int E, int r) {
-    int lo = 0, hi = E - 1;
+// Tiles are numbered by groups of column blocks (so that the fp32 output
+// columns being accumulated stay in L2), inside a group expert by expert,
+// inside an expert by column block and then by row block, so the CTAs
+// running side by side share one 256-column slice of W_e (read from DRAM
+// once, then from L2) and the expert's row blocks.  With mtot row blocks in
+// all, group gi starts at tile mtot * n0 (n0 = its first column block), and
+// expert e's tiles inside it at (eoff[e] / kGM) * (column blocks in group).
+struct GemmTile {
+    int m;   // row block (global)
+    int n;   // column block
+    int e;   // expert
+};
+
+__device__ __forceinline__ GemmTile tile_coords(const int32_t *eoff, int E, int n_blocks, int t) {
+#if EP_GEMM_ORDER == 0
+    {
+        GemmTile g;
+        g.m = t / n_blocks;
+        g.n = t - g.m * n_blocks;
+        int lo = 0, hi = E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(&eoff[mid]) <= g.m * kGM)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        g.e = lo;
+        return g;
+    }
+#endif
+    const int mtot = __ldg(&eoff[E]) / kGM;
+    const int ng = (EP_GEMM_NGROUP > 0 && EP_GEMM_NGROUP < n_blocks) ? EP_GEMM_NGROUP : n_blocks;
+    const int gi = t / (mtot * ng);
+    const int n0 = gi * ng, ngi = min(ng, n_blocks - n0);
+    const int lt = t - mtot * n0;
+    int lo = 0, hi = E - 1;   // largest e whose first tile in the group is <= lt
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(&eoff[mid]) <= r)
+        if (__ldg(&eoff[mid]) / kGM * ngi <= lt)
             lo = mid;
         else
             hi = mid - 1;
     }
-    return lo;
+    // an empty expert shares its first tile with the next one, so lo is never empty
+    const int m0 = __ldg(&eoff[lo]) / kGM;
+    const int mb = __ldg(&eoff[lo + 1]) / kGM - m0;
+    const int local = lt - m0 * ngi;
+    GemmTile g;
+    g.e = lo;
+    g.n = n0 + local / mb;
+    g.m = m0 + (local - (local / mb) * mb);
+    return g;
 }
 
 __global__ void __launch_bounds__(kGThreads, 1)
@@ -123,7 +200,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(g_smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
     uint8_t *sB = base + kGStages * kGABytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sB + kGStages * kGBBytes);
+    float *sT = reinterpret_cast<float *>(sB + kGStages * kGBBytes);   // [epilogue warps][32 rows][32 cols], swizzled
+    uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sT) + kGEpiWarps * kGStageT);
     uint64_t *empty = full + kGStages;
     uint64_t *acc_full = empty + kGStages;
     uint64_t *acc_empty = acc_full + kGAcc;
@@ -144,7 +222,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         for (int a = 0; a < kGAcc; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], 4);     // lane 0 of each epilogue warp
+            mbar_init(&acc_empty[a], kGEpiWarps);   // lane 0 of each epilogue warp
         }
         mbar_init(drain, 1);
         *s_abort = 0;
@@ -166,9 +244,20 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // ---- TMA producer ----
         if (lane == 0) {
             int it = 0;
+            uint64_t pol_w, pol_a;
+#if EP_GEMM_POLICY >= 1
+            asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol_w));
+#else
+            asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol_w));
+#endif
+#if EP_GEMM_POLICY == 1
+            asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_a));
+#else
+            asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol_a));
+#endif
             for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
-                const int m = tile / n_blocks, n = tile - m * n_blocks;
-                const int e = expert_of_row(p.eoff, p.E, m * kGM);
+                const GemmTile g = tile_coords(p.eoff, p.E, n_blocks, tile);
+                const int m = g.m, n = g.n, e = g.e;
                 for (int kb = 0; kb < k_blocks; ++kb, ++it) {
                     const int s = it % kGStages, use = it / kGStages;
                     if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1, p.wait_limit_ns)) {
@@ -177,8 +266,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&full[s], kGABytes + kGBBytes);
-                    tma_load_2d(sA + s * kGABytes, &map_a, kb * kGK, m * kGM, &full[s]);
-                    tma_load_2d(sB + s * kGBBytes, &map_b, kb * kGK, e * p.N + n * kGN, &full[s]);
+                    tma_load_2d(sA + s * kGABytes, &map_a, kb * kGK, m * kGM, &full[s], pol_a);
+                    tma_load_2d(sB + s * kGBBytes, &map_b, kb * kGK, e * p.N + n * kGN, &full[s], pol_w);
                 }
             }
             // on abort, let the loads already issued land before shared memory goes away
@@ -225,7 +314,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     } else {
         // ---- epilogue: scale by the pair's weight, add into the token's row ----
+        // A thread holds one row (its TMEM lane) of each 32-column chunk; the
+        // chunk is transposed through a swizzled shared-memory tile so that
+        // eight lanes cover 128 contiguous bytes of one token row and each
+        // warp-wide vector add touches 4 rows instead of 32.
         const int q = warp & 3;                    // TMEM lanes 32q .. 32q+31
+        constexpr int kChunks = (kGN / 32) / (kGEpiWarps / 4);                  // 32-column chunks per warp
+        const int c_lo = (warp - 2) / 4 * kChunks, c_hi = c_lo + kChunks;
+        float4 *tile4 = reinterpret_cast<float4 *>(sT + (warp - 2) * (kGStageT / 4));
         int local = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++local) {
             const int acc = local % kGAcc, ause = local / kGAcc;
@@ -237,27 +333,56 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int m = tile / n_blocks, n = tile - m * n_blocks;
-            const int r = m * kGM + q * 32 + lane;
+            const GemmTile g = tile_coords(p.eoff, p.E, n_blocks, tile);
+            const int r = g.m * kGM + q * 32 + lane;
             const int src = __ldg(&p.row_src[r]);
             float wt = 0.0f;
             if (src >= 0) wt = __ldg(&p.topk_w[(int64_t)src * p.K + __ldg(&p.row_slot[r])]);
-            float *orow = p.out_acc + (int64_t)(src >= 0 ? src : 0) * p.N + (int64_t)n * kGN;
-            for (int c = 0; c < kGN / 32; ++c) {
+#if EP_GEMM_EPI == 1
+            float *srow = sT + (warp - 2) * (kGStageT / 4) + lane * 36;   // this lane's staged row
+            float *orow = p.out_acc + (int64_t)(src >= 0 ? src : 0) * p.N + (int64_t)g.n * kGN;
+            for (int c = c_lo; c < c_hi; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kGN + c * 32), v);
-                if (src >= 0) {
+                bulk_wait_read<0>();                 // the previous chunk's reduction has read srow
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        atomicAdd(reinterpret_cast<float4 *>(orow + c * 32 + j),
-                                  make_float4(wt * __uint_as_float(v[j]), wt * __uint_as_float(v[j + 1]),
-                                              wt * __uint_as_float(v[j + 2]), wt * __uint_as_float(v[j + 3])));
-                }
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<float4 *>(srow + 4 * k) =
+                        make_float4(wt * __uint_as_float(v[4 * k]), wt * __uint_as_float(v[4 * k + 1]),
+                                    wt * __uint_as_float(v[4 * k + 2]), wt * __uint_as_float(v[4 * k + 3]));
+                fence_async_smem();                  // generic-proxy writes -> the bulk copy's reads
+                if (src >= 0) bulk_reduce_add_f32(orow + c * 32, srow, 32 * 4);
+                bulk_commit();
             }
+#else
+            const int sub = lane >> 3, k4 = lane & 7;  // reader: row i0 + sub, float4 k4 of the chunk
+            for (int c = c_lo; c < c_hi; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kGN + c * 32), v);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)                 // float4 k of row `lane` at slot k ^ (lane & 7)
+                    tile4[lane * 8 + (k ^ (lane & 7))] =
+                        make_float4(wt * __uint_as_float(v[4 * k]), wt * __uint_as_float(v[4 * k + 1]),
+                                    wt * __uint_as_float(v[4 * k + 2]), wt * __uint_as_float(v[4 * k + 3]));
+                __syncwarp();
+                float *ocol = p.out_acc + (int64_t)g.n * kGN + c * 32 + k4 * 4;
+#pragma unroll
+                for (int i0 = 0; i0 < 32; i0 += 4) {
+                    const int i = i0 + sub;
+                    const int t = __shfl_sync(0xffffffffu, src, i);
+                    const float4 val = tile4[i * 8 + (k4 ^ (i & 7))];
+                    if (t >= 0) atomicAdd(reinterpret_cast<float4 *>(ocol + (int64_t)t * p.N), val);
+                }
+                __syncwarp();
+            }
+#endif
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
         }
+#if EP_GEMM_EPI == 1
+        bulk_wait_all();                             // reductions done before shared memory goes away
+#endif
     }
     tc_fence_before();
     __syncthreads();
