@@ -169,13 +169,16 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
 
 
+# the sources of the step's kernels (layout, dispatch, combine) and their shared header
+STEP_KERNEL_SOURCES = ("combine.cu", "dispatch.cu", "ep_internal.cuh", "layout.cu")
+
+
 def kernel_source_digest() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "combine_ep_get_08_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in STEP_KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -399,12 +402,15 @@ def run_cuda(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     sptr = stream.cuda_stream
 
-    def one_step(ev=None):
+    def one_step(ev=None, split=False):
+        # The dispatch follows the layout with no event between them, so its
+        # launch overlaps the layout's tail (programmatic dependent launch);
+        # `split` puts an event between them to time each kernel alone.
         path.flush_l2()
         if ev is not None:
             ev[0].record(stream)
         path.layout(sptr)
-        if ev is not None:
+        if ev is not None and split:
             ev[1].record(stream)
         for r in range(reuse):
             path.dispatch(sptr)
@@ -440,14 +446,25 @@ def run_cuda(args, world, rank, local):
 
     # the low-latency mode has no layout launch (it is fused into the dispatch):
     # the empty event pair around it would only add the events' own overhead
-    lay_ms = [0.0 if ll else e[0].elapsed_time(e[1]) for e in evs]
-    dis_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    com_ms = [e[3].elapsed_time(e[4]) for e in evs]
-    # with reuse > 1 only the first dispatch/combine pair of a step carries events;
-    # the step's device time counts every call at that per-call time
-    step_ms = [l + reuse * (d + c) for l, d, c in zip(lay_ms, dis_ms, com_ms)]
-    total_ms = sum(step_ms)
     bracket_ms = bracket[0].elapsed_time(bracket[1])
+    # layout + first dispatch as one span (their launches overlap); with
+    # reuse > 1 only the first dispatch/combine pair of a step carries events
+    # and the further calls count at the per-call times measured below
+    ld_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    com_ms = [e[3].elapsed_time(e[4]) for e in evs]
+
+    # per-kernel times (events between layout and dispatch), for the
+    # breakdown and the roofline; not part of `value`
+    n_split = min(args.steps, 20)
+    evs_split = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_split)]
+    for i in range(n_split):
+        one_step(evs_split[i], split=True)
+    torch.cuda.synchronize()
+    lay_ms = [0.0 if ll else e[0].elapsed_time(e[1]) for e in evs_split]
+    dis_ms = [e[1].elapsed_time(e[2]) for e in evs_split]
+    mean_dis = statistics.mean(dis_ms)
+    step_ms = [ld + (reuse - 1) * mean_dis + reuse * c for ld, c in zip(ld_ms, com_ms)]
+    total_ms = sum(step_ms)
 
     b_dis = dispatch_bytes(wl.T, wl.H, wl.K, rows, wl.fp8)
     b_com = combine_bytes(wl.T, wl.H, wl.K)
@@ -461,6 +478,7 @@ def run_cuda(args, world, rank, local):
     e2e = run_e2e(path, args, stream, reuse, world, dev, bytes_step)
 
     lay_us, dis_us, com_us = (statistics.mean(v) * 1e3 for v in (lay_ms, dis_ms, com_ms))
+    ld_us = statistics.mean(ld_ms) * 1e3
     peak, peak_src = measured_peak()
     kern = {"layout": lay_us, "dispatch": dis_us, "combine": com_us}
     dom = "dispatch" if dis_us >= com_us else "combine"
@@ -488,6 +506,7 @@ def run_cuda(args, world, rank, local):
                       "between dispatch and combine",
             },
             "us_per_call": {k: round(v, 2) for k, v in kern.items()},
+            "us_layout_then_dispatch": round(ld_us, 2),
             "bytes_per_call": {"dispatch": b_dis, "combine": b_com},
             "gbs_per_call": {"dispatch": round(b_dis / dis_us / 1e3, 1),
                              "combine": round(b_com / com_us / 1e3, 1)},

@@ -159,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, EP_LSU_MINB) dispatch_bf16_kernel(Di
     int rows = -1;
     LlState st;
     int nblk = gridDim.x;
+    pdl_wait();   // the layout (or whatever ran before) is complete and visible
     if constexpr (LL) {
         extern __shared__ int32_t ll_smem[];
         st.ids = ll_smem;
@@ -331,8 +332,9 @@ __global__ void __launch_bounds__(kStagedThreads, 1) dispatch_bf16_staged_kernel
         }
         fence_async_smem();
         s_abort = 0;
-        s_rows = p.n_zero_units ? __ldg(&p.eoff[p.E]) : 0;
     }
+    pdl_wait();   // shared-memory set-up overlapped the previous kernel; global reads start here
+    if (threadIdx.x == 0) s_rows = p.n_zero_units ? __ldg(&p.eoff[p.E]) : 0;
     __syncthreads();
 
 #if EP_STAGED_PREFETCH
@@ -489,6 +491,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p
     int rows = -1;
     LlState st;
     int nblk = gridDim.x;
+    pdl_wait();   // the layout (or whatever ran before) is complete and visible
     if constexpr (LL) {
         extern __shared__ int32_t ll_smem[];
         st.ids = ll_smem;
@@ -598,6 +601,25 @@ cudaError_t dispatch_prepare() {
     return cudaSuccess;
 }
 
+// Launch that may start while the previous kernel on the stream finishes
+// (programmatic stream serialization); the kernels wait with pdl_wait()
+// before touching global memory.
+template <typename Kernel>
+static cudaError_t launch_pdl(Kernel kernel, int grid, int block, size_t smem, cudaStream_t s,
+                              const DispatchParams &p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 cudaError_t launch_dispatch_bf16(const DispatchParams &p_in, int num_sms, cudaStream_t s) {
     static int occ16 = 0, occ32 = 0;
     DispatchParams p = p_in;
@@ -612,23 +634,19 @@ cudaError_t launch_dispatch_bf16(const DispatchParams &p_in, int num_sms, cudaSt
         const int units = p.n_token_units + p.n_zero_units;
         const int grid = units < num_sms ? units : num_sms;
         const size_t smem = staged_smem_bytes(stages, row_bytes / splits);
-        if (v32)
-            dispatch_bf16_staged_kernel<32><<<grid, kStagedThreads, smem, s>>>(p);
-        else
-            dispatch_bf16_staged_kernel<16><<<grid, kStagedThreads, smem, s>>>(p);
-        return cudaGetLastError();
+        return v32 ? launch_pdl(dispatch_bf16_staged_kernel<32>, grid, kStagedThreads, smem, s, p)
+                   : launch_pdl(dispatch_bf16_staged_kernel<16>, grid, kStagedThreads, smem, s, p);
     }
     const int units = p.n_token_units + p.n_zero_units;
     if (v32) {
         const void *k = reinterpret_cast<const void *>(&dispatch_bf16_kernel<32, false>);
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ32), num_sms);
-        dispatch_bf16_kernel<32, false><<<grid, kThreads, 0, s>>>(p);
+        return launch_pdl(dispatch_bf16_kernel<32, false>, grid, kThreads, 0, s, p);
     } else {
         const void *k = reinterpret_cast<const void *>(&dispatch_bf16_kernel<16, false>);
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ16), num_sms);
-        dispatch_bf16_kernel<16, false><<<grid, kThreads, 0, s>>>(p);
+        return launch_pdl(dispatch_bf16_kernel<16, false>, grid, kThreads, 0, s, p);
     }
-    return cudaGetLastError();
 }
 
 // Low-latency launches: the register kernels with in-kernel destinations.
@@ -678,13 +696,12 @@ cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream
     if (v32) {
         const void *k = reinterpret_cast<const void *>(&dispatch_fp8_kernel<32, false>);
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ32), num_sms);
-        dispatch_fp8_kernel<32, false><<<grid, kThreads, 0, s>>>(p);
+        return launch_pdl(dispatch_fp8_kernel<32, false>, grid, kThreads, 0, s, p);
     } else {
         const void *k = reinterpret_cast<const void *>(&dispatch_fp8_kernel<16, false>);
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ16), num_sms);
-        dispatch_fp8_kernel<16, false><<<grid, kThreads, 0, s>>>(p);
+        return launch_pdl(dispatch_fp8_kernel<16, false>, grid, kThreads, 0, s, p);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace ep

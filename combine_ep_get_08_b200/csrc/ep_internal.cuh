@@ -329,6 +329,15 @@ __device__ __forceinline__ void bulk_wait_read() {
 
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" : : : "memory"); }
 
+// Programmatic dependent launch.  A kernel launched with programmatic
+// stream serialization may start while the kernel before it on the stream
+// is still running; griddepcontrol.wait blocks the calling thread until that
+// kernel has completed and its writes are visible, so every thread calls it
+// before its first read of global memory.  launch_dependents lets such a
+// dependent launch begin before this grid ends.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" : : : "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" : :); }
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy (bulk copy) reads of them.
 __device__ __forceinline__ void fence_async_smem() {

@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_kernel(LayoutParams 
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int c = blockIdx.x;
+    pdl_launch_dependents();   // a dispatch launched next may start its set-up now
     const int t_begin = min(p.T, c * p.tokens_per_chunk);
     const int t_end = min(p.T, t_begin + p.tokens_per_chunk);
     const int64_t p_begin = (int64_t)t_begin * K, p_end = (int64_t)t_end * K;
@@ -481,6 +482,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
     __shared__ int32_t s_tmp[2 * (kLayoutWarps + 1)];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_launch_dependents();   // a dispatch launched next may start its set-up now
     const int t_begin = min(p.T, c * p.tokens_per_chunk);
     const int t_end = min(p.T, t_begin + p.tokens_per_chunk);
     const int64_t p_begin = (int64_t)t_begin * K;
