@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
     const int vps = (V + p.splits - 1) / p.splits;
     const uint8_t *y = static_cast<const uint8_t *>(p.y);
     uint8_t *out = static_cast<uint8_t *>(p.out);
+    pdl_wait();   // the kernel before (the expert computation) is complete and visible
     for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
         const int t = u / p.splits, s = u - t * p.splits;
         if (threadIdx.x < p.K) {
@@ -115,8 +116,18 @@ cudaError_t launch_combine(const CombineParams &p_in, int num_sms, cudaStream_t 
     p.n_units = p.T * sp;
     const void *k = reinterpret_cast<const void *>(&combine_kernel<4>);
     const int grid = persistent_grid(p.n_units, blocks_per_sm(k, kThreads, 0, &occ), num_sms);
-    combine_kernel<4><<<grid, kThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    // programmatic stream serialization: the launch may overlap the end of
+    // the previous kernel; the kernel waits before its first global read
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_kernel<4>, p);
 }
 
 }  // namespace ep

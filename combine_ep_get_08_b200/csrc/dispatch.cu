@@ -682,8 +682,20 @@ cudaError_t launch_ll_dispatch(const DispatchParams &p_in, bool fp8, int num_sms
     p.n_token_units = p.T * p.splits;
     const int grid = persistent_grid(p.n_token_units, blocks_per_sm(k, kThreads, smem_max, slot), num_sms) +
                      (p.recv_count ? 1 : 0);
+    // programmatic stream serialization, as for the normal dispatch: the
+    // kernels wait (pdl_wait) before their first global read
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
     void *args[] = {&p};
-    return cudaLaunchKernel(k, dim3(grid), dim3(kThreads), args, smem, s);
+    return cudaLaunchKernelExC(&cfg, k, args);
 }
 
 // FP8 uses the register kernel: quantising from a staged ring with one
