@@ -110,8 +110,21 @@ __device__ bool grid_wait(const LayoutParams &p, int *s_flag) {
 
 __device__ __forceinline__ bool valid_expert(int64_t e, int E) { return e >= 0 && e < E; }
 
-// Brings the line holding *p (an in-bounds address) into L2; no register result.
-__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" : : "l"(p)); }
+// is_token_in_rank row of one token from its rank mask (R <= 64), four
+// bytes per store when the row is 4-byte aligned.
+__device__ __forceinline__ void write_in_rank_row(uint8_t *dst, int R, unsigned long long mask) {
+    if ((R & 3) == 0 && ((reinterpret_cast<uintptr_t>(dst) & 3) == 0)) {
+        for (int r = 0; r < R; r += 4) {
+            const unsigned int bits = (unsigned int)(mask >> r) & 0xfu;
+            const unsigned int word = (bits & 1u) | ((bits >> 1) & 1u) << 8 | ((bits >> 2) & 1u) << 16 |
+                                      ((bits >> 3) & 1u) << 24;
+            *reinterpret_cast<unsigned int *>(dst + r) = word;
+        }
+    } else {
+        for (int r = 0; r < R; ++r) dst[r] = (uint8_t)((mask >> r) & 1ull);
+    }
+}
+
 
 
 // Loads up to 8 consecutive expert ids of one token (all loads issued
@@ -479,6 +492,9 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
     int32_t *s_loff = s_eoff + (E + 1);             // [E+1] this CTA's rows: exclusive offsets per expert
     int32_t *s_er = s_loff + (E + 1);               // [steps][kLayoutThreads] pair: expert | rank << 16
     int32_t *s_qe = s_er + kClusterMaxPairs;        // [pairs] in this CTA's row order: pair | expert << 16
+    float *s_wp = reinterpret_cast<float *>(s_qe + kClusterMaxPairs);        // [pairs] weight, pair order
+    int16_t *s_ep = reinterpret_cast<int16_t *>(s_wp + kClusterMaxPairs);  // [pairs] expert (-1: none), pair order
+    int16_t *s_rk = s_ep + kClusterMaxPairs;                                // [E] rank of expert e
     __shared__ int32_t s_tmp[2 * (kLayoutWarps + 1)];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -491,22 +507,32 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
     const int steps = ppw / 32;
     const int w_lo = warp * ppw, w_hi = min(npairs, w_lo + ppw);          // this warp's local pairs
 
+    // every id and weight of this warp's range is requested before any is
+    // used; the shared-memory set-up runs while they are in flight
+    int64_t v_id[kClusterMaxSteps];
+    float v_w[kClusterMaxSteps];
+#pragma unroll
+    for (int j = 0; j < kClusterMaxSteps; ++j) {
+        const int i = w_lo + j * 32 + lane;
+        const bool in = j < steps && i < w_hi;
+        v_id[j] = in ? __ldg(p.topk_idx + p_begin + i) : (int64_t)-1;
+        v_w[j] = (in && p.topk_weights) ? __ldg(p.topk_weights + p_begin + i) : 0.0f;
+    }
     for (int i = tid; i < kLayoutWarps * ES; i += kLayoutThreads) s_cnt[i] = 0;
     for (int i = tid; i < ncols; i += kLayoutThreads) s_hist[i] = 0;
-    // the weights are read in row order at the end: bring them into L2 now
-    if (p.topk_weights && tid * 32 < npairs) prefetch_l2(p.topk_weights + p_begin + tid * 32);
-    // every id of this warp's range is requested before any is used
+    for (int e = tid; e < E; e += kLayoutThreads) s_rk[e] = (int16_t)(e / L);
 #pragma unroll
     for (int j = 0; j < kClusterMaxSteps; ++j) {
         if (j < steps) {
             const int i = w_lo + j * 32 + lane;
-            int e = -1;
-            if (i < w_hi) {
-                const int64_t v = __ldg(p.topk_idx + p_begin + i);
-                e = valid_expert(v, E) ? (int)v : -1;
-                if (e < 0 && v != -1) atomicOr(p.status, EP_DEV_BAD_EXPERT);   // -1: masked slot
-            }
+            const int64_t v = v_id[j];
+            const int e = valid_expert(v, E) ? (int)v : -1;
+            if (i < w_hi && e < 0 && v != -1) atomicOr(p.status, EP_DEV_BAD_EXPERT);   // -1: masked slot
             s_er[j * kLayoutThreads + tid] = e & 0xffff;
+            if (i < w_hi) {
+                s_ep[i] = (int16_t)e;
+                s_wp[i] = v_w[j];
+            }
         }
     }
     __syncthreads();
@@ -557,58 +583,70 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
         }
     }
     // distinct tokens per rank and is_token_in_rank rows, from the staged ids
-    for (int t = t_begin + tid; t < t_end; t += kLayoutThreads) {
-        const int i0 = (t - t_begin) * K;
-        if (R <= 64) {
-            unsigned long long mask = 0;
-            for (int k = 0; k < K; ++k) {
-                const int i = i0 + k, w = i / ppw, r = i - w * ppw;
-                const int e = cl_expert(s_er[(r >> 5) * kLayoutThreads + w * 32 + (r & 31)]);
-                if (e >= 0) mask |= 1ull << (e / L);
+    if (R <= 64 && K <= 32 && (K & (K - 1)) == 0) {
+        // a token's K pairs are K consecutive lanes of one warp: each lane
+        // contributes its pair's rank bit and a shuffle OR gives the token's mask
+        const int span = (npairs + 31) / 32 * 32;
+        for (int i = tid; i < span; i += kLayoutThreads) {
+            const int e = i < npairs ? s_ep[i] : -1;
+            const int r = e >= 0 ? s_rk[e] : -1;
+            unsigned int lo = (r >= 0 && r < 32) ? 1u << r : 0u;
+            unsigned int hi = r >= 32 ? 1u << (r - 32) : 0u;
+            for (int o = 1; o < K; o <<= 1) {
+                lo |= __shfl_xor_sync(0xffffffffu, lo, o);
+                hi |= __shfl_xor_sync(0xffffffffu, hi, o);
             }
-            for (unsigned long long m = mask; m; m &= m - 1) atomicAdd(&s_hist[E + __ffsll((long long)m) - 1], 1);
-            if (p.u_in_rank) {
-                uint8_t *dst = p.u_in_rank + (int64_t)t * R;
-                if ((R & 3) == 0 && ((reinterpret_cast<uintptr_t>(dst) & 3) == 0)) {
-                    for (int r = 0; r < R; r += 4) {
-                        const unsigned int bits = (unsigned int)(mask >> r) & 0xfu;
-                        const unsigned int word = (bits & 1u) | ((bits >> 1) & 1u) << 8 |
-                                                  ((bits >> 2) & 1u) << 16 | ((bits >> 3) & 1u) << 24;
-                        *reinterpret_cast<unsigned int *>(dst + r) = word;
+            if (i < npairs && i % K == 0) {
+                const int t = t_begin + i / K;
+                const unsigned long long mask = ((unsigned long long)hi << 32) | lo;
+                for (unsigned long long m = mask; m; m &= m - 1)
+                    atomicAdd(&s_hist[E + __ffsll((long long)m) - 1], 1);
+                if (p.u_in_rank) write_in_rank_row(p.u_in_rank + (int64_t)t * R, R, mask);
+            }
+        }
+    } else {
+        for (int t = t_begin + tid; t < t_end; t += kLayoutThreads) {
+            const int i0 = (t - t_begin) * K;
+            if (R <= 64) {
+                unsigned long long mask = 0;
+                for (int k = 0; k < K; ++k) {
+                    const int e = s_ep[i0 + k];
+                    if (e >= 0) mask |= 1ull << s_rk[e];
+                }
+                for (unsigned long long m = mask; m; m &= m - 1)
+                    atomicAdd(&s_hist[E + __ffsll((long long)m) - 1], 1);
+                if (p.u_in_rank) write_in_rank_row(p.u_in_rank + (int64_t)t * R, R, mask);
+            } else {
+                // more than 64 ranks: distinct ranks by pairwise comparison
+                uint8_t *dst = p.u_in_rank ? p.u_in_rank + (int64_t)t * R : nullptr;
+                if (dst)
+                    for (int r = 0; r < R; ++r) dst[r] = 0;
+                for (int k = 0; k < K; ++k) {
+                    const int e = s_ep[i0 + k];
+                    if (e < 0) continue;
+                    const int r = s_rk[e];
+                    bool dup = false;
+                    for (int k2 = 0; k2 < k; ++k2) {
+                        const int e2 = s_ep[i0 + k2];
+                        if (e2 >= 0 && s_rk[e2] == r) dup = true;
                     }
-                } else {
-                    for (int r = 0; r < R; ++r) dst[r] = (uint8_t)((mask >> r) & 1ull);
+                    if (!dup) atomicAdd(&s_hist[E + r], 1);
+                    if (dst) dst[r] = 1;
                 }
-            }
-        } else {
-            // more than 64 ranks: distinct ranks by pairwise comparison
-            uint8_t *dst = p.u_in_rank ? p.u_in_rank + (int64_t)t * R : nullptr;
-            if (dst)
-                for (int r = 0; r < R; ++r) dst[r] = 0;
-            for (int k = 0; k < K; ++k) {
-                const int i = i0 + k, w = i / ppw, rr = i - w * ppw;
-                const int e = cl_expert(s_er[(rr >> 5) * kLayoutThreads + w * 32 + (rr & 31)]);
-                if (e < 0) continue;
-                const int r = e / L;
-                bool dup = false;
-                for (int k2 = 0; k2 < k; ++k2) {
-                    const int i2 = i0 + k2, w2 = i2 / ppw, r2 = i2 - w2 * ppw;
-                    const int e2 = cl_expert(s_er[(r2 >> 5) * kLayoutThreads + w2 * 32 + (r2 & 31)]);
-                    if (e2 >= 0 && e2 / L == r) dup = true;
-                }
-                if (!dup) atomicAdd(&s_hist[E + r], 1);
-                if (dst) dst[r] = 1;
             }
         }
     }
     // every CTA's histogram complete and visible to the cluster
     cluster.sync();
     for (int j = tid; j < ncols; j += kLayoutThreads) {
+        int v[16];                                  // all remote reads in flight together
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) v[cc] = cc < C ? *cluster.map_shared_rank(s_hist + j, cc) : 0;
         int tot = 0, before = 0;
-        for (int cc = 0; cc < C; ++cc) {
-            const int v = *cluster.map_shared_rank(s_hist + j, cc);
-            tot += v;
-            before += cc < c ? v : 0;
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+            tot += v[cc];
+            before += cc < c ? v[cc] : 0;
         }
         s_tot[j] = tot;
         if (j < E) s_before[j] = before;
@@ -654,7 +692,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
         const int t = (int)(q / K);
         p.row_src[dst] = t;
         p.row_slot[dst] = (int)(q - (int64_t)t * K);
-        if (p.topk_weights) p.row_weight[dst] = __ldg(p.topk_weights + q);
+        if (p.topk_weights) p.row_weight[dst] = s_wp[i];
     }
     if (c == 0) {
         for (int e = tid; e < E; e += kLayoutThreads) {
@@ -689,7 +727,8 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
 
 size_t cluster_smem_bytes(int E, int R) {
     return sizeof(int32_t) * ((size_t)kLayoutWarps * (E + 1) + 2 * (size_t)(E + R) + E + 2 * (size_t)(E + 1) +
-                              2 * (size_t)kClusterMaxPairs);
+                              3 * (size_t)kClusterMaxPairs) +
+           sizeof(int16_t) * ((size_t)kClusterMaxPairs + E);
 }
 
 }  // namespace
