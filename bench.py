@@ -311,18 +311,19 @@ class Path:
         # lines behind for the next timed kernel to write back
         self.flush_sink = self.flush_buf.sum()
 
-    def layout(self, stream):
-        self.ep.ep_get_layout(self.h, self.idx, self.w, stream=stream)
+    def layout(self, stream, idx=None, w=None):
+        self.ep.ep_get_layout(self.h, self.idx if idx is None else idx, self.w if w is None else w, stream=stream)
 
-    def dispatch(self, stream, x=None):
+    def dispatch(self, stream, x=None, idx=None):
         x = self.x if x is None else x
         if self.wl.fp8:
             self.ep.ep_dispatch_fp8(self.h, x, self.recv, self.scales, stream=stream)
         else:
             self.ep.ep_dispatch(self.h, x, self.recv, stream=stream)
 
-    def combine(self, stream, out=None):
-        self.ep.ep_combine(self.h, self.y, self.w, self.out if out is None else out, stream=stream)
+    def combine(self, stream, out=None, w=None):
+        self.ep.ep_combine(self.h, self.y, self.w if w is None else w, self.out if out is None else out,
+                           stream=stream)
 
     def close(self):
         self.ep.ep_handle_destroy(self.h)
@@ -359,18 +360,20 @@ class LLPath(Path):
         self.flush_buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
         self.flush_sink = None
 
-    def layout(self, stream):
+    def layout(self, stream, idx=None, w=None):
         pass                                   # fused into the dispatch launch
 
-    def dispatch(self, stream, x=None):
+    def dispatch(self, stream, x=None, idx=None):
         x = self.x if x is None else x
+        idx = self.idx if idx is None else idx
         if self.wl.fp8:
-            self.ep.ep_ll_dispatch_fp8(self.h, self.idx, x, self.recv, self.scales, self.cnt, stream=stream)
+            self.ep.ep_ll_dispatch_fp8(self.h, idx, x, self.recv, self.scales, self.cnt, stream=stream)
         else:
-            self.ep.ep_ll_dispatch(self.h, self.idx, x, self.recv, self.cnt, stream=stream)
+            self.ep.ep_ll_dispatch(self.h, idx, x, self.recv, self.cnt, stream=stream)
 
-    def combine(self, stream, out=None):
-        self.ep.ep_ll_combine(self.h, self.y, self.w, self.out if out is None else out, stream=stream)
+    def combine(self, stream, out=None, w=None):
+        self.ep.ep_ll_combine(self.h, self.y, self.w if w is None else w, self.out if out is None else out,
+                              stream=stream)
 
 
 def run_cuda(args, world, rank, local):
@@ -533,44 +536,70 @@ def run_cuda(args, world, rank, local):
 
 
 def run_e2e(path, args, stream, reuse, world, dev, bytes_step):
-    """Host buffers in, host result out, through the same C-ABI calls."""
+    """Host buffers in, host result out, through the same C-ABI calls.
+
+    Every step copies its inputs (x, topk_idx, topk_weights) from pinned host
+    memory and its output back to pinned host memory.  Steps are independent,
+    so they are pipelined over two buffer slots: uploads on one stream,
+    kernels on the bench's stream, downloads on a third, ordered by events --
+    the kernels of step i overlap the upload of step i+1 and the download of
+    step i-1, and the two PCIe directions run at the same time."""
     import torch
     wl = path.wl
     x_h = wl.x.pin_memory()
     idx_h = wl.topk_idx.pin_memory()
     w_h = wl.topk_weights.pin_memory()
-    out_h = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
-    x_d = torch.empty_like(path.x)
+    out_h = [torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_d = [torch.empty_like(path.x) for _ in range(2)]
+    idx_d = [torch.empty_like(path.idx) for _ in range(2)]
+    w_d = [torch.empty_like(path.w) for _ in range(2)]
+    out_d = [torch.empty_like(path.out) for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in_ready", "in_free", "out_ready", "out_free")}
     sptr = stream.cuda_stream
-    n = max(3, min(args.steps, 20))
+    n = max(4, min(args.steps, 20))
 
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        path.idx.copy_(idx_h, non_blocking=True)
-        path.w.copy_(w_h, non_blocking=True)
-        path.layout(sptr)
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(ev["in_free"][b])
+            x_d[b].copy_(x_h, non_blocking=True)
+            idx_d[b].copy_(idx_h, non_blocking=True)
+            w_d[b].copy_(w_h, non_blocking=True)
+            ev["in_ready"][b].record(up)
+        stream.wait_event(ev["in_ready"][b])
+        if i >= 2:
+            stream.wait_event(ev["out_free"][b])
+        path.layout(sptr, idx=idx_d[b], w=w_d[b])
         for _ in range(reuse):
-            path.dispatch(sptr, x=x_d)
-            path.combine(sptr)
-        out_h.copy_(path.out, non_blocking=True)
+            path.dispatch(sptr, x=x_d[b], idx=idx_d[b])
+            path.combine(sptr, out=out_d[b], w=w_d[b])
+        ev["in_free"][b].record(stream)
+        ev["out_ready"][b].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev["out_ready"][b])
+            out_h[b].copy_(out_d[b], non_blocking=True)
+            ev["out_free"][b].record(down)
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(4):
+        e2e_step(i)
     torch.cuda.synchronize()
-    t = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
-    t[0].record(stream)
-    for _ in range(n):
-        e2e_step()
-    t[1].record(stream)
+    t0.record(up)
+    for i in range(n):
+        e2e_step(i)
+    t1.record(down)
     torch.cuda.synchronize()
-    ms = t[0].elapsed_time(t[1]) / n
+    ms = t0.elapsed_time(t1) / n
     ms = max_over_ranks(ms, world, dev)
     total = sum_over_ranks(bytes_step, world, dev)
     h2d = x_h.numel() * 2 + idx_h.numel() * 8 + w_h.numel() * 4
-    d2h = out_h.numel() * 2
+    d2h = out_h[0].numel() * 2
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelining": "two buffer slots; uploads, kernels and downloads on three streams"}
 
 
 # ----------------------------------------------------------------------------
