@@ -120,7 +120,6 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->sm_limit = 0;
     h->scale_layout = EP_SCALES_ROW_MAJOR;
     h->ll_M = 0;
-    h->layout_epoch = 0;
 
     auto fail = [&](int code) {
         delete h;
@@ -253,7 +252,6 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
     p.G = h->G;
     p.G_stride = (h->G + 3) / 4 * 4;
     p.tokens_per_chunk = h->tokens_per_chunk;
-    p.epoch = ++h->layout_epoch;
     p.pos = h->pos;
     p.row_src = h->row_src;
     p.row_slot = h->row_slot;
@@ -572,7 +570,6 @@ EP_API int ep_clear_status(ep_handle *h, ep_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     EP_CUDA(cudaMemsetAsync(h->status, 0, sizeof(unsigned int), s));
     EP_CUDA(cudaMemsetAsync(h->barrier, 0, sizeof(ep::GridBarrier), s));
-    h->layout_epoch = 0;
     return EP_OK;
 }
 

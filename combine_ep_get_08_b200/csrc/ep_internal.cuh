@@ -21,7 +21,8 @@ constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;
 
 struct GridBarrier {
     unsigned int count;          // arrivals so far (grows by G per layout launch)
-    unsigned int pad;
+    unsigned int epoch;          // completed grid-wide waits: advanced on the device, so a
+                                 // launch replayed from a CUDA graph finds its own target
 };
 
 // ---------------------------------------------------------------------------
@@ -35,7 +36,6 @@ struct LayoutParams {
     int G;                       // CTAs == chunks
     int G_stride;                // row stride of chunk_counts: G rounded up to 4
     int tokens_per_chunk;
-    unsigned int epoch;          // launch number on this handle (grid-wait target)
     // handle arrays
     int32_t *pos, *row_src, *row_slot;
     float *row_weight;
@@ -373,7 +373,6 @@ struct ep_handle {
     int sm_limit;                   // SMs dispatch / combine may occupy (0: all)
     int scale_layout;               // EP_SCALES_*
     int ll_M;                       // > 0: low-latency handle with ll_M slots per expert
-    unsigned int layout_epoch;      // layout launches since creation / ep_clear_status
     unsigned long long wait_limit_ns;
     int barrier_extra;
 };

@@ -439,12 +439,17 @@ bool make_map(CUtensorMap *map, const void *ptr, int64_t rows_total, int inner, 
 }  // namespace
 
 cudaError_t launch_gemm_combine(const GemmCombineArgs &g, int num_sms, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
+    // the kernel attribute belongs to each device's context: set it once per device
+    static int ready[64];
+    int dev = 0;
+    cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 != cudaSuccess) return e0;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE)) {
         const cudaError_t e = cudaFuncSetAttribute(gemm_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    (int)kGSmem);
         if (e != cudaSuccess) return e;
-        attr = true;
+        __atomic_store_n(&ready[dev], 1, __ATOMIC_RELEASE);
     }
     CUtensorMap map_a, map_b;
     if (!make_map(&map_a, g.act, g.cap, g.p.I, kGM) || !make_map(&map_b, g.w, (int64_t)g.p.E * g.p.N, g.p.I, kGN))

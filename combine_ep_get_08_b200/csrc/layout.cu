@@ -80,15 +80,20 @@ __device__ int block_exclusive_scan(int32_t *a, int n, int32_t *s_tmp /*[kLayout
 }
 
 // Grid-wide wait with a %globaltimer limit.  The arrival counter only grows:
-// launch number `epoch` (1, 2, ...) waits until it reaches epoch * G, so no
-// reset is needed between launches.  Returns false (and sets
-// EP_DEV_WAIT_TIMEOUT) if the other CTAs did not all arrive in time; the
-// caller then returns without touching memory again.
+// after `epoch` completed waits it holds epoch * G, and this wait ends when it
+// reaches (epoch + 1) * G, so no reset is needed between launches.  Each CTA
+// reads the epoch before it arrives, and CTA 0 advances it once every CTA has
+// arrived (so every CTA has read it): the target comes from the device, and a
+// launch replayed from a CUDA graph finds the right one.  Returns false (and
+// sets EP_DEV_WAIT_TIMEOUT) if the other CTAs did not all arrive in time; the
+// caller then returns without touching memory again (ep_clear_status resets
+// the counter and the epoch).
 __device__ bool grid_wait(const LayoutParams &p, int *s_flag) {
     __syncthreads();
     if (threadIdx.x == 0) {
         unsigned int *count = &p.barrier->count;
-        const unsigned int target = p.epoch * (unsigned int)(p.G + p.barrier_extra);
+        const unsigned int epoch = ld_acquire_u32(&p.barrier->epoch);
+        const unsigned int target = (epoch + 1) * (unsigned int)(p.G + p.barrier_extra);
         asm volatile("red.release.gpu.global.add.u32 [%0], 1;" : : "l"(count) : "memory");
         int ok = 1;
         if ((int)(ld_acquire_u32(count) - target) < 0) {
@@ -102,6 +107,7 @@ __device__ bool grid_wait(const LayoutParams &p, int *s_flag) {
             }
         }
         __threadfence();
+        if (ok && blockIdx.x == 0) atomicExch(&p.barrier->epoch, epoch + 1);
         *s_flag = ok;
     }
     __syncthreads();

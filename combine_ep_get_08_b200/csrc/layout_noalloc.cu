@@ -125,7 +125,6 @@ EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, 
     p.G = (int)G;
     p.G_stride = G_stride;
     p.tokens_per_chunk = tpc;
-    p.epoch = 1;   // the counter was just cleared: the wait targets G arrivals
     p.pos = pos;
     p.row_src = row_src;
     p.row_slot = row_slot;
