@@ -1,0 +1,68 @@
+"""The cross-GPU path of combine_ep_get_08_b200.dist through the CUDA kernels
+and NCCL, at the group size one GPU allows (world size 1: the all_to_all
+delivers every segment to this rank).  The exchange logic for several ranks
+is covered over gloo in test_dist_exchange.py.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import combine_ep_get_08_b200 as ep
+import oracle
+import workloads
+from ep_harness import combine_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from combine_ep_get_08_b200 import build_lib
+    build_lib.build()
+    oracle.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_dispatch_exchange_combine_nccl_one_rank():
+    import torch.distributed as dist
+
+    from combine_ep_get_08_b200 import dist as epd
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        wl = workloads.generate(None, T=512, H=1024, E=32, R=1, K=4, A=8, router="topk", seed=55)
+        cfg = ep.make_config(wl.T, wl.H, wl.E, 1, wl.K, wl.A)
+        h = ep.ep_handle_create(cfg)
+        try:
+            cap = ep.ep_capacity_rows(cfg)
+            x, idx, w = wl.x.to(dev), wl.topk_idx.to(dev), wl.topk_weights.to(dev)
+            send = torch.empty((cap, wl.H), dtype=torch.bfloat16, device=dev)
+            recv, plan = epd.dispatch(h, x, idx, w, send, cfg)
+            o = oracle.layout(wl.topk_idx.numpy(), wl.E, 1, wl.A)
+            assert plan.total_recv == o.rows and plan.total_send == o.rows
+            np.testing.assert_array_equal(plan.recv_expert_pairs.numpy().ravel(), o.num_tokens_per_expert)
+            np.testing.assert_array_equal(workloads.bf16_bits(recv),
+                                          oracle.dispatch_bf16(workloads.bf16_bits(wl.x), o.row_src))
+            y_send = torch.empty((cap, wl.H), dtype=torch.bfloat16, device=dev)
+            out = torch.empty_like(x)
+            epd.combine(h, recv, plan, w, out, y_send)        # identity experts
+            torch.cuda.synchronize()
+            x64 = (workloads.bf16_bits(wl.x).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            combine_close(out, x64 * wl.topk_weights.numpy().astype(np.float64).sum(1, keepdims=True))
+            assert ep.ep_get_status(h) == 0
+        finally:
+            ep.ep_handle_destroy(h)
+    finally:
+        dist.destroy_process_group()
