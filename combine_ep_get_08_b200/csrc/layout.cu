@@ -36,6 +36,11 @@
 
 #include "ep_internal.cuh"
 
+#ifndef EP_LAYOUT_TRIGGER_LATE
+#define EP_LAYOUT_TRIGGER_LATE 0   // 1: the cluster kernel lets a dependent launch start after its id
+                                   // loads (measured the same as at its start)
+#endif
+
 namespace ep {
 
 namespace {
@@ -504,7 +509,9 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
     __shared__ int32_t s_tmp[2 * (kLayoutWarps + 1)];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+#if !EP_LAYOUT_TRIGGER_LATE
     pdl_launch_dependents();   // a dispatch launched next may start its set-up now
+#endif
     const int t_begin = min(p.T, c * p.tokens_per_chunk);
     const int t_end = min(p.T, t_begin + p.tokens_per_chunk);
     const int64_t p_begin = (int64_t)t_begin * K;
@@ -541,6 +548,9 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
             }
         }
     }
+#if EP_LAYOUT_TRIGGER_LATE
+    pdl_launch_dependents();   // after this CTA's only DRAM reads
+#endif
     __syncthreads();
     int32_t *wrow = s_cnt + warp * ES;
 #pragma unroll 1
