@@ -21,12 +21,11 @@
 //              accumulate) from one thread; tcgen05.commit frees ring
 //              stages and hands finished accumulators to the epilogue;
 //   warps 2-5  epilogue, one warp per 32-lane quarter of TMEM (warp w reads
-//              lanes 32*(w%4)...): tcgen05.ld a row's columns, scale them
-//              by the pair's top-k weight,
-//              transpose each 32x32 chunk through shared memory and add it
-//              into an fp32 [T, N] accumulator with 16-byte vector atomics
-//              that cover 128 contiguous bytes per 8 lanes -- the combine,
-//              fused.  Padding rows add nothing.
+//              lanes 32*(w%4)...): tcgen05.ld a row's columns, scale them by
+//              the pair's top-k weight, transpose each 32x32 chunk through
+//              shared memory and add it into an fp32 [T, N] accumulator with
+//              16-byte vector atomics that cover 128 contiguous bytes per 8
+//              lanes -- the combine, fused.  Padding rows add nothing.
 // A second kernel rounds the fp32 accumulator to bf16.  Every wait on an
 // mbarrier is bounded; a timeout sets EP_DEV_WAIT_TIMEOUT, lets the copies
 // and MMAs in flight finish (bounded again), frees TMEM and returns.
@@ -39,20 +38,6 @@ namespace ep {
 
 namespace {
 
-#ifndef EP_GEMM_ORDER
-#define EP_GEMM_ORDER 1      // 1: tiles expert by expert, column block, row block; 0: row block, column block
-#endif
-#ifndef EP_GEMM_NGROUP
-#define EP_GEMM_NGROUP 0     // column blocks per pass over the experts (0: all of them)
-#endif
-#ifndef EP_GEMM_EPI
-#define EP_GEMM_EPI 0        // 0: thread vector atomics over transposed chunks; 1: a bulk reduce-add
-                             // (TMA engine) per 128-byte row chunk, measured 1% slower
-#endif
-#ifndef EP_GEMM_POLICY
-#define EP_GEMM_POLICY 0     // L2 hints on the TMA loads: 0 none; 1 W evict_first, act evict_last; 2 W evict_first
-#endif
-
 constexpr int kGM = 128;                              // rows per tile
 constexpr int kGN = 256;                              // output columns per tile
 constexpr int kGK = 64;                               // inner elements per stage: one 128-byte row
@@ -64,10 +49,7 @@ constexpr int kGEpiWarps = 4;                        // one per TMEM lane quarte
 constexpr int kGThreads = 64 + 32 * kGEpiWarps;
 constexpr int kGAcc = 2;                              // TMEM accumulators
 constexpr uint32_t kGTmemCols = kGAcc * kGN;          // 512: all of an SM's TMEM
-// one epilogue warp's 32x32 fp32 staging tile: transposed and swizzled for
-// thread atomics, or rows padded to 36 floats (16-byte aligned, no bank
-// conflicts) for bulk reductions
-constexpr uint32_t kGStageT = 32 * 36 * 4;
+constexpr uint32_t kGStageT = 32 * 32 * 4;           // one epilogue warp's 32x32 fp32 transpose tile
 constexpr size_t kGSmem = 1024 + kGStages * (size_t)(kGABytes + kGBBytes) + kGEpiWarps * kGStageT + 256;
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
@@ -85,15 +67,12 @@ __device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t saddr) {
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// 2-D tiled TMA load (no multicast) with an L2 eviction-priority policy.
-__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int x, int y, uint64_t *bar,
-                                            uint64_t policy) {
+// 2-D tiled TMA load into shared memory (no multicast), completing on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3}], [%4], %5;"
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         :
-        : "r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)),
-          "l"(policy)
+        : "r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -103,15 +82,6 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t 
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
         :
         : "r"(tmem_d), "l"(a), "l"(b), "r"(kGIdesc), "r"(accumulate));
-}
-
-// out[0 .. bytes/4) += src[...] in fp32, performed by the TMA engine in L2
-// (16-byte aligned addresses, bytes % 16 == 0; joins this thread's bulk group).
-__device__ __forceinline__ void bulk_reduce_add_f32(float *gdst, const float *ssrc, uint32_t bytes) {
-    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
-                 :
-                 : "l"(gdst), "r"(smem_u32(ssrc)), "r"(bytes)
-                 : "memory");
 }
 
 // Arrives once on `bar` when every tcgen05 operation this thread issued so far has completed.
@@ -138,13 +108,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" : : : "memory");
 }
 
-// Tiles are numbered by groups of column blocks (so that the fp32 output
-// columns being accumulated stay in L2), inside a group expert by expert,
-// inside an expert by column block and then by row block, so the CTAs
-// running side by side share one 256-column slice of W_e (read from DRAM
-// once, then from L2) and the expert's row blocks.  With mtot row blocks in
-// all, group gi starts at tile mtot * n0 (n0 = its first column block), and
-// expert e's tiles inside it at (eoff[e] / kGM) * (column blocks in group).
+// Tiles are numbered expert by expert; inside an expert by column block and
+// then by row block, so the CTAs running side by side share one 256-column
+// slice of W_e (read from DRAM once, then from L2) and the expert's row
+// blocks.  Expert e's tiles start at (eoff[e] / kGM) * n_blocks.
 struct GemmTile {
     int m;   // row block (global)
     int n;   // column block
@@ -152,32 +119,10 @@ struct GemmTile {
 };
 
 __device__ __forceinline__ GemmTile tile_coords(const int32_t *eoff, int E, int n_blocks, int t) {
-#if EP_GEMM_ORDER == 0
-    {
-        GemmTile g;
-        g.m = t / n_blocks;
-        g.n = t - g.m * n_blocks;
-        int lo = 0, hi = E - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(&eoff[mid]) <= g.m * kGM)
-                lo = mid;
-            else
-                hi = mid - 1;
-        }
-        g.e = lo;
-        return g;
-    }
-#endif
-    const int mtot = __ldg(&eoff[E]) / kGM;
-    const int ng = (EP_GEMM_NGROUP > 0 && EP_GEMM_NGROUP < n_blocks) ? EP_GEMM_NGROUP : n_blocks;
-    const int gi = t / (mtot * ng);
-    const int n0 = gi * ng, ngi = min(ng, n_blocks - n0);
-    const int lt = t - mtot * n0;
-    int lo = 0, hi = E - 1;   // largest e whose first tile in the group is <= lt
+    int lo = 0, hi = E - 1;   // largest e whose first tile is <= t
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(&eoff[mid]) / kGM * ngi <= lt)
+        if (__ldg(&eoff[mid]) / kGM * n_blocks <= t)
             lo = mid;
         else
             hi = mid - 1;
@@ -185,11 +130,11 @@ __device__ __forceinline__ GemmTile tile_coords(const int32_t *eoff, int E, int 
     // an empty expert shares its first tile with the next one, so lo is never empty
     const int m0 = __ldg(&eoff[lo]) / kGM;
     const int mb = __ldg(&eoff[lo + 1]) / kGM - m0;
-    const int local = lt - m0 * ngi;
+    const int local = t - m0 * n_blocks;
     GemmTile g;
     g.e = lo;
-    g.n = n0 + local / mb;
-    g.m = m0 + (local - (local / mb) * mb);
+    g.n = local / mb;
+    g.m = m0 + (local - g.n * mb);
     return g;
 }
 
@@ -244,17 +189,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // ---- TMA producer ----
         if (lane == 0) {
             int it = 0;
-            uint64_t pol_w, pol_a;
-#if EP_GEMM_POLICY >= 1
-            asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol_w));
-#else
-            asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol_w));
-#endif
-#if EP_GEMM_POLICY == 1
-            asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_a));
-#else
-            asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol_a));
-#endif
             for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
                 const GemmTile g = tile_coords(p.eoff, p.E, n_blocks, tile);
                 const int m = g.m, n = g.n, e = g.e;
@@ -266,8 +200,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&full[s], kGABytes + kGBBytes);
-                    tma_load_2d(sA + s * kGABytes, &map_a, kb * kGK, m * kGM, &full[s], pol_a);
-                    tma_load_2d(sB + s * kGBBytes, &map_b, kb * kGK, e * p.N + n * kGN, &full[s], pol_w);
+                    tma_load_2d(sA + s * kGABytes, &map_a, kb * kGK, m * kGM, &full[s]);
+                    tma_load_2d(sB + s * kGBBytes, &map_b, kb * kGK, e * p.N + n * kGN, &full[s]);
                 }
             }
             // on abort, let the loads already issued land before shared memory goes away
@@ -338,23 +272,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int src = __ldg(&p.row_src[r]);
             float wt = 0.0f;
             if (src >= 0) wt = __ldg(&p.topk_w[(int64_t)src * p.K + __ldg(&p.row_slot[r])]);
-#if EP_GEMM_EPI == 1
-            float *srow = sT + (warp - 2) * (kGStageT / 4) + lane * 36;   // this lane's staged row
-            float *orow = p.out_acc + (int64_t)(src >= 0 ? src : 0) * p.N + (int64_t)g.n * kGN;
-            for (int c = c_lo; c < c_hi; ++c) {
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kGN + c * 32), v);
-                bulk_wait_read<0>();                 // the previous chunk's reduction has read srow
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    *reinterpret_cast<float4 *>(srow + 4 * k) =
-                        make_float4(wt * __uint_as_float(v[4 * k]), wt * __uint_as_float(v[4 * k + 1]),
-                                    wt * __uint_as_float(v[4 * k + 2]), wt * __uint_as_float(v[4 * k + 3]));
-                fence_async_smem();                  // generic-proxy writes -> the bulk copy's reads
-                if (src >= 0) bulk_reduce_add_f32(orow + c * 32, srow, 32 * 4);
-                bulk_commit();
-            }
-#else
             const int sub = lane >> 3, k4 = lane & 7;  // reader: row i0 + sub, float4 k4 of the chunk
             for (int c = c_lo; c < c_hi; ++c) {
                 uint32_t v[32];
@@ -375,14 +292,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
                 __syncwarp();
             }
-#endif
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
         }
-#if EP_GEMM_EPI == 1
-        bulk_wait_all();                             // reductions done before shared memory goes away
-#endif
     }
     tc_fence_before();
     __syncthreads();
