@@ -9,16 +9,22 @@ group-limited top-8), bf16 dispatch + combine, identity experts (combine
 reads the dispatched rows).
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
-and torch.cuda.synchronize() on both sides.  Every kernel is timed with CUDA
-events on the stream it is launched on.  The 126 MB L2 is flushed (256 MiB
-write, outside the events) before each step and between dispatch and
-combine, where the expert GEMMs would run (a 256 MiB read: it leaves no dirty
-lines for the timed kernel to write back).  value = algorithmic bytes of
-dispatch + combine per step / device time of the step (layout + dispatch +
-combine), summed over ranks and divided by the max over ranks.
+and torch.cuda.synchronize() on both sides, timed with CUDA events on the
+stream the kernels are launched on.  The 126 MB L2 is flushed (a 256 MiB
+read, outside the events: it leaves no dirty lines for the timed kernel to
+write back) before each step and between dispatch and combine, where the
+expert GEMMs would run.  Layout and dispatch run back to back (the dispatch
+launch overlaps the layout's end) and are timed as one span; a separate pass
+with an event between them gives each kernel's own time for the breakdown
+and the roofline.  value = algorithmic bytes of dispatch + combine per step /
+device time of the step, summed over ranks and divided by the max over ranks.
+e2e: the same steps with their inputs uploaded from and outputs downloaded
+to pinned host memory, pipelined over two buffer slots.
 
 --impl reference times the CPU oracle (single thread) on a bounded sample of
-the same workload instead.  Multi-GPU (torchrun): every rank runs its own
+the same workload instead.  --expert-gemm times the expert GEMM with the
+fused combine (ep_expert_combine) in TFLOP/s.  --mode ll uses the
+low-latency static layout.  Multi-GPU (torchrun): every rank runs its own
 replica on its own GPU (independent batches, no collective on the data
 path); rank 0 prints one JSON line.
 """
