@@ -171,6 +171,14 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
                          int32_t *rank_offsets, ep_stream_t stream);
 
 /*
+ * Launch order.  ep_dispatch, ep_dispatch_fp8, ep_combine, ep_ll_dispatch,
+ * ep_ll_dispatch_fp8 and ep_ll_combine launch with programmatic stream
+ * serialization: the launch may begin while the previous kernel on the
+ * stream is still finishing, and the kernel waits for it (and for its writes
+ * to be visible) before it reads any global memory -- only its set-up and an
+ * L2 prefetch of its input run earlier.  Stream order is kept exactly as for
+ * an ordinary launch; the layout kernels let such a dependent start early.
+ *
  * bf16 dispatch: recv_x[pos[t,k], :] = x[t, :] for every pair, and zero
  * rows for the padding of each expert segment.  x is [T, H] bf16, recv_x is
  * [capacity, H] bf16; rows at or beyond `rows` are not written.  Uses the
