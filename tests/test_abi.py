@@ -75,3 +75,38 @@ def test_oracle_not_imported_by_product_path():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower(), f"{f} mentions the oracle"
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "ep.h"
+
+int main(void) {
+    ep_config c = {4096, 7168, 256, 8, 8, 128};
+    if (ep_validate_config(&c) != EP_OK) return 1;
+    if (ep_capacity_rows(&c) != 4096LL * 8 + 256LL * 127) return 2;
+    if (ep_scales_per_row(&c) != 56) return 3;
+    if (ep_scale_buffer_floats(&c, EP_SCALES_COL_MAJOR_TMA) != 56LL * ((ep_capacity_rows(&c) + 3) / 4 * 4)) return 4;
+    if (ep_ll_capacity_rows(&c, 4096) != 256LL * 4096) return 5;
+    if (ep_ll_capacity_rows(&c, 100) != EP_ERR_ARG) return 6;   /* fewer slots than tokens */
+    c.num_ranks = 7;
+    if (ep_validate_config(&c) != EP_ERR_ARG) return 7;
+    printf("ok %s\n", ep_status_string(EP_ERR_STATE));
+    return 0;
+}
+"""
+
+
+def test_header_is_c99_and_links(lib, tmp_path):
+    """A plain C99 program compiles against include/ep.h with warnings as
+    errors, links against libep_b200.so and runs its host-only calls."""
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(lib.LIB_PATH)
+    cmd = ["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+           str(src), "-o", str(exe), "-L", libdir, "-l:libep_b200.so", f"-Wl,-rpath,{libdir}"]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert r.stdout.startswith("ok ")
