@@ -42,7 +42,8 @@ struct CVec<4> {
 };
 
 template <int NW>
-__global__ void __launch_bounds__(kThreads) combine_kernel(CombineParams p) {
+// Four resident blocks per SM (62 registers, no spill); three measured 8% slower.
+__global__ void __launch_bounds__(kThreads, 4) combine_kernel(CombineParams p) {
     constexpr int VB = NW * 4;               // bytes per vector
     __shared__ int32_t s_src[kMaxTopk];
     __shared__ float s_w[kMaxTopk];
