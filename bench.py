@@ -670,6 +670,115 @@ EGEMM_DESC = ("one expert-parallel rank of a DeepSeek-V3 layer: 32 local experts
               "with the top-k weighted combine in the epilogue")
 
 
+def run_peer(args, world, rank, local):
+    """ep_dispatch_peer + ep_combine_peer on the named workload, its R
+    destination buffers all on this GPU (the addressing and store pattern of
+    the cross-GPU exchange, at this GPU's own bandwidth), timed beside
+    ep_dispatch + ep_combine on the same layout.  Layout is computed once,
+    outside the timed region."""
+    import numpy as np
+    import torch
+
+    import combine_ep_get_08_b200 as ep
+    import workloads
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    from combine_ep_get_08_b200 import build_lib
+    if rank == 0:
+        build_lib.build()
+    barrier(world)
+    base = workloads.CONFIGS[args.config]
+    if base["fp8"]:
+        base = dict(base, fp8=False)                  # the peer path moves bf16 rows
+    wl = workloads.generate(None, seed=base["seed"] + 1000 * rank,
+                            **{k: v for k, v in base.items() if k not in ("reuse", "seed")})
+    cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
+    h = ep.ep_handle_create(cfg)
+    if args.sm_limit:
+        ep.ep_set_sm_limit(h, args.sm_limit)
+    x, idx, tw = wl.x.to(dev), wl.topk_idx.to(dev), wl.topk_weights.to(dev)
+    roff = torch.empty(wl.R + 1, dtype=torch.int32, device=dev)
+    ep.ep_get_layout(h, idx, tw, rank_offsets=roff)
+    r = roff.cpu().numpy().astype(np.int64)
+    rows = int(r[-1])
+    seg = np.diff(r)
+    # destination d holds this source's block after R-1 other sources' blocks
+    # of the same size (row0 = (R-1) * seg[d]), as a balanced exchange would
+    row0 = (seg * (wl.R - 1)).astype(np.int32)
+    bufs = [torch.empty((int(seg[d] * wl.R) + 1, wl.H), dtype=torch.bfloat16, device=dev) for d in range(wl.R)]
+    bases = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device=dev)
+    row0_d = torch.from_numpy(row0).to(dev)
+    recv = torch.empty((max(ep.ep_capacity_rows(cfg), 1), wl.H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+    flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    cs = stream.cuda_stream
+    calls = {
+        "dispatch_peer": lambda: ep.ep_dispatch_peer(h, x, bases, row0_d, stream=cs),
+        "combine_peer": lambda: ep.ep_combine_peer(h, bases, row0_d, tw, out, stream=cs),
+        "dispatch": lambda: ep.ep_dispatch(h, x, recv, stream=cs),
+        "combine": lambda: ep.ep_combine(h, recv, tw, out, stream=cs),
+    }
+    for _ in range(args.warmup):
+        for f in calls.values():
+            f()
+    torch.cuda.synchronize()
+    ms = {k: [] for k in calls}
+    launches0 = ep.ep_launch_count()
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        for _ in range(args.steps):
+            for k, f in calls.items():
+                flush.sum()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                f()
+                e1.record(stream)
+                ms[k].append((e0, e1))
+        torch.cuda.synchronize()
+    barrier(world)
+    launches = ep.ep_launch_count() - launches0
+    us = {k: statistics.mean(a.elapsed_time(b) for a, b in v) * 1e3 for k, v in ms.items()}
+    b_dis = dispatch_bytes(wl.T, wl.H, wl.K, rows, False)
+    b_com = combine_bytes(wl.T, wl.H, wl.K)
+    peer_ms = sum(a.elapsed_time(b) for k in ("dispatch_peer", "combine_peer") for a, b in ms[k])
+    total_ms = max_over_ranks(peer_ms, world, dev)
+    all_bytes = sum_over_ranks((b_dis + b_com) * args.steps, world, dev)
+    peak, peak_src = measured_peak()
+    dom = "dispatch_peer" if us["dispatch_peer"] >= us["combine_peer"] else "combine_peer"
+    dom_bytes = b_dis if dom == "dispatch_peer" else b_com
+    status = ep.ep_get_status(h)
+    ep.ep_handle_destroy(h)
+    if rank == 0:
+        achieved = dom_bytes / (us[dom] * 1e-6) / 1e9
+        line = {
+            "metric": "peer dispatch + combine algorithmic GB/s", "unit": "GB/s",
+            "value": round(all_bytes / (total_ms * 1e-3) / 1e9, 1),
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workloads.DESCRIPTIONS[args.config] + " (bf16 rows)",
+                       "destinations": wl.R, "placement": "all destination buffers on this GPU",
+                       "rows": rows, "l2": "flushed (256 MiB read, outside the timed events) before each call"},
+            "kernels_us": {k: round(v, 2) for k, v in us.items()},
+            "peer_vs_local": {"dispatch": round(us["dispatch"] / us["dispatch_peer"], 3),
+                              "combine": round(us["combine"] / us["combine_peer"], 3)},
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                         "peak_source": peak_src, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": None},
+            "gpu_launches": int(launches), "clocks": sampler.summary(), "device_status": int(status),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def run_expert_gemm(args, world, rank, local):
     import numpy as np
     import torch
@@ -844,6 +953,8 @@ def main(argv=None):
                     help="layout: normal (padded, ep_get_layout) or low-latency static slots (ep_ll_*)")
     ap.add_argument("--ll-slots", type=int, default=0, help="slots per expert in --mode ll (0: T)")
     ap.add_argument("--ncu-ingest", metavar="REP", help="record DRAM traffic from an ncu report and exit")
+    ap.add_argument("--peer", action="store_true",
+                    help="time ep_dispatch_peer + ep_combine_peer (R destination buffers on this GPU)")
     ap.add_argument("--expert-gemm", action="store_true",
                     help="time ep_expert_combine (expert GEMM + fused combine) instead of the step")
     args = ap.parse_args(argv)
@@ -859,6 +970,8 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.expert_gemm:
         return run_expert_gemm(args, world, rank, local)
+    if args.peer:
+        return run_peer(args, world, rank, local)
     return run_cuda(args, world, rank, local)
 
 

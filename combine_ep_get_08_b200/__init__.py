@@ -19,6 +19,7 @@ LIB_PATH = os.environ.get("EP_B200_LIB", os.path.join(_HERE, "libep_b200.so"))
 EP_OK, EP_ERR_ARG, EP_ERR_CUDA, EP_ERR_UNSUPPORTED, EP_ERR_STATE, EP_ERR_DEVICE = 0, -1, -2, -3, -4, -5
 EP_DEV_BAD_EXPERT, EP_DEV_WAIT_TIMEOUT, EP_DEV_SLOT_OVERFLOW = 0x1, 0x2, 0x4
 EP_SCALES_ROW_MAJOR, EP_SCALES_COL_MAJOR_TMA = 0, 1
+EP_IPC_HANDLE_BYTES = 64
 
 
 class EpError(RuntimeError):
@@ -87,6 +88,11 @@ def _load():
             "ep_ll_dispatch": ([P] * 6, ctypes.c_int),
             "ep_ll_dispatch_fp8": ([P] * 7, ctypes.c_int),
             "ep_ll_combine": ([P] * 5, ctypes.c_int),
+            "ep_dispatch_peer": ([P] * 5, ctypes.c_int),
+            "ep_combine_peer": ([P] * 6, ctypes.c_int),
+            "ep_ipc_get_handle": ([P, P, ctypes.POINTER(I64)], ctypes.c_int),
+            "ep_ipc_open_handle": ([P, ctypes.POINTER(P)], ctypes.c_int),
+            "ep_ipc_close_handle": ([P], ctypes.c_int),
             "ep_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "ep_last_error": ([], ctypes.c_char_p),
             "ep_launch_count": ([], U64),
@@ -207,6 +213,38 @@ def ep_dispatch_fp8(h: int, x, recv_q, recv_scales, stream=None) -> None:
 
 def ep_combine(h: int, y, topk_weights, out, stream=None) -> None:
     _check("ep_combine", _load().ep_combine(h, _ptr(y), _ptr(topk_weights), _ptr(out), _stream(stream)))
+
+
+def ep_dispatch_peer(h: int, x, recv_bases, row0, stream=None) -> None:
+    """recv_bases: device int64 tensor of R buffer addresses; row0: device int32 [R]."""
+    _check("ep_dispatch_peer", _load().ep_dispatch_peer(h, _ptr(x), _ptr(recv_bases), _ptr(row0), _stream(stream)))
+
+
+def ep_combine_peer(h: int, y_bases, row0, topk_weights, out, stream=None) -> None:
+    _check("ep_combine_peer", _load().ep_combine_peer(h, _ptr(y_bases), _ptr(row0), _ptr(topk_weights), _ptr(out),
+                                                      _stream(stream)))
+
+
+def ep_ipc_get_handle(buf) -> tuple[bytes, int]:
+    """(handle bytes, byte offset of `buf` inside its allocation)."""
+    hd = ctypes.create_string_buffer(EP_IPC_HANDLE_BYTES)
+    off = ctypes.c_int64()
+    _check("ep_ipc_get_handle", _load().ep_ipc_get_handle(_ptr(buf), hd, ctypes.byref(off)))
+    return hd.raw, off.value
+
+
+def ep_ipc_open_handle(handle: bytes) -> int:
+    """Maps another process's allocation; returns its base address."""
+    if len(handle) != EP_IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {EP_IPC_HANDLE_BYTES} bytes, got {len(handle)}")
+    base = ctypes.c_void_p()
+    _check("ep_ipc_open_handle", _load().ep_ipc_open_handle(ctypes.create_string_buffer(handle, len(handle)),
+                                                            ctypes.byref(base)))
+    return base.value
+
+
+def ep_ipc_close_handle(base: int) -> None:
+    _check("ep_ipc_close_handle", _load().ep_ipc_close_handle(base))
 
 
 def ep_copy_routing(h: int, pos=None, row_src=None, row_slot=None, row_weight=None, stream=None) -> None:

@@ -8,7 +8,10 @@
 #include <cstring>
 #include <new>
 
+#include <cuda.h>
+
 #include "ep_internal.cuh"
+#include "peer.cuh"
 
 namespace {
 
@@ -404,6 +407,105 @@ EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner,
     cudaError_t e = ep::launch_gemm_combine(a, sms, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launch(expert_combine)");
     g_launches.fetch_add(2, std::memory_order_relaxed);
+    return EP_OK;
+}
+
+// ---- peer-memory exchange (one process per GPU) ----
+
+static int peer_common(const ep_handle *h, const void *x, const void *const *bases, const int32_t *row0,
+                       const float *topk_weights, void *out, bool combine, ep_stream_t stream) {
+    int rc = check_mode(h, false, true);
+    if (rc != EP_OK) return rc;
+    const ep_config &c = h->cfg;
+    if (c.num_tokens == 0) return EP_OK;
+    if (!bases || !row0 || !aligned(bases, 8) || !aligned(row0, 4)) return EP_ERR_ARG;
+    if (combine ? (!topk_weights || !out || !aligned(topk_weights, 4) || !aligned(out, 16))
+                : (!x || !aligned(x, 16)))
+        return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+
+    ep::PeerLaunch l{};
+    l.x = x;
+    l.base = const_cast<void *const *>(bases);
+    l.row0 = row0;
+    l.pos = h->pos;
+    l.row_src = h->row_src;
+    l.roff = h->roff;
+    l.w = topk_weights;
+    l.out = out;
+    l.T = c.num_tokens;
+    l.K = c.num_topk;
+    l.R = c.num_ranks;
+    l.H = c.hidden;
+    l.cap = h->cap;
+    l.zero_rows = c.expert_alignment > 1;
+    const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = combine ? ep::launch_combine_peer(l, sms, s) : ep::launch_dispatch_peer(l, sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, combine ? "launch(combine_peer)" : "launch(dispatch_peer)");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return EP_OK;
+}
+
+EP_API int ep_dispatch_peer(const ep_handle *h, const void *x, void *const *recv_bases, const int32_t *row0,
+                            ep_stream_t stream) {
+    return peer_common(h, x, const_cast<const void *const *>(recv_bases), row0, nullptr, nullptr, false, stream);
+}
+
+EP_API int ep_combine_peer(const ep_handle *h, const void *const *y_bases, const int32_t *row0,
+                           const float *topk_weights, void *out, ep_stream_t stream) {
+    return peer_common(h, nullptr, y_bases, row0, topk_weights, out, true, stream);
+}
+
+static_assert(sizeof(cudaIpcMemHandle_t) == EP_IPC_HANDLE_BYTES, "IPC handle size");
+
+// cuMemGetAddressRange through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*AddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+static AddressRangeFn address_range_fn() {
+    static AddressRangeFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<AddressRangeFn>(f);
+    }
+    return fn;
+}
+
+EP_API int ep_ipc_get_handle(const void *dev_ptr, void *handle, int64_t *offset) {
+    if (!dev_ptr || !handle || !offset) return EP_ERR_ARG;
+    AddressRangeFn range = address_range_fn();
+    if (!range) {
+        ep::record_error("cuMemGetAddressRange entry point unavailable");
+        return EP_ERR_UNSUPPORTED;
+    }
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS) return EP_ERR_ARG;
+    cudaIpcMemHandle_t hd;
+    cudaError_t e = cudaIpcGetMemHandle(&hd, reinterpret_cast<void *>(base));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaIpcGetMemHandle");
+    memcpy(handle, &hd, sizeof hd);
+    *offset = static_cast<int64_t>(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
+    return EP_OK;
+}
+
+EP_API int ep_ipc_open_handle(const void *handle, void **base) {
+    if (!handle || !base) return EP_ERR_ARG;
+    cudaIpcMemHandle_t hd;
+    memcpy(&hd, handle, sizeof hd);
+    cudaError_t e = cudaIpcOpenMemHandle(base, hd, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+    return EP_OK;
+}
+
+EP_API int ep_ipc_close_handle(void *base) {
+    if (!base) return EP_ERR_ARG;
+    cudaError_t e = cudaIpcCloseMemHandle(base);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaIpcCloseMemHandle");
     return EP_OK;
 }
 

@@ -27,6 +27,10 @@ gives the sizes).
 The functions take tensors on the group's device (CUDA with NCCL, CPU with
 gloo) and hold no arithmetic of their own: the rows are the dispatch
 kernel's output and the reduction is ep_combine.
+
+dispatch_peer / combine_peer (end of the file) do the same exchange inside
+the kernels: rows are stored straight into the other GPUs' buffers, mapped
+with CUDA IPC, so no send buffer and no all_to_all of rows remain.
 """
 from __future__ import annotations
 
@@ -140,4 +144,145 @@ def combine(h: int, y_recv: torch.Tensor, plan: ExchangePlan, topk_weights: torc
 
     return_rows(y_recv, plan, out=y_send, group=group)
     ep_combine(h, y_send, topk_weights, out, stream=stream)
+    return out
+
+
+# ---- the exchange inside the kernels: peer-memory dispatch / combine ----
+#
+# Instead of a send buffer plus all_to_all, ep_dispatch_peer stores every row
+# straight into the destination GPU's receive buffer (mapped into this process
+# with CUDA IPC), and ep_combine_peer reads the expert outputs back from the
+# destination GPUs.  The only collectives left are on the row counts (host
+# integers) and the barriers that order the ranks.
+
+
+@dataclass
+class PeerPlan:
+    world: int
+    send_rows: list      # rows this rank writes to each destination
+    recv_rows: list      # rows each source writes to this rank
+    row0: list           # first row of this rank's block in each destination's buffer
+    row0_dev: object     # the same as a device int32 tensor (for the kernels)
+
+    @property
+    def total_recv(self) -> int:
+        return int(sum(self.recv_rows))
+
+
+def peer_row0(send_rows, group=None, max_rows: int | None = None):
+    """Row starts of the peer exchange from every rank's send_rows.
+
+    Sources write their blocks into a destination's buffer in rank order, so
+    this rank's block in destination r starts after the rows of sources
+    0..me-1 bound for r.  One all_gather of the W counts; returns
+    (row0 [W], recv_rows [W]) as lists.  With max_rows, every rank checks that
+    no destination receives more rows than that (the same ValueError on every
+    rank, since all see the same counts)."""
+    import torch.distributed as dist
+
+    W = dist.get_world_size(group)
+    me = dist.get_rank(group)
+    mine = torch.as_tensor(send_rows, dtype=torch.int64).cpu().reshape(W)
+    backend = dist.get_backend(group)
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    parts = [torch.empty(W, dtype=torch.int64, device=dev) for _ in range(W)]
+    dist.all_gather(parts, mine.to(dev), group=group)
+    S = torch.stack([p.cpu() for p in parts])          # S[s, r]: rows source s sends to rank r
+    if max_rows is not None:
+        worst = int(S.sum(0).max())
+        if worst > max_rows:
+            raise ValueError(f"a rank would receive {worst} rows, more than the buffers' {max_rows}")
+    row0 = S[:me].sum(0)
+    return [int(v) for v in row0.tolist()], [int(v) for v in S[:, me].tolist()]
+
+
+class PeerBuffers:
+    """This rank's receive and expert-output buffers ([max_rows, H] bf16),
+    and every rank's, mapped here through CUDA IPC (device address tables
+    recv_bases / y_bases for the kernels).  Collective: every rank of the
+    group constructs it with the same sizes."""
+
+    def __init__(self, max_rows: int, hidden: int, group=None, device=None):
+        import torch.distributed as dist
+
+        from . import ep_ipc_get_handle, ep_ipc_open_handle
+
+        self.group = group
+        self.max_rows = int(max_rows)
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.recv = torch.zeros((max(self.max_rows, 1), hidden), dtype=torch.bfloat16, device=dev)
+        self.y = torch.zeros_like(self.recv)
+        mine = (ep_ipc_get_handle(self.recv), ep_ipc_get_handle(self.y))
+        W = dist.get_world_size(group)
+        me = dist.get_rank(group)
+        everyone = [None] * W
+        dist.all_gather_object(everyone, mine, group=group)
+        self._opened = {}                                  # handle bytes -> mapped base
+        recv_addr, y_addr = [], []
+        for r, pair in enumerate(everyone):
+            if r == me:
+                recv_addr.append(self.recv.data_ptr())
+                y_addr.append(self.y.data_ptr())
+                continue
+            for (hd, off), out in zip(pair, (recv_addr, y_addr)):
+                if hd not in self._opened:
+                    self._opened[hd] = ep_ipc_open_handle(hd)
+                out.append(self._opened[hd] + off)
+        self.recv_bases = torch.tensor(recv_addr, dtype=torch.int64, device=dev)
+        self.y_bases = torch.tensor(y_addr, dtype=torch.int64, device=dev)
+
+    def close(self) -> None:
+        """Unmaps the other ranks' buffers (after the last kernel that uses them)."""
+        from . import ep_ipc_close_handle
+
+        torch.cuda.synchronize()
+        for base in self._opened.values():
+            ep_ipc_close_handle(base)
+        self._opened = {}
+
+
+def _fence(group, stream) -> None:
+    """This rank's work so far is finished and every rank has reached here."""
+    import torch.distributed as dist
+
+    (stream if stream is not None else torch.cuda.current_stream()).synchronize()
+    dist.barrier(group=group)
+
+
+def dispatch_peer(h: int, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights, cfg, bufs: PeerBuffers,
+                  group=None, stream=None):
+    """Layout on this GPU, then the rows go straight into the destination
+    GPUs' receive buffers.  Returns (the rows this rank received, grouped by
+    source rank, as a view of bufs.recv; plan)."""
+    import torch.distributed as dist
+
+    from . import ep_dispatch_peer, ep_get_layout
+
+    W = dist.get_world_size(group)
+    if cfg.num_ranks != W:
+        raise ValueError("cfg.num_ranks must equal the process group's size")
+    roff = torch.empty((W + 1,), dtype=torch.int32, device=x.device)
+    ep_get_layout(h, topk_idx, topk_weights, None, None, None, None, roff, stream=stream)
+    r = roff.cpu()                                     # waits for the layout
+    send_rows = (r[1:] - r[:-1]).tolist()
+    row0, recv_rows = peer_row0(send_rows, group=group, max_rows=bufs.max_rows)
+    row0_dev = torch.tensor(row0, dtype=torch.int32, device=x.device)
+    plan = PeerPlan(world=W, send_rows=[int(v) for v in send_rows], recv_rows=recv_rows, row0=row0,
+                    row0_dev=row0_dev)
+    _fence(group, stream)                              # every destination is done with its last rows
+    ep_dispatch_peer(h, x, bufs.recv_bases, row0_dev, stream=stream)
+    _fence(group, stream)                              # every row has landed
+    return bufs.recv[:plan.total_recv], plan
+
+
+def combine_peer(h: int, plan: PeerPlan, topk_weights: torch.Tensor, out: torch.Tensor, bufs: PeerBuffers,
+                 group=None, stream=None) -> torch.Tensor:
+    """The expert outputs of this rank's received rows are in
+    bufs.y[:plan.total_recv] on every rank; reads this rank's rows back from
+    all of them and writes the weighted sum per token into `out`."""
+    from . import ep_combine_peer
+
+    _fence(group, stream)                              # every rank's expert outputs are complete
+    ep_combine_peer(h, bufs.y_bases, plan.row0_dev, topk_weights, out, stream=stream)
+    _fence(group, stream)                              # nobody overwrites y while it is read
     return out

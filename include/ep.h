@@ -345,6 +345,61 @@ EP_API int ep_ll_combine(const ep_handle *h, const void *y, const float *topk_we
 EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner, const void *w, int32_t n_out,
                              const float *topk_weights, float *out_acc, void *out, ep_stream_t stream);
 
+/*
+ * Peer-memory exchange between the GPUs of a node.  One process per GPU, R =
+ * the number of GPUs, rank r owning experts [r*L, (r+1)*L).  This is the
+ * exchange step of DeepEP's normal mode done inside the kernels: tokens
+ * travel over NVLink straight into the other GPUs' buffers
+ * ("blog.hotdry.top ... deepep-expert-parallel-alltoall", first section;
+ * "bowenzhou.top/repos/deepep/01-overview" section 1.3).
+ *
+ * With h's layout (num_ranks = R), the rows bound for rank r are the segment
+ * [rank_offsets[r], rank_offsets[r+1]).  Rank r's receive buffer holds the
+ * segments of all sources one after another (source order is the caller's
+ * choice); this source's block starts at row row0[r].  Row i of the segment
+ * goes to row row0[r] + i of rank r's buffer.
+ *
+ * ep_dispatch_peer writes each token row of x ([T, H] bf16) once per
+ * selected expert directly into the destination rank's buffer, and padding
+ * rows (expert_alignment > 1) as zeros.  The written bytes equal what
+ * ep_dispatch writes into segment r of a local buffer.  ep_combine_peer reads
+ * the expert-output rows from the same places (y_bases[r] has the row
+ * layout of rank r's receive buffer) and writes
+ *   out[t] = bf16_rn( sum_k topk_weights[t,k] * y[row of (t,k)] ),
+ * the ep_combine result.
+ *
+ * recv_bases / y_bases: DEVICE array of R device pointers (8-byte aligned
+ * array; each pointer 16-byte aligned), valid in this process: this GPU's own
+ * buffer for its rank, ep_ipc_open_handle results for the others.  row0:
+ * DEVICE array of R int32.  Each buffer must hold row0[r] + (rank_offsets[r+1]
+ * - rank_offsets[r]) rows of H bf16.  These contents are not checked on the
+ * host; a wrong value writes or reads outside the caller's buffers.  Null,
+ * misaligned or host-detectable errors return EP_ERR_ARG; a low-latency handle
+ * returns EP_ERR_STATE.  The calls issue plain loads and stores and never wait
+ * on another GPU.  The caller orders the ranks: every destination buffer is
+ * free before a dispatch starts, and every expert output is complete before a
+ * combine reads it (for example, a stream synchronise and a process-group
+ * barrier).
+ */
+EP_API int ep_dispatch_peer(const ep_handle *h, const void *x, void *const *recv_bases, const int32_t *row0,
+                            ep_stream_t stream);
+EP_API int ep_combine_peer(const ep_handle *h, const void *const *y_bases, const int32_t *row0,
+                           const float *topk_weights, void *out, ep_stream_t stream);
+
+/*
+ * CUDA IPC for those buffers.  ep_ipc_get_handle fills `handle`
+ * (EP_IPC_HANDLE_BYTES opaque bytes) for the allocation that contains
+ * dev_ptr and sets *offset to dev_ptr's byte offset inside it (allocators
+ * that sub-allocate return pointers inside a larger allocation).  In another
+ * process, ep_ipc_open_handle maps that allocation and returns its base;
+ * add the offset to reach dev_ptr.  ep_ipc_close_handle unmaps a base that
+ * ep_ipc_open_handle returned.  A process cannot open its own handles.
+ */
+#define EP_IPC_HANDLE_BYTES 64
+EP_API int ep_ipc_get_handle(const void *dev_ptr, void *handle, int64_t *offset);
+EP_API int ep_ipc_open_handle(const void *handle, void **base);
+EP_API int ep_ipc_close_handle(void *base);
+
 /* Synchronises `stream` and returns rows (= expert_offsets[E]) on the host. */
 EP_API int ep_get_num_rows(const ep_handle *h, int32_t *rows, ep_stream_t stream);
 

@@ -56,6 +56,15 @@ def test_host_only_calls(lib):
     with pytest.raises(lib.EpError):
         lib.ep_capacity_rows(bad[0])
     assert "invalid" in lib.ep_status_string(lib.EP_ERR_ARG)
+    # peer / IPC calls reject null arguments on the host, before any CUDA call
+    c = lib.library()
+    assert c.ep_dispatch_peer(None, None, None, None, None) == lib.EP_ERR_ARG
+    assert c.ep_combine_peer(None, None, None, None, None, None) == lib.EP_ERR_ARG
+    assert c.ep_ipc_get_handle(None, None, None) == lib.EP_ERR_ARG
+    assert c.ep_ipc_open_handle(None, None) == lib.EP_ERR_ARG
+    assert c.ep_ipc_close_handle(None) == lib.EP_ERR_ARG
+    with pytest.raises(ValueError):
+        lib.ep_ipc_open_handle(b"short")
     assert lib.ep_launch_count() == 0
 
 

@@ -88,3 +88,49 @@ def test_two_rank_exchange(tmp_path):
     for r in range(2):
         assert json.load(open(f"{out}.{r}")) == {"forward": True, "pairs": True, "rows_sum": True,
                                                  "reverse": True, "combine": True, "uneven": True}
+
+
+def _peer_rank_main(rank, world, port, out_path):
+    """peer_row0 over gloo: the blocks of all sources tile each destination's
+    rows in source order, with no gap and no overlap."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+
+    from combine_ep_get_08_b200 import dist as epd
+    oracle.build()
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    res = {}
+    try:
+        _, L, _, _ = _source(rank, world)
+        send = np.diff(L.rank_offsets).tolist()
+        row0, recv_rows = epd.peer_row0(send)
+        everyone = [None] * world
+        dist.all_gather_object(everyone, (send, row0, recv_rows))
+        ok = True
+        for r in range(world):
+            at = 0
+            for s in range(world):
+                s_send, s_row0, _ = everyone[s]
+                ok &= s_row0[r] == at                  # source s starts where s-1 ended
+                at += s_send[r]
+            ok &= sum(everyone[r][2]) == at            # rank r receives all of them
+            ok &= everyone[r][2] == [everyone[s][0][r] for s in range(world)]
+        res["tiling"] = bool(ok)
+        worst = max(sum(everyone[s][0][r] for s in range(world)) for r in range(world))
+        try:                                           # every rank raises the same error
+            epd.peer_row0(send, max_rows=worst - 1)
+            res["overflow"] = False
+        except ValueError:
+            res["overflow"] = True
+        epd.peer_row0(send, max_rows=worst)            # exactly enough rows is fine
+    finally:
+        dist.destroy_process_group()
+    with open(f"{out_path}.{rank}", "w") as f:
+        json.dump(res, f)
+
+
+def test_four_rank_peer_row0(tmp_path):
+    out = str(tmp_path / "peer")
+    mp.spawn(_peer_rank_main, args=(4, _free_port(), out), nprocs=4, join=True)
+    for r in range(4):
+        assert json.load(open(f"{out}.{r}")) == {"tiling": True, "overflow": True}
