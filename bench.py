@@ -176,7 +176,7 @@ def measured_peak():
 
 
 # the sources of the step's kernels (layout, dispatch, combine) and their shared header
-STEP_KERNEL_SOURCES = ("combine.cu", "dispatch.cu", "ep_internal.cuh", "layout.cu")
+STEP_KERNEL_SOURCES = ("combine.cu", "dispatch.cu", "ep_internal.cuh", "fp8_block.cuh", "layout.cu")
 
 
 def kernel_source_digest() -> str:
@@ -690,8 +690,7 @@ def run_peer(args, world, rank, local):
         build_lib.build()
     barrier(world)
     base = workloads.CONFIGS[args.config]
-    if base["fp8"]:
-        base = dict(base, fp8=False)                  # the peer path moves bf16 rows
+    fp8 = base["fp8"]
     wl = workloads.generate(None, seed=base["seed"] + 1000 * rank,
                             **{k: v for k, v in base.items() if k not in ("reuse", "seed")})
     cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
@@ -704,22 +703,39 @@ def run_peer(args, world, rank, local):
     r = roff.cpu().numpy().astype(np.int64)
     rows = int(r[-1])
     seg = np.diff(r)
-    # destination d holds this source's block after R-1 other sources' blocks
-    # of the same size (row0 = (R-1) * seg[d]), as a balanced exchange would
-    row0 = (seg * (wl.R - 1)).astype(np.int32)
-    bufs = [torch.empty((int(seg[d] * wl.R) + 1, wl.H), dtype=torch.bfloat16, device=dev) for d in range(wl.R)]
-    bases = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device=dev)
+    # destination d holds this source's block after another source's block of
+    # the same size (row0 = seg[d]): non-zero offsets, 2x the rows in memory
+    row0 = seg.astype(np.int32)
+    n_d = [int(2 * seg[d]) + 1 for d in range(wl.R)]
+    ybufs = [torch.empty((n, wl.H), dtype=torch.bfloat16, device=dev) for n in n_d]
+    y_bases = torch.tensor([b.data_ptr() for b in ybufs], dtype=torch.int64, device=dev)
     row0_d = torch.from_numpy(row0).to(dev)
-    recv = torch.empty((max(ep.ep_capacity_rows(cfg), 1), wl.H), dtype=torch.bfloat16, device=dev)
+    cap = max(ep.ep_capacity_rows(cfg), 1)
+    y_local = torch.empty((cap, wl.H), dtype=torch.bfloat16, device=dev)
     out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
     flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     cs = stream.cuda_stream
+    if fp8:
+        qbufs = [torch.empty((n, wl.H), dtype=torch.uint8, device=dev) for n in n_d]
+        sbufs = [torch.empty((n, wl.H // 128), dtype=torch.float32, device=dev) for n in n_d]
+        q_bases = torch.tensor([b.data_ptr() for b in qbufs], dtype=torch.int64, device=dev)
+        s_bases = torch.tensor([b.data_ptr() for b in sbufs], dtype=torch.int64, device=dev)
+        recv_q = torch.empty((cap, wl.H), dtype=torch.uint8, device=dev)
+        recv_s = torch.empty((cap, wl.H // 128), dtype=torch.float32, device=dev)
+        d_peer = lambda: ep.ep_dispatch_peer_fp8(h, x, q_bases, s_bases, row0_d, stream=cs)  # noqa: E731
+        d_local = lambda: ep.ep_dispatch_fp8(h, x, recv_q, recv_s, stream=cs)  # noqa: E731
+    else:
+        rbufs = [torch.empty((n, wl.H), dtype=torch.bfloat16, device=dev) for n in n_d]
+        r_bases = torch.tensor([b.data_ptr() for b in rbufs], dtype=torch.int64, device=dev)
+        recv = torch.empty((cap, wl.H), dtype=torch.bfloat16, device=dev)
+        d_peer = lambda: ep.ep_dispatch_peer(h, x, r_bases, row0_d, stream=cs)  # noqa: E731
+        d_local = lambda: ep.ep_dispatch(h, x, recv, stream=cs)  # noqa: E731
     calls = {
-        "dispatch_peer": lambda: ep.ep_dispatch_peer(h, x, bases, row0_d, stream=cs),
-        "combine_peer": lambda: ep.ep_combine_peer(h, bases, row0_d, tw, out, stream=cs),
-        "dispatch": lambda: ep.ep_dispatch(h, x, recv, stream=cs),
-        "combine": lambda: ep.ep_combine(h, recv, tw, out, stream=cs),
+        "dispatch_peer": d_peer,
+        "combine_peer": lambda: ep.ep_combine_peer(h, y_bases, row0_d, tw, out, stream=cs),
+        "dispatch": d_local,
+        "combine": lambda: ep.ep_combine(h, y_local, tw, out, stream=cs),
     }
     for _ in range(args.warmup):
         for f in calls.values():
@@ -743,7 +759,7 @@ def run_peer(args, world, rank, local):
     barrier(world)
     launches = ep.ep_launch_count() - launches0
     us = {k: statistics.mean(a.elapsed_time(b) for a, b in v) * 1e3 for k, v in ms.items()}
-    b_dis = dispatch_bytes(wl.T, wl.H, wl.K, rows, False)
+    b_dis = dispatch_bytes(wl.T, wl.H, wl.K, rows, fp8)
     b_com = combine_bytes(wl.T, wl.H, wl.K)
     peer_ms = sum(a.elapsed_time(b) for k in ("dispatch_peer", "combine_peer") for a, b in ms[k])
     total_ms = max_over_ranks(peer_ms, world, dev)
@@ -760,8 +776,8 @@ def run_peer(args, world, rank, local):
             "value": round(all_bytes / (total_ms * 1e-3) / 1e9, 1),
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workloads.DESCRIPTIONS[args.config] + " (bf16 rows)",
+            "vs_baseline": None, "dtype": "e4m3+bf16" if fp8 else "bf16", "data": "synthetic",
+            "config": {"workload": workloads.DESCRIPTIONS[args.config], "name": args.config,
                        "destinations": wl.R, "placement": "all destination buffers on this GPU",
                        "rows": rows, "l2": "flushed (256 MiB read, outside the timed events) before each call"},
             "kernels_us": {k: round(v, 2) for k, v in us.items()},

@@ -89,6 +89,7 @@ def _load():
             "ep_ll_dispatch_fp8": ([P] * 7, ctypes.c_int),
             "ep_ll_combine": ([P] * 5, ctypes.c_int),
             "ep_dispatch_peer": ([P] * 5, ctypes.c_int),
+            "ep_dispatch_peer_fp8": ([P] * 6, ctypes.c_int),
             "ep_combine_peer": ([P] * 6, ctypes.c_int),
             "ep_ipc_get_handle": ([P, P, ctypes.POINTER(I64)], ctypes.c_int),
             "ep_ipc_open_handle": ([P, ctypes.POINTER(P)], ctypes.c_int),
@@ -218,6 +219,12 @@ def ep_combine(h: int, y, topk_weights, out, stream=None) -> None:
 def ep_dispatch_peer(h: int, x, recv_bases, row0, stream=None) -> None:
     """recv_bases: device int64 tensor of R buffer addresses; row0: device int32 [R]."""
     _check("ep_dispatch_peer", _load().ep_dispatch_peer(h, _ptr(x), _ptr(recv_bases), _ptr(row0), _stream(stream)))
+
+
+def ep_dispatch_peer_fp8(h: int, x, recv_bases, scale_bases, row0, stream=None) -> None:
+    """recv_bases / scale_bases: device int64 tensors of R code / scale buffer addresses."""
+    _check("ep_dispatch_peer_fp8", _load().ep_dispatch_peer_fp8(h, _ptr(x), _ptr(recv_bases), _ptr(scale_bases),
+                                                                _ptr(row0), _stream(stream)))
 
 
 def ep_combine_peer(h: int, y_bases, row0, topk_weights, out, stream=None) -> None:

@@ -17,9 +17,9 @@
 // 32-byte (sm_100 256-bit) vector loads and stores when rows and pointers
 // allow, else 16-byte ones; a bulk-copy (TMA engine) variant measured no
 // faster on this write-bound pattern.
-#include <cuda_fp8.h>
 
 #include "ep_internal.cuh"
+#include "fp8_block.cuh"
 
 namespace ep {
 
@@ -446,15 +446,6 @@ __global__ void __launch_bounds__(kStagedThreads, 1) dispatch_bf16_staged_kernel
     }
 }
 
-// Two floats -> two E4M3 codes (round to nearest even, saturate to +-448),
-// first argument in the low byte.
-__device__ __forceinline__ unsigned int e4m3x2(float a, float b) {
-    return (unsigned int)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-}
-
-// EPT bf16 elements per thread (16: 16-byte accesses, 32: 32-byte accesses);
-// TPB = 128 / EPT consecutive lanes share one 1x128 block and reduce its
-// amax with shuffles.  Each thread stores EPT code bytes per received row.
 // Index of the scale of received row `row`, block b, in either layout.
 // Column-major scales come in groups of scale_group_rows rows (the whole
 // buffer, or one expert's M slots), each group [H/128][scale_ld].
@@ -464,37 +455,9 @@ __device__ __forceinline__ int64_t scale_index(const DispatchParams &p, int row,
     return ((int64_t)g * NB + b) * p.scale_ld + (row - g * p.scale_group_rows);
 }
 
-template <int EPT>
-struct Fp8Io;
-template <>
-struct Fp8Io<16> {
-    static __device__ __forceinline__ void load(const uint8_t *src, unsigned int (&w)[8]) {
-        const uint4 a = ld_stream_v4(src), b = ld_stream_v4(src + 16);
-        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-    }
-    static __device__ __forceinline__ void store(uint8_t *dst, const unsigned int (&q)[8]) {
-        st_v4(dst, make_uint4(q[0], q[1], q[2], q[3]));
-    }
-};
-template <>
-struct Fp8Io<32> {
-    static __device__ __forceinline__ void load(const uint8_t *src, unsigned int (&w)[16]) {
-        const u32x8 a = ld_stream_v8(src), b = ld_stream_v8(src + 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            w[i] = a.v[i];
-            w[8 + i] = b.v[i];
-        }
-    }
-    static __device__ __forceinline__ void store(uint8_t *dst, const unsigned int (&q)[8]) {
-        u32x8 v;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v.v[i] = q[i];
-        st_v8(dst, v);
-    }
-};
-
+// EPT bf16 elements per thread (16: 16-byte accesses, 32: 32-byte accesses);
+// TPB = 128 / EPT consecutive lanes share one 1x128 block and reduce its
+// amax with shuffles.  Each thread stores EPT code bytes per received row.
 template <int EPT, bool LL>
 __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p) {
     constexpr int TPB = 128 / EPT;
@@ -552,19 +515,8 @@ __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p
                         for (int i = 0; i < NW; ++i) w[i] = 0;
                     }
                 }
-                float amax = 0.0f;
-#pragma unroll
-                for (int i = 0; i < NW; ++i) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
-#pragma unroll
-                for (int o = TPB / 2; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                const float a = fmaxf(amax, 1e-4f);
-                const float inv = 448.0f / a;    // IEEE round-to-nearest divide
-                const float scale = a / 448.0f;
                 unsigned int q[8];
-#pragma unroll
-                for (int i = 0; i < NW / 2; ++i)
-                    q[i] = e4m3x2(bf16_lo(w[2 * i]) * inv, bf16_hi(w[2 * i]) * inv) |
-                           (e4m3x2(bf16_lo(w[2 * i + 1]) * inv, bf16_hi(w[2 * i + 1]) * inv) << 16);
+                const float scale = quantize_block<TPB, NW>(w, q);
                 if (act) {
                     const int b = g / TPB;
                     const bool lead = (g % TPB) == 0;

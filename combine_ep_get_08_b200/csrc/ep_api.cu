@@ -412,15 +412,21 @@ EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner,
 
 // ---- peer-memory exchange (one process per GPU) ----
 
-static int peer_common(const ep_handle *h, const void *x, const void *const *bases, const int32_t *row0,
-                       const float *topk_weights, void *out, bool combine, ep_stream_t stream) {
+enum class PeerOp { kDispatch, kDispatchFp8, kCombine };
+
+static int peer_common(const ep_handle *h, PeerOp op, const void *x, const void *const *bases,
+                       float *const *scale_bases, const int32_t *row0, const float *topk_weights, void *out,
+                       ep_stream_t stream) {
     int rc = check_mode(h, false, true);
     if (rc != EP_OK) return rc;
     const ep_config &c = h->cfg;
+    if (op == PeerOp::kDispatchFp8 && (c.hidden % 128 != 0 || !scale_bases || !aligned(scale_bases, 8)))
+        return EP_ERR_ARG;
+    if (op == PeerOp::kDispatchFp8 && h->scale_layout != EP_SCALES_ROW_MAJOR) return EP_ERR_UNSUPPORTED;
     if (c.num_tokens == 0) return EP_OK;
     if (!bases || !row0 || !aligned(bases, 8) || !aligned(row0, 4)) return EP_ERR_ARG;
-    if (combine ? (!topk_weights || !out || !aligned(topk_weights, 4) || !aligned(out, 16))
-                : (!x || !aligned(x, 16)))
+    if (op == PeerOp::kCombine ? (!topk_weights || !out || !aligned(topk_weights, 4) || !aligned(out, 16))
+                               : (!x || !aligned(x, 16)))
         return EP_ERR_ARG;
     DeviceGuard g(h->device);
     if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
@@ -428,6 +434,7 @@ static int peer_common(const ep_handle *h, const void *x, const void *const *bas
     ep::PeerLaunch l{};
     l.x = x;
     l.base = const_cast<void *const *>(bases);
+    l.sbase = scale_bases;
     l.row0 = row0;
     l.pos = h->pos;
     l.row_src = h->row_src;
@@ -442,20 +449,36 @@ static int peer_common(const ep_handle *h, const void *x, const void *const *bas
     l.zero_rows = c.expert_alignment > 1;
     const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = combine ? ep::launch_combine_peer(l, sms, s) : ep::launch_dispatch_peer(l, sms, s);
-    if (e != cudaSuccess) return cuda_fail(e, combine ? "launch(combine_peer)" : "launch(dispatch_peer)");
+    cudaError_t e;
+    const char *what;
+    switch (op) {
+        case PeerOp::kDispatch: e = ep::launch_dispatch_peer(l, sms, s); what = "launch(dispatch_peer)"; break;
+        case PeerOp::kDispatchFp8:
+            e = ep::launch_dispatch_fp8_peer(l, sms, s);
+            what = "launch(dispatch_fp8_peer)";
+            break;
+        default: e = ep::launch_combine_peer(l, sms, s); what = "launch(combine_peer)"; break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, what);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return EP_OK;
 }
 
 EP_API int ep_dispatch_peer(const ep_handle *h, const void *x, void *const *recv_bases, const int32_t *row0,
                             ep_stream_t stream) {
-    return peer_common(h, x, const_cast<const void *const *>(recv_bases), row0, nullptr, nullptr, false, stream);
+    return peer_common(h, PeerOp::kDispatch, x, const_cast<const void *const *>(recv_bases), nullptr, row0,
+                       nullptr, nullptr, stream);
+}
+
+EP_API int ep_dispatch_peer_fp8(const ep_handle *h, const void *x, void *const *recv_bases,
+                                float *const *scale_bases, const int32_t *row0, ep_stream_t stream) {
+    return peer_common(h, PeerOp::kDispatchFp8, x, const_cast<const void *const *>(recv_bases), scale_bases, row0,
+                       nullptr, nullptr, stream);
 }
 
 EP_API int ep_combine_peer(const ep_handle *h, const void *const *y_bases, const int32_t *row0,
                            const float *topk_weights, void *out, ep_stream_t stream) {
-    return peer_common(h, nullptr, y_bases, row0, topk_weights, out, true, stream);
+    return peer_common(h, PeerOp::kCombine, nullptr, y_bases, nullptr, row0, topk_weights, out, stream);
 }
 
 static_assert(sizeof(cudaIpcMemHandle_t) == EP_IPC_HANDLE_BYTES, "IPC handle size");

@@ -20,6 +20,7 @@
 // multicast, no wait on another GPU (the caller orders the ranks on the host).
 #include <cuda_bf16.h>
 
+#include "fp8_block.cuh"
 #include "peer.cuh"
 
 namespace ep {
@@ -37,6 +38,7 @@ __device__ __forceinline__ unsigned int pack_bf16x2(float lo, float hi) {
 struct PeerParams {
     const uint8_t *x;              // [T, H] bf16 (dispatch)
     uint8_t *const *base;          // [R] receive / expert-output buffers
+    float *const *sbase;           // [R] scale buffers (FP8 dispatch), else null
     const int32_t *row0;           // [R] first row of this source's block in each
     const int32_t *pos;            // [T, K]
     const int32_t *row_src;        // [cap]
@@ -47,9 +49,11 @@ struct PeerParams {
     int splits;                    // column ranges per token
 };
 
-// Per-rank addressing, staged in shared memory once per CTA.
+// Per-rank addressing, staged in shared memory once per CTA (layout of
+// peer_smem_bytes: R row-buffer bases, R scale-buffer bases, row0, roff).
 struct PeerTable {
     uint8_t **base;                // [R]
+    float **sbase;                 // [R] (FP8 dispatch)
     int32_t *row0;                 // [R]
     int32_t *roff;                 // [R+1]
 };
@@ -57,10 +61,12 @@ struct PeerTable {
 __device__ __forceinline__ PeerTable load_table(const PeerParams &p, unsigned char *smem) {
     PeerTable t;
     t.base = reinterpret_cast<uint8_t **>(smem);
-    t.row0 = reinterpret_cast<int32_t *>(smem + sizeof(void *) * p.R);
+    t.sbase = reinterpret_cast<float **>(smem + sizeof(void *) * p.R);
+    t.row0 = reinterpret_cast<int32_t *>(smem + 2 * sizeof(void *) * p.R);
     t.roff = t.row0 + p.R;
     for (int i = threadIdx.x; i < p.R; i += blockDim.x) {
         t.base[i] = p.base[i];
+        t.sbase[i] = p.sbase ? p.sbase[i] : nullptr;
         t.row0[i] = __ldg(&p.row0[i]);
     }
     for (int i = threadIdx.x; i <= p.R; i += blockDim.x) t.roff[i] = __ldg(&p.roff[i]);
@@ -82,10 +88,21 @@ __device__ __forceinline__ int rank_of_row(const int32_t *roff, int R, int row) 
     return lo;
 }
 
+// Where this rank's received row `row` lives: destination rank and row index there.
+struct PeerSlot {
+    int r;
+    int row;
+};
+
+__device__ __forceinline__ PeerSlot peer_slot(const PeerTable &t, int R, int row) {
+    const int r = rank_of_row(t.roff, R, row);
+    return PeerSlot{r, t.row0[r] + row - t.roff[r]};
+}
+
 // Address of this rank's received row `row` in its destination's buffer.
 __device__ __forceinline__ uint8_t *peer_row(const PeerTable &t, int R, int row, int row_bytes) {
-    const int r = rank_of_row(t.roff, R, row);
-    return t.base[r] + (int64_t)(t.row0[r] + row - t.roff[r]) * row_bytes;
+    const PeerSlot sl = peer_slot(t, R, row);
+    return t.base[sl.r] + (int64_t)sl.row * row_bytes;
 }
 
 // Units [0, T*splits): one column range of one token to its K rows;
@@ -120,6 +137,78 @@ __global__ void __launch_bounds__(kPThreads) dispatch_peer_kernel(PeerParams p, 
                 if (__ldg(&p.row_src[r]) >= 0) continue;
                 uint8_t *o = peer_row(tab, p.R, r, row_bytes);
                 for (int v = threadIdx.x; v < nv; v += kPThreads) st_v4(o + (int64_t)v * 16, make_uint4(0, 0, 0, 0));
+            }
+        }
+    }
+}
+
+// FP8 dispatch into peer buffers: one token per unit; 8 lanes quantise one
+// 1x128 block (16 elements each, 16-byte stores), then store its codes and,
+// from the block's first lane, its scale into each of the K destination rows.
+// Units after the tokens: padding rows (codes 0, scales 0).
+__global__ void __launch_bounds__(kPThreads) dispatch_fp8_peer_kernel(PeerParams p, int n_zero_units) {
+    constexpr int EPT = 16, TPB = 128 / EPT, NW = EPT / 2;
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ uint8_t *s_dst[kMaxTopk];
+    __shared__ float *s_sc[kMaxTopk];
+    const PeerTable tab = load_table(p, smem);
+    const int NB = p.H / 128, nthr_row = p.H / EPT;
+    const int rows = tab.roff[p.R];
+    for (int u = blockIdx.x; u < p.T + n_zero_units; u += gridDim.x) {
+        if (u < p.T) {
+            const uint8_t *xr = p.x + (int64_t)u * p.H * 2;
+            unsigned int w[NW];
+            if (threadIdx.x < nthr_row) {
+                Fp8Io<EPT>::load(xr + (int64_t)threadIdx.x * EPT * 2, w);
+            } else {
+#pragma unroll
+                for (int i = 0; i < NW; ++i) w[i] = 0;
+            }
+            if (threadIdx.x < p.K) {
+                const int d = __ldg(&p.pos[(int64_t)u * p.K + threadIdx.x]);
+                if (d >= 0) {
+                    const PeerSlot sl = peer_slot(tab, p.R, d);
+                    s_dst[threadIdx.x] = tab.base[sl.r] + (int64_t)sl.row * p.H;
+                    s_sc[threadIdx.x] = tab.sbase[sl.r] + (int64_t)sl.row * NB;
+                } else {
+                    s_dst[threadIdx.x] = nullptr;
+                    s_sc[threadIdx.x] = nullptr;
+                }
+            }
+            __syncthreads();
+            for (int g0 = 0; g0 < nthr_row; g0 += kPThreads) {      // uniform trip count: every lane shuffles
+                const int g = g0 + threadIdx.x;
+                const bool act = g < nthr_row;
+                if (g0 > 0) {
+                    if (act) {
+                        Fp8Io<EPT>::load(xr + (int64_t)g * EPT * 2, w);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < NW; ++i) w[i] = 0;
+                    }
+                }
+                unsigned int q[8];
+                const float scale = quantize_block<TPB, NW>(w, q);
+                if (act) {
+                    const int b = g / TPB;
+                    const bool lead = (g % TPB) == 0;
+                    for (int k = 0; k < p.K; ++k) {
+                        if (!s_dst[k]) continue;
+                        Fp8Io<EPT>::store(s_dst[k] + (int64_t)g * EPT, q);
+                        if (lead) s_sc[k][b] = scale;
+                    }
+                }
+            }
+            __syncthreads();
+        } else {
+            const int r0 = (u - p.T) * kZeroRowsPerUnit, r1 = min(rows, r0 + kZeroRowsPerUnit);
+            for (int r = r0; r < r1; ++r) {
+                if (__ldg(&p.row_src[r]) >= 0) continue;
+                const PeerSlot sl = peer_slot(tab, p.R, r);
+                uint8_t *o = tab.base[sl.r] + (int64_t)sl.row * p.H;
+                float *sc = tab.sbase[sl.r] + (int64_t)sl.row * NB;
+                for (int v = threadIdx.x; v < p.H / 16; v += kPThreads) st_v4(o + (int64_t)v * 16, make_uint4(0, 0, 0, 0));
+                for (int b = threadIdx.x; b < NB; b += kPThreads) sc[b] = 0.0f;
             }
         }
     }
@@ -199,6 +288,26 @@ cudaError_t launch_dispatch_peer(const PeerLaunch &l, int num_sms, cudaStream_t 
     const int units = p.T * p.splits + n_zero;
     const int grid = units < 4 * num_sms ? units : 4 * num_sms;
     dispatch_peer_kernel<<<grid, kPThreads, peer_smem_bytes(l.R), s>>>(p, n_zero);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_fp8_peer(const PeerLaunch &l, int num_sms, cudaStream_t s) {
+    PeerParams p{};
+    p.x = static_cast<const uint8_t *>(l.x);
+    p.base = reinterpret_cast<uint8_t *const *>(l.base);
+    p.sbase = l.sbase;
+    p.row0 = l.row0;
+    p.pos = l.pos;
+    p.row_src = l.row_src;
+    p.roff = l.roff;
+    p.T = l.T;
+    p.K = l.K;
+    p.R = l.R;
+    p.H = l.H;
+    const int n_zero = l.zero_rows ? (int)((l.cap + kZeroRowsPerUnit - 1) / kZeroRowsPerUnit) : 0;
+    const int units = p.T + n_zero;
+    const int grid = units < 4 * num_sms ? units : 4 * num_sms;
+    dispatch_fp8_peer_kernel<<<grid, kPThreads, peer_smem_bytes(l.R), s>>>(p, n_zero);
     return cudaGetLastError();
 }
 

@@ -8,6 +8,7 @@ namespace ep {
 struct PeerLaunch {
     const void *x;            // [T, H] bf16 (dispatch)
     void *const *base;        // device array [R]: each rank's row buffer, mapped here
+    float *const *sbase;      // device array [R]: each rank's scale buffer (FP8 dispatch), else null
     const int32_t *row0;      // device array [R]: first row of this source's block there
     const int32_t *pos;       // [T, K] this rank's layout
     const int32_t *row_src;   // [cap]
@@ -20,9 +21,10 @@ struct PeerLaunch {
 };
 
 cudaError_t launch_dispatch_peer(const PeerLaunch &l, int num_sms, cudaStream_t s);
+cudaError_t launch_dispatch_fp8_peer(const PeerLaunch &l, int num_sms, cudaStream_t s);
 cudaError_t launch_combine_peer(const PeerLaunch &l, int num_sms, cudaStream_t s);
 
 // Bytes of dynamic shared memory the peer kernels take for R ranks.
-inline size_t peer_smem_bytes(int R) { return sizeof(void *) * R + sizeof(int32_t) * (2 * R + 1); }
+inline size_t peer_smem_bytes(int R) { return 2 * sizeof(void *) * R + sizeof(int32_t) * (2 * R + 1); }
 
 }  // namespace ep

@@ -197,39 +197,47 @@ def peer_row0(send_rows, group=None, max_rows: int | None = None):
 
 
 class PeerBuffers:
-    """This rank's receive and expert-output buffers ([max_rows, H] bf16),
-    and every rank's, mapped here through CUDA IPC (device address tables
-    recv_bases / y_bases for the kernels).  Collective: every rank of the
-    group constructs it with the same sizes."""
+    """This rank's receive buffer ([max_rows, H] bf16, or E4M3 codes
+    [max_rows, H] uint8 plus fp32 scales [max_rows, H/128] with fp8=True) and
+    expert-output buffer ([max_rows, H] bf16), and every rank's, mapped here
+    through CUDA IPC (device address tables recv_bases, scale_bases and
+    y_bases for the kernels).  Collective: every rank of the group constructs
+    it with the same arguments."""
 
-    def __init__(self, max_rows: int, hidden: int, group=None, device=None):
+    def __init__(self, max_rows: int, hidden: int, group=None, device=None, fp8: bool = False):
         import torch.distributed as dist
 
         from . import ep_ipc_get_handle, ep_ipc_open_handle
 
+        if fp8 and hidden % 128:
+            raise ValueError("FP8 rows need hidden % 128 == 0")
         self.group = group
+        self.fp8 = fp8
         self.max_rows = int(max_rows)
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-        self.recv = torch.zeros((max(self.max_rows, 1), hidden), dtype=torch.bfloat16, device=dev)
-        self.y = torch.zeros_like(self.recv)
-        mine = (ep_ipc_get_handle(self.recv), ep_ipc_get_handle(self.y))
+        n = max(self.max_rows, 1)
+        self.recv = torch.zeros((n, hidden), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
+        self.recv_scales = torch.zeros((n, hidden // 128), dtype=torch.float32, device=dev) if fp8 else None
+        self.y = torch.zeros((n, hidden), dtype=torch.bfloat16, device=dev)
+        local = [self.recv, self.y] + ([self.recv_scales] if fp8 else [])
+        mine = [ep_ipc_get_handle(t) for t in local]
         W = dist.get_world_size(group)
         me = dist.get_rank(group)
         everyone = [None] * W
         dist.all_gather_object(everyone, mine, group=group)
         self._opened = {}                                  # handle bytes -> mapped base
-        recv_addr, y_addr = [], []
-        for r, pair in enumerate(everyone):
-            if r == me:
-                recv_addr.append(self.recv.data_ptr())
-                y_addr.append(self.y.data_ptr())
-                continue
-            for (hd, off), out in zip(pair, (recv_addr, y_addr)):
+        addr = [[] for _ in local]                         # per buffer kind, per rank
+        for r, handles in enumerate(everyone):
+            for i, (hd, off) in enumerate(handles):
+                if r == me:
+                    addr[i].append(local[i].data_ptr())
+                    continue
                 if hd not in self._opened:
                     self._opened[hd] = ep_ipc_open_handle(hd)
-                out.append(self._opened[hd] + off)
-        self.recv_bases = torch.tensor(recv_addr, dtype=torch.int64, device=dev)
-        self.y_bases = torch.tensor(y_addr, dtype=torch.int64, device=dev)
+                addr[i].append(self._opened[hd] + off)
+        table = [torch.tensor(a, dtype=torch.int64, device=dev) for a in addr]
+        self.recv_bases, self.y_bases = table[0], table[1]
+        self.scale_bases = table[2] if fp8 else None
 
     def close(self) -> None:
         """Unmaps the other ranks' buffers (after the last kernel that uses them)."""
@@ -252,11 +260,12 @@ def _fence(group, stream) -> None:
 def dispatch_peer(h: int, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights, cfg, bufs: PeerBuffers,
                   group=None, stream=None):
     """Layout on this GPU, then the rows go straight into the destination
-    GPUs' receive buffers.  Returns (the rows this rank received, grouped by
-    source rank, as a view of bufs.recv; plan)."""
+    GPUs' receive buffers (E4M3 codes and scales if bufs.fp8).  Returns (the
+    rows this rank received, grouped by source rank -- a view of bufs.recv,
+    or (codes, scales) views with FP8 -- and the plan)."""
     import torch.distributed as dist
 
-    from . import ep_dispatch_peer, ep_get_layout
+    from . import ep_dispatch_peer, ep_dispatch_peer_fp8, ep_get_layout
 
     W = dist.get_world_size(group)
     if cfg.num_ranks != W:
@@ -270,9 +279,15 @@ def dispatch_peer(h: int, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights,
     plan = PeerPlan(world=W, send_rows=[int(v) for v in send_rows], recv_rows=recv_rows, row0=row0,
                     row0_dev=row0_dev)
     _fence(group, stream)                              # every destination is done with its last rows
-    ep_dispatch_peer(h, x, bufs.recv_bases, row0_dev, stream=stream)
+    if bufs.fp8:
+        ep_dispatch_peer_fp8(h, x, bufs.recv_bases, bufs.scale_bases, row0_dev, stream=stream)
+    else:
+        ep_dispatch_peer(h, x, bufs.recv_bases, row0_dev, stream=stream)
     _fence(group, stream)                              # every row has landed
-    return bufs.recv[:plan.total_recv], plan
+    n = plan.total_recv
+    if bufs.fp8:
+        return (bufs.recv[:n], bufs.recv_scales[:n]), plan
+    return bufs.recv[:n], plan
 
 
 def combine_peer(h: int, plan: PeerPlan, topk_weights: torch.Tensor, out: torch.Tensor, bufs: PeerBuffers,

@@ -383,6 +383,18 @@ EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner,
  */
 EP_API int ep_dispatch_peer(const ep_handle *h, const void *x, void *const *recv_bases, const int32_t *row0,
                             ep_stream_t stream);
+
+/*
+ * FP8 form of ep_dispatch_peer: each destination receives E4M3 codes
+ * (recv_bases[r]: [rows, H] bytes) and fp32 scales (scale_bases[r]: DEVICE
+ * array of R pointers, each to [rows, H/128] floats, row-major, 4-byte
+ * aligned), the bytes ep_dispatch_fp8 writes into segment r of a local
+ * buffer; padding rows get codes 0 and scales 0.  Needs H % 128 == 0 (else
+ * EP_ERR_ARG) and the handle's row-major scale layout (else
+ * EP_ERR_UNSUPPORTED).  Combine takes bf16 expert outputs, as ep_combine_peer.
+ */
+EP_API int ep_dispatch_peer_fp8(const ep_handle *h, const void *x, void *const *recv_bases,
+                                float *const *scale_bases, const int32_t *row0, ep_stream_t stream);
 EP_API int ep_combine_peer(const ep_handle *h, const void *const *y_bases, const int32_t *row0,
                            const float *topk_weights, void *out, ep_stream_t stream);
 

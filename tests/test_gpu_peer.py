@@ -4,7 +4,8 @@ CPU oracle, with W ranks' buffers on one GPU and one handle per source rank.
 Every source s routes its own tokens over all E experts (num_ranks = W).
 Destination r's buffer must hold, for s = 0..W-1 in order, exactly the rows
 the oracle lays out for rank r from source s, starting at row0_s[r] =
-rows that sources 0..s-1 send to r; rows past them stay untouched.  The peer
+rows that sources 0..s-1 send to r; rows past them stay untouched.  The FP8
+form must write the oracle's E4M3 codes and fp32 scales the same way.  The peer
 combine, reading stand-in expert outputs from the W buffers, must equal the
 oracle's weighted sum within the combine tolerance, and ep_combine on the
 same rows gathered into one local buffer bit for bit (same fp32 order).
@@ -42,7 +43,7 @@ def _sources(W, T, H, E, K, A, router, seed, idx_edit=None):
     return out
 
 
-def run_peer(W, T, H, E, K, A, router="topk", seed=500, idx_edit=None):
+def run_peer(W, T, H, E, K, A, router="topk", seed=500, idx_edit=None, fp8=False):
     dev = torch.device("cuda")
     wls = _sources(W, T, H, E, K, A, router, seed, idx_edit)
     orc = [oracle.layout(wl.topk_idx.numpy(), E, W, A, topk_weights=wl.topk_weights.numpy()) for wl in wls]
@@ -59,23 +60,46 @@ def run_peer(W, T, H, E, K, A, router="topk", seed=500, idx_edit=None):
             roff = torch.empty(W + 1, dtype=torch.int32, device=dev)
             ep.ep_get_layout(h, wl.topk_idx.to(dev), wl.topk_weights.to(dev), rank_offsets=roff)
             np.testing.assert_array_equal(roff.cpu().numpy(), orc[len(handles) - 1].rank_offsets)
-        recv = [torch.full((max_rows, H), SENTINEL, dtype=torch.int16, device=dev).view(torch.bfloat16)
-                for _ in range(W)]
-        bases = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device=dev)
         row0_d = [torch.from_numpy(row0[s].astype(np.int32)).to(dev) for s in range(W)]
-        for s, (h, wl) in enumerate(zip(handles, wls)):
-            ep.ep_dispatch_peer(h, wl.x.to(dev), bases, row0_d[s])
-        torch.cuda.synchronize()
-        # destination r: the blocks of sources 0..W-1 in order, then untouched rows
-        rows_of = [oracle.dispatch_bf16(workloads.bf16_bits(wl.x), o.row_src) for wl, o in zip(wls, orc)]
-        for r in range(W):
-            want = np.concatenate([rows_of[s][orc[s].rank_offsets[r]:orc[s].rank_offsets[r + 1]]
-                                   for s in range(W)] + [np.zeros((0, H), np.uint16)])
-            got = workloads.bf16_bits(recv[r])
-            n = int(recv_total[r])
-            assert n == want.shape[0]
-            np.testing.assert_array_equal(got[:n], want, err_msg=f"rows received by rank {r}")
-            assert bool((recv[r][n:].view(torch.int16) == SENTINEL).all()), f"rank {r}: rows past the blocks"
+        xb = [workloads.bf16_bits(wl.x) for wl in wls]
+        if fp8:
+            codes = [torch.full((max_rows, H), 0x5A, dtype=torch.uint8, device=dev) for _ in range(W)]
+            scales = [torch.full((max_rows, H // 128), -3.0, dtype=torch.float32, device=dev) for _ in range(W)]
+            bases = torch.tensor([t.data_ptr() for t in codes], dtype=torch.int64, device=dev)
+            sbases = torch.tensor([t.data_ptr() for t in scales], dtype=torch.int64, device=dev)
+            for s, (h, wl) in enumerate(zip(handles, wls)):
+                ep.ep_dispatch_peer_fp8(h, wl.x.to(dev), bases, sbases, row0_d[s])
+            torch.cuda.synchronize()
+            ref = [oracle.dispatch_fp8(xb[s], orc[s].row_src) for s in range(W)]
+            for r in range(W):
+                n = int(recv_total[r])
+                segs = [(orc[s].rank_offsets[r], orc[s].rank_offsets[r + 1]) for s in range(W)]
+                want_q = np.concatenate([ref[s][0][a:b] for s, (a, b) in enumerate(segs)] + [np.zeros((0, H), np.uint8)])
+                want_s = np.concatenate([ref[s][1][a:b] for s, (a, b) in enumerate(segs)]
+                                        + [np.zeros((0, H // 128), np.float32)])
+                np.testing.assert_array_equal(codes[r][:n].cpu().numpy(), want_q, err_msg=f"codes at rank {r}")
+                np.testing.assert_array_equal(scales[r][:n].cpu().numpy().view(np.uint32), want_s.view(np.uint32),
+                                              err_msg=f"scales at rank {r}")
+                assert bool((codes[r][n:] == 0x5A).all()) and bool((scales[r][n:] == -3.0).all())
+            del codes, scales
+        else:
+            recv = [torch.full((max_rows, H), SENTINEL, dtype=torch.int16, device=dev).view(torch.bfloat16)
+                    for _ in range(W)]
+            bases = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device=dev)
+            for s, (h, wl) in enumerate(zip(handles, wls)):
+                ep.ep_dispatch_peer(h, wl.x.to(dev), bases, row0_d[s])
+            torch.cuda.synchronize()
+            # destination r: the blocks of sources 0..W-1 in order, then untouched rows
+            rows_of = [oracle.dispatch_bf16(xb[s], orc[s].row_src) for s in range(W)]
+            for r in range(W):
+                want = np.concatenate([rows_of[s][orc[s].rank_offsets[r]:orc[s].rank_offsets[r + 1]]
+                                       for s in range(W)] + [np.zeros((0, H), np.uint16)])
+                got = workloads.bf16_bits(recv[r])
+                n = int(recv_total[r])
+                assert n == want.shape[0]
+                np.testing.assert_array_equal(got[:n], want, err_msg=f"rows received by rank {r}")
+                assert bool((recv[r][n:].view(torch.int16) == SENTINEL).all()), f"rank {r}: rows past the blocks"
+            del recv
         # combine: stand-in expert outputs in every rank's buffer (seeded N(0,1))
         gen = torch.Generator(device=dev)
         gen.manual_seed(seed + 1)
@@ -113,8 +137,11 @@ CASES = [
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"W{c['W']}T{c['T']}H{c['H']}E{c['E']}K{c['K']}A{c['A']}")
-def test_peer_parity(case):
-    run_peer(**case)
+@pytest.mark.parametrize("fp8", [False, True])
+def test_peer_parity(case, fp8):
+    if fp8 and case["H"] % 128:
+        pytest.skip("FP8 needs H % 128 == 0")
+    run_peer(**case, fp8=fp8)
 
 
 def test_peer_empty_segments_and_masked_slots():
@@ -139,6 +166,7 @@ def test_peer_empty_segments_and_masked_slots():
         return idx
 
     run_peer(W, 120, 256, E, 3, 2, router="topk", seed=510, idx_edit=dedup)
+    run_peer(W, 120, 256, E, 3, 2, router="topk", seed=510, idx_edit=dedup, fp8=True)
 
 
 def test_peer_argument_errors():
@@ -161,6 +189,9 @@ def test_peer_argument_errors():
         assert e.value.code == ep.EP_ERR_ARG
         with pytest.raises(ep.EpError) as e:
             ep.ep_combine_peer(h, bases, row0, None, buf)
+        assert e.value.code == ep.EP_ERR_ARG
+        with pytest.raises(ep.EpError) as e:             # FP8 needs H % 128 == 0
+            ep.ep_dispatch_peer_fp8(h, wl.x.to(dev), bases, bases, row0)
         assert e.value.code == ep.EP_ERR_ARG
     finally:
         ep.ep_handle_destroy(h)

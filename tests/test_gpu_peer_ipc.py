@@ -8,7 +8,8 @@ Both processes share one GPU here; the kernels never wait on each other
 program a node with one GPU per rank runs.  Checks: each rank receives,
 source by source, exactly the rows the oracle lays out for it (bit for bit);
 with experts that double their rows (exact in bf16), each rank's combine
-matches the oracle's weighted sum of its own doubled rows.
+matches the oracle's weighted sum of its own doubled rows; the FP8 dispatch
+delivers the oracle's codes and scales the same way.
 """
 import json
 import os
@@ -77,6 +78,21 @@ def _rank_main(rank, port, out_path):
         ref = oracle.combine(_double_bits(rows), o.pos, wl.topk_weights.numpy())
         got = out.float().cpu().numpy().astype(np.float64)
         res["combine"] = bool(np.allclose(got, ref, rtol=1e-2, atol=1e-3))
+        # the FP8 form into a second set of mapped buffers: codes and scales
+        fbufs = epd.PeerBuffers(max_rows=W * (T * K + E * (A - 1)), hidden=H, fp8=True)
+        try:
+            (q, sc), plan8 = epd.dispatch_peer(h, wl.x.to(dev), wl.topk_idx.to(dev), wl.topk_weights.to(dev),
+                                               ep.make_config(T, H, E, W, K, A), fbufs)
+            ref = [oracle.dispatch_fp8(workloads.bf16_bits(wl_s.x), os_.row_src) for wl_s, os_, _ in srcs]
+            a = [(os_.rank_offsets[rank], os_.rank_offsets[rank + 1]) for _, os_, _ in srcs]
+            want_q = np.concatenate([rq[0][lo:hi] for rq, (lo, hi) in zip(ref, a)])
+            want_s = np.concatenate([rq[1][lo:hi] for rq, (lo, hi) in zip(ref, a)])
+            res["fp8"] = bool(np.array_equal(q.cpu().numpy(), want_q)) and \
+                bool(np.array_equal(sc.cpu().numpy().view(np.uint32), want_s.view(np.uint32))) and \
+                plan8.recv_rows == plan.recv_rows
+        finally:
+            dist.barrier()
+            fbufs.close()
         res["status"] = ep.ep_get_status(h)
     finally:
         if h is not None:
@@ -98,4 +114,5 @@ def test_two_process_peer_exchange(tmp_path):
     out = str(tmp_path / "res")
     mp.spawn(_rank_main, args=(_free_port(), out), nprocs=W, join=True)
     for r in range(W):
-        assert json.load(open(f"{out}.{r}")) == {"forward": True, "recv_rows": True, "combine": True, "status": 0}
+        assert json.load(open(f"{out}.{r}")) == {"forward": True, "recv_rows": True, "combine": True, "fp8": True,
+                                                 "status": 0}
