@@ -262,7 +262,8 @@ def run_reference(args, world, rank):
         "config": {"workload": workloads.DESCRIPTIONS[args.config], "sample_tokens": sample_T},
         "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": f"each step: oracle layout + dispatch + combine over the first "
-                                   f"{sample_T} of {wl.T} tokens of the workload (single thread)"},
+                                   f"{sample_T} of {wl.T} tokens of the workload (single thread)",
+                         "host": host_cpu()},
         "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -523,6 +524,8 @@ def run_cuda(args, world, rank, local):
             },
             "us_per_call": {k: round(v, 2) for k, v in kern.items()},
             "us_layout_then_dispatch": round(ld_us, 2),
+            "us_p10_p50_p90": {k: pct(v) for k, v in (("layout_then_dispatch", ld_ms), ("layout", lay_ms),
+                                                       ("dispatch", dis_ms), ("combine", com_ms))},
             "bytes_per_call": {"dispatch": b_dis, "combine": b_com},
             "gbs_per_call": {"dispatch": round(b_dis / dis_us / 1e3, 1),
                              "combine": round(b_com / com_us / 1e3, 1)},
@@ -542,12 +545,35 @@ def run_cuda(args, world, rank, local):
             line["cpu_baseline"] = {
                 "value": round(gbs, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
                 "sample": f"{n} full step(s) of the same workload (layout + dispatch + combine, "
-                          f"{el:.1f} s, single thread)"}
+                          f"{el:.1f} s, single thread)", "host": host_cpu()}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def pct(ms_list) -> list:
+    """10th, 50th and 90th percentile of event times in ms, as µs."""
+    v = sorted(ms_list)
+    if not v:
+        return [None, None, None]
+    at = lambda q: v[min(len(v) - 1, int(round(q * (len(v) - 1))))]  # noqa: E731
+    return [round(at(q) * 1e3, 2) for q in (0.1, 0.5, 0.9)]
+
+
+def host_cpu() -> dict:
+    """The host the oracle baseline ran on: CPU model and logical CPUs."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
 
 
 def run_graph(path, one_step, args, stream, reuse, world, dev, bytes_step):
@@ -889,7 +915,8 @@ def run_expert_gemm(args, world, rank, local):
             el = time.perf_counter() - t0
             line["cpu_baseline"] = {
                 "value": round(2.0 * wl.K * N * I * n_tok / el / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
-                "kind": "oracle", "sample": f"{n_tok} token(s) of the same workload ({el:.1f} s, single thread, fp64)"}
+                "kind": "oracle", "sample": f"{n_tok} token(s) of the same workload ({el:.1f} s, single thread, fp64)",
+                "host": host_cpu()}
         print(json.dumps(line), flush=True)
     ep.ep_handle_destroy(h)
     if world > 1:
