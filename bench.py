@@ -682,9 +682,38 @@ def run_e2e(path, args, stream, reuse, world, dev, bytes_step):
     total = sum_over_ranks(bytes_step, world, dev)
     h2d = x_h.numel() * 2 + idx_h.numel() * 8 + w_h.numel() * 4
     d2h = out_h[0].numel() * 2
+
+    # the PCIe floor of a pipelined step: one step's uploads and its download
+    # issued together on the two copy streams, no kernels
+    def copies_ms(do_up, do_down, reps=5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(up)
+        down.wait_event(a)
+        for _ in range(reps):
+            if do_up:
+                with torch.cuda.stream(up):
+                    x_d[0].copy_(x_h, non_blocking=True)
+                    idx_d[0].copy_(idx_h, non_blocking=True)
+                    w_d[0].copy_(w_h, non_blocking=True)
+            if do_down:
+                with torch.cuda.stream(down):
+                    out_h[1].copy_(out_d[1], non_blocking=True)
+        up.wait_stream(down)
+        b.record(up)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    h2d_ms, d2h_ms, both_ms = copies_ms(True, False), copies_ms(False, True), copies_ms(True, True)
+    floor_ms = max_over_ranks(both_ms, world, dev)
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "pipelining": "two buffer slots; uploads, kernels and downloads on three streams"}
+            "pipelining": "two buffer slots; uploads, kernels and downloads on three streams",
+            "pcie": {"h2d_gbs_alone": round(h2d / (h2d_ms * 1e-3) / 1e9, 1),
+                     "d2h_gbs_alone": round(d2h / (d2h_ms * 1e-3) / 1e9, 1),
+                     "floor_ms_per_step": round(floor_ms, 4),
+                     "frac": round(floor_ms / ms, 4),
+                     "note": "floor = one step's uploads and download issued together, no kernels"}}
 
 
 # ----------------------------------------------------------------------------
