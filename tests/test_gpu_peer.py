@@ -133,6 +133,7 @@ CASES = [
     dict(W=8, T=1000, H=512, E=64, K=8, A=128, router="group", seed=503),    # mostly padding
     dict(W=4, T=1, H=64, E=8, K=2, A=1, router="topk", seed=504),
     dict(W=8, T=2048, H=2048, E=256, K=8, A=1, router="zipf", seed=505),     # skewed ranks
+    dict(W=32, T=24, H=128, E=64, K=4, A=2, router="topk", seed=506),        # many ranks, some empty segments
 ]
 
 
