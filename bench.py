@@ -132,21 +132,29 @@ class ClockSampler:
         except Exception:  # noqa: BLE001 - clocks are reported as unavailable
             self._nvml = None
 
-    def _run(self):
+    def _sample(self):
         nv = self._nvml
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for b, name in self.REASONS.items():
+                if bits & b:
+                    self.reasons.add(name)
+        except Exception:  # noqa: BLE001
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for b, name in self.REASONS.items():
-                    if bits & b:
-                        self.reasons.add(name)
-            except Exception:  # noqa: BLE001
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):
         if self._nvml is not None:
+            # a short region (tens of ms) would otherwise see the sampling
+            # thread only at the interpreter's default 5 ms switch interval
+            self._switch = sys.getswitchinterval()
+            sys.setswitchinterval(self.period / 4)
+            self._sample()
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
         return self
@@ -155,6 +163,8 @@ class ClockSampler:
         self._stop.set()
         if self._thread is not None:
             self._thread.join()
+            self._sample()
+            sys.setswitchinterval(self._switch)
 
     def summary(self):
         if not self.samples:

@@ -79,3 +79,50 @@ def test_reference_arm_other_ranks_are_silent():
 def test_warmup_floor():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_clock_sampler_with_fake_nvml(monkeypatch):
+    """Clock sampling reads NVML only (a fake here): a sample on entry and on
+    exit even for a short region, event-reason bits mapped to names, the
+    interpreter's switch interval restored."""
+    import sys
+    import time
+    import types
+
+    import bench
+
+    unexpected = []
+
+    class FakeNvml(types.ModuleType):
+        NVML_CLOCK_SM = 0
+
+        def nvmlInit(self):
+            pass
+
+        def nvmlDeviceGetHandleByIndex(self, i):
+            return ("dev", i)
+
+        def nvmlDeviceGetMaxClockInfo(self, h, kind):
+            return 1965
+
+        def nvmlDeviceGetClockInfo(self, h, kind):
+            return 1950
+
+        def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+            return 0x4 | 0x1                     # sw_power_cap + idle
+
+        def __getattr__(self, name):             # anything else (a setter, a reset) is recorded
+            unexpected.append(name)
+            raise AttributeError(name)
+
+    fake = FakeNvml("pynvml")
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    before = sys.getswitchinterval()
+    s = bench.ClockSampler(0)
+    with s:
+        time.sleep(0.01)
+    out = s.summary()
+    assert out["samples"] >= 2 and out["sm_mhz"] == 1950 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"]
+    assert sys.getswitchinterval() == before
+    assert unexpected == []                      # read-only: no other NVML call
