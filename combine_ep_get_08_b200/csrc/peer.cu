@@ -14,10 +14,13 @@
 //     base[r] + (row0[r] + row - rank_offsets[r]) * row_bytes,
 // base[r] being rank r's buffer mapped into this process (CUDA IPC; this
 // GPU's own buffer for r == this rank), so the copy to the other GPU is the
-// gather's own store stream -- no staging buffer, no second pass.  The
-// combine reads the expert outputs back from the same places and reduces
-// them as ep_combine does.  Plain loads and stores only: no TMA, no
-// multicast, no wait on another GPU (the caller orders the ranks on the host).
+// gather's own store stream -- no staging buffer, no second pass.  The FP8
+// form quantises each 1x128 block once (the block step shared with the
+// local FP8 dispatch) and stores the E4M3 codes and the block's scale into
+// the destination's code and scale rows.  The combine reads the expert
+// outputs back from the same places and reduces them as ep_combine does.
+// Plain loads and stores only: no TMA, no multicast, no wait on another GPU
+// (the caller orders the ranks on the host).
 #include <cuda_bf16.h>
 
 #include "fp8_block.cuh"
