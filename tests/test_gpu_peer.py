@@ -196,3 +196,31 @@ def test_peer_argument_errors():
         assert e.value.code == ep.EP_ERR_ARG
     finally:
         ep.ep_handle_destroy(h)
+
+
+def test_peer_empty_batch_launches_nothing():
+    dev = torch.device("cuda")
+    h = ep.ep_handle_create(ep.make_config(0, 256, 8, 2, 2, 1))
+    try:
+        ep.ep_get_layout(h, torch.empty((0, 2), dtype=torch.int64, device=dev))
+        buf = torch.zeros((4, 256), dtype=torch.bfloat16, device=dev)
+        bases = torch.tensor([buf.data_ptr()] * 2, dtype=torch.int64, device=dev)
+        row0 = torch.zeros(2, dtype=torch.int32, device=dev)
+        n0 = ep.ep_launch_count()
+        ep.ep_dispatch_peer(h, None, bases, row0)
+        ep.ep_dispatch_peer_fp8(h, None, bases, bases, row0)
+        ep.ep_combine_peer(h, bases, row0, None, None)
+        assert ep.ep_launch_count() == n0
+        assert bool((buf == 0).all())
+    finally:
+        ep.ep_handle_destroy(h)
+
+
+def test_ipc_handle_offset_inside_an_allocation():
+    """The handle names the whole allocation; the offset locates the pointer in it."""
+    dev = torch.device("cuda")
+    t = torch.empty((64, 256), dtype=torch.bfloat16, device=dev)
+    hd0, off0 = ep.ep_ipc_get_handle(t)
+    hd1, off1 = ep.ep_ipc_get_handle(t[3:])
+    assert len(hd0) == ep.EP_IPC_HANDLE_BYTES and hd0 == hd1
+    assert off1 - off0 == 3 * 256 * 2 and off0 >= 0
