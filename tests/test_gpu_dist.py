@@ -1,7 +1,10 @@
 """The cross-GPU path of combine_ep_get_08_b200.dist through the CUDA kernels
 and NCCL, at the group size one GPU allows (world size 1: the all_to_all
-delivers every segment to this rank).  The exchange logic for several ranks
-is covered over gloo in test_dist_exchange.py.
+delivers every segment to this rank), and the peer-memory exchange
+(dispatch_peer / combine_peer, bf16 and FP8) over the same NCCL group.  The
+exchange logic for several ranks is covered over gloo in
+test_dist_exchange.py, and the peer exchange across two processes in
+test_gpu_peer_ipc.py.
 """
 import os
 import socket
@@ -61,6 +64,28 @@ def test_dispatch_exchange_combine_nccl_one_rank():
             torch.cuda.synchronize()
             x64 = (workloads.bf16_bits(wl.x).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
             combine_close(out, x64 * wl.topk_weights.numpy().astype(np.float64).sum(1, keepdims=True))
+            assert ep.ep_get_status(h) == 0
+
+            # the exchange inside the kernels over the same NCCL group: bf16 and FP8
+            for fp8 in (False, True):
+                bufs = epd.PeerBuffers(max_rows=cap, hidden=wl.H, fp8=fp8)
+                try:
+                    got, pplan = epd.dispatch_peer(h, x, idx, w, cfg, bufs)
+                    assert pplan.recv_rows == [o.rows] and pplan.row0 == [0]
+                    xb = workloads.bf16_bits(wl.x)
+                    if fp8:
+                        q, sc = got
+                        oq, osc = oracle.dispatch_fp8(xb, o.row_src)
+                        np.testing.assert_array_equal(q.cpu().numpy(), oq)
+                        np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), osc.view(np.uint32))
+                    else:
+                        np.testing.assert_array_equal(workloads.bf16_bits(got), oracle.dispatch_bf16(xb, o.row_src))
+                    bufs.y[:pplan.total_recv] = recv               # identity experts
+                    out_p = torch.empty_like(x)
+                    epd.combine_peer(h, pplan, w, out_p, bufs)
+                    assert torch.equal(out_p.view(torch.int16), out.view(torch.int16))
+                finally:
+                    bufs.close()
             assert ep.ep_get_status(h) == 0
         finally:
             ep.ep_handle_destroy(h)
