@@ -652,24 +652,33 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
             }
         }
     }
-    // every CTA's histogram complete and visible to the cluster
-    cluster.sync();
-    for (int j = tid; j < ncols; j += kLayoutThreads) {
-        int v[16];                                  // all remote reads in flight together
+    if (C > 1) {
+        // every CTA's histogram complete and visible to the cluster
+        cluster.sync();
+        for (int j = tid; j < ncols; j += kLayoutThreads) {
+            int v[16];                              // all remote reads in flight together
 #pragma unroll
-        for (int cc = 0; cc < 16; ++cc) v[cc] = cc < C ? *cluster.map_shared_rank(s_hist + j, cc) : 0;
-        int tot = 0, before = 0;
+            for (int cc = 0; cc < 16; ++cc) v[cc] = cc < C ? *cluster.map_shared_rank(s_hist + j, cc) : 0;
+            int tot = 0, before = 0;
 #pragma unroll
-        for (int cc = 0; cc < 16; ++cc) {
-            tot += v[cc];
-            before += cc < c ? v[cc] : 0;
+            for (int cc = 0; cc < 16; ++cc) {
+                tot += v[cc];
+                before += cc < c ? v[cc] : 0;
+            }
+            s_tot[j] = tot;
+            if (j < E) s_before[j] = before;
         }
-        s_tot[j] = tot;
-        if (j < E) s_before[j] = before;
+        // this CTA is done reading the others' shared memory; it must not exit
+        // before they are done reading its own (waited for at the end)
+        cluster.barrier_arrive();
+    } else {
+        // one CTA (small batches): its histogram is the total, no cluster exchange
+        __syncthreads();
+        for (int j = tid; j < ncols; j += kLayoutThreads) {
+            s_tot[j] = s_hist[j];
+            if (j < E) s_before[j] = 0;
+        }
     }
-    // this CTA is done reading the others' shared memory; it must not exit
-    // before they are done reading its own (waited for at the end)
-    cluster.barrier_arrive();
     __syncthreads();
     for (int e = tid; e < E; e += kLayoutThreads) {
         s_eoff[e] = (s_tot[e] + p.A - 1) / p.A * p.A;
@@ -738,7 +747,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
             if (p.topk_weights) p.row_weight[r] = 0.0f;
         }
     }
-    cluster.barrier_wait();
+    if (C > 1) cluster.barrier_wait();
 }
 
 size_t cluster_smem_bytes(int E, int R) {

@@ -43,7 +43,7 @@ def test_dispatch_exchange_combine_nccl_one_rank():
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    dist.init_process_group("nccl", rank=0, world_size=1)
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=dev)
     try:
         wl = workloads.generate(None, T=512, H=1024, E=32, R=1, K=4, A=8, router="topk", seed=55)
         cfg = ep.make_config(wl.T, wl.H, wl.E, 1, wl.K, wl.A)
