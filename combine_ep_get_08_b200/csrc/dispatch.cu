@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kStagedThreads, 1) dispatch_bf16_staged_kernel
 #if EP_PDL_PREFETCH && EP_STAGED_PREFETCH
     // an L2 prefetch may run before the wait: L2 is where writes land, so a
     // line prefetched while the previous kernel still writes it is updated there
-    if (threadIdx.x == 0) {
+    if (p.prefetch_x && threadIdx.x == 0) {
         const uint64_t pol_x = policy_evict_last();
         for (int i = 0; i < n_cta; ++i) {
             const int u = blockIdx.x + i * gridDim.x;
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kStagedThreads, 1) dispatch_bf16_staged_kernel
     // bring all of this CTA's x chunks into L2 up front: HBM serves a short
     // burst of reads, then only the stream of received-row writes, and the
     // chunks stay in L2 (evict_last) while that stream passes through
-    if (threadIdx.x == 0) {
+    if (p.prefetch_x && threadIdx.x == 0) {
 #if EP_STAGED_PREFETCH == 1
         const uint64_t pol_x = policy_evict_last();
 #else
@@ -471,6 +471,16 @@ __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p
     int rows = -1;
     LlState st;
     int nblk = gridDim.x;
+    if constexpr (!LL) {
+        // this CTA's token rows into L2 (evict_last) before the dependency
+        // wait, as in the staged bf16 kernel: L2 is where writes land, so a
+        // line prefetched while the previous kernel still writes it is updated
+        if (p.prefetch_x && threadIdx.x == 0) {
+            const uint64_t pol_x = policy_evict_last();
+            for (int t = blockIdx.x; t < p.n_token_units; t += gridDim.x)
+                bulk_prefetch_l2(x + (int64_t)t * p.H * 2, (uint32_t)p.H * 2, pol_x);
+        }
+    }
     pdl_wait();   // the layout (or whatever ran before) is complete and visible
     if constexpr (LL) {
         extern __shared__ int32_t ll_smem[];

@@ -132,6 +132,8 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     if (e != cudaSuccess) return fail(cuda_fail(e, "cudaGetDevice"));
     e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
     if (e != cudaSuccess) return fail(cuda_fail(e, "cudaDeviceGetAttribute"));
+    e = cudaDeviceGetAttribute(&h->l2_bytes, cudaDevAttrL2CacheSize, h->device);
+    if (e != cudaSuccess) return fail(cuda_fail(e, "cudaDeviceGetAttribute(L2)"));
 
     const int T = cfg->num_tokens, E = cfg->num_experts, R = cfg->num_ranks, K = cfg->num_topk;
 
@@ -313,6 +315,9 @@ static int dispatch_common(const ep_handle *h, const void *x, void *recv, float 
     p.n_zero_units = c.expert_alignment > 1
                          ? (int)((h->cap + ep::kZeroRowsPerUnit - 1) / ep::kZeroRowsPerUnit)
                          : 0;
+    // x is pulled into L2 ahead of the gather only when it fits in half of it:
+    // a larger x pinned with evict_last would push out its own rows before use
+    p.prefetch_x = (int64_t)c.num_tokens * c.hidden * 2 <= (int64_t)h->l2_bytes / 2;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
     cudaError_t e = fp8 ? ep::launch_dispatch_fp8(p, sms, s) : ep::launch_dispatch_bf16(p, sms, s);

@@ -68,6 +68,7 @@ struct DispatchParams {
     int stages;                  // shared-memory ring depth (staged kernel)
     int groups;                  // consumer groups (staged kernel)
     int scale_group_rows;        // column-major scales: rows per [H/128][scale_ld] group
+    int prefetch_x;              // 1: each CTA prefetches its x rows into L2 before the dependency wait
     // low-latency static layout (ll_M > 0): destinations computed in-kernel
     // from topk_idx, e*ll_M + slot; no padding rows, no zero fill
     int ll_M;                    // fixed slots per expert
@@ -355,6 +356,7 @@ struct ep_handle {
     ep_config cfg;
     int device;
     int num_sms;
+    int l2_bytes;                   // the device's L2 size
     int64_t cap;
     // layout launch shape
     ep::LayoutPlan plan;
