@@ -39,6 +39,17 @@ from dataclasses import dataclass
 import torch
 
 
+def _join(stream) -> None:
+    """The host continues once the work enqueued so far is finished.  With
+    the current stream (stream None) syncing it is enough; with another
+    stream the whole device is synced, since torch collectives, host reads
+    and small uploads are ordered against the current stream only."""
+    if stream is None:
+        torch.cuda.current_stream().synchronize()
+    else:
+        torch.cuda.synchronize()
+
+
 @dataclass
 class ExchangePlan:
     world: int
@@ -132,6 +143,8 @@ def dispatch(h: int, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights, send
     cnt = torch.empty((cfg.num_experts,), dtype=torch.int32, device=x.device)
     ep_get_layout(h, topk_idx, topk_weights, cnt, stream=stream)
     ep_dispatch(h, x, send, stream=stream)
+    if stream is not None:
+        _join(stream)                                  # the collectives below run on the current stream
     plan = plan_exchange(cnt, cfg.expert_alignment, group=group, device=x.device)
     return exchange_rows(send, plan, group=group), plan
 
@@ -143,6 +156,8 @@ def combine(h: int, y_recv: torch.Tensor, plan: ExchangePlan, topk_weights: torc
     from . import ep_combine
 
     return_rows(y_recv, plan, out=y_send, group=group)
+    if stream is not None:
+        _join(stream)                                  # the rows came in on the current stream
     ep_combine(h, y_send, topk_weights, out, stream=stream)
     return out
 
@@ -253,7 +268,7 @@ def _fence(group, stream) -> None:
     """This rank's work so far is finished and every rank has reached here."""
     import torch.distributed as dist
 
-    (stream if stream is not None else torch.cuda.current_stream()).synchronize()
+    _join(stream)
     dist.barrier(group=group)
 
 
@@ -272,9 +287,11 @@ def dispatch_peer(h: int, x: torch.Tensor, topk_idx: torch.Tensor, topk_weights,
         raise ValueError("cfg.num_ranks must equal the process group's size")
     roff = torch.empty((W + 1,), dtype=torch.int32, device=x.device)
     ep_get_layout(h, topk_idx, topk_weights, None, None, None, None, roff, stream=stream)
-    r = roff.cpu()                                     # waits for the layout
+    _join(stream)
+    r = roff.cpu()
     send_rows = (r[1:] - r[:-1]).tolist()
     row0, recv_rows = peer_row0(send_rows, group=group, max_rows=bufs.max_rows)
+    # uploaded on the current stream; the fence below finishes it before the launch
     row0_dev = torch.tensor(row0, dtype=torch.int32, device=x.device)
     plan = PeerPlan(world=W, send_rows=[int(v) for v in send_rows], recv_rows=recv_rows, row0=row0,
                     row0_dev=row0_dev)
