@@ -86,6 +86,26 @@ def test_dispatch_exchange_combine_nccl_one_rank():
                     assert torch.equal(out_p.view(torch.int16), out.view(torch.int16))
                 finally:
                     bufs.close()
+            # the same on a caller-given side stream (host reads and collectives
+            # must wait for the kernels enqueued there)
+            side = torch.cuda.Stream(dev)
+            recv2, plan2 = epd.dispatch(h, x, idx, w, send, cfg, stream=side)
+            assert plan2.total_recv == o.rows
+            np.testing.assert_array_equal(workloads.bf16_bits(recv2), workloads.bf16_bits(recv))
+            out2 = torch.empty_like(x)
+            epd.combine(h, recv2, plan2, w, out2, y_send, stream=side)
+            side.synchronize()
+            assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
+            bufs = epd.PeerBuffers(max_rows=cap, hidden=wl.H)
+            try:
+                got, pplan = epd.dispatch_peer(h, x, idx, w, cfg, bufs, stream=side)
+                np.testing.assert_array_equal(workloads.bf16_bits(got), workloads.bf16_bits(recv))
+                bufs.y[:pplan.total_recv] = recv
+                out3 = torch.empty_like(x)
+                epd.combine_peer(h, pplan, w, out3, bufs, stream=side)
+                assert torch.equal(out3.view(torch.int16), out.view(torch.int16))
+            finally:
+                bufs.close()
             assert ep.ep_get_status(h) == 0
         finally:
             ep.ep_handle_destroy(h)
