@@ -375,7 +375,8 @@ EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner,
  * - rank_offsets[r]) rows of H bf16.  These contents are not checked on the
  * host; a wrong value writes or reads outside the caller's buffers.  Null,
  * misaligned or host-detectable errors return EP_ERR_ARG; a low-latency handle
- * returns EP_ERR_STATE.  The calls issue plain loads and stores and never wait
+ * returns EP_ERR_STATE; an empty batch (T = 0) returns EP_OK and launches
+ * nothing.  The calls issue plain loads and stores and never wait
  * on another GPU.  The caller orders the ranks: every destination buffer is
  * free before a dispatch starts, and every expert output is complete before a
  * combine reads it (for example, a stream synchronise and a process-group
@@ -383,6 +384,8 @@ EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner,
  */
 EP_API int ep_dispatch_peer(const ep_handle *h, const void *x, void *const *recv_bases, const int32_t *row0,
                             ep_stream_t stream);
+EP_API int ep_combine_peer(const ep_handle *h, const void *const *y_bases, const int32_t *row0,
+                           const float *topk_weights, void *out, ep_stream_t stream);
 
 /*
  * FP8 form of ep_dispatch_peer: each destination receives E4M3 codes
@@ -395,8 +398,6 @@ EP_API int ep_dispatch_peer(const ep_handle *h, const void *x, void *const *recv
  */
 EP_API int ep_dispatch_peer_fp8(const ep_handle *h, const void *x, void *const *recv_bases,
                                 float *const *scale_bases, const int32_t *row0, ep_stream_t stream);
-EP_API int ep_combine_peer(const ep_handle *h, const void *const *y_bases, const int32_t *row0,
-                           const float *topk_weights, void *out, ep_stream_t stream);
 
 /*
  * CUDA IPC for those buffers.  ep_ipc_get_handle fills `handle`
