@@ -92,7 +92,9 @@ def test_two_rank_exchange(tmp_path):
 
 def _peer_rank_main(rank, world, port, out_path):
     """peer_row0 over gloo: the blocks of all sources tile each destination's
-    rows in source order, with no gap and no overlap."""
+    rows in source order, with no gap and no overlap, and placing the oracle's
+    segments at those rows (what the peer dispatch does) gives exactly the
+    receive buffer of the all_to_all exchange."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import torch.distributed as dist
 
@@ -123,6 +125,18 @@ def _peer_rank_main(rank, world, port, out_path):
         except ValueError:
             res["overflow"] = True
         epd.peer_row0(send, max_rows=worst)            # exactly enough rows is fine
+        # the peer placement gives the receive buffer the all_to_all gives:
+        # source s's segment for this rank at row0_s[me], sources in order
+        _, _, _, rows = _source(rank, world)
+        plan = epd.plan_exchange(L.num_tokens_per_expert, A)
+        recv = epd.exchange_rows(torch.from_numpy(np.ascontiguousarray(rows).view(np.int32).copy()), plan)
+        buf = np.full((plan.total_recv, H), 0xBEEF, np.uint16)
+        for s in range(world):
+            _, Ls, _, rows_s = _source(s, world)
+            a, b = Ls.rank_offsets[rank], Ls.rank_offsets[rank + 1]
+            r0 = everyone[s][1][rank]
+            buf[r0:r0 + b - a] = rows_s[a:b]
+        res["same_as_all_to_all"] = bool(np.array_equal(buf, recv.numpy().view(np.uint16)))
     finally:
         dist.destroy_process_group()
     with open(f"{out_path}.{rank}", "w") as f:
@@ -133,4 +147,4 @@ def test_four_rank_peer_row0(tmp_path):
     out = str(tmp_path / "peer")
     mp.spawn(_peer_rank_main, args=(4, _free_port(), out), nprocs=4, join=True)
     for r in range(4):
-        assert json.load(open(f"{out}.{r}")) == {"tiling": True, "overflow": True}
+        assert json.load(open(f"{out}.{r}")) == {"tiling": True, "overflow": True, "same_as_all_to_all": True}
