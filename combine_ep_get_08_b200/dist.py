@@ -254,6 +254,12 @@ class PeerBuffers:
         self.recv_bases, self.y_bases = table[0], table[1]
         self.scale_bases = table[2] if fp8 else None
 
+    def __enter__(self) -> "PeerBuffers":
+        return self
+
+    def __exit__(self, *exc) -> None:
+        self.close()
+
     def close(self) -> None:
         """Unmaps the other ranks' buffers (after the last kernel that uses them)."""
         from . import ep_ipc_close_handle
