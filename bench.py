@@ -46,6 +46,7 @@ if ROOT not in sys.path:
 
 METRIC = "dispatch+combine µs/call and effective HBM GB/s (% of B200 peak) at 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0          # the B200 specification figure (~8 TB/s)
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -393,8 +394,151 @@ class LLPath(Path):
                               stream=stream)
 
 
+def make_path(name, mode, dev, rank, ll_slots=0):
+    """The named workload (rank-seeded) and its device buffers and handle."""
+    import workloads
+    base = workloads.CONFIGS[name]
+    wl = workloads.generate(name, seed=base["seed"] + 1000 * rank)
+    path = LLPath(wl, dev, ll_slots or max(wl.T, 1)) if mode == "ll" else Path(wl, dev)
+    return wl, path
+
+
+def step_fn(path, reuse, sptr, stream):
+    """One step: flush, layout, then `reuse` dispatch/flush/combine calls.
+    ev: 5 events (before the layout, unused, after the first dispatch, after
+    the flush that follows it, after the first combine); sp: the stream to
+    launch on (the bench's stream unless being captured)."""
+    def one_step(ev=None, sp=None):
+        # The dispatch follows the layout with no event between them, so its
+        # launch overlaps the layout's tail (programmatic dependent launch).
+        sp = sptr if sp is None else sp
+        path.flush_l2()
+        if ev is not None:
+            ev[0].record(stream)
+        path.layout(sp)
+        for r in range(reuse):
+            path.dispatch(sp)
+            if ev is not None and r == 0:
+                ev[2].record(stream)
+            path.flush_l2()
+            if ev is not None and r == 0:
+                ev[3].record(stream)
+            path.combine(sp)
+            if ev is not None and r == 0:
+                ev[4].record(stream)
+    return one_step
+
+
+def split_pass(path, n, stream, sptr):
+    """Each kernel timed alone (events between layout, dispatch and combine),
+    and the L2 write-back each one leaves behind: the 256 MiB read flush that
+    follows a kernel also writes back the dirty lines the kernel left in L2,
+    so (flush after the kernel) - (flush of a clean L2) is the time of that
+    write-back, charged to the kernel in `with_writeback`."""
+    import torch
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(n)]
+    for e in evs:
+        e[0].record(stream)
+        path.flush_l2()
+        e[1].record(stream)
+        path.layout(sptr)
+        e[2].record(stream)
+        path.dispatch(sptr)
+        e[3].record(stream)
+        path.flush_l2()                     # writes back what the dispatch left dirty
+        e[4].record(stream)
+        path.combine(sptr)
+        e[5].record(stream)
+        path.flush_l2()                     # writes back what the combine left dirty
+        e[6].record(stream)
+        path.flush_l2()                     # a clean L2: the flush alone
+        e[7].record(stream)
+    torch.cuda.synchronize()
+    el = lambda e, i, j: e[i].elapsed_time(e[j])  # noqa: E731
+    return {"layout": [el(e, 1, 2) for e in evs], "dispatch": [el(e, 2, 3) for e in evs],
+            "combine": [el(e, 4, 5) for e in evs], "flush_after_dispatch": [el(e, 3, 4) for e in evs],
+            "flush_after_combine": [el(e, 5, 6) for e in evs], "flush_clean": [el(e, 6, 7) for e in evs]}
+
+
+def kernel_figures(wl, rows, split, ll, peak):
+    """Per-kernel means, GB/s and roofline fractions (of the measured peak and
+    of the 8 TB/s B200 figure), plain and with the L2 write-back charged."""
+    b_dis = dispatch_bytes(wl.T, wl.H, wl.K, rows, wl.fp8)
+    b_com = combine_bytes(wl.T, wl.H, wl.K)
+    mean = {k: statistics.mean(v) * 1e3 for k, v in split.items()}      # µs
+    lay = 0.0 if ll else mean["layout"]
+    wb_dis = max(0.0, mean["flush_after_dispatch"] - mean["flush_clean"])
+    wb_com = max(0.0, mean["flush_after_combine"] - mean["flush_clean"])
+    out = {
+        "us_per_call": {"layout": round(lay, 2), "dispatch": round(mean["dispatch"], 2),
+                        "combine": round(mean["combine"], 2)},
+        "bytes_per_call": {"dispatch": b_dis, "combine": b_com},
+        "gbs_per_call": {"dispatch": round(b_dis / mean["dispatch"] / 1e3, 1),
+                         "combine": round(b_com / mean["combine"] / 1e3, 1)},
+        "frac_of_measured": {"dispatch": round(b_dis / mean["dispatch"] / 1e3 / peak, 4),
+                             "combine": round(b_com / mean["combine"] / 1e3 / peak, 4)},
+        "frac_of_8tbs": {"dispatch": round(b_dis / mean["dispatch"] / 1e3 / SPEC_HBM_GBS, 4),
+                         "combine": round(b_com / mean["combine"] / 1e3 / SPEC_HBM_GBS, 4)},
+        "with_writeback": {
+            "dispatch_us": round(mean["dispatch"] + wb_dis, 2), "combine_us": round(mean["combine"] + wb_com, 2),
+            "dispatch_gbs": round(b_dis / (mean["dispatch"] + wb_dis) / 1e3, 1),
+            "combine_gbs": round(b_com / (mean["combine"] + wb_com) / 1e3, 1),
+            "dispatch_frac": round(b_dis / (mean["dispatch"] + wb_dis) / 1e3 / peak, 4),
+            "combine_frac": round(b_com / (mean["combine"] + wb_com) / 1e3 / peak, 4),
+            "flush_clean_us": round(mean["flush_clean"], 2),
+            "how": "kernel time + (256 MiB read flush right after the kernel - the same flush of a clean L2): "
+                   "the write-back of the lines the kernel left dirty in L2"},
+        "us_p10_p50_p90": {k: pct(split[k]) for k in ("layout", "dispatch", "combine")},
+    }
+    return out
+
+
+def config_summary(name, mode, args, dev, rank, stream, peak, steps, warmup):
+    """One workload measured on its own (no barrier, this rank only): the
+    step as `value` times it, per-kernel times with and without the L2
+    write-back, and for latency-bound steps the CUDA-graph replay."""
+    import torch
+
+    import combine_ep_get_08_b200 as ep
+    import workloads
+    ll = mode == "ll"
+    wl, path = make_path(name, mode, dev, rank)
+    try:
+        reuse = wl.reuse
+        sptr = stream.cuda_stream
+        one_step = step_fn(path, reuse, sptr, stream)
+        for _ in range(warmup):
+            one_step()
+        torch.cuda.synchronize()
+        rows = int(path.cnt.sum()) if ll else ep.ep_get_num_rows(path.h)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        for e in evs:
+            one_step(e)
+        torch.cuda.synchronize()
+        ld_ms = [e[0].elapsed_time(e[2]) for e in evs]
+        com_ms = [e[3].elapsed_time(e[4]) for e in evs]
+        split = split_pass(path, steps, stream, sptr)
+        fig = kernel_figures(wl, rows, split, ll, peak)
+        mean_dis = statistics.mean(split["dispatch"])
+        step_ms = statistics.mean([ld + (reuse - 1) * mean_dis + reuse * c for ld, c in zip(ld_ms, com_ms)])
+        bytes_step = reuse * (fig["bytes_per_call"]["dispatch"] + fig["bytes_per_call"]["combine"])
+        entry = {"workload": workloads.DESCRIPTIONS[name] + (" (low-latency static layout)" if ll else ""),
+                 "steps": steps, "rows": rows, "reuse": reuse,
+                 "step_us": round(step_ms * 1e3, 2), "step_gbs": round(bytes_step / (step_ms * 1e-3) / 1e9, 1),
+                 "us_layout_then_dispatch": round(statistics.mean(ld_ms) * 1e3, 2)}
+        entry.update(fig)
+        if bytes_step < L2_FLUSH_BYTES // 8:
+            entry["graph"] = run_graph(path, one_step, args, stream, reuse, 1, dev, bytes_step)
+        entry["device_status"] = int(ep.ep_get_status(path.h))
+        return entry
+    finally:
+        path.close()
+
+
+PER_CONFIG = (("tiny", "normal"), ("decode", "normal"), ("decode", "ll"), ("skew", "normal"), ("large", "normal"))
+
+
 def run_cuda(args, world, rank, local):
-    import numpy as np
     import torch
 
     import combine_ep_get_08_b200 as ep
@@ -412,38 +556,14 @@ def run_cuda(args, world, rank, local):
     barrier(world)
     ep.library()
 
-    base = workloads.CONFIGS[args.config]
-    wl = workloads.generate(args.config, seed=base["seed"] + 1000 * rank)
-    reuse = base["reuse"] if args.reuse is None else args.reuse
     ll = args.mode == "ll"
-    path = LLPath(wl, dev, args.ll_slots or max(wl.T, 1)) if ll else Path(wl, dev)
+    wl, path = make_path(args.config, args.mode, dev, rank, args.ll_slots)
+    reuse = wl.reuse if args.reuse is None else args.reuse
     if args.sm_limit:
         ep.ep_set_sm_limit(path.h, args.sm_limit)
     stream = torch.cuda.current_stream(dev)
     sptr = stream.cuda_stream
-
-    def one_step(ev=None, split=False, sp=None):
-        # The dispatch follows the layout with no event between them, so its
-        # launch overlaps the layout's tail (programmatic dependent launch);
-        # `split` puts an event between them to time each kernel alone.  `sp`:
-        # the stream to launch on (the bench's stream unless being captured).
-        sp = sptr if sp is None else sp
-        path.flush_l2()
-        if ev is not None:
-            ev[0].record(stream)
-        path.layout(sp)
-        if ev is not None and split:
-            ev[1].record(stream)
-        for r in range(reuse):
-            path.dispatch(sp)
-            if ev is not None and r == 0:
-                ev[2].record(stream)
-            path.flush_l2()
-            if ev is not None and r == 0:
-                ev[3].record(stream)
-            path.combine(sp)
-            if ev is not None and r == 0:
-                ev[4].record(stream)
+    one_step = step_fn(path, reuse, sptr, stream)
 
     for _ in range(args.warmup):
         one_step()
@@ -466,30 +586,23 @@ def run_cuda(args, world, rank, local):
     barrier(world)
     launches = ep.ep_launch_count() - launches0
 
-    # the low-latency mode has no layout launch (it is fused into the dispatch):
-    # the empty event pair around it would only add the events' own overhead
     bracket_ms = bracket[0].elapsed_time(bracket[1])
     # layout + first dispatch as one span (their launches overlap); with
     # reuse > 1 only the first dispatch/combine pair of a step carries events
-    # and the further calls count at the per-call times measured below
+    # and the further calls count at the per-call time measured below
     ld_ms = [e[0].elapsed_time(e[2]) for e in evs]
     com_ms = [e[3].elapsed_time(e[4]) for e in evs]
 
-    # per-kernel times (events between layout and dispatch), for the
-    # breakdown and the roofline; not part of `value`
-    n_split = min(args.steps, 20)
-    evs_split = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_split)]
-    for i in range(n_split):
-        one_step(evs_split[i], split=True)
-    torch.cuda.synchronize()
-    lay_ms = [0.0 if ll else e[0].elapsed_time(e[1]) for e in evs_split]
-    dis_ms = [e[1].elapsed_time(e[2]) for e in evs_split]
-    mean_dis = statistics.mean(dis_ms)
+    # per-kernel times (events between the kernels) and the L2 write-back
+    # each leaves, for the breakdown and the roofline; not part of `value`
+    split = split_pass(path, min(args.steps, 20), stream, sptr)
+    peak, peak_src = measured_peak()
+    fig = kernel_figures(wl, rows, split, ll, peak)
+    mean_dis = statistics.mean(split["dispatch"])
     step_ms = [ld + (reuse - 1) * mean_dis + reuse * c for ld, c in zip(ld_ms, com_ms)]
     total_ms = sum(step_ms)
 
-    b_dis = dispatch_bytes(wl.T, wl.H, wl.K, rows, wl.fp8)
-    b_com = combine_bytes(wl.T, wl.H, wl.K)
+    b_dis, b_com = fig["bytes_per_call"]["dispatch"], fig["bytes_per_call"]["combine"]
     bytes_step = reuse * (b_dis + b_com)
     my_bytes = bytes_step * args.steps
     all_bytes = sum_over_ranks(my_bytes, world, dev)
@@ -504,17 +617,23 @@ def run_cuda(args, world, rank, local):
     small = bytes_step < L2_FLUSH_BYTES // 8
     graph = run_graph(path, one_step, args, stream, reuse, world, dev, bytes_step) if small else None
 
-    lay_us, dis_us, com_us = (statistics.mean(v) * 1e3 for v in (lay_ms, dis_ms, com_ms))
-    ld_us = statistics.mean(ld_ms) * 1e3
-    peak, peak_src = measured_peak()
-    kern = {"layout": lay_us, "dispatch": dis_us, "combine": com_us}
-    dom = "dispatch" if dis_us >= com_us else "combine"
+    kern = fig["us_per_call"]
+    dom = "dispatch" if kern["dispatch"] >= kern["combine"] else "combine"
     dom_bytes = b_dis if dom == "dispatch" else b_com
     achieved = dom_bytes / (kern[dom] * 1e-6) / 1e9
+    wb = fig["with_writeback"]
     kname, traffic = ncu_traffic(dom, args.config + ("-ll" if ll else ""))
     clocks = sampler.summary()
     status_end = ep.ep_get_status(path.h)
     path.close()
+
+    per_config = None
+    if world == 1 and not args.no_per_config and args.config == "dsv3" and not ll and not args.sm_limit:
+        n = max(5, min(args.steps, 20))
+        per_config = {}
+        for name, mode in PER_CONFIG:
+            per_config[name + ("_ll" if mode == "ll" else "")] = config_summary(
+                name, mode, args, dev, rank, stream, peak, n, args.warmup)
 
     if rank == 0:
         line = {
@@ -532,16 +651,18 @@ def run_cuda(args, world, rank, local):
                 "l2": "flushed (256 MiB read, outside the timed events) before each step and "
                       "between dispatch and combine",
             },
-            "us_per_call": {k: round(v, 2) for k, v in kern.items()},
-            "us_layout_then_dispatch": round(ld_us, 2),
-            "us_p10_p50_p90": {k: pct(v) for k, v in (("layout_then_dispatch", ld_ms), ("layout", lay_ms),
-                                                       ("dispatch", dis_ms), ("combine", com_ms))},
-            "bytes_per_call": {"dispatch": b_dis, "combine": b_com},
-            "gbs_per_call": {"dispatch": round(b_dis / dis_us / 1e3, 1),
-                             "combine": round(b_com / com_us / 1e3, 1)},
+            "us_per_call": kern,
+            "us_layout_then_dispatch": round(statistics.mean(ld_ms) * 1e3, 2),
+            "us_p10_p50_p90": dict(fig["us_p10_p50_p90"], layout_then_dispatch=pct(ld_ms)),
+            "bytes_per_call": fig["bytes_per_call"],
+            "gbs_per_call": fig["gbs_per_call"],
+            "frac_of_8tbs": fig["frac_of_8tbs"],
             "roofline": {"bound": "hbm", "kernel": dom if kname is None else f"{dom}: {kname}",
                          "achieved": round(achieved, 1), "peak": peak, "peak_source": peak_src,
-                         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic},
+                         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "with_writeback": {"us": wb[dom + "_us"], "achieved": wb[dom + "_gbs"],
+                                            "frac": wb[dom + "_frac"], "how": wb["how"]}},
+            "with_writeback": wb,
             "e2e": e2e,
             "gpu_launches": int(launches),
             "clocks": clocks,
@@ -550,6 +671,8 @@ def run_cuda(args, world, rank, local):
         }
         if graph is not None:
             line["graph"] = graph
+        if per_config is not None:
+            line["per_config"] = per_config
         if world == 1 and not args.no_cpu_baseline:
             gbs, n, el, _ = oracle_sample(wl, args.cpu_budget)
             line["cpu_baseline"] = {
@@ -1030,6 +1153,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds for the oracle baseline")
     ap.add_argument("--ref-tokens", type=int, default=4096, help="tokens per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per_config block (the other four workloads, measured after dsv3)")
     ap.add_argument("--sm-limit", type=int, default=0, help="SMs dispatch/combine may occupy (0: all)")
     ap.add_argument("--mode", choices=["normal", "ll"], default="normal",
                     help="layout: normal (padded, ep_get_layout) or low-latency static slots (ep_ll_*)")

@@ -72,6 +72,7 @@ def _load():
             "ep_handle_get_view": ([P, ctypes.POINTER(ep_handle_view)], ctypes.c_int),
             "ep_get_layout": ([P] + [P] * 7 + [P], ctypes.c_int),
             "ep_get_layout_noalloc": ([CFG] + [P] * 13, ctypes.c_int),
+            "ep_layout_shape": ([CFG, ctypes.POINTER(I32), ctypes.POINTER(I32), ctypes.POINTER(I64)], ctypes.c_int),
             "ep_dispatch": ([P, P, P, P], ctypes.c_int),
             "ep_dispatch_fp8": ([P, P, P, P, P], ctypes.c_int),
             "ep_combine": ([P, P, P, P, P], ctypes.c_int),
@@ -201,6 +202,14 @@ def ep_get_layout_noalloc(cfg: ep_config, topk_idx, topk_weights, pos, row_src, 
         ctypes.byref(cfg), _ptr(topk_idx), _ptr(topk_weights), _ptr(pos), _ptr(row_src), _ptr(row_slot),
         _ptr(row_weight), _ptr(num_tokens_per_expert), _ptr(num_tokens_per_rank), _ptr(is_token_in_rank),
         _ptr(expert_offsets), _ptr(rank_offsets), _ptr(status), _stream(stream)))
+
+
+def ep_layout_shape(cfg: ep_config) -> tuple[int, int, int]:
+    """(cluster, ctas, noalloc_scratch_bytes) of the layout launch on the current device."""
+    cl, ctas, need = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int64()
+    _check("ep_layout_shape", _load().ep_layout_shape(ctypes.byref(cfg), ctypes.byref(cl), ctypes.byref(ctas),
+                                                      ctypes.byref(need)))
+    return cl.value, ctas.value, need.value
 
 
 def ep_dispatch(h: int, x, recv_x, stream=None) -> None:

@@ -52,7 +52,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_report: bool = False
     objs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc, *ARCH, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-dc" if False else "-c",
+        cmd = [nvcc, *ARCH, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c",
                src, "-o", obj]
         if ptxas_report:
             cmd += ["-Xptxas", "-v"]

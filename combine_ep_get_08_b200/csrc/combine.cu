@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 4) combine_kernel(CombineParams p) {
 // DeepSeek-V3 shape): the fp32 accumulation needs the register kernel's
 // four resident blocks per SM.
 cudaError_t launch_combine(const CombineParams &p_in, int num_sms, cudaStream_t s) {
-    static int occ = 0;
+    static OccupancyCache occ;
     CombineParams p = p_in;
     // a small batch splits each row over several CTAs (at least half a
     // block of vectors each) so that it still spreads over the SMs

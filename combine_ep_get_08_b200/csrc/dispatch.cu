@@ -600,7 +600,7 @@ static cudaError_t launch_pdl(Kernel kernel, int grid, int block, size_t smem, c
 }
 
 cudaError_t launch_dispatch_bf16(const DispatchParams &p_in, int num_sms, cudaStream_t s) {
-    static int occ16 = 0, occ32 = 0;
+    static OccupancyCache occ16, occ32;
     DispatchParams p = p_in;
     const bool v32 = (p.H % 16 == 0) && ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
     const int row_bytes = p.H * 2;
@@ -634,7 +634,7 @@ cudaError_t launch_dispatch_bf16(const DispatchParams &p_in, int num_sms, cudaSt
 static size_t ll_smem_bytes(int E) { return sizeof(int32_t) * (size_t)(kMaxTopk + E); }
 
 cudaError_t launch_ll_dispatch(const DispatchParams &p_in, bool fp8, int num_sms, cudaStream_t s) {
-    static int occ[4] = {0, 0, 0, 0};
+    static OccupancyCache occ[4];
     DispatchParams p = p_in;
     p.n_zero_units = 0;
     const size_t smem = ll_smem_bytes(p.E);
@@ -642,7 +642,7 @@ cudaError_t launch_ll_dispatch(const DispatchParams &p_in, bool fp8, int num_sms
     const bool v32 = (fp8 || p.H % 16 == 0) &&
                      ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
     const void *k;
-    int *slot;
+    OccupancyCache *slot;
     if (fp8) {
         p.splits = 1;
         k = v32 ? reinterpret_cast<const void *>(&dispatch_fp8_kernel<32, true>)
@@ -681,7 +681,7 @@ cudaError_t launch_ll_dispatch(const DispatchParams &p_in, bool fp8, int num_sms
 // consumer group per SM measured slower (the quantisation needs the
 // register kernel's four resident blocks per SM).
 cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream_t s) {
-    static int occ16 = 0, occ32 = 0;
+    static OccupancyCache occ16, occ32;
     const int units = p.n_token_units + p.n_zero_units;
     const bool v32 = ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
     if (v32) {

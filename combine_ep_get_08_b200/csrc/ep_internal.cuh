@@ -148,13 +148,25 @@ void record_error(const char *msg);
 int record_cuda_error(cudaError_t e, const char *what);   // returns EP_ERR_CUDA
 void count_launch();
 
+// Resident blocks per SM of one kernel instance, cached per device ordinal
+// (0 = not yet known); launchers keep one as a function-local static.
+constexpr int kMaxDevices = 64;
+struct OccupancyCache {
+    int per_device[kMaxDevices];
+};
+
 // Resident blocks per SM of `kernel` at `threads` threads and `smem` dynamic
-// shared memory, cached in *slot (0 = not yet known).
-inline int blocks_per_sm(const void *kernel, int threads, size_t smem, int *slot) {
-    int v = __atomic_load_n(slot, __ATOMIC_RELAXED);
+// shared memory on the current device, through the cache.  Entries are read
+// and written atomically, so host threads may launch concurrently; two that
+// race both compute the same value.
+inline int blocks_per_sm(const void *kernel, int threads, size_t smem, OccupancyCache *cache) {
+    int dev = -1;
+    int *slot = nullptr;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) slot = &cache->per_device[dev];
+    int v = slot ? __atomic_load_n(slot, __ATOMIC_RELAXED) : 0;
     if (v > 0) return v;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, threads, smem) != cudaSuccess || v < 1) v = 1;
-    __atomic_store_n(slot, v, __ATOMIC_RELAXED);
+    if (slot) __atomic_store_n(slot, v, __ATOMIC_RELAXED);
     return v;
 }
 inline int persistent_grid(int units, int per_sm, int num_sms) {

@@ -357,7 +357,7 @@ cudaError_t launch_gemm_combine(const GemmCombineArgs &g, int num_sms, cudaStrea
     int dev = 0;
     cudaError_t e0 = cudaGetDevice(&dev);
     if (e0 != cudaSuccess) return e0;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     if (!__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE)) {
         const cudaError_t e = cudaFuncSetAttribute(gemm_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    (int)kGSmem);

@@ -767,10 +767,10 @@ const void *layout_kernel_ptr() { return reinterpret_cast<const void *>(&layout_
 // Per device, once: kernel attributes (dynamic shared memory for the
 // largest supported E and R, clusters of 16) and the largest cluster size
 // that can be resident with one 1024-thread CTA per SM.
-static int g_max_cluster[64];
+static int g_max_cluster[kMaxDevices];
 
 cudaError_t layout_prepare(int device) {
-    if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+    if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
     if (__atomic_load_n(&g_max_cluster[device], __ATOMIC_ACQUIRE) > 0) return cudaSuccess;
     const void *coop = reinterpret_cast<const void *>(&layout_kernel);
     const void *clus = reinterpret_cast<const void *>(&layout_cluster_kernel);
@@ -806,7 +806,7 @@ cudaError_t layout_prepare(int device) {
 LayoutPlan plan_layout(int device, int T, int E, int R, int K, int num_sms) {
     LayoutPlan pl{};
     const int64_t pairs = (int64_t)T * K;
-    const int cmax = (device >= 0 && device < 64) ? __atomic_load_n(&g_max_cluster[device], __ATOMIC_ACQUIRE) : 0;
+    const int cmax = (device >= 0 && device < kMaxDevices) ? __atomic_load_n(&g_max_cluster[device], __ATOMIC_ACQUIRE) : 0;
     if (cmax >= 1) {
         // about kClusterPairsTarget pairs per CTA, at most kClusterMaxPairs
         int C = (int)((pairs + kClusterPairsTarget - 1) / kClusterPairsTarget);

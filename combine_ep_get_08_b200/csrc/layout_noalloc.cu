@@ -24,7 +24,7 @@ constexpr size_t kCountsOffset = 256;
 
 static __device__ __align__(256) unsigned char g_layout_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
+using ep::kMaxDevices;
 
 struct DeviceSetup {
     bool ready;
@@ -57,6 +57,26 @@ int setup_device(int dev, DeviceSetup *out) {
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Bytes of the array a layout of this launch shape uses: none for the
+// cluster kernel; the arrival counter and the chunk histograms (E + R rows of
+// G rounded up to 4 int32) for the cooperative kernel.
+size_t scratch_need(const ep::LayoutPlan &plan, int E, int R) {
+    if (plan.cluster) return 0;
+    const size_t G_stride = ((size_t)plan.G + 3) / 4 * 4;
+    return kCountsOffset + sizeof(int32_t) * G_stride * (size_t)(E + R);
+}
+
+// The current device, checked against the table size.
+int current_device(int *dev) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return ep::record_cuda_error(e, "cudaGetDevice");
+    if (*dev < 0 || *dev >= kMaxDevices) {
+        ep::record_error("device ordinal beyond the 64 this library tracks");
+        return EP_ERR_UNSUPPORTED;
+    }
+    return EP_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -79,12 +99,8 @@ EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, 
         return EP_ERR_ARG;
 
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return ep::record_cuda_error(e, "cudaGetDevice");
-    if (dev < 0 || dev >= kMaxDevices) {
-        ep::record_error("ep_get_layout_noalloc: device ordinal beyond the 64 this library tracks");
-        return EP_ERR_UNSUPPORTED;
-    }
+    rc = current_device(&dev);
+    if (rc != EP_OK) return rc;
     DeviceSetup s;
     rc = setup_device(dev, &s);
     if (rc != EP_OK) return rc;
@@ -95,7 +111,7 @@ EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, 
     const int64_t G = plan.G;
     const int tpc = plan.tokens_per_chunk;
     const int G_stride = (int)((G + 3) / 4 * 4);
-    const size_t need = plan.cluster ? 0 : kCountsOffset + sizeof(int32_t) * (size_t)G_stride * (E + R);
+    const size_t need = scratch_need(plan, E, R);
     if (need > kScratchBytes) {
         char msg[160];
         snprintf(msg, sizeof msg, "ep_get_layout_noalloc: %zu bytes of scratch needed, the fixed array holds %zu",
@@ -107,7 +123,7 @@ EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // the array keeps the previous call's contents: the arrival counter and
     // the histogram rows (whose tail past G is read as zeros) start at zero
-    e = need ? cudaMemsetAsync(s.scratch, 0, need, st) : cudaSuccess;
+    cudaError_t e = need ? cudaMemsetAsync(s.scratch, 0, need, st) : cudaSuccess;
     if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, sizeof(uint32_t), st);
     if (e != cudaSuccess) return ep::record_cuda_error(e, "cudaMemsetAsync(layout scratch)");
 
@@ -142,6 +158,23 @@ EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, 
     e = ep::launch_layout(p, plan, st);
     if (e != cudaSuccess) return ep::record_cuda_error(e, "launch(layout)");
     ep::count_launch();
+    return EP_OK;
+}
+
+EP_API int ep_layout_shape(const ep_config *cfg, int32_t *cluster, int32_t *ctas, int64_t *noalloc_scratch_bytes) {
+    int rc = ep_validate_config(cfg);
+    if (rc != EP_OK) return rc;
+    int dev = 0;
+    rc = current_device(&dev);
+    if (rc != EP_OK) return rc;
+    DeviceSetup s;
+    rc = setup_device(dev, &s);
+    if (rc != EP_OK) return rc;
+    const ep::LayoutPlan plan =
+        ep::plan_layout(dev, cfg->num_tokens, cfg->num_experts, cfg->num_ranks, cfg->num_topk, s.num_sms);
+    if (cluster) *cluster = plan.cluster ? 1 : 0;
+    if (ctas) *ctas = plan.G;
+    if (noalloc_scratch_bytes) *noalloc_scratch_bytes = (int64_t)scratch_need(plan, cfg->num_experts, cfg->num_ranks);
     return EP_OK;
 }
 

@@ -156,10 +156,16 @@ EP_API int ep_handle_get_view(const ep_handle *h, ep_handle_view *out);
  *   is_token_in_rank [T, R] uint8 (0/1), expert_offsets [E+1] int32,
  *   rank_offsets [R+1] int32.
  * topk_idx/topk_weights need 8/4-byte alignment only.  One kernel launch:
- * a thread-block cluster of up to 16 CTAs (at most 8192 pairs each) that
+ * a thread-block cluster of up to 16 CTAs (at most 4096 pairs each) that
  * exchanges its histograms in distributed shared memory, or, for larger
  * batches, a cooperative grid whose one grid-wide wait is bounded
  * (EP_DEV_WAIT_TIMEOUT).
+ * Defined by: the V1 layout tensors num_tokens_per_rank, is_token_in_rank
+ * and num_tokens_per_expert of bowenzhou.top "deepep/01-overview" section
+ * 1.4; the per-expert queue order (tokens in order, then k) of the
+ * moe_dispatch loop in the "lesson14_deepep" practice task, whose counts sum
+ * to T*K (its conservation assert); expert_alignment / do_zero_padding of
+ * section 1.1 of the same overview page for the padded offsets.
  * An id of -1 marks an unused top-k slot (the token selects fewer than K
  * experts): that pair gets pos = -1, no row, is not counted and adds
  * nothing in combine.  Any other id outside [0, E) also gets pos = -1 and
@@ -183,6 +189,10 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
  * rows for the padding of each expert segment.  x is [T, H] bf16, recv_x is
  * [capacity, H] bf16; rows at or beyond `rows` are not written.  Uses the
  * layout last computed in h (a layout may serve any number of dispatches).
+ * Defined by: do_expand (one received row per (token, expert) pair) and
+ * do_zero_padding of EPBuffer.dispatch, bowenzhou.top "deepep/01-overview"
+ * section 1.1; the moe_dispatch loop of the "lesson14_deepep" practice task
+ * (each token row appended to the queue of each expert it selected).
  */
 EP_API int ep_dispatch(const ep_handle *h, const void *x, void *recv_x, ep_stream_t stream);
 
@@ -195,6 +205,12 @@ EP_API int ep_dispatch(const ep_handle *h, const void *x, void *recv_x, ep_strea
  * (16-byte aligned); recv_scales is fp32, 4-byte aligned, in the handle's
  * scale layout (ep_set_scale_layout; default [capacity, H/128] row-major).
  * Needs H % 128 == 0.
+ * Defined by: FP8 transport with the sender quantising and the receiver
+ * restoring, "2kiu.com/news/5702702" section 2.3; one scaling factor per
+ * block, "m.nlpx.cn/news/135159" section 4.1.  The 1x128 block, E4M3 and
+ * fp32 scale are the configuration this library targets; the 1e-4 floor and
+ * the stored dequantisation factor are this library's readings of what the
+ * pages leave open.
  */
 EP_API int ep_dispatch_fp8(const ep_handle *h, const void *x, void *recv_q, float *recv_scales,
                            ep_stream_t stream);
@@ -205,6 +221,9 @@ EP_API int ep_dispatch_fp8(const ep_handle *h, const void *x, void *recv_q, floa
  * starting from 0.  y is [capacity, H] bf16 in the received-row layout of h
  * (expert outputs), topk_weights [T, K] fp32 (4-byte aligned), out [T, H]
  * bf16.  Padding rows are never read; pairs with pos = -1 add nothing.
+ * Defined by: moe_combine of the "lesson14_deepep" practice task (for each
+ * token, weight * expert output added back for k = 0..K-1); combine(x,
+ * handle) of the golden path, bowenzhou.top "deepep/01-overview" section 1.3.
  */
 EP_API int ep_combine(const ep_handle *h, const void *y, const float *topk_weights, void *out,
                       ep_stream_t stream);
@@ -245,12 +264,27 @@ EP_API int ep_copy_routing(const ep_handle *h, int32_t *pos, int32_t *row_src, i
  * clears the part it uses (stream-ordered memset), so calls that overlap on
  * the GPU -- on two streams, or from two threads -- race and must not be
  * issued.  No cudaMalloc, cudaFree or other allocating call is made.
+ * The set-up is kept per device for the life of the process: after a
+ * cudaDeviceReset the library's device state (this set-up, kernel
+ * attributes, every handle) is stale, and calls after a reset in the same
+ * process are not supported.
  */
 EP_API int ep_get_layout_noalloc(const ep_config *cfg, const int64_t *topk_idx, const float *topk_weights,
                                  int32_t *pos, int32_t *row_src, int32_t *row_slot, float *row_weight,
                                  int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
                                  uint8_t *is_token_in_rank, int32_t *expert_offsets, int32_t *rank_offsets,
                                  uint32_t *status, ep_stream_t stream);
+
+/*
+ * Launch shape of the layout for cfg on the current device, host only (the
+ * first query on a device does the same one-time set-up as the first
+ * ep_get_layout_noalloc call): *cluster = 1 when one thread-block cluster
+ * computes it (no scratch), 0 for the cooperative kernel; *ctas = CTAs
+ * launched; *noalloc_scratch_bytes = bytes of the fixed array that
+ * ep_get_layout_noalloc would use (0 for the cluster kernel; a call that
+ * needs more than the array's 256 KiB is rejected).  Any pointer may be NULL.
+ */
+EP_API int ep_layout_shape(const ep_config *cfg, int32_t *cluster, int32_t *ctas, int64_t *noalloc_scratch_bytes);
 
 /*
  * ---- Low-latency (static, masked) layout ----

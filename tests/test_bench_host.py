@@ -126,3 +126,26 @@ def test_clock_sampler_with_fake_nvml(monkeypatch):
     assert out["reasons"] == ["sw_power_cap"]
     assert sys.getswitchinterval() == before
     assert unexpected == []                      # read-only: no other NVML call
+
+
+def test_kernel_figures_writeback_arithmetic():
+    """with_writeback charges each kernel (flush right after it) - (flush of a
+    clean L2); fractions divide algorithmic bytes by time and the peak."""
+    import bench
+    import workloads
+    wl = workloads.generate("dsv3", with_x=False)
+    ms = lambda v: [v * 1e-3] * 3  # noqa: E731  (µs -> ms samples)
+    split = {"layout": ms(13.0), "dispatch": ms(90.0), "combine": ms(80.0),
+             "flush_after_dispatch": ms(50.0), "flush_after_combine": ms(42.0), "flush_clean": ms(40.0)}
+    f = bench.kernel_figures(wl, 32768, split, False, 6500.0)
+    b = 528482304
+    assert f["bytes_per_call"] == {"dispatch": b, "combine": b}
+    assert f["us_per_call"] == {"layout": 13.0, "dispatch": 90.0, "combine": 80.0}
+    wb = f["with_writeback"]
+    assert wb["dispatch_us"] == 100.0 and wb["combine_us"] == 82.0
+    assert abs(wb["dispatch_gbs"] - b / 100e-6 / 1e9) < 0.1
+    assert abs(wb["dispatch_frac"] - b / 100e-6 / 1e9 / 6500.0) < 1e-4
+    assert abs(f["frac_of_8tbs"]["combine"] - b / 80e-6 / 1e9 / 8000.0) < 1e-4
+    # a flush that ran faster than the clean one charges nothing
+    split["flush_after_combine"] = ms(39.0)
+    assert bench.kernel_figures(wl, 32768, split, True, 6500.0)["with_writeback"]["combine_us"] == 80.0

@@ -71,6 +71,18 @@ def test_masked_slots_and_skew():
     run_case(wl, I=256, N=512, idx=idx)
 
 
+def test_bench_shape():
+    """The shape the bench times: one expert-parallel rank of a DeepSeek-V3
+    layer (32 local experts, 4096 tokens x top-8, alignment 128), inner 2048
+    -> 7168 outputs: 32-deep k-block accumulation over 28 column blocks and
+    ~288 row tiles.  256 tokens (both ends and a seeded sample), all 7168
+    columns each, against the oracle."""
+    wl = workloads.generate(None, T=4096, H=7168, E=32, R=8, K=8, A=128, router="topk", seed=5, with_x=False)
+    rng = np.random.default_rng(17)
+    tok = np.unique(np.concatenate([np.arange(32), np.arange(4064, 4096), rng.integers(32, 4064, 200)]))
+    run_case(wl, I=2048, N=7168, check_tokens=tok, seed=5)
+
+
 def test_rejects_unaligned_experts():
     dev = torch.device("cuda")
     wl = workloads.generate(None, T=64, H=128, E=8, R=2, K=2, A=64, router="topk", seed=94)

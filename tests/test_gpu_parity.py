@@ -25,11 +25,22 @@ def _built():
         pytest.skip("no CUDA device")
 
 
-def run_full(wl, fp8: bool, y_seed=99, check_rows=None, check_tokens=None):
+ROW_CHUNK = 16384      # received rows compared per oracle call (bounds host memory)
+TOKEN_CHUNK = 2048     # tokens compared per oracle call
+
+
+def _chunks(sel, n):
+    for i in range(0, len(sel), n):
+        yield sel[i:i + n]
+
+
+def run_full(wl, fp8: bool, y_seed=99, check_rows=None, check_tokens=None, sm_limit=0):
     """Layout + dispatch + combine on the GPU, compared with the oracle.
 
     check_rows / check_tokens: compare only these received rows / tokens
-    (indexing happens on the device); None compares everything."""
+    (indexing happens on the device); None compares every row and every
+    token, in chunks so that host memory stays bounded at any size.
+    sm_limit: cap on the SMs dispatch and combine occupy (0: all)."""
     dev = torch.device("cuda")
     idx, w = wl.topk_idx.numpy(), wl.topk_weights.numpy()
     o = oracle.layout(idx, wl.E, wl.R, wl.A, topk_weights=w)
@@ -37,28 +48,33 @@ def run_full(wl, fp8: bool, y_seed=99, check_rows=None, check_tokens=None):
     g = gpu_layout(wl)
     try:
         assert_layout_equal(g, o)
+        if sm_limit:
+            ep.ep_set_sm_limit(g.handle, sm_limit)
         x_d = wl.x.to(dev)
         xb = workloads.bf16_bits(wl.x)
         cap = g.cap
         sel = np.arange(g.rows, dtype=np.int32) if check_rows is None else np.asarray(check_rows, np.int32)
-        sel_d = torch.from_numpy(sel).long().to(dev)
         if fp8:
             q = torch.full((max(cap, 1), wl.H), 0x5A, dtype=torch.uint8, device=dev)
             s = torch.full((max(cap, 1), wl.H // 128), -3.0, dtype=torch.float32, device=dev)
             ep.ep_dispatch_fp8(g.handle, x_d, q, s)
-            q_h = q[sel_d].cpu().numpy()
-            s_h = s[sel_d].cpu().numpy()
-            oq, osc = oracle.dispatch_fp8(xb, o.row_src, sel)
-            np.testing.assert_array_equal(q_h, oq, err_msg="fp8 codes")
-            np.testing.assert_array_equal(s_h.view(np.uint32), osc.view(np.uint32), err_msg="fp8 scales")
+            for part in _chunks(sel, ROW_CHUNK):
+                part_d = torch.from_numpy(part).long().to(dev)
+                oq, osc = oracle.dispatch_fp8(xb, o.row_src, part)
+                np.testing.assert_array_equal(q[part_d].cpu().numpy(), oq, err_msg="fp8 codes")
+                np.testing.assert_array_equal(s[part_d].cpu().numpy().view(np.uint32), osc.view(np.uint32),
+                                              err_msg="fp8 scales")
             if cap > g.rows:                      # rows beyond `rows` are untouched
                 assert bool((q[g.rows:cap] == 0x5A).all())
+                assert bool((s[g.rows:cap] == -3.0).all())
             del q, s
         else:
             recv = torch.full((max(cap, 1), wl.H), 12345, dtype=torch.int16, device=dev).view(torch.bfloat16)
             ep.ep_dispatch(g.handle, x_d, recv)
-            r_h = workloads.bf16_bits(recv[sel_d])
-            np.testing.assert_array_equal(r_h, oracle.dispatch_bf16(xb, o.row_src, sel), err_msg="bf16 rows")
+            for part in _chunks(sel, ROW_CHUNK):
+                part_d = torch.from_numpy(part).long().to(dev)
+                np.testing.assert_array_equal(workloads.bf16_bits(recv[part_d]),
+                                              oracle.dispatch_bf16(xb, o.row_src, part), err_msg="bf16 rows")
             if cap > g.rows:
                 assert bool((recv[g.rows:cap].view(torch.int16) == 12345).all())
             del recv
@@ -70,15 +86,15 @@ def run_full(wl, fp8: bool, y_seed=99, check_rows=None, check_tokens=None):
         out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
         ep.ep_combine(g.handle, y_d, w_d, out)
         tsel = np.arange(wl.T, dtype=np.int32) if check_tokens is None else np.asarray(check_tokens, np.int32)
-        if len(tsel):
-            need = o.pos[tsel]                     # [n, K] rows those tokens read (-1: masked slot)
+        for part in _chunks(tsel, TOKEN_CHUNK):
+            need = o.pos[part]                     # [n, K] rows those tokens read (-1: masked slot)
             uniq, inv = np.unique(need[need >= 0], return_inverse=True)
             small_pos = np.full(need.shape, -1, np.int32)
             small_pos[need >= 0] = inv
             y_small = workloads.bf16_bits(y_d[torch.from_numpy(uniq).long().to(dev)]) if len(uniq) \
                 else np.zeros((1, wl.H), np.uint16)
-            ref = oracle.combine(y_small, small_pos, w[tsel])
-            combine_close(out[torch.from_numpy(tsel).long().to(dev)], ref)
+            ref = oracle.combine(y_small, small_pos, w[part])
+            combine_close(out[torch.from_numpy(part).long().to(dev)], ref)
         assert ep.ep_get_status(g.handle) == 0
     finally:
         ep.ep_handle_destroy(g.handle)
@@ -93,7 +109,11 @@ SMALL = [
     dict(T=1, H=8, E=1, R=1, K=1, A=1, router="topk", seed=25),
     dict(T=300, H=1024, E=8, R=2, K=8, A=300, router="topk", seed=26),      # A > T*K/E
     dict(T=20000, H=64, E=64, R=8, K=8, A=4, router="topk", seed=27),        # beyond one cluster: cooperative
-    dict(T=16384, H=64, E=256, R=64, K=8, A=2, router="group", seed=28),     # 16-CTA cluster, 8192 pairs each
+    dict(T=16384, H=64, E=256, R=64, K=8, A=2, router="group", seed=28),     # 131072 pairs: cooperative
+    dict(T=8192, H=64, E=256, R=64, K=8, A=2, router="group", seed=30),      # 16-CTA cluster, 4096 pairs each
+    # staged bf16 dispatch whose CTAs walk more than one window of staged
+    # destinations (4096 / K = 64 units per window, ~82 units per CTA)
+    dict(T=12000, H=128, E=128, R=8, K=64, A=1, router="topk", seed=29),
 ]
 
 
@@ -114,20 +134,14 @@ def test_small_parity(spec, fp8):
 
 @pytest.mark.parametrize("name", ["dsv3", "decode", "skew", "large"])
 def test_full_size_parity(name):
-    """Full-size workloads in the launch configuration the bench uses:
-    full layout bit-exact, sampled received rows and tokens."""
+    """Full-size workloads, same seeds and launch configuration as the bench:
+    every layout array, every received row (bf16 rows, or FP8 codes and
+    scales) and every combined token against the oracle."""
     wl = workloads.generate(name)
-    rng = np.random.default_rng(5)
-    cap = wl.T * wl.K + wl.E * (wl.A - 1)
-    o = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A)
-    rows = o.rows
-    sel_rows = np.unique(np.concatenate([[0, rows - 1], rng.integers(0, rows, 1500),
-                                         np.flatnonzero(o.row_src < 0)[:200]]))
-    sel_tok = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 300)]))
-    run_full(wl, wl.fp8, check_rows=sel_rows, check_tokens=sel_tok)
+    run_full(wl, wl.fp8)
     if name == "dsv3":
-        # bench's dsv3 step is bf16; also check the FP8 variant on the same routing
-        run_full(wl, True, check_rows=sel_rows, check_tokens=sel_tok)
+        # the bench's dsv3 step is bf16; the FP8 dispatch on the same routing too
+        run_full(wl, True)
 
 
 def test_identity_round_trip_bf16():
@@ -262,29 +276,15 @@ def test_host_argument_errors():
 
 
 @pytest.mark.parametrize("sms", [1, 7, 24])
-def test_sm_limit_same_results(sms):
-    """Capping dispatch/combine to a few SMs changes the launch, not the results."""
-    dev = torch.device("cuda")
+@pytest.mark.parametrize("fp8", [False, True])
+def test_sm_limit_parity(sms, fp8):
+    """Dispatch and combine capped to a few SMs (ep_set_sm_limit, the num_sms
+    budget of bowenzhou.top "deepep/01-overview" section 1.1) against the
+    oracle.  With one SM the staged bf16 dispatch runs all 1200 tokens in one
+    CTA, so it walks three windows of staged destinations (512 units each at
+    K = 8); the FP8 and combine grids shrink to the cap."""
     wl = workloads.generate(None, T=1200, H=2048, E=64, R=8, K=8, A=4, router="topk", seed=61)
-    outs = []
-    for limit in (0, sms):
-        g = gpu_layout(wl)
-        try:
-            ep.ep_set_sm_limit(g.handle, limit)
-            x = wl.x.to(dev)
-            recv = torch.zeros((g.cap, wl.H), dtype=torch.bfloat16, device=dev)
-            ep.ep_dispatch(g.handle, x, recv)
-            q = torch.zeros((g.cap, wl.H), dtype=torch.uint8, device=dev)
-            sc = torch.zeros((g.cap, wl.H // 128), dtype=torch.float32, device=dev)
-            ep.ep_dispatch_fp8(g.handle, x, q, sc)
-            out = torch.empty_like(x)
-            ep.ep_combine(g.handle, recv, wl.topk_weights.to(dev), out)
-            torch.cuda.synchronize()
-            outs.append([t.cpu() for t in (recv[:g.rows], q[:g.rows], sc[:g.rows], out)])
-        finally:
-            ep.ep_handle_destroy(g.handle)
-    for a, b in zip(*outs):
-        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    run_full(wl, fp8, sm_limit=sms)
 
 
 def test_masked_slots_parity():

@@ -8,7 +8,9 @@ keeps its scratch in a fixed array inside the library.  This test calls it
 through the C ABI several times in a row -- on workloads of different shapes,
 so each call reuses an array the previous one left dirty -- and checks every
 output against the handle-based entry point bit for bit (the layout is
-integer data: the tolerance is zero).
+integer data: the tolerance is zero), and the calls that use the array
+against the CPU oracle too.  ep_layout_shape confirms which calls run the
+cooperative kernel, the one that keeps its scratch in the array.
 
 This file is collected last on purpose, and it also passes alone in a fresh
 process.
@@ -18,6 +20,7 @@ import pytest
 import torch
 
 import combine_ep_get_08_b200 as ep
+import oracle
 import workloads
 from ep_harness import gpu_layout
 
@@ -28,6 +31,7 @@ pytestmark = pytest.mark.gpu
 def _built():
     from combine_ep_get_08_b200 import build_lib
     build_lib.build()
+    oracle.build()
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
 
@@ -84,28 +88,53 @@ def assert_same(na, g):
             np.testing.assert_array_equal(a, b.reshape(a.shape), err_msg=k)
 
 
+def uses_scratch(wl) -> bool:
+    """Whether the layout of wl runs the cooperative kernel (and so keeps its
+    scratch in the fixed array), from the library's own launch plan."""
+    cluster, ctas, need = ep.ep_layout_shape(ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A))
+    assert ctas >= 1
+    assert (need > 0) == (cluster == 0)
+    return need > 0
+
+
+def assert_oracle(na, wl):
+    o = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A, topk_weights=wl.topk_weights.numpy())
+    assert o.status == 0 and na["rows"] == o.rows
+    for k in KEYS:
+        a, b = na[k], getattr(o, k)
+        np.testing.assert_array_equal(a.reshape(-1), b.reshape(-1), err_msg=f"{k} vs oracle")
+
+
 def test_matches_handle_layout_calls_in_a_row():
     shapes = [
-        workloads.generate("dsv3", with_x=False),                       # an 8-CTA cluster
-        workloads.generate(None, T=700, H=256, E=64, R=8, K=6, A=5,
-                           router="topk", seed=77, with_x=False),
-        workloads.generate(None, T=20000, H=64, E=64, R=8, K=8, A=3,    # beyond one cluster: the
-                           router="topk", seed=78, with_x=False),       # cooperative kernel and its scratch
-        workloads.generate("skew", with_x=False),                        # expert_alignment 128
-        workloads.generate("decode", with_x=False),                      # one CTA, no grid-wide wait
-        workloads.generate("dsv3", seed=11, with_x=False),               # back to the first shape
+        (workloads.generate("dsv3", with_x=False), False),              # a thread-block cluster
+        (workloads.generate(None, T=700, H=256, E=64, R=8, K=6, A=5,
+                            router="topk", seed=77, with_x=False), False),
+        (workloads.generate(None, T=20000, H=64, E=64, R=8, K=8, A=3,   # beyond one cluster: the
+                            router="topk", seed=78, with_x=False), True),  # cooperative kernel, the array
+        (workloads.generate("skew", with_x=False), False),               # expert_alignment 128
+        (workloads.generate("decode", with_x=False), False),             # one CTA, no grid-wide wait
+        (workloads.generate(None, T=12000, H=64, E=128, R=16, K=8, A=2,  # the array again, other
+                            router="group", seed=79, with_x=False), True),  # columns and chunk count
+        (workloads.generate("dsv3", seed=11, with_x=False), False),      # back to the first shape
     ]
-    for wl in shapes:
-        assert_same(noalloc_layout(wl), handle_layout(wl))
+    for wl, scratch in shapes:
+        assert uses_scratch(wl) == scratch
+        na = noalloc_layout(wl)
+        assert_same(na, handle_layout(wl))
+        if scratch:
+            assert_oracle(na, wl)
 
 
 def test_same_call_twice():
     wl = workloads.generate("large", with_x=False)
+    assert uses_scratch(wl)                    # 131 072 pairs: the cooperative kernel
     first = noalloc_layout(wl)
     second = noalloc_layout(wl)
     for k in KEYS:
         np.testing.assert_array_equal(first[k], second[k], err_msg=k)
     assert_same(second, handle_layout(wl))
+    assert_oracle(second, wl)
 
 
 def test_rejects_sizes_beyond_the_array():
