@@ -187,7 +187,7 @@ def measured_peak():
 
 
 # the sources of the step's kernels (layout, dispatch, combine) and their shared header
-STEP_KERNEL_SOURCES = ("combine.cu", "dispatch.cu", "ep_internal.cuh", "fp8_block.cuh", "layout.cu")
+STEP_KERNEL_SOURCES = ("combine.cu", "dispatch.cu", "dispatch_lb.cu", "ep_internal.cuh", "fp8_block.cuh", "layout.cu")
 
 
 def kernel_source_digest() -> str:
@@ -394,12 +394,41 @@ class LLPath(Path):
                               stream=stream)
 
 
+class FusedPath(Path):
+    """Layout and the step's first dispatch in one call (ep_layout_dispatch:
+    a counts pre-pass, then the dispatch ranks its chunks and places them by
+    decoupled look-back); later dispatches of the step reuse the handle."""
+
+    def __init__(self, wl, dev):
+        super().__init__(wl, dev)
+        self._pending = None
+
+    def layout(self, stream, idx=None, w=None):
+        self._pending = (self.idx if idx is None else idx, self.w if w is None else w)
+
+    def dispatch(self, stream, x=None, idx=None):
+        if self._pending is None:
+            return super().dispatch(stream, x=x)
+        x = self.x if x is None else x
+        idx, w = self._pending
+        self._pending = None
+        if self.wl.fp8:
+            self.ep.ep_layout_dispatch_fp8(self.h, idx, w, x, self.recv, self.scales, stream=stream)
+        else:
+            self.ep.ep_layout_dispatch(self.h, idx, w, x, self.recv, stream=stream)
+
+
 def make_path(name, mode, dev, rank, ll_slots=0):
     """The named workload (rank-seeded) and its device buffers and handle."""
     import workloads
     base = workloads.CONFIGS[name]
     wl = workloads.generate(name, seed=base["seed"] + 1000 * rank)
-    path = LLPath(wl, dev, ll_slots or max(wl.T, 1)) if mode == "ll" else Path(wl, dev)
+    if mode == "ll":
+        path = LLPath(wl, dev, ll_slots or max(wl.T, 1))
+    elif mode == "fused":
+        path = FusedPath(wl, dev)
+    else:
+        path = Path(wl, dev)
     return wl, path
 
 
@@ -501,7 +530,7 @@ def config_summary(name, mode, args, dev, rank, stream, peak, steps, warmup):
 
     import combine_ep_get_08_b200 as ep
     import workloads
-    ll = mode == "ll"
+    ll = mode in ("ll", "fused")        # no separate layout launch
     wl, path = make_path(name, mode, dev, rank)
     try:
         reuse = wl.reuse
@@ -522,7 +551,7 @@ def config_summary(name, mode, args, dev, rank, stream, peak, steps, warmup):
         mean_dis = statistics.mean(split["dispatch"])
         step_ms = statistics.mean([ld + (reuse - 1) * mean_dis + reuse * c for ld, c in zip(ld_ms, com_ms)])
         bytes_step = reuse * (fig["bytes_per_call"]["dispatch"] + fig["bytes_per_call"]["combine"])
-        entry = {"workload": workloads.DESCRIPTIONS[name] + (" (low-latency static layout)" if ll else ""),
+        entry = {"workload": workloads.DESCRIPTIONS[name] + MODE_NOTE[mode],
                  "steps": steps, "rows": rows, "reuse": reuse,
                  "step_us": round(step_ms * 1e3, 2), "step_gbs": round(bytes_step / (step_ms * 1e-3) / 1e9, 1),
                  "us_layout_then_dispatch": round(statistics.mean(ld_ms) * 1e3, 2)}
@@ -535,7 +564,10 @@ def config_summary(name, mode, args, dev, rank, stream, peak, steps, warmup):
         path.close()
 
 
-PER_CONFIG = (("tiny", "normal"), ("decode", "normal"), ("decode", "ll"), ("skew", "normal"), ("large", "normal"))
+PER_CONFIG = (("dsv3", "fused"), ("tiny", "normal"), ("decode", "normal"), ("decode", "ll"), ("decode", "fused"),
+              ("skew", "normal"), ("skew", "fused"), ("large", "normal"), ("large", "fused"))
+MODE_NOTE = {"normal": "", "ll": " (low-latency static layout)",
+             "fused": " (layout fused into the dispatch: ep_layout_dispatch)"}
 
 
 def run_cuda(args, world, rank, local):
@@ -556,7 +588,7 @@ def run_cuda(args, world, rank, local):
     barrier(world)
     ep.library()
 
-    ll = args.mode == "ll"
+    ll = args.mode in ("ll", "fused")   # no separate layout launch
     wl, path = make_path(args.config, args.mode, dev, rank, args.ll_slots)
     reuse = wl.reuse if args.reuse is None else args.reuse
     if args.sm_limit:
@@ -622,17 +654,18 @@ def run_cuda(args, world, rank, local):
     dom_bytes = b_dis if dom == "dispatch" else b_com
     achieved = dom_bytes / (kern[dom] * 1e-6) / 1e9
     wb = fig["with_writeback"]
-    kname, traffic = ncu_traffic(dom, args.config + ("-ll" if ll else ""))
+    kname, traffic = ncu_traffic(dom, args.config + ("" if args.mode == "normal" else "-" + args.mode))
     clocks = sampler.summary()
     status_end = ep.ep_get_status(path.h)
     path.close()
 
     per_config = None
-    if world == 1 and not args.no_per_config and args.config == "dsv3" and not ll and not args.sm_limit:
+    if world == 1 and not args.no_per_config and args.config == "dsv3" and args.mode == "normal" \
+            and not args.sm_limit:
         n = max(5, min(args.steps, 20))
         per_config = {}
         for name, mode in PER_CONFIG:
-            per_config[name + ("_ll" if mode == "ll" else "")] = config_summary(
+            per_config[name + ("" if mode == "normal" else "_" + mode)] = config_summary(
                 name, mode, args, dev, rank, stream, peak, n, args.warmup)
 
     if rank == 0:
@@ -644,8 +677,11 @@ def run_cuda(args, world, rank, local):
             "config": {
                 "workload": workloads.DESCRIPTIONS[args.config], "name": args.config,
                 "rows": rows, "reuse": reuse,
-                "layout_mode": (f"low-latency static: {path.M} slots per expert, layout fused into "
-                                "the dispatch launch" if ll else "normal: padded expert-major rows"),
+                "layout_mode": {"ll": f"low-latency static: {getattr(path, 'M', 0)} slots per expert, layout "
+                                      "fused into the dispatch launch",
+                                "fused": "normal padded expert-major rows; layout and dispatch in one call "
+                                         "(counts pre-pass + dispatch with decoupled look-back)",
+                                "normal": "normal: padded expert-major rows (ep_get_layout, then ep_dispatch)"}[args.mode],
                 "parallelism": f"replicas x{world} (independent batches, no data-path collective)",
                 "sm_limit": args.sm_limit or None,
                 "l2": "flushed (256 MiB read, outside the timed events) before each step and "
@@ -1156,8 +1192,9 @@ def main(argv=None):
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per_config block (the other four workloads, measured after dsv3)")
     ap.add_argument("--sm-limit", type=int, default=0, help="SMs dispatch/combine may occupy (0: all)")
-    ap.add_argument("--mode", choices=["normal", "ll"], default="normal",
-                    help="layout: normal (padded, ep_get_layout) or low-latency static slots (ep_ll_*)")
+    ap.add_argument("--mode", choices=["normal", "ll", "fused"], default="normal",
+                    help="layout: normal (padded, ep_get_layout then ep_dispatch), fused (ep_layout_dispatch) "
+                         "or low-latency static slots (ep_ll_*)")
     ap.add_argument("--ll-slots", type=int, default=0, help="slots per expert in --mode ll (0: T)")
     ap.add_argument("--ncu-ingest", metavar="REP", help="record DRAM traffic from an ncu report and exit")
     ap.add_argument("--peer", action="store_true",
@@ -1166,7 +1203,7 @@ def main(argv=None):
                     help="time ep_expert_combine (expert GEMM + fused combine) instead of the step")
     args = ap.parse_args(argv)
     if args.ncu_ingest:
-        return ncu_ingest(args.ncu_ingest, args.config + ("-ll" if args.mode == "ll" else ""))
+        return ncu_ingest(args.ncu_ingest, args.config + ("" if args.mode == "normal" else "-" + args.mode))
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_env()

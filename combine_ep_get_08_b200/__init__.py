@@ -74,6 +74,8 @@ def _load():
             "ep_get_layout_noalloc": ([CFG] + [P] * 13, ctypes.c_int),
             "ep_layout_shape": ([CFG, ctypes.POINTER(I32), ctypes.POINTER(I32), ctypes.POINTER(I64)], ctypes.c_int),
             "ep_dispatch": ([P, P, P, P], ctypes.c_int),
+            "ep_layout_dispatch": ([P] * 11, ctypes.c_int),
+            "ep_layout_dispatch_fp8": ([P] * 12, ctypes.c_int),
             "ep_dispatch_fp8": ([P, P, P, P, P], ctypes.c_int),
             "ep_combine": ([P, P, P, P, P], ctypes.c_int),
             "ep_copy_routing": ([P, P, P, P, P, P], ctypes.c_int),
@@ -214,6 +216,24 @@ def ep_layout_shape(cfg: ep_config) -> tuple[int, int, int]:
 
 def ep_dispatch(h: int, x, recv_x, stream=None) -> None:
     _check("ep_dispatch", _load().ep_dispatch(h, _ptr(x), _ptr(recv_x), _stream(stream)))
+
+
+def ep_layout_dispatch(h: int, topk_idx, topk_weights, x, recv_x, num_tokens_per_expert=None,
+                       num_tokens_per_rank=None, is_token_in_rank=None, expert_offsets=None, rank_offsets=None,
+                       stream=None) -> None:
+    _check("ep_layout_dispatch", _load().ep_layout_dispatch(
+        h, _ptr(topk_idx), _ptr(topk_weights), _ptr(x), _ptr(recv_x), _ptr(num_tokens_per_expert),
+        _ptr(num_tokens_per_rank), _ptr(is_token_in_rank), _ptr(expert_offsets), _ptr(rank_offsets),
+        _stream(stream)))
+
+
+def ep_layout_dispatch_fp8(h: int, topk_idx, topk_weights, x, recv_q, recv_scales, num_tokens_per_expert=None,
+                           num_tokens_per_rank=None, is_token_in_rank=None, expert_offsets=None,
+                           rank_offsets=None, stream=None) -> None:
+    _check("ep_layout_dispatch_fp8", _load().ep_layout_dispatch_fp8(
+        h, _ptr(topk_idx), _ptr(topk_weights), _ptr(x), _ptr(recv_q), _ptr(recv_scales),
+        _ptr(num_tokens_per_expert), _ptr(num_tokens_per_rank), _ptr(is_token_in_rank), _ptr(expert_offsets),
+        _ptr(rank_offsets), _stream(stream)))
 
 
 def ep_dispatch_fp8(h: int, x, recv_q, recv_scales, stream=None) -> None:

@@ -1,0 +1,699 @@
+// dispatch_lb.cu -- the layout fused with the dispatch (sm_100a).
+//
+// ep_layout_dispatch / ep_layout_dispatch_fp8 compute exactly what
+// ep_get_layout followed by ep_dispatch / ep_dispatch_fp8 computes, in two
+// launches that overlap:
+//
+//   layout_counts_kernel   one CTA per super-chunk of kLbSuper token chunks:
+//     the expert and distinct-rank histograms of its tokens and their
+//     is_token_in_rank rows.  The last CTA to arrive (an arrival counter,
+//     nobody waits) adds the histograms up, forms the padded expert offsets
+//     (expert_alignment, bowenzhou.top "deepep/01-overview" section 1.1) and,
+//     for each super-chunk, the row where its pairs of each expert start.
+//
+//   dispatch_lb_kernel     one CTA per SM.  CTAs take token chunks in launch
+//     order from an atomic ticket.  A chunk's pairs are ranked with warp
+//     ballots, so that inside an expert the rows follow (token, k) order --
+//     the order in which the moe_dispatch loop of the "lesson14_deepep"
+//     practice task appends tokens to each expert's queue.  The chunk then
+//     publishes its per-expert counts and finds how many pairs of each
+//     expert the earlier chunks of its super-chunk hold by decoupled
+//     look-back (the single-pass scan of Merrill and Garland, "Single-pass
+//     Parallel Prefix Scan with Decoupled Look-back", 2016): each chunk
+//     publishes first its own count (an aggregate) and, once known, its
+//     running total (an inclusive prefix); a chunk reads its predecessors'
+//     words back to the first running total.  Chunks are taken in launch
+//     order and publish their aggregate before they wait, so every wait is
+//     on a chunk whose CTA is running and will publish without waiting; every
+//     wait is bounded by %globaltimer (EP_DEV_WAIT_TIMEOUT).  All of this
+//     reads only topk_idx, so it runs before the dependency wait, beside the
+//     pre-pass.  After it, a pair's row is its super-chunk's base + the
+//     look-back prefix + its rank, and the chunk's x rows stream through a
+//     shared-memory ring of bulk copies (TMA engine, no multicast) to their
+//     rows: a plain copy (bf16), or the fused 1x128-block FP8 E4M3
+//     quantisation of "m.nlpx.cn/news/135159" section 4.1.  One warp writes
+//     the padding rows (zeros, and -1 routing) with bulk copies meanwhile.
+//
+// With lb = 0 the same kernel takes the positions from the handle (a layout
+// computed earlier) and is a chunked, dynamically scheduled dispatch.
+#include "ep_internal.cuh"
+#include "fp8_block.cuh"
+
+#ifndef EP_LB_FP8_GROUPS
+#define EP_LB_FP8_GROUPS 2          // FP8 consumer groups per CTA (quantisation needs more warps)
+#endif
+#ifndef EP_LB_RING_BYTES
+#define EP_LB_RING_BYTES (112 * 1024)
+#endif
+
+namespace ep {
+
+namespace {
+
+constexpr int kGroupWarps = 7;          // warps per consumer group
+constexpr int kGroupThreads = kGroupWarps * 32;
+constexpr int kLayoutRankWarps = 8;     // warps that rank a chunk's pairs
+constexpr int kMaxStages = 16;
+constexpr int kZeroBytes = 8192;        // zeroed shared memory the padding warp copies from
+constexpr int kFp8Ept = 32;             // FP8: bf16 elements per consumer thread
+
+template <int G>
+struct Shape {
+    static constexpr int kSetThreads = 32 + G * kGroupThreads;   // producer warp + consumer groups
+    static constexpr int kThreads = kSetThreads + 32;            // + the padding warp
+    static constexpr int kPadWarp = kThreads / 32 - 1;
+};
+
+__host__ __device__ __forceinline__ size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Dynamic shared memory carve-up (same on host and device).
+struct Carve {
+    size_t ring, bars, zeros, pos, e16, rk16, cnt, base, agg, total;
+};
+__host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int E) {
+    Carve c;
+    size_t o = 0;
+    c.ring = o;  o += up((size_t)stages * chunk_bytes, 128);
+    c.bars = o;  o += 2 * kMaxStages * sizeof(uint64_t);
+    c.zeros = o; o += kZeroBytes;
+    c.pos = o;   o += (size_t)kLbMaxPairs * sizeof(int32_t);
+    c.e16 = o;   o += (size_t)kLbMaxPairs * sizeof(int16_t);
+    c.rk16 = o;  o += (size_t)kLbMaxPairs * sizeof(int16_t);
+    c.cnt = o;   o += (size_t)kLayoutRankWarps * (E + 1) * sizeof(int32_t);
+    c.base = o;  o += (size_t)E * sizeof(int32_t);
+    c.agg = o;   o += (size_t)E * sizeof(int32_t);
+    c.total = up(o, 128);
+    return c;
+}
+
+// named barrier 1: the producer warp and the consumer groups (the padding
+// warp runs on its own and never takes part)
+__device__ __forceinline__ void set_sync(int nthreads) {
+    asm volatile("bar.sync 1, %0;" : : "r"(nthreads) : "memory");
+}
+
+// Look-back word of (chunk, expert): the count in the low 32 bits; the high
+// 32 bits are tag << 1 | inclusive, tag = the launch's epoch tag (1 ..
+// 2^31 - 1), so zeroed words and words of earlier launches read as "not
+// published yet".
+__device__ __forceinline__ unsigned long long lb_word(unsigned int tag, bool inclusive, int v) {
+    return ((unsigned long long)((tag << 1) | (inclusive ? 1u : 0u)) << 32) | (unsigned int)v;
+}
+__device__ __forceinline__ unsigned int lb_tag(unsigned long long w) { return (unsigned int)(w >> 33); }
+__device__ __forceinline__ bool lb_inclusive(unsigned long long w) { return (w >> 32) & 1ull; }
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" : : "l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ bool valid_id(int64_t e, int E) { return e >= 0 && e < E; }
+
+__device__ __forceinline__ int64_t scale_at(const LbParams &p, int row, int b, int NB) {
+    return p.scale_ld == 0 ? (int64_t)row * NB + b : (int64_t)b * p.scale_ld + row;
+}
+
+// ---------------------------------------------------------------------------
+// Counts pre-pass
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kLayoutThreads, 1) layout_counts_kernel(LbParams p) {
+    extern __shared__ int32_t smem_c[];
+    const int E = p.E, R = p.R, K = p.K, L = p.L, ncols = E + R;
+    int32_t *s_hist = smem_c;            // [E+R] this super-chunk's counts, later the totals
+    int32_t *s_eoff = s_hist + ncols;    // [E+1] padded expert offsets
+    __shared__ int32_t s_tmp[kLayoutWarps + 1];
+    __shared__ int s_last;
+    const int tid = threadIdx.x;
+    pdl_launch_dependents();             // the dispatch may start its own layout work now
+
+    const int tps = p.tpc * kLbSuper;
+    const int t0 = min(p.T, (int)blockIdx.x * tps), t1 = min(p.T, t0 + tps);
+    for (int j = tid; j < ncols; j += kLayoutThreads) s_hist[j] = 0;
+    __syncthreads();
+    for (int64_t q = (int64_t)t0 * K + tid; q < (int64_t)t1 * K; q += kLayoutThreads) {
+        const int64_t e = __ldg(p.topk_idx + q);
+        if (valid_id(e, E))
+            atomicAdd(&s_hist[e], 1);
+        else if (e != -1)
+            atomicOr(p.status, EP_DEV_BAD_EXPERT);   // -1: a masked top-k slot
+    }
+    // distinct ranks of each token, and its is_token_in_rank row
+    for (int t = t0 + tid; t < t1; t += kLayoutThreads) {
+        const int64_t *row = p.topk_idx + (int64_t)t * K;
+        uint8_t *dst = p.u_in_rank ? p.u_in_rank + (int64_t)t * R : nullptr;
+        if (R <= 64) {
+            unsigned long long mask = 0;
+            for (int k = 0; k < K; ++k) {
+                const int64_t e = __ldg(row + k);
+                if (valid_id(e, E)) mask |= 1ull << (int)(e / L);
+            }
+            for (unsigned long long m = mask; m; m &= m - 1) atomicAdd(&s_hist[E + __ffsll((long long)m) - 1], 1);
+            if (dst)
+                for (int r = 0; r < R; ++r) dst[r] = (uint8_t)((mask >> r) & 1ull);
+        } else {
+            if (dst)
+                for (int r = 0; r < R; ++r) dst[r] = 0;
+            for (int k = 0; k < K; ++k) {
+                const int64_t e = __ldg(row + k);
+                if (!valid_id(e, E)) continue;
+                const int r = (int)(e / L);
+                bool dup = false;
+                for (int k2 = 0; k2 < k; ++k2) {
+                    const int64_t e2 = __ldg(row + k2);
+                    if (valid_id(e2, E) && (int)(e2 / L) == r) dup = true;
+                }
+                if (!dup) atomicAdd(&s_hist[E + r], 1);
+                if (dst) dst[r] = 1;
+            }
+        }
+    }
+    __syncthreads();
+    int32_t *mine = p.super_hist + (size_t)blockIdx.x * ncols;
+    for (int j = tid; j < ncols; j += kLayoutThreads) mine[j] = s_hist[j];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&p.ctl->pre_arrivals, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+
+    // the last CTA: every histogram is published
+    __threadfence();
+    const int ns = gridDim.x;
+    for (int j = tid; j < ncols; j += kLayoutThreads) {
+        int tot = 0;
+#pragma unroll 4
+        for (int s = 0; s < ns; ++s) tot += __ldcg(p.super_hist + (size_t)s * ncols + j);
+        s_hist[j] = tot;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kLayoutThreads) s_eoff[e] = (s_hist[e] + p.A - 1) / p.A * p.A;
+    __syncthreads();
+    const int rows = block_exclusive_scan(s_eoff, E, s_tmp);
+    if (tid == 0) s_eoff[E] = rows;
+    __syncthreads();
+    for (int e = tid; e < E; e += kLayoutThreads) {
+        p.cnt[e] = s_hist[e];
+        if (p.u_cnt) p.u_cnt[e] = s_hist[e];
+        int run = s_eoff[e];
+#pragma unroll 4
+        for (int s = 0; s < ns; ++s) {
+            p.super_base[(size_t)s * E + e] = run;
+            run += __ldcg(p.super_hist + (size_t)s * ncols + e);
+        }
+    }
+    for (int e = tid; e <= E; e += kLayoutThreads) {
+        p.eoff[e] = s_eoff[e];
+        if (p.u_eoff) p.u_eoff[e] = s_eoff[e];
+    }
+    for (int r = tid; r < R; r += kLayoutThreads) {
+        p.rank_tok[r] = s_hist[E + r];
+        if (p.u_rank_tok) p.u_rank_tok[r] = s_hist[E + r];
+    }
+    for (int r = tid; r <= R; r += kLayoutThreads) {
+        p.roff[r] = s_eoff[r * L];
+        if (p.u_roff) p.u_roff[r] = s_eoff[r * L];
+    }
+    if (tid == 0) atomicExch(&p.ctl->pre_arrivals, 0u);   // every CTA has arrived: ready for the next launch
+}
+
+// ---------------------------------------------------------------------------
+// Padding rows: the padding warp takes experts blockIdx.x + (lane + 32 i) *
+// gridDim.x and writes their padding rows (rows eoff[e] + cnt[e] ..
+// eoff[e+1]) with bulk shared->global copies of a zeroed block: zero bf16
+// rows, or zero codes and zero scales; with lb = 1 also their routing
+// (row_src = row_slot = -1, row_weight = 0).
+// ---------------------------------------------------------------------------
+template <bool FP8>
+__device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros, int lane) {
+    pdl_wait();   // offsets and counts come from the kernel before
+    const int row_bytes = FP8 ? p.H : 2 * p.H;
+    const int NB = p.H / 128;
+    uint8_t *recv = static_cast<uint8_t *>(p.recv);
+    for (int e = blockIdx.x + lane * gridDim.x; e < p.E; e += 32 * gridDim.x) {
+        const int r0 = __ldcg(p.eoff + e) + __ldcg(p.cnt + e), r1 = __ldcg(p.eoff + e + 1);
+        for (int r = r0; r < r1; ++r) {
+            if (p.lb) {
+                p.row_src[r] = -1;
+                p.row_slot[r] = -1;
+                if (p.topk_weights) p.row_weight[r] = 0.0f;
+            }
+            uint8_t *o = recv + (int64_t)r * row_bytes;
+            for (int off = 0; off < row_bytes; off += kZeroBytes)
+                bulk_s2g(o + off, zeros, (uint32_t)min(kZeroBytes, row_bytes - off));
+            if (FP8)
+                for (int b = 0; b < NB; ++b) p.recv_scale[scale_at(p, r, b, NB)] = 0.0f;
+        }
+        bulk_commit();
+    }
+    bulk_wait_all();
+}
+
+// bf16 unit: copy the staged part of a token row to its K rows.
+template <int VB>
+__device__ __forceinline__ void copy_unit(const LbParams &p, const uint8_t *src, const int32_t *dsts, int part,
+                                          int gtid, uint64_t pol) {
+    const int row_bytes = 2 * p.H, chunk = p.chunk_bytes, nv = chunk / VB;
+    uint8_t *recv = static_cast<uint8_t *>(p.recv);
+    for (int v = gtid; v < nv; v += kGroupThreads) {
+        if constexpr (VB == 32) {
+            const uint4 a = *reinterpret_cast<const uint4 *>(src + v * 32);
+            const uint4 b = *reinterpret_cast<const uint4 *>(src + v * 32 + 16);
+            u32x8 val;
+            val.v[0] = a.x; val.v[1] = a.y; val.v[2] = a.z; val.v[3] = a.w;
+            val.v[4] = b.x; val.v[5] = b.y; val.v[6] = b.z; val.v[7] = b.w;
+            for (int k = 0; k < p.K; ++k) {
+                const int dst = dsts[k];
+                if (dst >= 0) st_v8_policy(recv + (int64_t)dst * row_bytes + (int64_t)part * chunk + v * 32, val, pol);
+            }
+        } else {
+            const uint4 val = *reinterpret_cast<const uint4 *>(src + v * 16);
+            for (int k = 0; k < p.K; ++k) {
+                const int dst = dsts[k];
+                if (dst >= 0) st_v4_policy(recv + (int64_t)dst * row_bytes + (int64_t)part * chunk + v * 16, val, pol);
+            }
+        }
+    }
+}
+
+// FP8 unit: thread gtid quantises elements [gtid*32, gtid*32+32) of the
+// staged part (4 consecutive lanes per 1x128 block) and stores the 32 code
+// bytes to each of the K rows; the block's first lane stores its scale.
+__device__ __forceinline__ void quantise_unit(const LbParams &p, const uint8_t *src, const int32_t *dsts, int part,
+                                              int gtid, uint64_t pol) {
+    constexpr int TPB = 128 / kFp8Ept, NW = kFp8Ept / 2;
+    const int U = p.chunk_bytes / 2;           // elements per unit (a multiple of 128)
+    const bool act = gtid * kFp8Ept < U;       // whole blocks of 4 lanes are active or idle
+    unsigned int w[NW];
+    if (act) {
+#pragma unroll
+        for (int i = 0; i < NW / 4; ++i) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(src + gtid * 2 * kFp8Ept + 16 * i);
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < NW; ++i) w[i] = 0;
+    }
+    unsigned int q[8];
+    const float scale = quantize_block<TPB, NW>(w, q);   // every lane of the warp takes part
+    if (!act) return;
+    const int col = part * U + gtid * kFp8Ept;
+    const int NB = p.H / 128, b = col / 128;
+    const bool lead = (gtid % TPB) == 0;
+    u32x8 v;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v.v[i] = q[i];
+    uint8_t *recv = static_cast<uint8_t *>(p.recv);
+    for (int k = 0; k < p.K; ++k) {
+        const int dst = dsts[k];
+        if (dst < 0) continue;
+        uint8_t *o = recv + (int64_t)dst * p.H + col;
+        if (p.vec32) {
+            st_v8_policy(o, v, pol);
+        } else {   // a 16-byte aligned buffer
+            st_v4_policy(o, make_uint4(q[0], q[1], q[2], q[3]), pol);
+            st_v4_policy(o + 16, make_uint4(q[4], q[5], q[6], q[7]), pol);
+        }
+        if (lead) p.recv_scale[scale_at(p, dst, b, NB)] = scale;
+    }
+}
+
+template <int VB, bool FP8, int G>
+__global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbParams p) {
+    using S = Shape<G>;
+    constexpr int NSET = S::kSetThreads;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const Carve cv = carve(p.stages, p.chunk_bytes, p.E);
+    uint8_t *ring = smem + cv.ring;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + cv.bars);
+    uint64_t *empty = full + kMaxStages;
+    uint8_t *zeros = smem + cv.zeros;
+    int32_t *s_pos = reinterpret_cast<int32_t *>(smem + cv.pos);
+    int16_t *s_e = reinterpret_cast<int16_t *>(smem + cv.e16);
+    int16_t *s_rk = reinterpret_cast<int16_t *>(smem + cv.rk16);
+    int32_t *s_cnt = reinterpret_cast<int32_t *>(smem + cv.cnt);
+    int32_t *s_base = reinterpret_cast<int32_t *>(smem + cv.base);
+    int32_t *s_agg = reinterpret_cast<int32_t *>(smem + cv.agg);
+    __shared__ int s_ticket;
+    __shared__ int s_abort;
+    __shared__ unsigned int s_tag;
+    volatile int *abort_flag = &s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int E = p.E, K = p.K, ES = E + 1, NS = p.stages, chunk = p.chunk_bytes;
+    const int row_bytes = 2 * p.H;   // bytes of an x row
+    const bool padding = p.A > 1;
+    const uint8_t *x = static_cast<const uint8_t *>(p.x);
+
+    if (padding) {
+        for (int i = tid; i < kZeroBytes / 16; i += S::kThreads) reinterpret_cast<uint4 *>(zeros)[i] = make_uint4(0, 0, 0, 0);
+        fence_async_smem();
+    }
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kGroupWarps);
+        }
+        fence_async_smem();
+        s_abort = 0;
+        // the previous launch's tag is stable: it changes only after every CTA
+        // of that launch finished, and that launch completed before this one
+        s_tag = (__ldcg(&p.ctl->epoch) % 0x7fffffffu) + 1u;
+    }
+    __syncthreads();
+
+    if (warp == S::kPadWarp) {
+        if (padding) pad_rows<FP8>(p, zeros, lane);
+    } else {
+        const uint64_t pol_out = policy_evict_first();
+        const uint64_t pol_x = policy_evict_last();
+        int unit_base = 0;     // units of earlier chunks of this CTA (ring stage and phase)
+        int issued = 0;        // producer: units whose load was issued
+        bool waited = false;
+        // the producer's load of chunk unit i (lane 0 of warp 0); false on a timeout
+        auto issue = [&](int t0, int i) -> bool {
+            const int g = unit_base + i, s = g % NS;
+            if (g >= NS && !mbar_wait_bounded(&empty[s], ((g / NS) - 1) & 1, p.wait_limit_ns)) return false;
+            const int t = t0 + i / p.splits, part = i - (i / p.splits) * p.splits;
+            mbar_arrive_expect_tx(&full[s], chunk);
+            bulk_g2s(ring + (size_t)s * chunk, x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk, &full[s]);
+            ++issued;
+            return true;
+        };
+        for (;;) {
+            set_sync(NSET);
+            if (tid == 0) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
+            set_sync(NSET);
+            const int c = s_ticket;
+            if (c >= p.nchunks || *abort_flag) break;
+            const int t0 = c * p.tpc, t1 = min(p.T, t0 + p.tpc);
+            const int nt = t1 - t0, nu = nt * p.splits, n = nt * K;
+            const int64_t q0 = (int64_t)t0 * K;
+
+            // the chunk's first units into the ring (their stages are free: every
+            // earlier unit was consumed before the last set barrier) and all of
+            // its x rows into L2
+            if (tid == 0) {
+                if (p.prefetch_x)
+                    for (int t = t0; t < t1; ++t) bulk_prefetch_l2(x + (int64_t)t * row_bytes, (uint32_t)row_bytes, pol_x);
+                for (int i = 0; i < min(NS, nu); ++i)
+                    if (!issue(t0, i)) {
+                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *abort_flag = 1;
+                        break;
+                    }
+            }
+            __syncwarp();
+
+            const int ppw = (n + kLayoutRankWarps * 32 - 1) / (kLayoutRankWarps * 32) * 32;   // pairs per ranking warp
+            if (p.lb) {
+                // ranks: warp w walks pairs [w*ppw, (w+1)*ppw) 32 at a time; a
+                // lane's rank is its warp's running count of its expert plus the
+                // lanes below it with the same expert (ballots over the id bits)
+                if (warp < kLayoutRankWarps) {
+                    int32_t *wrow = s_cnt + warp * ES;
+                    for (int e = lane; e < ES; e += 32) wrow[e] = 0;
+                    __syncwarp();
+                    const int lo = warp * ppw, hi = min(n, lo + ppw);
+                    for (int j0 = lo; j0 < hi; j0 += 32 * 8) {
+                        int64_t v[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int i = j0 + u * 32 + lane;
+                            v[u] = i < hi ? __ldg(p.topk_idx + q0 + i) : (int64_t)-1;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            if (j0 + u * 32 >= hi) break;   // warp-uniform
+                            const int i = j0 + u * 32 + lane;
+                            const int e = valid_id(v[u], E) ? (int)v[u] : -1;
+                            if (i < hi && e < 0 && v[u] != -1) atomicOr(p.status, EP_DEV_BAD_EXPERT);
+                            unsigned int peers = __ballot_sync(0xffffffffu, e >= 0);
+                            if (e < 0) peers = ~peers;
+                            for (int bit = 0; bit < p.id_bits; ++bit) {
+                                const int bv = (e >> bit) & 1;
+                                const unsigned int bal = __ballot_sync(0xffffffffu, bv);
+                                peers &= bv ? bal : ~bal;
+                            }
+                            const int lrank = __popc(peers & lanemask_lt());
+                            const int base = e >= 0 ? wrow[e] : 0;
+                            __syncwarp();
+                            if (e >= 0 && lrank == 0) wrow[e] = base + __popc(peers);
+                            __syncwarp();
+                            if (i < hi) {
+                                s_e[i] = (int16_t)e;
+                                s_rk[i] = (int16_t)(base + lrank);
+                            }
+                        }
+                    }
+                }
+                set_sync(NSET);
+                // each expert's counts become exclusive prefixes over the ranking
+                // warps; their total is the chunk's aggregate
+                for (int e = tid; e < E; e += NSET) {
+                    int run = 0;
+#pragma unroll
+                    for (int w = 0; w < kLayoutRankWarps; ++w) {
+                        const int vv = s_cnt[w * ES + e];
+                        s_cnt[w * ES + e] = run;
+                        run += vv;
+                    }
+                    s_agg[e] = run;
+                }
+                set_sync(NSET);
+                // publish, then look back over the earlier chunks of the super-chunk
+                const int c0 = c / kLbSuper * kLbSuper;
+                const unsigned int tag = s_tag;
+                unsigned long long *fl = p.flags;
+                if (!(p.stall_first_chunk && c == 0))
+                    for (int e = tid; e < E; e += NSET)
+                        st_relaxed_u64(fl + (size_t)c * E + e, lb_word(tag, c == c0, s_agg[e]));
+                if (c > c0) {
+                    const int np = c - c0;   // predecessors, at most kLbSuper - 1
+                    for (int e = tid; e < E; e += NSET) {
+                        unsigned long long v[kLbSuper - 1];
+#pragma unroll
+                        for (int k = 0; k < kLbSuper - 1; ++k)
+                            v[k] = k < np ? ld_relaxed_u64(fl + (size_t)(c - 1 - k) * E + e) : 0ull;
+                        int sum = 0;
+                        bool ok = true;
+#pragma unroll
+                        for (int k = 0; k < kLbSuper - 1; ++k) {
+                            if (k >= np) break;
+                            unsigned long long wv = v[k];
+                            if (lb_tag(wv) != tag) {   // not published yet: wait for it, bounded
+                                const unsigned long long tw0 = globaltimer_ns();
+                                for (;;) {
+                                    wv = ld_relaxed_u64(fl + (size_t)(c - 1 - k) * E + e);
+                                    if (lb_tag(wv) == tag) break;
+                                    if (globaltimer_ns() - tw0 > p.wait_limit_ns) {
+                                        ok = false;
+                                        break;
+                                    }
+                                }
+                                if (!ok) break;
+                            }
+                            sum += (int)(unsigned int)wv;
+                            if (lb_inclusive(wv)) break;
+                        }
+                        if (!ok) {
+                            atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                            *abort_flag = 1;
+                        } else {
+                            st_relaxed_u64(fl + (size_t)c * E + e, lb_word(tag, true, sum + s_agg[e]));
+                        }
+                        s_base[e] = sum;
+                    }
+                } else {
+                    for (int e = tid; e < E; e += NSET) s_base[e] = 0;
+                }
+                set_sync(NSET);
+            }
+            if (*abort_flag) break;
+            if (!waited) {
+                pdl_wait();   // the pre-pass (or the layout) is complete and visible
+                waited = true;
+            }
+            if (p.lb) {
+                const int sb = c / kLbSuper;
+                for (int e = tid; e < E; e += NSET) s_base[e] += __ldcg(p.super_base + (size_t)sb * E + e);
+                set_sync(NSET);
+                for (int i = tid; i < n; i += NSET) {
+                    const int e = s_e[i];
+                    int dst = -1;
+                    if (e >= 0) {
+                        dst = s_base[e] + s_cnt[(i / ppw) * ES + e] + s_rk[i];
+                        const int tl = i / K;
+                        p.row_src[dst] = t0 + tl;
+                        p.row_slot[dst] = i - tl * K;
+                        if (p.topk_weights) p.row_weight[dst] = __ldg(p.topk_weights + q0 + i);
+                    }
+                    s_pos[i] = dst;
+                    p.pos[q0 + i] = dst;
+                }
+            } else {
+                for (int i = tid; i < n; i += NSET) s_pos[i] = __ldg(p.pos + q0 + i);
+            }
+            set_sync(NSET);
+
+            if (warp == 0) {
+                if (lane == 0)
+                    for (int i = min(NS, nu); i < nu && !*abort_flag; ++i)
+                        if (!issue(t0, i)) {
+                            atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                            *abort_flag = 1;
+                            break;
+                        }
+                __syncwarp();
+            } else {
+                const int grp = (tid - 32) / kGroupThreads, gtid = (tid - 32) - grp * kGroupThreads;
+                // units whose CTA-wide index is grp modulo G belong to this group
+                for (int i = ((grp - unit_base % G) % G + G) % G; i < nu; i += G) {
+                    const int g = unit_base + i, s = g % NS;
+                    // the warp decides together, so that no lane is left alone at a __syncwarp
+                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (g / NS) & 1, p.wait_limit_ns))) {
+                        if (lane == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    const int tl = i / p.splits, part = i - tl * p.splits;
+                    if constexpr (FP8)
+                        quantise_unit(p, ring + (size_t)s * chunk, s_pos + tl * K, part, gtid, pol_out);
+                    else
+                        copy_unit<VB>(p, ring + (size_t)s * chunk, s_pos + tl * K, part, gtid, pol_out);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[s]);
+                }
+            }
+            unit_base += nu;
+            set_sync(NSET);   // every unit of the chunk consumed: the ring is free
+            if (*abort_flag) break;
+        }
+        if (!waited) pdl_wait();   // no chunk: nothing read, but keep the dependency
+        if (*abort_flag && tid == 0) {
+            // let every issued load land before the CTA's shared memory goes away
+            for (int j = max(0, issued - NS); j < issued; ++j)
+                mbar_wait_bounded(&full[j % NS], (j / NS) & 1, p.wait_limit_ns);
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // the last CTA to finish leaves the control words ready for the next
+        // launch: every CTA took its last ticket before it got here
+        __threadfence();
+        if (atomicAdd(&p.ctl->done, 1u) == gridDim.x - 1) {
+            __threadfence();
+            atomicExch(&p.ctl->ticket, 0u);
+            atomicExch(&p.ctl->done, 0u);
+            atomicExch(&p.ctl->epoch, s_tag);
+        }
+    }
+}
+
+// Units per token and bytes per unit: bf16 rows split into the fewest
+// power-of-two parts of at most 8 KB; FP8 rows into the fewest parts of at
+// most 224 x 32 elements that hold whole 1x128 blocks.
+bool lb_unit_shape(int H, bool fp8, int VB, int *splits, int *chunk_bytes) {
+    if (fp8) {
+        for (int sp = 1; sp <= H / 128; ++sp) {
+            if (H % sp || (H / sp) % 128 || H / sp > kGroupThreads * kFp8Ept) continue;
+            *splits = sp;
+            *chunk_bytes = 2 * (H / sp);
+            return true;
+        }
+        return false;
+    }
+    const int row_bytes = 2 * H;
+    for (int sp = 1; sp <= 64; sp *= 2) {
+        if (row_bytes % (sp * VB) || row_bytes / sp > 8192) continue;
+        *splits = sp;
+        *chunk_bytes = row_bytes / sp;
+        return true;
+    }
+    return false;
+}
+
+template <typename Kern>
+cudaError_t launch_pdl_lb(Kern kernel, int grid, int block, size_t smem, cudaStream_t s, const LbParams &p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+constexpr int kFp8Groups = EP_LB_FP8_GROUPS;
+constexpr size_t kSmemLimit = 227 * 1024;
+
+}  // namespace
+
+LbPlan plan_lb(int T, int K, int num_sms) {
+    LbPlan pl{};
+    if (T <= 0) {
+        pl.nchunks = 0;
+        pl.tpc = 1;
+        pl.nsuper = 1;
+        return pl;
+    }
+    // about one chunk per SM, at most kLbMaxPairs pairs each
+    const int64_t pairs = (int64_t)T * K;
+    int64_t n = (pairs + kLbMaxPairs - 1) / kLbMaxPairs;
+    if (n < num_sms) n = num_sms < T ? num_sms : T;
+    int tpc = (int)((T + n - 1) / n);
+    while ((int64_t)tpc * K > kLbMaxPairs && tpc > 1) --tpc;
+    pl.tpc = tpc;
+    pl.nchunks = (T + tpc - 1) / tpc;
+    pl.nsuper = (pl.nchunks + kLbSuper - 1) / kLbSuper;
+    return pl;
+}
+
+cudaError_t dispatch_lb_prepare() {
+    const void *kernels[] = {reinterpret_cast<const void *>(&dispatch_lb_kernel<32, false, 1>),
+                             reinterpret_cast<const void *>(&dispatch_lb_kernel<16, false, 1>),
+                             reinterpret_cast<const void *>(&dispatch_lb_kernel<32, true, kFp8Groups>)};
+    for (const void *k : kernels) {
+        const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_layout_counts(const LbParams &p, cudaStream_t s) {
+    const size_t smem = sizeof(int32_t) * ((size_t)(p.E + p.R) + p.E + 1);
+    layout_counts_kernel<<<p.nsuper, kLayoutThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_lb(const LbParams &p_in, bool fp8, int num_sms, cudaStream_t s) {
+    LbParams p = p_in;
+    const bool v32 = !fp8 && p.H % 16 == 0 &&
+                     ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
+    const int VB = v32 ? 32 : 16;
+    p.vec32 = (reinterpret_cast<uintptr_t>(p.recv) & 31) == 0;
+    if (!lb_unit_shape(p.H, fp8, VB, &p.splits, &p.chunk_bytes)) return cudaErrorInvalidValue;
+    const size_t fixed = carve(0, p.chunk_bytes, p.E).total;
+    int ns = (int)(EP_LB_RING_BYTES / p.chunk_bytes);
+    while (ns > 0 && carve(ns, p.chunk_bytes, p.E).total > kSmemLimit) --ns;
+    ns = ns > kMaxStages ? kMaxStages : ns;
+    if (ns < 2 || fixed > kSmemLimit) return cudaErrorInvalidValue;
+    p.stages = ns;
+    const size_t smem = carve(ns, p.chunk_bytes, p.E).total;
+    const int grid = p.nchunks < num_sms ? p.nchunks : num_sms;
+    if (grid <= 0) return cudaSuccess;
+    if (fp8)
+        return launch_pdl_lb(dispatch_lb_kernel<32, true, kFp8Groups>, grid, Shape<kFp8Groups>::kThreads, smem, s, p);
+    return v32 ? launch_pdl_lb(dispatch_lb_kernel<32, false, 1>, grid, Shape<1>::kThreads, smem, s, p)
+               : launch_pdl_lb(dispatch_lb_kernel<16, false, 1>, grid, Shape<1>::kThreads, smem, s, p);
+}
+
+}  // namespace ep

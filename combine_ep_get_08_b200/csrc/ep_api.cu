@@ -4,6 +4,7 @@
 // shapes once per handle and enqueues kernels.  No host synchronisation,
 // allocation or copy on the layout/dispatch/combine calls.
 #include <atomic>
+#include <cstddef>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -153,7 +154,9 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->tokens_per_chunk = h->plan.tokens_per_chunk;
 
     e = ep::dispatch_prepare();
+    if (e == cudaSuccess) e = ep::dispatch_lb_prepare();
     if (e != cudaSuccess) return fail(cuda_fail(e, "cudaFuncSetAttribute(dispatch)"));
+    h->lb = ep::plan_lb(T, K, h->num_sms);
 
     // carve one allocation
     const size_t A256 = 256;
@@ -175,6 +178,12 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     const size_t o_chunk = take(h->plan.cluster ? 0 : sizeof(int32_t) * (size_t)((G + 3) / 4 * 4) * (E + R));
     const size_t o_bar = take(sizeof(ep::GridBarrier));
     const size_t o_stat = take(sizeof(unsigned int));
+    // the fused layout + dispatch: control words, super-chunk histograms and
+    // bases, look-back words
+    const size_t o_lbctl = take(sizeof(ep::LbControl));
+    const size_t o_lbhist = take(sizeof(int32_t) * (size_t)h->lb.nsuper * (E + R));
+    const size_t o_lbbase = take(sizeof(int32_t) * (size_t)h->lb.nsuper * E);
+    const size_t o_lbflags = take(sizeof(unsigned long long) * (size_t)h->lb.nchunks * E);
     h->block_bytes = off;
     e = cudaMalloc(&h->block, h->block_bytes);
     if (e != cudaSuccess) return fail(cuda_fail(e, "cudaMalloc(handle)"));
@@ -195,6 +204,10 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->chunk_counts = reinterpret_cast<int32_t *>(b + o_chunk);
     h->barrier = reinterpret_cast<ep::GridBarrier *>(b + o_bar);
     h->status = reinterpret_cast<unsigned int *>(b + o_stat);
+    h->lb_ctl = reinterpret_cast<ep::LbControl *>(b + o_lbctl);
+    h->lb_super_hist = reinterpret_cast<int32_t *>(b + o_lbhist);
+    h->lb_super_base = reinterpret_cast<int32_t *>(b + o_lbbase);
+    h->lb_flags = reinterpret_cast<unsigned long long *>(b + o_lbflags);
     *out = h;
     return EP_OK;
 }
@@ -282,6 +295,15 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
     return EP_OK;
 }
 
+#ifndef EP_FP8_CHUNKED
+#define EP_FP8_CHUNKED 0   // 1: ep_dispatch_fp8 runs the chunked, staged kernel of dispatch_lb.cu
+#endif
+#ifndef EP_BF16_CHUNKED
+#define EP_BF16_CHUNKED 0  // 1: ep_dispatch does too
+#endif
+
+static ep::LbParams lb_params(const ep_handle *h, const void *x, void *recv, float *scales, int lb);
+
 static int dispatch_common(const ep_handle *h, const void *x, void *recv, float *scales, bool fp8,
                            ep_stream_t stream) {
     int rc = check_mode(h, false, true);
@@ -320,7 +342,11 @@ static int dispatch_common(const ep_handle *h, const void *x, void *recv, float 
     p.prefetch_x = (int64_t)c.num_tokens * c.hidden * 2 <= (int64_t)h->l2_bytes / 2;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
-    cudaError_t e = fp8 ? ep::launch_dispatch_fp8(p, sms, s) : ep::launch_dispatch_bf16(p, sms, s);
+    cudaError_t e;
+    if (fp8 ? EP_FP8_CHUNKED : EP_BF16_CHUNKED)
+        e = ep::launch_dispatch_lb(lb_params(h, x, recv, scales, 0), fp8, sms, s);
+    else
+        e = fp8 ? ep::launch_dispatch_fp8(p, sms, s) : ep::launch_dispatch_bf16(p, sms, s);
     if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(dispatch_fp8)" : "launch(dispatch)");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return EP_OK;
@@ -333,6 +359,99 @@ EP_API int ep_dispatch(const ep_handle *h, const void *x, void *recv_x, ep_strea
 EP_API int ep_dispatch_fp8(const ep_handle *h, const void *x, void *recv_q, float *recv_scales,
                            ep_stream_t stream) {
     return dispatch_common(h, x, recv_q, recv_scales, true, stream);
+}
+
+// The handle's arrays and the fused path's scratch, for the chunked dispatch
+// kernel (lb = 1: layout in the kernel; lb = 0: positions from the handle).
+static ep::LbParams lb_params(const ep_handle *h, const void *x, void *recv, float *scales, int lb) {
+    const ep_config &c = h->cfg;
+    ep::LbParams p{};
+    p.x = x;
+    p.recv = recv;
+    p.recv_scale = scales;
+    p.scale_ld = h->scale_layout == EP_SCALES_COL_MAJOR_TMA ? (int)((h->cap + 3) / 4 * 4) : 0;
+    p.pos = h->pos;
+    p.row_src = h->row_src;
+    p.row_slot = h->row_slot;
+    p.row_weight = h->row_weight;
+    p.cnt = h->cnt;
+    p.rank_tok = h->rank_tok;
+    p.eoff = h->eoff;
+    p.roff = h->roff;
+    p.super_hist = h->lb_super_hist;
+    p.super_base = h->lb_super_base;
+    p.flags = h->lb_flags;
+    p.ctl = h->lb_ctl;
+    p.status = h->status;
+    p.wait_limit_ns = h->wait_limit_ns;
+    p.stall_first_chunk = lb && h->barrier_extra > 0;
+    p.T = c.num_tokens;
+    p.K = c.num_topk;
+    p.E = c.num_experts;
+    p.R = c.num_ranks;
+    p.L = c.num_experts / c.num_ranks;
+    p.A = c.expert_alignment;
+    p.H = c.hidden;
+    p.id_bits = 0;
+    while ((1 << p.id_bits) < c.num_experts) ++p.id_bits;
+    p.nchunks = h->lb.nchunks;
+    p.tpc = h->lb.tpc;
+    p.nsuper = h->lb.nsuper;
+    p.lb = lb;
+    p.prefetch_x = (int64_t)c.num_tokens * c.hidden * 2 <= (int64_t)h->l2_bytes / 2;
+    return p;
+}
+
+static int layout_dispatch_common(ep_handle *h, const int64_t *topk_idx, const float *topk_weights, const void *x,
+                                  void *recv, float *scales, bool fp8, int32_t *num_tokens_per_expert,
+                                  int32_t *num_tokens_per_rank, uint8_t *is_token_in_rank, int32_t *expert_offsets,
+                                  int32_t *rank_offsets, ep_stream_t stream) {
+    int rc = check_mode(h, false, false);
+    if (rc != EP_OK) return rc;
+    const ep_config &c = h->cfg;
+    if (fp8 && c.hidden % 128 != 0) return EP_ERR_ARG;
+    if (c.num_tokens > 0 && (!topk_idx || !x || !recv || (fp8 && !scales))) return EP_ERR_ARG;
+    if (!aligned(topk_idx, 8) || !aligned(topk_weights, 4) || !aligned(x, 16) || !aligned(recv, 16) ||
+        !aligned(scales, 4) || !aligned(num_tokens_per_expert, 4) || !aligned(num_tokens_per_rank, 4) ||
+        !aligned(expert_offsets, 4) || !aligned(rank_offsets, 4))
+        return EP_ERR_ARG;
+    DeviceGuard g(h->device);
+    if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    ep::LbParams p = lb_params(h, x, recv, scales, 1);
+    p.topk_idx = topk_idx;
+    p.topk_weights = topk_weights;
+    p.u_cnt = num_tokens_per_expert;
+    p.u_rank_tok = num_tokens_per_rank;
+    p.u_in_rank = is_token_in_rank;
+    p.u_eoff = expert_offsets;
+    p.u_roff = rank_offsets;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = ep::launch_layout_counts(p, s);
+    if (e != cudaSuccess) return cuda_fail(e, "launch(layout_counts)");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    h->has_layout = true;
+    if (c.num_tokens == 0) return EP_OK;
+    const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
+    e = ep::launch_dispatch_lb(p, fp8, sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(layout_dispatch_fp8)" : "launch(layout_dispatch)");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return EP_OK;
+}
+
+EP_API int ep_layout_dispatch(ep_handle *h, const int64_t *topk_idx, const float *topk_weights, const void *x,
+                              void *recv_x, int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+                              uint8_t *is_token_in_rank, int32_t *expert_offsets, int32_t *rank_offsets,
+                              ep_stream_t stream) {
+    return layout_dispatch_common(h, topk_idx, topk_weights, x, recv_x, nullptr, false, num_tokens_per_expert,
+                                  num_tokens_per_rank, is_token_in_rank, expert_offsets, rank_offsets, stream);
+}
+
+EP_API int ep_layout_dispatch_fp8(ep_handle *h, const int64_t *topk_idx, const float *topk_weights, const void *x,
+                                  void *recv_q, float *recv_scales, int32_t *num_tokens_per_expert,
+                                  int32_t *num_tokens_per_rank, uint8_t *is_token_in_rank, int32_t *expert_offsets,
+                                  int32_t *rank_offsets, ep_stream_t stream) {
+    return layout_dispatch_common(h, topk_idx, topk_weights, x, recv_q, recv_scales, true, num_tokens_per_expert,
+                                  num_tokens_per_rank, is_token_in_rank, expert_offsets, rank_offsets, stream);
 }
 
 static int combine_common(const ep_handle *h, const void *y, const float *topk_weights, void *out,
@@ -700,6 +819,8 @@ EP_API int ep_clear_status(ep_handle *h, ep_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     EP_CUDA(cudaMemsetAsync(h->status, 0, sizeof(unsigned int), s));
     EP_CUDA(cudaMemsetAsync(h->barrier, 0, sizeof(ep::GridBarrier), s));
+    if (h->lb_ctl)   // arrival counters and tickets; the epoch stays, so earlier look-back words never match
+        EP_CUDA(cudaMemsetAsync(h->lb_ctl, 0, offsetof(ep::LbControl, epoch), s));
     return EP_OK;
 }
 

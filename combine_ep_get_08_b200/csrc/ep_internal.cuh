@@ -112,6 +112,66 @@ struct GemmCombineArgs {
 // memset of the accumulator, the GEMM (one CTA per SM, num_sms CTAs) and the bf16 rounding
 cudaError_t launch_gemm_combine(const GemmCombineArgs &g, int num_sms, cudaStream_t s);
 
+// ---------------------------------------------------------------------------
+// Layout fused with the dispatch (dispatch_lb.cu): a counts pre-pass over
+// super-chunks, then a dispatch whose CTAs take token chunks by ticket, rank
+// their pairs and find each chunk's place by decoupled look-back.
+// ---------------------------------------------------------------------------
+constexpr int kLbSuper = 16;          // token chunks per super-chunk (one pre-pass CTA each)
+constexpr int kLbMaxPairs = 4096;     // (token, k) pairs per chunk at most
+
+// Device-side control words of the fused path (in the handle's allocation,
+// zeroed at creation; each kernel leaves them as it found them).
+struct LbControl {
+    unsigned int pre_arrivals;   // pre-pass CTAs that published their histogram (reset by the last)
+    unsigned int ticket;         // next chunk to take (reset by the last dispatch CTA)
+    unsigned int done;           // dispatch CTAs finished (reset by the last)
+    unsigned int epoch;          // tag of the last completed dispatch launch (look-back flags)
+};
+
+struct LbPlan {
+    int nchunks;                 // token chunks
+    int tpc;                     // tokens per chunk
+    int nsuper;                  // super-chunks = pre-pass CTAs
+};
+LbPlan plan_lb(int T, int K, int num_sms);
+
+struct LbParams {
+    const int64_t *topk_idx;     // [T, K]
+    const float *topk_weights;   // [T, K] or null
+    const void *x;               // [T, H] bf16
+    void *recv;                  // [cap, H] bf16 or e4m3
+    float *recv_scale;           // FP8: row-major [cap, H/128] or column-major [H/128][scale_ld]
+    int scale_ld;                // 0: row-major scales
+    // routing (the handle's arrays)
+    int32_t *pos, *row_src, *row_slot;
+    float *row_weight;
+    int32_t *cnt, *rank_tok, *eoff, *roff;
+    // caller copies of the counts and offsets (may be null)
+    int32_t *u_cnt, *u_rank_tok, *u_eoff, *u_roff;
+    uint8_t *u_in_rank;
+    // scratch
+    int32_t *super_hist;         // [nsuper][E+R] pre-pass histograms
+    int32_t *super_base;         // [nsuper][E] first row of each expert's pairs in a super-chunk
+    unsigned long long *flags;   // [nchunks][E] look-back words
+    LbControl *ctl;
+    unsigned int *status;
+    unsigned long long wait_limit_ns;
+    int stall_first_chunk;       // test hook: chunk 0 never publishes, so its successors' waits run out
+    int T, K, E, R, L, A, H, id_bits;
+    int nchunks, tpc, nsuper;
+    int lb;                      // 1: the layout is computed in the kernel; 0: positions from pos
+    int splits;                  // row parts per token (units per token)
+    int chunk_bytes;             // bytes of x per unit
+    int stages;                  // ring depth
+    int prefetch_x;              // 1: the chunk's x rows are prefetched into L2 at its start
+    int vec32;                   // FP8: 1 when recv is 32-byte aligned (32-byte code stores)
+};
+cudaError_t launch_layout_counts(const LbParams &p, cudaStream_t s);
+// The fused (lb = 1) or handle-driven (lb = 0) chunked dispatch, bf16 or FP8.
+cudaError_t launch_dispatch_lb(const LbParams &p, bool fp8, int num_sms, cudaStream_t s);
+cudaError_t dispatch_lb_prepare();
+
 // Layout launch shape: the cluster kernel (G CTAs in one thread-block
 // cluster, exchange through distributed shared memory) when a CTA can hold
 // its share of the pairs, else the cooperative kernel (G CTAs, one grid-wide
@@ -357,6 +417,46 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" : : : "memory");
 }
 
+// Exclusive scan of a[0..n) in shared memory, in place, by a CTA of
+// kLayoutThreads threads; returns the total.  Caller must have synchronised
+// after writing a[].
+__device__ __forceinline__ int block_exclusive_scan(int32_t *a, int n, int32_t *s_tmp /*[kLayoutWarps+1]*/) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (n + kLayoutThreads - 1) / kLayoutThreads;
+    const int b = min(n, tid * per), e = min(n, b + per);
+    int sum = 0;
+    for (int i = b; i < e; ++i) sum += a[i];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_tmp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int v = lane < kLayoutWarps ? s_tmp[lane] : 0;
+        int iv = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int u = __shfl_up_sync(0xffffffffu, iv, o);
+            if (lane >= o) iv += u;
+        }
+        if (lane < kLayoutWarps) s_tmp[lane] = iv - v;
+        if (lane == 31) s_tmp[kLayoutWarps] = iv;
+    }
+    __syncthreads();
+    int run = s_tmp[warp] + incl - sum;
+    for (int i = b; i < e; ++i) {
+        int v = a[i];
+        a[i] = run;
+        run += v;
+    }
+    const int total = s_tmp[kLayoutWarps];
+    __syncthreads();
+    return total;
+}
+
 // bf16 pair in a 32-bit word -> two floats (exact)
 __device__ __forceinline__ float bf16_lo(unsigned int u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(unsigned int u) { return __uint_as_float(u & 0xffff0000u); }
@@ -389,4 +489,9 @@ struct ep_handle {
     int ll_M;                       // > 0: low-latency handle with ll_M slots per expert
     unsigned long long wait_limit_ns;
     int barrier_extra;
+    // fused layout + dispatch
+    ep::LbPlan lb;
+    ep::LbControl *lb_ctl;
+    int32_t *lb_super_hist, *lb_super_base;
+    unsigned long long *lb_flags;
 };

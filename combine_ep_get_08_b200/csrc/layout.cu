@@ -45,45 +45,6 @@ namespace ep {
 
 namespace {
 
-// Exclusive scan of a[0..n) in shared memory, in place; returns the total.
-// Caller must have synchronised after writing a[].
-__device__ int block_exclusive_scan(int32_t *a, int n, int32_t *s_tmp /*[kLayoutWarps+1]*/) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int per = (n + kLayoutThreads - 1) / kLayoutThreads;
-    const int b = min(n, tid * per), e = min(n, b + per);
-    int sum = 0;
-    for (int i = b; i < e; ++i) sum += a[i];
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-    }
-    if (lane == 31) s_tmp[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int v = lane < kLayoutWarps ? s_tmp[lane] : 0;
-        int iv = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int u = __shfl_up_sync(0xffffffffu, iv, o);
-            if (lane >= o) iv += u;
-        }
-        if (lane < kLayoutWarps) s_tmp[lane] = iv - v;
-        if (lane == 31) s_tmp[kLayoutWarps] = iv;
-    }
-    __syncthreads();
-    int run = s_tmp[warp] + incl - sum;
-    for (int i = b; i < e; ++i) {
-        int v = a[i];
-        a[i] = run;
-        run += v;
-    }
-    const int total = s_tmp[kLayoutWarps];
-    __syncthreads();
-    return total;
-}
-
 // Grid-wide wait with a %globaltimer limit.  The arrival counter only grows:
 // after `epoch` completed waits it holds epoch * G, and this wait ends when it
 // reaches (epoch + 1) * G, so no reset is needed between launches.  Each CTA

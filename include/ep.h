@@ -35,7 +35,8 @@
  *     any launch and leave all outputs untouched;
  *   - work is enqueued on `stream` (NULL = legacy default stream) and is
  *     asynchronous: no host synchronisation, allocation or copy happens in
- *     ep_get_layout, ep_dispatch, ep_dispatch_fp8 or ep_combine;
+ *     ep_get_layout, ep_dispatch, ep_dispatch_fp8, ep_layout_dispatch(_fp8)
+ *     or ep_combine;
  *   - errors found on the device (an expert id outside [0, E), a bounded
  *     in-kernel wait that gave up) set sticky bits in the handle's status
  *     word, read with ep_get_status; outputs of that call are unspecified
@@ -214,6 +215,39 @@ EP_API int ep_dispatch(const ep_handle *h, const void *x, void *recv_x, ep_strea
  */
 EP_API int ep_dispatch_fp8(const ep_handle *h, const void *x, void *recv_q, float *recv_scales,
                            ep_stream_t stream);
+
+/*
+ * Layout and dispatch in one call: the results of ep_get_layout followed by
+ * ep_dispatch (or ep_dispatch_fp8), bit for bit -- the handle's routing
+ * arrays, the caller's copies of the counts and offsets (each optional, as
+ * in ep_get_layout), and the received rows (or codes and scales) -- so that
+ * ep_combine, and further ep_dispatch calls, work on the handle afterwards.
+ * Arguments as in ep_get_layout and ep_dispatch / ep_dispatch_fp8.
+ *
+ * Two launches that overlap: a counts pre-pass (one CTA per 16 token chunks;
+ * the last CTA to finish forms the padded offsets) and the dispatch, whose
+ * CTAs take token chunks in launch order from an atomic ticket, rank their
+ * chunk's pairs, and find how many pairs of each expert earlier chunks hold
+ * by decoupled look-back over per-chunk counts (a published single-pass scan
+ * method: Merrill and Garland, 2016) -- all before they wait for the
+ * pre-pass, so the layout work overlaps it and the copy starts as soon as
+ * the offsets exist.  Each look-back wait is bounded (ep_set_wait_limit;
+ * EP_DEV_WAIT_TIMEOUT, outputs then unspecified).  With extra_arrivals > 0
+ * set by ep_set_wait_limit, the first chunk never publishes its counts: a
+ * test hook that makes the waits of the chunks after it run out.
+ * Defined by: the same passages as ep_get_layout and ep_dispatch (the
+ * queue order of the "lesson14_deepep" moe_dispatch loop; do_expand,
+ * expert_alignment and do_zero_padding of bowenzhou.top "deepep/01-overview"
+ * section 1.1).
+ */
+EP_API int ep_layout_dispatch(ep_handle *h, const int64_t *topk_idx, const float *topk_weights, const void *x,
+                              void *recv_x, int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+                              uint8_t *is_token_in_rank, int32_t *expert_offsets, int32_t *rank_offsets,
+                              ep_stream_t stream);
+EP_API int ep_layout_dispatch_fp8(ep_handle *h, const int64_t *topk_idx, const float *topk_weights, const void *x,
+                                  void *recv_q, float *recv_scales, int32_t *num_tokens_per_expert,
+                                  int32_t *num_tokens_per_rank, uint8_t *is_token_in_rank, int32_t *expert_offsets,
+                                  int32_t *rank_offsets, ep_stream_t stream);
 
 /*
  * Combine: out[t, :] = bf16_rn( sum_{k=0..K-1} topk_weights[t,k] *
@@ -486,9 +520,10 @@ EP_API int ep_set_sm_limit(ep_handle *h, int32_t num_sms);
 /*
  * Limit for each bounded in-kernel wait, in nanoseconds of %globaltimer
  * (default 1e9).  `extra_arrivals` > 0 makes the layout's grid-wide wait
- * expect that many CTAs that never arrive: a test hook that exercises the
- * timeout path without hanging (the wait gives up after limit_ns and sets
- * EP_DEV_WAIT_TIMEOUT).  Use 0 in normal operation.
+ * expect that many CTAs that never arrive, and makes the first chunk of
+ * ep_layout_dispatch(_fp8) never publish its counts: test hooks that
+ * exercise the timeout paths without hanging (the waits give up after
+ * limit_ns and set EP_DEV_WAIT_TIMEOUT).  Use 0 in normal operation.
  */
 EP_API int ep_set_wait_limit(ep_handle *h, uint64_t limit_ns, int32_t extra_arrivals);
 

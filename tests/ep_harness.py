@@ -11,6 +11,14 @@ import combine_ep_get_08_b200 as ep
 import workloads
 
 RTOL, ATOL = 1e-2, 1e-3   # combine tolerance (fp32 accumulation, bf16 output)
+ROW_CHUNK = 16384         # received rows compared per oracle call (bounds host memory)
+TOKEN_CHUNK = 2048        # tokens compared per oracle call
+
+
+def chunks(sel, n):
+    """Consecutive slices of at most n entries of sel."""
+    for i in range(0, len(sel), n):
+        yield sel[i:i + n]
 
 
 @dataclass

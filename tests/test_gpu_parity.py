@@ -11,7 +11,7 @@ import torch
 import combine_ep_get_08_b200 as ep
 import oracle
 import workloads
-from ep_harness import (assert_layout_equal, combine_close, expert_outputs, gpu_layout)
+from ep_harness import ROW_CHUNK, TOKEN_CHUNK, assert_layout_equal, chunks as _chunks, combine_close, gpu_layout
 
 pytestmark = pytest.mark.gpu
 
@@ -23,15 +23,6 @@ def _built():
     oracle.build()
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-
-
-ROW_CHUNK = 16384      # received rows compared per oracle call (bounds host memory)
-TOKEN_CHUNK = 2048     # tokens compared per oracle call
-
-
-def _chunks(sel, n):
-    for i in range(0, len(sel), n):
-        yield sel[i:i + n]
 
 
 def run_full(wl, fp8: bool, y_seed=99, check_rows=None, check_tokens=None, sm_limit=0):
