@@ -1164,13 +1164,14 @@ def ncu_ingest(rep: str, workload: str) -> int:
         data = {}
     if data.get("source_digest") != digest:
         data = {"source_digest": digest, "roles": {}}
-    data["how"] = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none on the "
-                   "bench command; caches are flushed between replays; mean over the captured launches")
-    data.setdefault("roles", {})[workload] = {
+    data["how"] = ("one capture per kernel: ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum "
+                   "--clock-control none -k <kernel> -s <warm-up launches> -c 1 on the bench command; "
+                   "caches are flushed between replays; each capture's roles are merged into its workload")
+    data.setdefault("roles", {}).setdefault(workload, {}).update({
         role: {"kernel": e["kernel"], "launches": e["n"], "dram_bytes_read": round(e["rd"] / e["n"]),
                "dram_bytes_write": round(e["wr"] / e["n"]),
                "dram_bytes_per_launch": round((e["rd"] + e["wr"]) / e["n"])}
-        for role, e in per_role.items()}
+        for role, e in per_role.items()})
     with open(path, "w") as f:
         json.dump(data, f, indent=1)
         f.write("\n")

@@ -32,6 +32,12 @@ constexpr int kThreads = 256;
                              // overlapping the layout (layout + dispatch 104.7 -> 101.9 us at the
                              // DeepSeek-V3 shape); 0: after it
 #endif
+#ifndef EP_FP8_PIPE
+#define EP_FP8_PIPE 0        // 1: the FP8 register kernel requests the next token's row before storing
+#endif
+#ifndef EP_FP8_MINB
+#define EP_FP8_MINB 1        // resident blocks per SM the FP8 register kernel is compiled for
+#endif
 #ifndef EP_LSU_UNROLL
 #define EP_LSU_UNROLL 1      // vectors loaded per thread before its K stores (LSU bf16 path)
 #endif
@@ -459,7 +465,7 @@ __device__ __forceinline__ int64_t scale_index(const DispatchParams &p, int row,
 // TPB = 128 / EPT consecutive lanes share one 1x128 block and reduce its
 // amax with shuffles.  Each thread stores EPT code bytes per received row.
 template <int EPT, bool LL>
-__global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p) {
+__global__ void __launch_bounds__(kThreads, EP_FP8_MINB) dispatch_fp8_kernel(DispatchParams p) {
     constexpr int TPB = 128 / EPT;
     constexpr int NW = EPT / 2;              // bf16x2 words loaded per thread
     __shared__ int32_t s_dst[kMaxTopk];
@@ -495,7 +501,50 @@ __global__ void __launch_bounds__(kThreads) dispatch_fp8_kernel(DispatchParams p
             }
         }
     }
-    for (int u = blockIdx.x; u < total; u += nblk) {
+    int u = blockIdx.x;
+#if EP_FP8_PIPE
+    if (!LL && nthr_row <= kThreads) {
+        // software-pipelined token loop: the next token's row is requested
+        // before this token's codes are stored, so one row's loads are always
+        // in flight behind the stores
+        const bool act = threadIdx.x < nthr_row;
+        unsigned int w[NW];
+        if (act && u < p.n_token_units) {
+            Fp8Io<EPT>::load(x + (int64_t)u * p.H * 2 + (int64_t)threadIdx.x * EPT * 2, w);
+        } else {
+#pragma unroll
+            for (int i = 0; i < NW; ++i) w[i] = 0;
+        }
+        for (; u < p.n_token_units; u += nblk) {
+            if (threadIdx.x < p.K) s_dst[threadIdx.x] = __ldg(&p.pos[(int64_t)u * p.K + threadIdx.x]);
+            __syncthreads();
+            const int un = u + nblk;
+            unsigned int wn[NW];
+            if (act && un < p.n_token_units) {
+                Fp8Io<EPT>::load(x + (int64_t)un * p.H * 2 + (int64_t)threadIdx.x * EPT * 2, wn);
+            } else {
+#pragma unroll
+                for (int i = 0; i < NW; ++i) wn[i] = 0;
+            }
+            unsigned int q[8];
+            const float scale = quantize_block<TPB, NW>(w, q);
+            if (act) {
+                const int b = threadIdx.x / TPB;
+                const bool lead = (threadIdx.x % TPB) == 0;
+                for (int k = 0; k < p.K; ++k) {
+                    const int dst = s_dst[k];
+                    if (dst < 0) continue;
+                    Fp8Io<EPT>::store(recv + (int64_t)dst * p.H + (int64_t)threadIdx.x * EPT, q);
+                    if (lead) p.recv_scale[scale_index(p, dst, b, NB)] = scale;
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < NW; ++i) w[i] = wn[i];
+        }
+    }
+#endif
+    for (; u < total; u += nblk) {
         if (u < p.n_token_units) {
             const int t = u;
             const uint8_t *xr = x + (int64_t)t * p.H * 2;

@@ -633,7 +633,16 @@ cudaError_t launch_pdl_lb(Kern kernel, int grid, int block, size_t smem, cudaStr
 }
 
 constexpr int kFp8Groups = EP_LB_FP8_GROUPS;
-constexpr size_t kSmemLimit = 227 * 1024;
+
+// Dynamic shared memory the chunked kernels may use on each device: the
+// opt-in limit per block less their static shared memory (0: not set up).
+int g_smem_limit[kMaxDevices];
+
+size_t smem_limit() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    return (size_t)__atomic_load_n(&g_smem_limit[dev], __ATOMIC_ACQUIRE);
+}
 
 }  // namespace
 
@@ -658,13 +667,29 @@ LbPlan plan_lb(int T, int K, int num_sms) {
 }
 
 cudaError_t dispatch_lb_prepare() {
+    int dev = -1, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (__atomic_load_n(&g_smem_limit[dev], __ATOMIC_ACQUIRE) > 0) return cudaSuccess;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
     const void *kernels[] = {reinterpret_cast<const void *>(&dispatch_lb_kernel<32, false, 1>),
                              reinterpret_cast<const void *>(&dispatch_lb_kernel<16, false, 1>),
                              reinterpret_cast<const void *>(&dispatch_lb_kernel<32, true, kFp8Groups>)};
+    size_t static_max = 0;
     for (const void *k : kernels) {
-        const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, k);
+        if (e != cudaSuccess) return e;
+        static_max = fa.sharedSizeBytes > static_max ? fa.sharedSizeBytes : static_max;
+    }
+    const int limit = optin - (int)up(static_max, 128);
+    for (const void *k : kernels) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
         if (e != cudaSuccess) return e;
     }
+    __atomic_store_n(&g_smem_limit[dev], limit, __ATOMIC_RELEASE);
     return cudaSuccess;
 }
 
@@ -681,11 +706,12 @@ cudaError_t launch_dispatch_lb(const LbParams &p_in, bool fp8, int num_sms, cuda
     const int VB = v32 ? 32 : 16;
     p.vec32 = (reinterpret_cast<uintptr_t>(p.recv) & 31) == 0;
     if (!lb_unit_shape(p.H, fp8, VB, &p.splits, &p.chunk_bytes)) return cudaErrorInvalidValue;
+    const size_t limit = smem_limit();
     const size_t fixed = carve(0, p.chunk_bytes, p.E).total;
     int ns = (int)(EP_LB_RING_BYTES / p.chunk_bytes);
-    while (ns > 0 && carve(ns, p.chunk_bytes, p.E).total > kSmemLimit) --ns;
+    while (ns > 0 && carve(ns, p.chunk_bytes, p.E).total > limit) --ns;
     ns = ns > kMaxStages ? kMaxStages : ns;
-    if (ns < 2 || fixed > kSmemLimit) return cudaErrorInvalidValue;
+    if (ns < 2 || fixed > limit) return cudaErrorInvalidValue;
     p.stages = ns;
     const size_t smem = carve(ns, p.chunk_bytes, p.E).total;
     const int grid = p.nchunks < num_sms ? p.nchunks : num_sms;
