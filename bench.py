@@ -539,7 +539,7 @@ def config_summary(name, mode, args, dev, rank, stream, peak, steps, warmup):
         for _ in range(warmup):
             one_step()
         torch.cuda.synchronize()
-        rows = int(path.cnt.sum()) if ll else ep.ep_get_num_rows(path.h)
+        rows = int(path.cnt.sum()) if isinstance(path, LLPath) else ep.ep_get_num_rows(path.h)
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
         for e in evs:
             one_step(e)
@@ -600,7 +600,7 @@ def run_cuda(args, world, rank, local):
     for _ in range(args.warmup):
         one_step()
     torch.cuda.synchronize()
-    rows = int(path.cnt.sum()) if ll else ep.ep_get_num_rows(path.h)
+    rows = int(path.cnt.sum()) if isinstance(path, LLPath) else ep.ep_get_num_rows(path.h)
     status = ep.ep_get_status(path.h)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
