@@ -9,7 +9,8 @@
 //     is_token_in_rank rows.  The last CTA to arrive (an arrival counter,
 //     nobody waits) adds the histograms up, forms the padded expert offsets
 //     (expert_alignment, bowenzhou.top "deepep/01-overview" section 1.1) and,
-//     for each super-chunk, the row where its pairs of each expert start.
+//     for each super-chunk, how many pairs of each expert earlier
+//     super-chunks hold.
 //
 //   dispatch_lb_kernel     one CTA per SM.  CTAs take token chunks in launch
 //     order from an atomic ticket.  A chunk's pairs are ranked with warp
@@ -27,12 +28,18 @@
 //     on a chunk whose CTA is running and will publish without waiting; every
 //     wait is bounded by %globaltimer (EP_DEV_WAIT_TIMEOUT).  All of this
 //     reads only topk_idx, so it runs before the dependency wait, beside the
-//     pre-pass.  After it, a pair's row is its super-chunk's base + the
-//     look-back prefix + its rank, and the chunk's x rows stream through a
-//     shared-memory ring of bulk copies (TMA engine, no multicast) to their
-//     rows: a plain copy (bf16), or the fused 1x128-block FP8 E4M3
-//     quantisation of "m.nlpx.cn/news/135159" section 4.1.  One warp writes
-//     the padding rows (zeros, and -1 routing) with bulk copies meanwhile.
+//     pre-pass.  After it, a pair's row is the expert's offset + the pairs of
+//     earlier super-chunks + the look-back prefix + its rank; the chunk's
+//     routing is written and a per-chunk ready flag released.  Then every
+//     CTA copies its share of the token rows in interleaved order (CTA b
+//     takes row parts b, b + G, ...; each waits, bounded, for the ready flags
+//     of the chunks it reads): the x rows stream through a shared-memory ring
+//     of bulk copies (TMA engine, no multicast) to their rows, as a plain copy
+//     (bf16) or with the fused 1x128-block FP8 E4M3 quantisation of
+//     "m.nlpx.cn/news/135159" section 4.1.  No CTA copies before it has
+//     finished every chunk it took, so a copy waits only on chunks that
+//     running CTAs complete without waiting on copies.  One warp writes the
+//     padding rows (zeros, and -1 routing) with bulk copies meanwhile.
 //
 // With lb = 0 the same kernel takes the positions from the handle (a layout
 // computed earlier) and is a chunked, dynamically scheduled dispatch.
@@ -111,6 +118,10 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
     return v;
 }
 
+__device__ __forceinline__ void st_release_u32(unsigned int *p, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" : : "l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ bool valid_id(int64_t e, int E) { return e >= 0 && e < E; }
 
 __device__ __forceinline__ int64_t scale_at(const LbParams &p, int row, int b, int NB) {
@@ -180,13 +191,22 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_counts_kernel(LbPara
     __syncthreads();
     if (!s_last) return;
 
-    // the last CTA: every histogram is published
+    // the last CTA: every histogram is published.  Per column, the totals and
+    // (experts) the pairs in earlier super-chunks, eight loads in flight
     __threadfence();
     const int ns = gridDim.x;
     for (int j = tid; j < ncols; j += kLayoutThreads) {
         int tot = 0;
-#pragma unroll 4
-        for (int s = 0; s < ns; ++s) tot += __ldcg(p.super_hist + (size_t)s * ncols + j);
+        for (int s0 = 0; s0 < ns; s0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = s0 + k < ns ? __ldcg(p.super_hist + (size_t)(s0 + k) * ncols + j) : 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                if (j < E && s0 + k < ns) p.super_base[(size_t)(s0 + k) * E + j] = tot;
+                tot += v[k];
+            }
+        }
         s_hist[j] = tot;
     }
     __syncthreads();
@@ -198,12 +218,6 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_counts_kernel(LbPara
     for (int e = tid; e < E; e += kLayoutThreads) {
         p.cnt[e] = s_hist[e];
         if (p.u_cnt) p.u_cnt[e] = s_hist[e];
-        int run = s_eoff[e];
-#pragma unroll 4
-        for (int s = 0; s < ns; ++s) {
-            p.super_base[(size_t)s * E + e] = run;
-            run += __ldcg(p.super_hist + (size_t)s * ncols + e);
-        }
     }
     for (int e = tid; e <= E; e += kLayoutThreads) {
         p.eoff[e] = s_eoff[e];
@@ -370,180 +384,215 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         if (padding) pad_rows<FP8>(p, zeros, lane);
     } else {
         const uint64_t pol_out = policy_evict_first();
-        const uint64_t pol_x = policy_evict_last();
-        int unit_base = 0;     // units of earlier chunks of this CTA (ring stage and phase)
-        int issued = 0;        // producer: units whose load was issued
-        bool waited = false;
-        // the producer's load of chunk unit i (lane 0 of warp 0); false on a timeout
-        auto issue = [&](int t0, int i) -> bool {
-            const int g = unit_base + i, s = g % NS;
-            if (g >= NS && !mbar_wait_bounded(&empty[s], ((g / NS) - 1) & 1, p.wait_limit_ns)) return false;
-            const int t = t0 + i / p.splits, part = i - (i / p.splits) * p.splits;
+        const unsigned int tag = s_tag;
+        // Copy order: this CTA's units are u = blockIdx.x + i * gridDim.x (unit
+        // u = part u % splits of token u / splits), so at any moment the CTAs
+        // write the rows of neighbouring tokens, which lie close together in
+        // every expert segment; contiguous token chunks per CTA measured 8%
+        // slower on the write stream.
+        const int GC = gridDim.x;
+        const int total_units = p.T * p.splits;
+        const int n_cta = total_units > (int)blockIdx.x ? (total_units - (int)blockIdx.x + GC - 1) / GC : 0;
+        int issued = 0;   // producer (thread 0): units whose load was issued
+        // the producer's load of this CTA's unit i into stage i % NS; false on a timeout
+        auto issue = [&](int i) -> bool {
+            const int s = i % NS;
+            if (i >= NS && !mbar_wait_bounded(&empty[s], ((i / NS) - 1) & 1, p.wait_limit_ns)) return false;
+            const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
             mbar_arrive_expect_tx(&full[s], chunk);
             bulk_g2s(ring + (size_t)s * chunk, x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk, &full[s]);
             ++issued;
             return true;
         };
-        for (;;) {
+        auto prefetch_x = [&]() {   // this CTA's x chunks into L2 (thread 0)
+            const uint64_t pol_x = policy_evict_last();
+            for (int i = 0; i < n_cta; ++i) {
+                const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
+                bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
+            }
+        };
+        // x is an input: the first units go into the ring now, overlapping the layout
+        if (tid == 0) {
+            if (p.prefetch_x && !p.lb) prefetch_x();
+            for (int i = 0; i < min(NS, n_cta); ++i)
+                if (!issue(i)) {
+                    atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+        }
+        __syncwarp();
+
+        // ---- phase 1: the layout of every chunk this CTA takes ----
+        for (bool first = true; p.lb; first = false) {
             set_sync(NSET);
             if (tid == 0) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
             set_sync(NSET);
             const int c = s_ticket;
             if (c >= p.nchunks || *abort_flag) break;
             const int t0 = c * p.tpc, t1 = min(p.T, t0 + p.tpc);
-            const int nt = t1 - t0, nu = nt * p.splits, n = nt * K;
+            const int nt = t1 - t0, n = nt * K;
             const int64_t q0 = (int64_t)t0 * K;
-
-            // the chunk's first units into the ring (their stages are free: every
-            // earlier unit was consumed before the last set barrier) and all of
-            // its x rows into L2
-            if (tid == 0) {
-                if (p.prefetch_x)
-                    for (int t = t0; t < t1; ++t) bulk_prefetch_l2(x + (int64_t)t * row_bytes, (uint32_t)row_bytes, pol_x);
-                for (int i = 0; i < min(NS, nu); ++i)
-                    if (!issue(t0, i)) {
-                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                        *abort_flag = 1;
-                        break;
-                    }
-            }
-            __syncwarp();
-
             const int ppw = (n + kLayoutRankWarps * 32 - 1) / (kLayoutRankWarps * 32) * 32;   // pairs per ranking warp
-            if (p.lb) {
-                // ranks: warp w walks pairs [w*ppw, (w+1)*ppw) 32 at a time; a
-                // lane's rank is its warp's running count of its expert plus the
-                // lanes below it with the same expert (ballots over the id bits)
-                if (warp < kLayoutRankWarps) {
-                    int32_t *wrow = s_cnt + warp * ES;
-                    for (int e = lane; e < ES; e += 32) wrow[e] = 0;
-                    __syncwarp();
-                    const int lo = warp * ppw, hi = min(n, lo + ppw);
-                    for (int j0 = lo; j0 < hi; j0 += 32 * 8) {
-                        int64_t v[8];
+            // ranks: warp w walks pairs [w*ppw, (w+1)*ppw) 32 at a time; a lane's
+            // rank is its warp's running count of its expert plus the lanes below
+            // it with the same expert (ballots over the id bits)
+            if (warp < kLayoutRankWarps) {
+                int32_t *wrow = s_cnt + warp * ES;
+                for (int e = lane; e < ES; e += 32) wrow[e] = 0;
+                __syncwarp();
+                const int lo = warp * ppw, hi = min(n, lo + ppw);
+                for (int j0 = lo; j0 < hi; j0 += 32 * 8) {
+                    int64_t v[8];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int i = j0 + u * 32 + lane;
-                            v[u] = i < hi ? __ldg(p.topk_idx + q0 + i) : (int64_t)-1;
+                    for (int u = 0; u < 8; ++u) {
+                        const int i = j0 + u * 32 + lane;
+                        v[u] = i < hi ? __ldg(p.topk_idx + q0 + i) : (int64_t)-1;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        if (j0 + u * 32 >= hi) break;   // warp-uniform
+                        const int i = j0 + u * 32 + lane;
+                        const int e = valid_id(v[u], E) ? (int)v[u] : -1;
+                        if (i < hi && e < 0 && v[u] != -1) atomicOr(p.status, EP_DEV_BAD_EXPERT);
+                        unsigned int peers = __ballot_sync(0xffffffffu, e >= 0);
+                        if (e < 0) peers = ~peers;
+                        for (int bit = 0; bit < p.id_bits; ++bit) {
+                            const int bv = (e >> bit) & 1;
+                            const unsigned int bal = __ballot_sync(0xffffffffu, bv);
+                            peers &= bv ? bal : ~bal;
                         }
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            if (j0 + u * 32 >= hi) break;   // warp-uniform
-                            const int i = j0 + u * 32 + lane;
-                            const int e = valid_id(v[u], E) ? (int)v[u] : -1;
-                            if (i < hi && e < 0 && v[u] != -1) atomicOr(p.status, EP_DEV_BAD_EXPERT);
-                            unsigned int peers = __ballot_sync(0xffffffffu, e >= 0);
-                            if (e < 0) peers = ~peers;
-                            for (int bit = 0; bit < p.id_bits; ++bit) {
-                                const int bv = (e >> bit) & 1;
-                                const unsigned int bal = __ballot_sync(0xffffffffu, bv);
-                                peers &= bv ? bal : ~bal;
-                            }
-                            const int lrank = __popc(peers & lanemask_lt());
-                            const int base = e >= 0 ? wrow[e] : 0;
-                            __syncwarp();
-                            if (e >= 0 && lrank == 0) wrow[e] = base + __popc(peers);
-                            __syncwarp();
-                            if (i < hi) {
-                                s_e[i] = (int16_t)e;
-                                s_rk[i] = (int16_t)(base + lrank);
-                            }
+                        const int lrank = __popc(peers & lanemask_lt());
+                        const int base = e >= 0 ? wrow[e] : 0;
+                        __syncwarp();
+                        if (e >= 0 && lrank == 0) wrow[e] = base + __popc(peers);
+                        __syncwarp();
+                        if (i < hi) {
+                            s_e[i] = (int16_t)e;
+                            s_rk[i] = (int16_t)(base + lrank);
                         }
                     }
                 }
-                set_sync(NSET);
-                // each expert's counts become exclusive prefixes over the ranking
-                // warps; their total is the chunk's aggregate
-                for (int e = tid; e < E; e += NSET) {
-                    int run = 0;
-#pragma unroll
-                    for (int w = 0; w < kLayoutRankWarps; ++w) {
-                        const int vv = s_cnt[w * ES + e];
-                        s_cnt[w * ES + e] = run;
-                        run += vv;
-                    }
-                    s_agg[e] = run;
-                }
-                set_sync(NSET);
-                // publish, then look back over the earlier chunks of the super-chunk
-                const int c0 = c / kLbSuper * kLbSuper;
-                const unsigned int tag = s_tag;
-                unsigned long long *fl = p.flags;
-                if (!(p.stall_first_chunk && c == 0))
-                    for (int e = tid; e < E; e += NSET)
-                        st_relaxed_u64(fl + (size_t)c * E + e, lb_word(tag, c == c0, s_agg[e]));
-                if (c > c0) {
-                    const int np = c - c0;   // predecessors, at most kLbSuper - 1
-                    for (int e = tid; e < E; e += NSET) {
-                        unsigned long long v[kLbSuper - 1];
-#pragma unroll
-                        for (int k = 0; k < kLbSuper - 1; ++k)
-                            v[k] = k < np ? ld_relaxed_u64(fl + (size_t)(c - 1 - k) * E + e) : 0ull;
-                        int sum = 0;
-                        bool ok = true;
-#pragma unroll
-                        for (int k = 0; k < kLbSuper - 1; ++k) {
-                            if (k >= np) break;
-                            unsigned long long wv = v[k];
-                            if (lb_tag(wv) != tag) {   // not published yet: wait for it, bounded
-                                const unsigned long long tw0 = globaltimer_ns();
-                                for (;;) {
-                                    wv = ld_relaxed_u64(fl + (size_t)(c - 1 - k) * E + e);
-                                    if (lb_tag(wv) == tag) break;
-                                    if (globaltimer_ns() - tw0 > p.wait_limit_ns) {
-                                        ok = false;
-                                        break;
-                                    }
-                                }
-                                if (!ok) break;
-                            }
-                            sum += (int)(unsigned int)wv;
-                            if (lb_inclusive(wv)) break;
-                        }
-                        if (!ok) {
-                            atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                            *abort_flag = 1;
-                        } else {
-                            st_relaxed_u64(fl + (size_t)c * E + e, lb_word(tag, true, sum + s_agg[e]));
-                        }
-                        s_base[e] = sum;
-                    }
-                } else {
-                    for (int e = tid; e < E; e += NSET) s_base[e] = 0;
-                }
-                set_sync(NSET);
-            }
-            if (*abort_flag) break;
-            if (!waited) {
-                pdl_wait();   // the pre-pass (or the layout) is complete and visible
-                waited = true;
-            }
-            if (p.lb) {
-                const int sb = c / kLbSuper;
-                for (int e = tid; e < E; e += NSET) s_base[e] += __ldcg(p.super_base + (size_t)sb * E + e);
-                set_sync(NSET);
-                for (int i = tid; i < n; i += NSET) {
-                    const int e = s_e[i];
-                    int dst = -1;
-                    if (e >= 0) {
-                        dst = s_base[e] + s_cnt[(i / ppw) * ES + e] + s_rk[i];
-                        const int tl = i / K;
-                        p.row_src[dst] = t0 + tl;
-                        p.row_slot[dst] = i - tl * K;
-                        if (p.topk_weights) p.row_weight[dst] = __ldg(p.topk_weights + q0 + i);
-                    }
-                    s_pos[i] = dst;
-                    p.pos[q0 + i] = dst;
-                }
-            } else {
-                for (int i = tid; i < n; i += NSET) s_pos[i] = __ldg(p.pos + q0 + i);
             }
             set_sync(NSET);
+            // each expert's counts become exclusive prefixes over the ranking
+            // warps; their total is the chunk's aggregate
+            for (int e = tid; e < E; e += NSET) {
+                int run = 0;
+#pragma unroll
+                for (int w = 0; w < kLayoutRankWarps; ++w) {
+                    const int vv = s_cnt[w * ES + e];
+                    s_cnt[w * ES + e] = run;
+                    run += vv;
+                }
+                s_agg[e] = run;
+            }
+            set_sync(NSET);
+            // publish, then look back over the earlier chunks of the super-chunk
+            const int c0 = c / kLbSuper * kLbSuper;
+            unsigned long long *fl = p.flags;
+            if (!(p.stall_first_chunk && c == 0))
+                for (int e = tid; e < E; e += NSET)
+                    st_relaxed_u64(fl + (size_t)c * E + e, lb_word(tag, c == c0, s_agg[e]));
+            if (c > c0) {
+                const int np = c - c0;   // predecessors, at most kLbSuper - 1
+                for (int e = tid; e < E; e += NSET) {
+                    unsigned long long v[kLbSuper - 1];
+#pragma unroll
+                    for (int k = 0; k < kLbSuper - 1; ++k)
+                        v[k] = k < np ? ld_relaxed_u64(fl + (size_t)(c - 1 - k) * E + e) : 0ull;
+                    int sum = 0;
+                    bool ok = true;
+#pragma unroll
+                    for (int k = 0; k < kLbSuper - 1; ++k) {
+                        if (k >= np) break;
+                        unsigned long long wv = v[k];
+                        if (lb_tag(wv) != tag) {   // not published yet: wait for it, bounded
+                            const unsigned long long tw0 = globaltimer_ns();
+                            for (;;) {
+                                wv = ld_relaxed_u64(fl + (size_t)(c - 1 - k) * E + e);
+                                if (lb_tag(wv) == tag) break;
+                                if (globaltimer_ns() - tw0 > p.wait_limit_ns) {
+                                    ok = false;
+                                    break;
+                                }
+                            }
+                            if (!ok) break;
+                        }
+                        sum += (int)(unsigned int)wv;
+                        if (lb_inclusive(wv)) break;
+                    }
+                    if (!ok) {
+                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *abort_flag = 1;
+                    } else {
+                        st_relaxed_u64(fl + (size_t)c * E + e, lb_word(tag, true, sum + s_agg[e]));
+                    }
+                    s_base[e] = sum;
+                }
+            } else {
+                for (int e = tid; e < E; e += NSET) s_base[e] = 0;
+            }
+            set_sync(NSET);
+            if (*abort_flag) break;
+            if (first) pdl_wait();   // the pre-pass is complete and visible
+            // rows: expert offset + this super-chunk's earlier pairs + the look-back
+            // prefix + the rank inside the chunk
+            const int sb = c / kLbSuper;
+            for (int e = tid; e < E; e += NSET)
+                s_base[e] += __ldcg(p.eoff + e) + __ldcg(p.super_base + (size_t)sb * E + e);
+            set_sync(NSET);
+            for (int i = tid; i < n; i += NSET) {
+                const int e = s_e[i];
+                int dst = -1;
+                if (e >= 0) {
+                    dst = s_base[e] + s_cnt[(i / ppw) * ES + e] + s_rk[i];
+                    const int tl = i / K;
+                    p.row_src[dst] = t0 + tl;
+                    p.row_slot[dst] = i - tl * K;
+                    if (p.topk_weights) p.row_weight[dst] = __ldg(p.topk_weights + q0 + i);
+                }
+                p.pos[q0 + i] = dst;
+            }
+            __threadfence();   // this thread's rows before the chunk's ready flag
+            set_sync(NSET);
+            if (tid == 0) st_release_u32(p.ready + c, tag);
+        }
+        pdl_wait();            // (a no-op after the first wait) the layout before is complete and visible
+        if (p.lb && tid == 0 && p.prefetch_x && !*abort_flag) prefetch_x();
 
+        // ---- phase 2: the copy, window by window of staged destinations ----
+        const int win = max(1, kLbMaxPairs / K);
+        for (int w0 = 0; w0 < n_cta && !*abort_flag; w0 += win) {
+            const int wn = min(win, n_cta - w0);
+            if (p.lb) {
+                // every chunk behind this window's tokens has published its rows
+                for (int i = tid; i < wn; i += NSET) {
+                    const int t = ((int)blockIdx.x + (w0 + i) * GC) / p.splits;
+                    const unsigned int *rf = p.ready + t / p.tpc;
+                    if (ld_acquire_u32(rf) != tag) {
+                        const unsigned long long tw0 = globaltimer_ns();
+                        while (ld_acquire_u32(rf) != tag)
+                            if (globaltimer_ns() - tw0 > p.wait_limit_ns) {
+                                atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                                *abort_flag = 1;
+                                break;
+                            }
+                    }
+                }
+                set_sync(NSET);
+                if (*abort_flag) break;
+            }
+            for (int i = tid; i < wn * K; i += NSET) {
+                const int t = ((int)blockIdx.x + (w0 + i / K) * GC) / p.splits;
+                const int32_t *pp = p.pos + (int64_t)t * K + (i % K);
+                s_pos[i] = p.lb ? __ldcg(pp) : __ldg(pp);
+            }
+            set_sync(NSET);
             if (warp == 0) {
                 if (lane == 0)
-                    for (int i = min(NS, nu); i < nu && !*abort_flag; ++i)
-                        if (!issue(t0, i)) {
+                    for (int i = max(issued, w0); i < w0 + wn && !*abort_flag; ++i)
+                        if (!issue(i)) {
                             atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
                             *abort_flag = 1;
                             break;
@@ -551,29 +600,26 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
                 __syncwarp();
             } else {
                 const int grp = (tid - 32) / kGroupThreads, gtid = (tid - 32) - grp * kGroupThreads;
-                // units whose CTA-wide index is grp modulo G belong to this group
-                for (int i = ((grp - unit_base % G) % G + G) % G; i < nu; i += G) {
-                    const int g = unit_base + i, s = g % NS;
+                // unit i belongs to consumer group i % G
+                for (int i = w0 + ((grp - w0 % G) % G + G) % G; i < w0 + wn; i += G) {
+                    const int s = i % NS;
                     // the warp decides together, so that no lane is left alone at a __syncwarp
-                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (g / NS) & 1, p.wait_limit_ns))) {
+                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (i / NS) & 1, p.wait_limit_ns))) {
                         if (lane == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
                         *abort_flag = 1;
                         break;
                     }
-                    const int tl = i / p.splits, part = i - tl * p.splits;
+                    const int u = (int)blockIdx.x + i * GC, part = u % p.splits;
                     if constexpr (FP8)
-                        quantise_unit(p, ring + (size_t)s * chunk, s_pos + tl * K, part, gtid, pol_out);
+                        quantise_unit(p, ring + (size_t)s * chunk, s_pos + (i - w0) * K, part, gtid, pol_out);
                     else
-                        copy_unit<VB>(p, ring + (size_t)s * chunk, s_pos + tl * K, part, gtid, pol_out);
+                        copy_unit<VB>(p, ring + (size_t)s * chunk, s_pos + (i - w0) * K, part, gtid, pol_out);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[s]);
                 }
             }
-            unit_base += nu;
-            set_sync(NSET);   // every unit of the chunk consumed: the ring is free
-            if (*abort_flag) break;
+            set_sync(NSET);   // every unit of the window consumed
         }
-        if (!waited) pdl_wait();   // no chunk: nothing read, but keep the dependency
         if (*abort_flag && tid == 0) {
             // let every issued load land before the CTA's shared memory goes away
             for (int j = max(0, issued - NS); j < issued; ++j)

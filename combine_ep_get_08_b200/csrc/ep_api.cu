@@ -184,6 +184,7 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     const size_t o_lbhist = take(sizeof(int32_t) * (size_t)h->lb.nsuper * (E + R));
     const size_t o_lbbase = take(sizeof(int32_t) * (size_t)h->lb.nsuper * E);
     const size_t o_lbflags = take(sizeof(unsigned long long) * (size_t)h->lb.nchunks * E);
+    const size_t o_lbready = take(sizeof(unsigned int) * (size_t)h->lb.nchunks);
     h->block_bytes = off;
     e = cudaMalloc(&h->block, h->block_bytes);
     if (e != cudaSuccess) return fail(cuda_fail(e, "cudaMalloc(handle)"));
@@ -208,6 +209,7 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->lb_super_hist = reinterpret_cast<int32_t *>(b + o_lbhist);
     h->lb_super_base = reinterpret_cast<int32_t *>(b + o_lbbase);
     h->lb_flags = reinterpret_cast<unsigned long long *>(b + o_lbflags);
+    h->lb_ready = reinterpret_cast<unsigned int *>(b + o_lbready);
     *out = h;
     return EP_OK;
 }
@@ -381,6 +383,7 @@ static ep::LbParams lb_params(const ep_handle *h, const void *x, void *recv, flo
     p.super_hist = h->lb_super_hist;
     p.super_base = h->lb_super_base;
     p.flags = h->lb_flags;
+    p.ready = h->lb_ready;
     p.ctl = h->lb_ctl;
     p.status = h->status;
     p.wait_limit_ns = h->wait_limit_ns;

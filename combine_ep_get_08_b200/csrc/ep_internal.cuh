@@ -152,8 +152,9 @@ struct LbParams {
     uint8_t *u_in_rank;
     // scratch
     int32_t *super_hist;         // [nsuper][E+R] pre-pass histograms
-    int32_t *super_base;         // [nsuper][E] first row of each expert's pairs in a super-chunk
+    int32_t *super_base;         // [nsuper][E] pairs of each expert in earlier super-chunks
     unsigned long long *flags;   // [nchunks][E] look-back words
+    unsigned int *ready;         // [nchunks] launch tag once the chunk's routing is written
     LbControl *ctl;
     unsigned int *status;
     unsigned long long wait_limit_ns;
@@ -494,4 +495,5 @@ struct ep_handle {
     ep::LbControl *lb_ctl;
     int32_t *lb_super_hist, *lb_super_base;
     unsigned long long *lb_flags;
+    unsigned int *lb_ready;
 };
