@@ -235,21 +235,35 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_counts_kernel(LbPara
 }
 
 // ---------------------------------------------------------------------------
-// Padding rows: the padding warp takes experts blockIdx.x + (lane + 32 i) *
-// gridDim.x and writes their padding rows (rows eoff[e] + cnt[e] ..
-// eoff[e+1]) with bulk shared->global copies of a zeroed block: zero bf16
-// rows, or zero codes and zero scales; with lb = 1 also their routing
-// (row_src = row_slot = -1, row_weight = 0).
+// Padding rows: the padding warp takes experts blockIdx.x, blockIdx.x +
+// gridDim.x, ... and its 32 lanes share each expert's padding rows (rows
+// eoff[e] + cnt[e] .. eoff[e+1]); every row is written with bulk
+// shared->global copies of a zeroed block: a zero bf16 row, or zero codes and
+// (row-major, when 16-byte sized) zero scales; with lb = 1 also its routing
+// (row_src = row_slot = -1, row_weight = 0).  Before that, with lb = 1 and
+// prefetch_x, lane 0 pulls this CTA's x chunks into L2 (issued here, after the
+// dependency wait, so it does not delay the latency-bound layout work).
 // ---------------------------------------------------------------------------
 template <bool FP8>
-__device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros, int lane) {
+__device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros, int lane, int n_cta, int chunk) {
     pdl_wait();   // offsets and counts come from the kernel before
+    if (p.lb && p.prefetch_x && lane == 0) {
+        const uint64_t pol_x = policy_evict_last();
+        const uint8_t *x = static_cast<const uint8_t *>(p.x);
+        for (int i = 0; i < n_cta; ++i) {
+            const int u = (int)blockIdx.x + i * (int)gridDim.x, t = u / p.splits, part = u - t * p.splits;
+            bulk_prefetch_l2(x + (int64_t)t * 2 * p.H + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
+        }
+    }
+    if (p.A <= 1) return;
     const int row_bytes = FP8 ? p.H : 2 * p.H;
     const int NB = p.H / 128;
+    const bool bulk_scales = FP8 && p.scale_ld == 0 && (NB * 4) % 16 == 0 &&
+                             (reinterpret_cast<uintptr_t>(p.recv_scale) & 15) == 0;
     uint8_t *recv = static_cast<uint8_t *>(p.recv);
-    for (int e = blockIdx.x + lane * gridDim.x; e < p.E; e += 32 * gridDim.x) {
+    for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
         const int r0 = __ldcg(p.eoff + e) + __ldcg(p.cnt + e), r1 = __ldcg(p.eoff + e + 1);
-        for (int r = r0; r < r1; ++r) {
+        for (int r = r0 + lane; r < r1; r += 32) {
             if (p.lb) {
                 p.row_src[r] = -1;
                 p.row_slot[r] = -1;
@@ -258,8 +272,12 @@ __device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros
             uint8_t *o = recv + (int64_t)r * row_bytes;
             for (int off = 0; off < row_bytes; off += kZeroBytes)
                 bulk_s2g(o + off, zeros, (uint32_t)min(kZeroBytes, row_bytes - off));
-            if (FP8)
-                for (int b = 0; b < NB; ++b) p.recv_scale[scale_at(p, r, b, NB)] = 0.0f;
+            if (FP8) {
+                if (bulk_scales)
+                    bulk_s2g(p.recv_scale + (int64_t)r * NB, zeros, (uint32_t)(NB * 4));
+                else
+                    for (int b = 0; b < NB; ++b) p.recv_scale[scale_at(p, r, b, NB)] = 0.0f;
+            }
         }
         bulk_commit();
     }
@@ -367,6 +385,10 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         for (int i = tid; i < kZeroBytes / 16; i += S::kThreads) reinterpret_cast<uint4 *>(zeros)[i] = make_uint4(0, 0, 0, 0);
         fence_async_smem();
     }
+    // this CTA's units: u = blockIdx.x + i * gridDim.x (see the copy phase)
+    const int GC = gridDim.x;
+    const int total_units = p.T * p.splits;
+    const int n_cta = total_units > (int)blockIdx.x ? (total_units - (int)blockIdx.x + GC - 1) / GC : 0;
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
@@ -381,7 +403,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     __syncthreads();
 
     if (warp == S::kPadWarp) {
-        if (padding) pad_rows<FP8>(p, zeros, lane);
+        pad_rows<FP8>(p, zeros, lane, n_cta, chunk);
     } else {
         const uint64_t pol_out = policy_evict_first();
         const unsigned int tag = s_tag;
@@ -390,9 +412,6 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         // write the rows of neighbouring tokens, which lie close together in
         // every expert segment; contiguous token chunks per CTA measured 8%
         // slower on the write stream.
-        const int GC = gridDim.x;
-        const int total_units = p.T * p.splits;
-        const int n_cta = total_units > (int)blockIdx.x ? (total_units - (int)blockIdx.x + GC - 1) / GC : 0;
         int issued = 0;   // producer (thread 0): units whose load was issued
         // the producer's load of this CTA's unit i into stage i % NS; false on a timeout
         auto issue = [&](int i) -> bool {
@@ -404,16 +423,19 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
             ++issued;
             return true;
         };
-        auto prefetch_x = [&]() {   // this CTA's x chunks into L2 (thread 0)
-            const uint64_t pol_x = policy_evict_last();
-            for (int i = 0; i < n_cta; ++i) {
-                const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
-                bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
-            }
-        };
-        // x is an input: the first units go into the ring now, overlapping the layout
+        // the first chunk's ticket is requested before anything else
+        if (p.lb && tid == 0) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
+        // x is an input: the first units go into the ring now, overlapping the
+        // layout (with lb = 0 all of this CTA's x chunks also go into L2 now;
+        // with lb = 1 the padding warp does that after the dependency wait)
         if (tid == 0) {
-            if (p.prefetch_x && !p.lb) prefetch_x();
+            if (p.prefetch_x && !p.lb) {
+                const uint64_t pol_x = policy_evict_last();
+                for (int i = 0; i < n_cta; ++i) {
+                    const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
+                    bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
+                }
+            }
             for (int i = 0; i < min(NS, n_cta); ++i)
                 if (!issue(i)) {
                     atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
@@ -426,7 +448,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         // ---- phase 1: the layout of every chunk this CTA takes ----
         for (bool first = true; p.lb; first = false) {
             set_sync(NSET);
-            if (tid == 0) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
+            if (tid == 0 && !first) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
             set_sync(NSET);
             const int c = s_ticket;
             if (c >= p.nchunks || *abort_flag) break;
@@ -559,7 +581,6 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
             if (tid == 0) st_release_u32(p.ready + c, tag);
         }
         pdl_wait();            // (a no-op after the first wait) the layout before is complete and visible
-        if (p.lb && tid == 0 && p.prefetch_x && !*abort_flag) prefetch_x();
 
         // ---- phase 2: the copy, window by window of staged destinations ----
         const int win = max(1, kLbMaxPairs / K);
