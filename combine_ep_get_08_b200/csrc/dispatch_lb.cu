@@ -49,6 +49,9 @@
 #ifndef EP_LB_FP8_GROUPS
 #define EP_LB_FP8_GROUPS 2          // FP8 consumer groups per CTA (quantisation needs more warps)
 #endif
+#ifndef EP_LB_DYN
+#define EP_LB_DYN 1                 // copy phase: row parts claimed in batches (0: fixed interleaved order)
+#endif
 #ifndef EP_LB_RING_BYTES
 #define EP_LB_RING_BYTES (112 * 1024)
 #endif
@@ -63,6 +66,10 @@ constexpr int kLayoutRankWarps = 8;     // warps that rank a chunk's pairs
 constexpr int kMaxStages = 16;
 constexpr int kZeroBytes = 8192;        // zeroed shared memory the padding warp copies from
 constexpr int kFp8Ept = 32;             // FP8: bf16 elements per consumer thread
+#ifndef EP_LB_DYN_BATCH
+#define EP_LB_DYN_BATCH 4
+#endif
+constexpr int kDynBatch = EP_LB_DYN_BATCH;   // row parts per claim of the dynamic copy
 
 template <int G>
 struct Shape {
@@ -75,7 +82,7 @@ __host__ __device__ __forceinline__ size_t up(size_t v, size_t a) { return (v + 
 
 // Dynamic shared memory carve-up (same on host and device).
 struct Carve {
-    size_t ring, bars, zeros, pos, e16, rk16, cnt, base, agg, total;
+    size_t ring, bars, zeros, pos, e16, rk16, cnt, base, agg, unit, stpos, total;
 };
 __host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int E) {
     Carve c;
@@ -89,6 +96,10 @@ __host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int
     c.cnt = o;   o += (size_t)kLayoutRankWarps * (E + 1) * sizeof(int32_t);
     c.base = o;  o += (size_t)E * sizeof(int32_t);
     c.agg = o;   o += (size_t)E * sizeof(int32_t);
+    o = up(o, 128);
+    c.unit = o;  o += (size_t)kMaxStages * sizeof(int32_t);
+    o = up(o, 128);                      // bulk-copy destinations: 16-byte aligned
+    c.stpos = o; o += (size_t)kMaxStages * kMaxTopk * sizeof(int32_t);
     c.total = up(o, 128);
     return c;
 }
@@ -116,6 +127,12 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
     unsigned long long v;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Orders generic-proxy global memory accesses this thread has observed
+// before its later async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" : : : "memory");
 }
 
 __device__ __forceinline__ void st_release_u32(unsigned int *p, unsigned int v) {
@@ -370,6 +387,8 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     int32_t *s_cnt = reinterpret_cast<int32_t *>(smem + cv.cnt);
     int32_t *s_base = reinterpret_cast<int32_t *>(smem + cv.base);
     int32_t *s_agg = reinterpret_cast<int32_t *>(smem + cv.agg);
+    int32_t *s_unit = reinterpret_cast<int32_t *>(smem + cv.unit);     // [stages] row part in each stage (-1: end)
+    int32_t *s_stpos = reinterpret_cast<int32_t *>(smem + cv.stpos);   // [stages][K] its destinations
     __shared__ int s_ticket;
     __shared__ int s_abort;
     __shared__ unsigned int s_tag;
@@ -436,7 +455,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
                     bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
                 }
             }
-            for (int i = 0; i < min(NS, n_cta); ++i)
+            for (int i = 0; i < (p.dyn ? 0 : min(NS, n_cta)); ++i)
                 if (!issue(i)) {
                     atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
                     *abort_flag = 1;
@@ -582,9 +601,86 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         }
         pdl_wait();            // (a no-op after the first wait) the layout before is complete and visible
 
-        // ---- phase 2: the copy, window by window of staged destinations ----
+        // ---- phase 2, dynamic: row parts claimed in batches of kDynBatch ----
+        // The producer claims a batch from ctl->units (the next claim is
+        // requested before the current batch is issued), and per row part puts
+        // its x bytes and its K destinations (a second bulk copy, K*4 bytes) into
+        // one stage, completing on the stage's barrier.  Consumer group grp takes
+        // the stages g = grp, grp + G, ...; a part of -1 ends the group's loop.
+        // CTAs on SMs that move bytes faster take more parts.
+        if (p.dyn) {
+            if (warp == 0) {
+                if (lane == 0) {
+                    int g = 0;
+                    unsigned int claim = atomicAdd(&p.ctl->units, 1u);
+                    while (!*abort_flag) {
+                        const int u0 = (int)claim * kDynBatch;
+                        if (u0 >= total_units) break;
+                        const unsigned int next = atomicAdd(&p.ctl->units, 1u);
+                        for (int u = u0; u < min(total_units, u0 + kDynBatch) && !*abort_flag; ++u, ++g) {
+                            const int s = g % NS;
+                            bool ok = g < NS || mbar_wait_bounded(&empty[s], ((g / NS) - 1) & 1, p.wait_limit_ns);
+                            const int t = u / p.splits, part = u - t * p.splits;
+                            if (ok && p.lb) {   // the chunk's rows are written (released by its CTA)
+                                const unsigned int *rf = p.ready + t / p.tpc;
+                                if (ld_acquire_u32(rf) != tag) {
+                                    const unsigned long long tw0 = globaltimer_ns();
+                                    while (ok && ld_acquire_u32(rf) != tag) ok = globaltimer_ns() - tw0 <= p.wait_limit_ns;
+                                }
+                                fence_proxy_async_global();   // those generic writes, before the bulk read below
+                            }
+                            if (!ok) {
+                                atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                                *abort_flag = 1;
+                                break;
+                            }
+                            s_unit[s] = u;
+                            mbar_arrive_expect_tx(&full[s], (uint32_t)(chunk + K * 4));
+                            bulk_g2s(ring + (size_t)s * chunk, x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk,
+                                     &full[s]);
+                            bulk_g2s(s_stpos + s * kMaxTopk, p.pos + (int64_t)t * K, (uint32_t)(K * 4), &full[s]);
+                            ++issued;
+                        }
+                        claim = next;
+                    }
+                    // one end marker per consumer group
+                    for (int k = 0; k < G && !*abort_flag; ++k, ++g) {
+                        const int s = g % NS;
+                        if (g >= NS && !mbar_wait_bounded(&empty[s], ((g / NS) - 1) & 1, p.wait_limit_ns)) {
+                            atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                            *abort_flag = 1;
+                            break;
+                        }
+                        s_unit[s] = -1;
+                        mbar_arrive(&full[s]);
+                    }
+                }
+                __syncwarp();
+            } else {
+                const int grp = (tid - 32) / kGroupThreads, gtid = (tid - 32) - grp * kGroupThreads;
+                for (int g = grp;; g += G) {
+                    const int s = g % NS;
+                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (g / NS) & 1, p.wait_limit_ns))) {
+                        if (lane == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    const int u = s_unit[s];
+                    if (u < 0) break;
+                    const int part = u % p.splits;
+                    if constexpr (FP8)
+                        quantise_unit(p, ring + (size_t)s * chunk, s_stpos + s * kMaxTopk, part, gtid, pol_out);
+                    else
+                        copy_unit<VB>(p, ring + (size_t)s * chunk, s_stpos + s * kMaxTopk, part, gtid, pol_out);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[s]);
+                }
+            }
+        }
+
+        // ---- phase 2, static: the copy, window by window of staged destinations ----
         const int win = max(1, kLbMaxPairs / K);
-        for (int w0 = 0; w0 < n_cta && !*abort_flag; w0 += win) {
+        for (int w0 = 0; w0 < n_cta && !*abort_flag && !p.dyn; w0 += win) {
             const int wn = min(win, n_cta - w0);
             if (p.lb) {
                 // every chunk behind this window's tokens has published its rows
@@ -655,6 +751,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         if (atomicAdd(&p.ctl->done, 1u) == gridDim.x - 1) {
             __threadfence();
             atomicExch(&p.ctl->ticket, 0u);
+            atomicExch(&p.ctl->units, 0u);
             atomicExch(&p.ctl->done, 0u);
             atomicExch(&p.ctl->epoch, s_tag);
         }
@@ -772,6 +869,8 @@ cudaError_t launch_dispatch_lb(const LbParams &p_in, bool fp8, int num_sms, cuda
                      ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
     const int VB = v32 ? 32 : 16;
     p.vec32 = (reinterpret_cast<uintptr_t>(p.recv) & 31) == 0;
+    // dynamic copy: each part's K destinations arrive by a bulk copy (16-byte multiple)
+    p.dyn = EP_LB_DYN && p.K % 4 == 0 && (reinterpret_cast<uintptr_t>(p.pos) & 15) == 0;
     if (!lb_unit_shape(p.H, fp8, VB, &p.splits, &p.chunk_bytes)) return cudaErrorInvalidValue;
     const size_t limit = smem_limit();
     const size_t fixed = carve(0, p.chunk_bytes, p.E).total;

@@ -126,6 +126,7 @@ struct LbControl {
     unsigned int pre_arrivals;   // pre-pass CTAs that published their histogram (reset by the last)
     unsigned int ticket;         // next chunk to take (reset by the last dispatch CTA)
     unsigned int done;           // dispatch CTAs finished (reset by the last)
+    unsigned int units;          // next batch of row parts to copy (dynamic copy; reset by the last)
     unsigned int epoch;          // tag of the last completed dispatch launch (look-back flags)
 };
 
@@ -167,6 +168,7 @@ struct LbParams {
     int stages;                  // ring depth
     int prefetch_x;              // 1: the chunk's x rows are prefetched into L2 at its start
     int vec32;                   // FP8: 1 when recv is 32-byte aligned (32-byte code stores)
+    int dyn;                     // 1: row parts are claimed in batches from ctl->units (K % 4 == 0)
 };
 cudaError_t launch_layout_counts(const LbParams &p, cudaStream_t s);
 // The fused (lb = 1) or handle-driven (lb = 0) chunked dispatch, bf16 or FP8.
