@@ -10,13 +10,15 @@
 // restore-after-receive scheme of "2kiu.com/news/5702702" section 2.3, with
 // one fp32 scale per 1x128 block of a token row.
 //
-// Work is split into units of similar byte volume, walked by a persistent
-// grid: units [0, T*splits) copy one column range of one token to its K
-// rows; units after that zero-fill the padding among kZeroRowsPerUnit
-// consecutive received rows (only when expert_alignment > 1).  Copies use
-// 32-byte (sm_100 256-bit) vector loads and stores when rows and pointers
-// allow, else 16-byte ones; a bulk-copy (TMA engine) variant measured no
-// faster on this write-bound pattern.
+// These are the register kernels: ep_dispatch / ep_dispatch_fp8 use them for
+// batches too small to fill the GPU (fewer than two tokens per SM), and the
+// low-latency layout uses them always; larger batches go to the chunked
+// kernel of dispatch_lb.cu.  Work is split into units of similar byte
+// volume, walked by a persistent grid: units [0, T*splits) copy one column
+// range of one token to its K rows; units after that zero-fill the padding
+// among kZeroRowsPerUnit consecutive received rows (only when
+// expert_alignment > 1).  Copies use 32-byte (sm_100 256-bit) vector loads
+// and stores when rows and pointers allow, else 16-byte ones.
 
 #include "ep_internal.cuh"
 #include "fp8_block.cuh"
@@ -27,11 +29,6 @@ namespace {
 
 constexpr int kThreads = 256;
 
-#ifndef EP_PDL_PREFETCH
-#define EP_PDL_PREFETCH 1    // the staged kernel's L2 prefetch of x runs before its dependency wait,
-                             // overlapping the layout (layout + dispatch 104.7 -> 101.9 us at the
-                             // DeepSeek-V3 shape); 0: after it
-#endif
 #ifndef EP_FP8_PIPE
 #define EP_FP8_PIPE 1        // the FP8 register kernel requests the next token's row before storing this
                              // one's codes (skew 94.6 -> 88.0 us, large 270.8 -> 260.8 us in one run)
@@ -227,233 +224,6 @@ __global__ void __launch_bounds__(kThreads, EP_LSU_MINB) dispatch_bf16_kernel(Di
     }
 }
 
-// ---------------------------------------------------------------------------
-// Staged path (bf16): a producer warp streams row chunks of x into a ring of
-// shared-memory stages with bulk global->shared copies (TMA engine; each
-// stage's "full" mbarrier counts the bytes in).  Consumer groups of 7 warps
-// take every kStagedGroups-th unit: a group waits for its stage, reads each
-// vector of it once and stores it to the unit's K received rows, then
-// releases the stage on its "empty" mbarrier.  Loads run ahead of the
-// stores, and several groups keep enough stores in flight per SM to cover
-// HBM write latency.  Every wait is bounded; a timeout sets
-// EP_DEV_WAIT_TIMEOUT.
-// ---------------------------------------------------------------------------
-#ifndef EP_DISPATCH_STAGED
-#define EP_DISPATCH_STAGED 1
-#endif
-#ifndef EP_STAGED_CHUNK_MAX
-#define EP_STAGED_CHUNK_MAX 8192    // bytes of a row per unit (rows split into chunks)
-#endif
-#ifndef EP_STAGED_SMEM
-#define EP_STAGED_SMEM (112 * 1024) // shared-memory ring budget per CTA
-#endif
-#ifndef EP_STAGED_PREFETCH
-#define EP_STAGED_PREFETCH 1        // 0: none, 1: L2 prefetch of the CTA's x rows (evict_last), 2: evict_normal
-#endif
-#ifndef EP_STAGED_STORE_EVICT_FIRST
-#define EP_STAGED_STORE_EVICT_FIRST 1
-#endif
-#ifndef EP_STAGED_GROUPS
-#define EP_STAGED_GROUPS 1          // consumer groups working on different stages at once
-#endif
-constexpr int kGroupWarps = 7;                     // warps per consumer group
-constexpr int kGroupThreads = kGroupWarps * 32;
-constexpr int kStagedGroups = EP_STAGED_GROUPS;
-// warp 0 produces, then kStagedGroups consumer groups, then one zero-fill warp
-constexpr int kStagedThreads = 32 + kStagedGroups * kGroupThreads + 32;
-constexpr int kZeroWarp = (kStagedThreads / 32) - 1;
-constexpr int kZeroSmemBytes = 8192;   // zeroed shared memory the zero-fill warp copies from
-constexpr int kStagedMaxStages = 16;
-constexpr int kStagedPosInts = 4096;  // staged pos entries (units x K) per window
-
-__host__ __device__ __forceinline__ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-__host__ __device__ __forceinline__ size_t staged_smem_bytes(int stages, int chunk) {
-    return align_up((size_t)stages * chunk, 128) + 2 * kStagedMaxStages * sizeof(uint64_t) +
-           kStagedPosInts * sizeof(int32_t) + kZeroSmemBytes;
-}
-
-// The zero-fill warp: lane l takes zero units blockIdx.x + (l + 32 i) * gridDim.x
-// and writes every padding row among them with bulk shared->global copies
-// from a zeroed shared-memory block (the TMA engine does the writing, so no
-// consumer thread is spent on it).
-__device__ __forceinline__ void zero_fill_warp(const DispatchParams &p, int rows, int row_bytes,
-                                               const uint8_t *zeros, int lane) {
-    uint8_t *recv = static_cast<uint8_t *>(p.recv);
-    for (int z = blockIdx.x + lane * gridDim.x; z < p.n_zero_units; z += 32 * gridDim.x) {
-        const int r0 = z * kZeroRowsPerUnit, r1 = min(rows, r0 + kZeroRowsPerUnit);
-        for (int r = r0; r < r1; ++r) {
-            if (__ldg(&p.row_src[r]) >= 0) continue;
-            uint8_t *o = recv + (int64_t)r * row_bytes;
-            for (int off = 0; off < row_bytes; off += kZeroSmemBytes)
-                bulk_s2g(o + off, zeros, (uint32_t)min(kZeroSmemBytes, row_bytes - off));
-        }
-        bulk_commit();
-    }
-    bulk_wait_all();
-}
-
-template <int VB>
-__device__ __forceinline__ typename Vec<VB>::T lds_vec(const uint8_t *p);
-template <>
-__device__ __forceinline__ uint4 lds_vec<16>(const uint8_t *p) {
-    return *reinterpret_cast<const uint4 *>(p);
-}
-template <>
-__device__ __forceinline__ u32x8 lds_vec<32>(const uint8_t *p) {
-    const uint4 a = *reinterpret_cast<const uint4 *>(p), b = *reinterpret_cast<const uint4 *>(p + 16);
-    u32x8 r;
-    r.v[0] = a.x; r.v[1] = a.y; r.v[2] = a.z; r.v[3] = a.w;
-    r.v[4] = b.x; r.v[5] = b.y; r.v[6] = b.z; r.v[7] = b.w;
-    return r;
-}
-
-template <int VB>
-__global__ void __launch_bounds__(kStagedThreads, 1) dispatch_bf16_staged_kernel(DispatchParams p) {
-    static_assert(kStagedThreads <= 1024, "too many consumer groups");
-    using V = Vec<VB>;
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int NS = p.stages;
-    const int row_bytes = p.H * 2;
-    const int chunk = row_bytes / p.splits;
-    uint8_t *buf = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + align_up((size_t)NS * chunk, 128));
-    uint64_t *empty = full + kStagedMaxStages;
-    int32_t *s_pos = reinterpret_cast<int32_t *>(empty + kStagedMaxStages);
-    uint8_t *zeros = reinterpret_cast<uint8_t *>(s_pos + kStagedPosInts);
-    __shared__ int s_abort;
-    __shared__ int s_rows;
-    volatile int *abort_flag = &s_abort;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_cta = p.n_token_units > (int)blockIdx.x
-                          ? (p.n_token_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
-                          : 0;
-    const int win = max(1, kStagedPosInts / p.K);
-    const uint8_t *x = static_cast<const uint8_t *>(p.x);
-    uint8_t *recv = static_cast<uint8_t *>(p.recv);
-
-    if (p.n_zero_units) {
-        for (int i = threadIdx.x; i < kZeroSmemBytes / 16; i += kStagedThreads)
-            reinterpret_cast<uint4 *>(zeros)[i] = make_uint4(0, 0, 0, 0);
-        fence_async_smem();
-    }
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kGroupWarps);
-        }
-        fence_async_smem();
-        s_abort = 0;
-    }
-#if EP_PDL_PREFETCH && EP_STAGED_PREFETCH
-    // an L2 prefetch may run before the wait: L2 is where writes land, so a
-    // line prefetched while the previous kernel still writes it is updated there
-    if (p.prefetch_x && threadIdx.x == 0) {
-        const uint64_t pol_x = policy_evict_last();
-        for (int i = 0; i < n_cta; ++i) {
-            const int u = blockIdx.x + i * gridDim.x;
-            const int t = u / p.splits, part = u - t * p.splits;
-            bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk, pol_x);
-        }
-    }
-#endif
-    pdl_wait();   // shared-memory set-up overlapped the previous kernel; global reads start here
-    if (threadIdx.x == 0) s_rows = p.n_zero_units ? __ldg(&p.eoff[p.E]) : 0;
-    __syncthreads();
-
-#if EP_STAGED_PREFETCH && !EP_PDL_PREFETCH
-    // bring all of this CTA's x chunks into L2 up front: HBM serves a short
-    // burst of reads, then only the stream of received-row writes, and the
-    // chunks stay in L2 (evict_last) while that stream passes through
-    if (p.prefetch_x && threadIdx.x == 0) {
-#if EP_STAGED_PREFETCH == 1
-        const uint64_t pol_x = policy_evict_last();
-#else
-        uint64_t pol_x;
-        asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol_x));
-#endif
-        for (int i = 0; i < n_cta; ++i) {
-            const int u = blockIdx.x + i * gridDim.x;
-            const int t = u / p.splits, part = u - t * p.splits;
-            bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk, pol_x);
-        }
-    }
-#endif
-#if EP_STAGED_STORE_EVICT_FIRST
-    const uint64_t pol_out = policy_evict_first();
-#endif
-
-    int issued = 0;   // producer: units whose load was issued
-    for (int w0 = 0; w0 < n_cta; w0 += win) {
-        const int wn = min(win, n_cta - w0);
-        for (int i = threadIdx.x; i < wn * p.K; i += kStagedThreads) {
-            const int u = blockIdx.x + (w0 + i / p.K) * gridDim.x;
-            s_pos[i] = __ldg(&p.pos[(int64_t)(u / p.splits) * p.K + (i % p.K)]);
-        }
-        __syncthreads();
-        if (warp == 0) {
-            if (lane == 0) {
-                for (int i = w0; i < w0 + wn && !*abort_flag; ++i) {
-                    const int s = i % NS, use = i / NS;
-                    if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1, p.wait_limit_ns)) {
-                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                        *abort_flag = 1;
-                        break;
-                    }
-                    const int u = blockIdx.x + i * gridDim.x;
-                    const int t = u / p.splits, part = u - t * p.splits;
-                    mbar_arrive_expect_tx(&full[s], chunk);
-                    bulk_g2s(buf + (size_t)s * chunk, x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk,
-                             &full[s]);
-                    ++issued;
-                }
-            }
-        } else if (warp == kZeroWarp) {
-            if (w0 == 0) zero_fill_warp(p, s_rows, row_bytes, zeros, lane);
-        } else {
-            const int grp = (threadIdx.x - 32) / kGroupThreads;
-            const int gtid = (threadIdx.x - 32) - grp * kGroupThreads;
-            const int nv = chunk / VB;
-            for (int i = w0 + ((grp - w0 % kStagedGroups + kStagedGroups) % kStagedGroups); i < w0 + wn;
-                 i += kStagedGroups) {
-                const int s = i % NS;
-                if (!mbar_wait_bounded(&full[s], (i / NS) & 1, p.wait_limit_ns)) {
-                    atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                    *abort_flag = 1;
-                    break;
-                }
-                const int part = (blockIdx.x + i * gridDim.x) % p.splits;
-                const uint8_t *src = buf + (size_t)s * chunk;
-                const int32_t *dsts = s_pos + (i - w0) * p.K;
-                for (int v = gtid; v < nv; v += kGroupThreads) {
-                    const typename V::T val = lds_vec<VB>(src + v * VB);
-                    for (int k = 0; k < p.K; ++k) {
-                        const int dst = dsts[k];
-                        if (dst >= 0)
-#if EP_STAGED_STORE_EVICT_FIRST
-                            V::store(recv + (int64_t)dst * row_bytes + (int64_t)part * chunk + (int64_t)v * VB, val,
-                                     pol_out);
-#else
-                            V::store(recv + (int64_t)dst * row_bytes + (int64_t)part * chunk + (int64_t)v * VB, val);
-#endif
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-            }
-        }
-        __syncthreads();
-        if (*abort_flag) break;
-    }
-    if (n_cta == 0 && warp == kZeroWarp) zero_fill_warp(p, s_rows, row_bytes, zeros, lane);
-    if (*abort_flag && threadIdx.x == 0) {
-        // let every issued load land before the CTA's shared memory goes away
-        for (int j = max(0, issued - NS); j < issued; ++j)
-            mbar_wait_bounded(&full[j % NS], (j / NS) & 1, p.wait_limit_ns);
-    }
-}
-
 // Index of the scale of received row `row`, block b, in either layout.
 // Column-major scales come in groups of scale_group_rows rows (the whole
 // buffer, or one expert's M slots), each group [H/128][scale_ld].
@@ -481,8 +251,8 @@ __global__ void __launch_bounds__(kThreads, EP_FP8_MINB) dispatch_fp8_kernel(Dis
     int nblk = gridDim.x;
     if constexpr (!LL) {
         // this CTA's token rows into L2 (evict_last) before the dependency
-        // wait, as in the staged bf16 kernel: L2 is where writes land, so a
-        // line prefetched while the previous kernel still writes it is updated
+        // wait: L2 is where writes land, so a line prefetched while the
+        // previous kernel still writes it is updated
         if (p.prefetch_x && threadIdx.x == 0) {
             const uint64_t pol_x = policy_evict_last();
             for (int t = blockIdx.x; t < p.n_token_units; t += gridDim.x)
@@ -606,31 +376,6 @@ __global__ void __launch_bounds__(kThreads, EP_FP8_MINB) dispatch_fp8_kernel(Dis
 
 }  // namespace
 
-// Staged launch shape for rows of row_bytes with VB-byte vectors: the row is
-// split into the fewest power-of-two chunks of at most EP_STAGED_CHUNK_MAX
-// bytes (a multiple of VB); 0 stages means "use the register kernel".
-static void staged_shape(int row_bytes, int VB, int *splits, int *stages) {
-    int sp = 1;
-    while (sp <= 64 && (row_bytes / sp > EP_STAGED_CHUNK_MAX || row_bytes % (sp * VB) != 0)) sp *= 2;
-    *splits = sp;
-    *stages = 0;
-    if (!EP_DISPATCH_STAGED || sp > 64 || row_bytes % (sp * VB) != 0) return;
-    int ns = EP_STAGED_SMEM / (row_bytes / sp);
-    ns = ns > kStagedMaxStages ? kStagedMaxStages : ns;
-    if (ns >= 3) *stages = ns;
-}
-
-cudaError_t dispatch_prepare() {
-    const int smem = (int)staged_smem_bytes(kStagedMaxStages, EP_STAGED_CHUNK_MAX);
-    const void *kernels[] = {reinterpret_cast<const void *>(&dispatch_bf16_staged_kernel<32>),
-                             reinterpret_cast<const void *>(&dispatch_bf16_staged_kernel<16>)};
-    for (const void *k : kernels) {
-        const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
-}
-
 // Launch that may start while the previous kernel on the stream finishes
 // (programmatic stream serialization); the kernels wait with pdl_wait()
 // before touching global memory.
@@ -650,33 +395,20 @@ static cudaError_t launch_pdl(Kernel kernel, int grid, int block, size_t smem, c
     return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-cudaError_t launch_dispatch_bf16(const DispatchParams &p_in, int num_sms, cudaStream_t s) {
+// The register kernel: batches too small to fill the GPU (ep_dispatch routes
+// larger ones to the chunked kernel of dispatch_lb.cu).
+cudaError_t launch_dispatch_bf16(const DispatchParams &p, int num_sms, cudaStream_t s) {
     static OccupancyCache occ16, occ32;
-    DispatchParams p = p_in;
     const bool v32 = (p.H % 16 == 0) && ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
-    const int row_bytes = p.H * 2;
-    int splits = 1, stages = 0;
-    staged_shape(row_bytes, v32 ? 32 : 16, &splits, &stages);
-    if (stages > 0 && p.T * splits >= 4 * num_sms) {
-        p.splits = splits;
-        p.stages = stages;
-        p.n_token_units = p.T * splits;
-        const int units = p.n_token_units + p.n_zero_units;
-        const int grid = units < num_sms ? units : num_sms;
-        const size_t smem = staged_smem_bytes(stages, row_bytes / splits);
-        return v32 ? launch_pdl(dispatch_bf16_staged_kernel<32>, grid, kStagedThreads, smem, s, p)
-                   : launch_pdl(dispatch_bf16_staged_kernel<16>, grid, kStagedThreads, smem, s, p);
-    }
     const int units = p.n_token_units + p.n_zero_units;
     if (v32) {
         const void *k = reinterpret_cast<const void *>(&dispatch_bf16_kernel<32, false>);
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ32), num_sms);
         return launch_pdl(dispatch_bf16_kernel<32, false>, grid, kThreads, 0, s, p);
-    } else {
-        const void *k = reinterpret_cast<const void *>(&dispatch_bf16_kernel<16, false>);
-        const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ16), num_sms);
-        return launch_pdl(dispatch_bf16_kernel<16, false>, grid, kThreads, 0, s, p);
     }
+    const void *k = reinterpret_cast<const void *>(&dispatch_bf16_kernel<16, false>);
+    const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ16), num_sms);
+    return launch_pdl(dispatch_bf16_kernel<16, false>, grid, kThreads, 0, s, p);
 }
 
 // Low-latency launches: the register kernels with in-kernel destinations.
@@ -728,9 +460,7 @@ cudaError_t launch_ll_dispatch(const DispatchParams &p_in, bool fp8, int num_sms
     return cudaLaunchKernelExC(&cfg, k, args);
 }
 
-// FP8 uses the register kernel: quantising from a staged ring with one
-// consumer group per SM measured slower (the quantisation needs the
-// register kernel's four resident blocks per SM).
+// The FP8 register kernel, four resident blocks per SM.
 cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream_t s) {
     static OccupancyCache occ16, occ32;
     const int units = p.n_token_units + p.n_zero_units;

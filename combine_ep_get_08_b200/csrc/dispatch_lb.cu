@@ -30,27 +30,25 @@
 //     reads only topk_idx, so it runs before the dependency wait, beside the
 //     pre-pass.  After it, a pair's row is the expert's offset + the pairs of
 //     earlier super-chunks + the look-back prefix + its rank; the chunk's
-//     routing is written and a per-chunk ready flag released.  Then every
-//     CTA copies its share of the token rows in interleaved order (CTA b
-//     takes row parts b, b + G, ...; each waits, bounded, for the ready flags
-//     of the chunks it reads): the x rows stream through a shared-memory ring
-//     of bulk copies (TMA engine, no multicast) to their rows, as a plain copy
-//     (bf16) or with the fused 1x128-block FP8 E4M3 quantisation of
-//     "m.nlpx.cn/news/135159" section 4.1.  No CTA copies before it has
+//     routing is written and a per-chunk ready flag released.  Then the CTAs
+//     copy: each claims row parts in small batches from an atomic counter (a
+//     part waits, bounded, for the ready flag of its token's chunk), and the
+//     x bytes and the token's destinations stream through a shared-memory
+//     ring of bulk copies (TMA engine, no multicast) to the token's K rows, as
+//     a plain copy (bf16) or with the fused 1x128-block FP8 E4M3 quantisation
+//     of "m.nlpx.cn/news/135159" section 4.1.  No CTA copies before it has
 //     finished every chunk it took, so a copy waits only on chunks that
 //     running CTAs complete without waiting on copies.  One warp writes the
 //     padding rows (zeros, and -1 routing) with bulk copies meanwhile.
 //
 // With lb = 0 the same kernel takes the positions from the handle (a layout
-// computed earlier) and is a chunked, dynamically scheduled dispatch.
+// computed earlier): it is the dispatch of ep_dispatch / ep_dispatch_fp8 for
+// batches that fill the GPU.
 #include "ep_internal.cuh"
 #include "fp8_block.cuh"
 
 #ifndef EP_LB_FP8_GROUPS
 #define EP_LB_FP8_GROUPS 2          // FP8 consumer groups per CTA (quantisation needs more warps)
-#endif
-#ifndef EP_LB_DYN
-#define EP_LB_DYN 1                 // copy phase: row parts claimed in batches (0: fixed interleaved order)
 #endif
 #ifndef EP_LB_RING_BYTES
 #define EP_LB_RING_BYTES (112 * 1024)
@@ -66,10 +64,13 @@ constexpr int kLayoutRankWarps = 8;     // warps that rank a chunk's pairs
 constexpr int kMaxStages = 16;
 constexpr int kZeroBytes = 8192;        // zeroed shared memory the padding warp copies from
 constexpr int kFp8Ept = 32;             // FP8: bf16 elements per consumer thread
-#ifndef EP_LB_DYN_BATCH
-#define EP_LB_DYN_BATCH 4
+constexpr int kStageDst = kMaxTopk + 4;  // int32 per stage for a token's destinations (+ alignment lead)
+#ifndef EP_LB_DYN_TOKENS_BF16
+#define EP_LB_DYN_TOKENS_BF16 1     // tokens per claim of the dynamic copy, bf16 (dsv3: 1 -> 90.8 us,
+#endif                              // 2 -> 92.4 us, 4 -> 94.7 us)
+#ifndef EP_LB_DYN_TOKENS_FP8
+#define EP_LB_DYN_TOKENS_FP8 4      // tokens per claim, FP8
 #endif
-constexpr int kDynBatch = EP_LB_DYN_BATCH;   // row parts per claim of the dynamic copy
 
 template <int G>
 struct Shape {
@@ -82,7 +83,7 @@ __host__ __device__ __forceinline__ size_t up(size_t v, size_t a) { return (v + 
 
 // Dynamic shared memory carve-up (same on host and device).
 struct Carve {
-    size_t ring, bars, zeros, pos, e16, rk16, cnt, base, agg, unit, stpos, total;
+    size_t ring, bars, zeros, e16, rk16, cnt, base, agg, unit, stpos, total;
 };
 __host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int E) {
     Carve c;
@@ -90,7 +91,6 @@ __host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int
     c.ring = o;  o += up((size_t)stages * chunk_bytes, 128);
     c.bars = o;  o += 2 * kMaxStages * sizeof(uint64_t);
     c.zeros = o; o += kZeroBytes;
-    c.pos = o;   o += (size_t)kLbMaxPairs * sizeof(int32_t);
     c.e16 = o;   o += (size_t)kLbMaxPairs * sizeof(int16_t);
     c.rk16 = o;  o += (size_t)kLbMaxPairs * sizeof(int16_t);
     c.cnt = o;   o += (size_t)kLayoutRankWarps * (E + 1) * sizeof(int32_t);
@@ -99,7 +99,7 @@ __host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int
     o = up(o, 128);
     c.unit = o;  o += (size_t)kMaxStages * sizeof(int32_t);
     o = up(o, 128);                      // bulk-copy destinations: 16-byte aligned
-    c.stpos = o; o += (size_t)kMaxStages * kMaxTopk * sizeof(int32_t);
+    c.stpos = o; o += (size_t)kMaxStages * kStageDst * sizeof(int32_t);
     c.total = up(o, 128);
     return c;
 }
@@ -381,14 +381,13 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + cv.bars);
     uint64_t *empty = full + kMaxStages;
     uint8_t *zeros = smem + cv.zeros;
-    int32_t *s_pos = reinterpret_cast<int32_t *>(smem + cv.pos);
     int16_t *s_e = reinterpret_cast<int16_t *>(smem + cv.e16);
     int16_t *s_rk = reinterpret_cast<int16_t *>(smem + cv.rk16);
     int32_t *s_cnt = reinterpret_cast<int32_t *>(smem + cv.cnt);
     int32_t *s_base = reinterpret_cast<int32_t *>(smem + cv.base);
     int32_t *s_agg = reinterpret_cast<int32_t *>(smem + cv.agg);
-    int32_t *s_unit = reinterpret_cast<int32_t *>(smem + cv.unit);     // [stages] row part in each stage (-1: end)
-    int32_t *s_stpos = reinterpret_cast<int32_t *>(smem + cv.stpos);   // [stages][K] its destinations
+    int32_t *s_unit = reinterpret_cast<int32_t *>(smem + cv.unit);     // [stages] row part | lead << 28 (-1: end)
+    int32_t *s_stpos = reinterpret_cast<int32_t *>(smem + cv.stpos);   // [stages][kStageDst] its destinations
     __shared__ int s_ticket;
     __shared__ int s_abort;
     __shared__ unsigned int s_tag;
@@ -404,7 +403,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         for (int i = tid; i < kZeroBytes / 16; i += S::kThreads) reinterpret_cast<uint4 *>(zeros)[i] = make_uint4(0, 0, 0, 0);
         fence_async_smem();
     }
-    // this CTA's units: u = blockIdx.x + i * gridDim.x (see the copy phase)
+    // this CTA's share of the row parts for the L2 prefetch of x: b, b + G, ...
     const int GC = gridDim.x;
     const int total_units = p.T * p.splits;
     const int n_cta = total_units > (int)blockIdx.x ? (total_units - (int)blockIdx.x + GC - 1) / GC : 0;
@@ -426,41 +425,19 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     } else {
         const uint64_t pol_out = policy_evict_first();
         const unsigned int tag = s_tag;
-        // Copy order: this CTA's units are u = blockIdx.x + i * gridDim.x (unit
-        // u = part u % splits of token u / splits), so at any moment the CTAs
-        // write the rows of neighbouring tokens, which lie close together in
-        // every expert segment; contiguous token chunks per CTA measured 8%
-        // slower on the write stream.
-        int issued = 0;   // producer (thread 0): units whose load was issued
-        // the producer's load of this CTA's unit i into stage i % NS; false on a timeout
-        auto issue = [&](int i) -> bool {
-            const int s = i % NS;
-            if (i >= NS && !mbar_wait_bounded(&empty[s], ((i / NS) - 1) & 1, p.wait_limit_ns)) return false;
-            const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
-            mbar_arrive_expect_tx(&full[s], chunk);
-            bulk_g2s(ring + (size_t)s * chunk, x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk, &full[s]);
-            ++issued;
-            return true;
-        };
+        int issued = 0;   // producer (thread 0): row parts whose load was issued
         // the first chunk's ticket is requested before anything else
         if (p.lb && tid == 0) s_ticket = (int)atomicAdd(&p.ctl->ticket, 1u);
-        // x is an input: the first units go into the ring now, overlapping the
-        // layout (with lb = 0 all of this CTA's x chunks also go into L2 now;
-        // with lb = 1 the padding warp does that after the dependency wait)
-        if (tid == 0) {
-            if (p.prefetch_x && !p.lb) {
-                const uint64_t pol_x = policy_evict_last();
-                for (int i = 0; i < n_cta; ++i) {
-                    const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
-                    bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
-                }
+        // x is an input: with lb = 0 a share of it (row parts b, b + G, ... --
+        // together all of x) goes into L2 now, overlapping the kernel before;
+        // with lb = 1 the padding warp does that after the dependency wait,
+        // where it cannot delay the latency-bound layout phases
+        if (tid == 0 && p.prefetch_x && !p.lb) {
+            const uint64_t pol_x = policy_evict_last();
+            for (int i = 0; i < n_cta; ++i) {
+                const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
+                bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
             }
-            for (int i = 0; i < (p.dyn ? 0 : min(NS, n_cta)); ++i)
-                if (!issue(i)) {
-                    atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                    *abort_flag = 1;
-                    break;
-                }
         }
         __syncwarp();
 
@@ -601,23 +578,25 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         }
         pdl_wait();            // (a no-op after the first wait) the layout before is complete and visible
 
-        // ---- phase 2, dynamic: row parts claimed in batches of kDynBatch ----
+        // ---- phase 2: the copy; row parts claimed in batches of dyn_batch ----
         // The producer claims a batch from ctl->units (the next claim is
         // requested before the current batch is issued), and per row part puts
-        // its x bytes and its K destinations (a second bulk copy, K*4 bytes) into
+        // its x bytes and its token's K destinations (a second bulk copy) into
         // one stage, completing on the stage's barrier.  Consumer group grp takes
         // the stages g = grp, grp + G, ...; a part of -1 ends the group's loop.
-        // CTAs on SMs that move bytes faster take more parts.
-        if (p.dyn) {
+        // CTAs on SMs that move bytes faster take more parts: against a fixed
+        // interleaved order (CTA b taking parts b, b + G, ...) this measured
+        // dsv3 bf16 96.1 -> 90.8 us and large FP8 (fused) 277.2 -> 237.1 us.
+        {
             if (warp == 0) {
                 if (lane == 0) {
                     int g = 0;
                     unsigned int claim = atomicAdd(&p.ctl->units, 1u);
                     while (!*abort_flag) {
-                        const int u0 = (int)claim * kDynBatch;
+                        const int u0 = (int)claim * p.dyn_batch;
                         if (u0 >= total_units) break;
                         const unsigned int next = atomicAdd(&p.ctl->units, 1u);
-                        for (int u = u0; u < min(total_units, u0 + kDynBatch) && !*abort_flag; ++u, ++g) {
+                        for (int u = u0; u < min(total_units, u0 + p.dyn_batch) && !*abort_flag; ++u, ++g) {
                             const int s = g % NS;
                             bool ok = g < NS || mbar_wait_bounded(&empty[s], ((g / NS) - 1) & 1, p.wait_limit_ns);
                             const int t = u / p.splits, part = u - t * p.splits;
@@ -634,11 +613,18 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
                                 *abort_flag = 1;
                                 break;
                             }
-                            s_unit[s] = u;
-                            mbar_arrive_expect_tx(&full[s], (uint32_t)(chunk + K * 4));
+                            // the token's K destinations: the 16-byte aligned span that holds
+                            // them (pos is followed by other arrays of the handle's allocation,
+                            // so the span never leaves it); the consumers skip `lead` entries
+                            const int64_t b0 = (int64_t)t * K * 4, a0 = b0 & ~(int64_t)15;
+                            const int lead = (int)(b0 - a0) / 4;
+                            const uint32_t span = (uint32_t)((b0 + K * 4 - a0 + 15) & ~(int64_t)15);
+                            s_unit[s] = u | (lead << 28);
+                            mbar_arrive_expect_tx(&full[s], (uint32_t)chunk + span);
                             bulk_g2s(ring + (size_t)s * chunk, x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk,
                                      &full[s]);
-                            bulk_g2s(s_stpos + s * kMaxTopk, p.pos + (int64_t)t * K, (uint32_t)(K * 4), &full[s]);
+                            bulk_g2s(s_stpos + s * kStageDst, reinterpret_cast<const uint8_t *>(p.pos) + a0, span,
+                                     &full[s]);
                             ++issued;
                         }
                         claim = next;
@@ -665,78 +651,21 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
                         *abort_flag = 1;
                         break;
                     }
-                    const int u = s_unit[s];
-                    if (u < 0) break;
+                    const int su = s_unit[s];
+                    if (su < 0) break;
+                    const int u = su & 0x0fffffff, lead = su >> 28;
                     const int part = u % p.splits;
+                    const int32_t *dsts = s_stpos + s * kStageDst + lead;
                     if constexpr (FP8)
-                        quantise_unit(p, ring + (size_t)s * chunk, s_stpos + s * kMaxTopk, part, gtid, pol_out);
+                        quantise_unit(p, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
                     else
-                        copy_unit<VB>(p, ring + (size_t)s * chunk, s_stpos + s * kMaxTopk, part, gtid, pol_out);
+                        copy_unit<VB>(p, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[s]);
                 }
             }
         }
 
-        // ---- phase 2, static: the copy, window by window of staged destinations ----
-        const int win = max(1, kLbMaxPairs / K);
-        for (int w0 = 0; w0 < n_cta && !*abort_flag && !p.dyn; w0 += win) {
-            const int wn = min(win, n_cta - w0);
-            if (p.lb) {
-                // every chunk behind this window's tokens has published its rows
-                for (int i = tid; i < wn; i += NSET) {
-                    const int t = ((int)blockIdx.x + (w0 + i) * GC) / p.splits;
-                    const unsigned int *rf = p.ready + t / p.tpc;
-                    if (ld_acquire_u32(rf) != tag) {
-                        const unsigned long long tw0 = globaltimer_ns();
-                        while (ld_acquire_u32(rf) != tag)
-                            if (globaltimer_ns() - tw0 > p.wait_limit_ns) {
-                                atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                                *abort_flag = 1;
-                                break;
-                            }
-                    }
-                }
-                set_sync(NSET);
-                if (*abort_flag) break;
-            }
-            for (int i = tid; i < wn * K; i += NSET) {
-                const int t = ((int)blockIdx.x + (w0 + i / K) * GC) / p.splits;
-                const int32_t *pp = p.pos + (int64_t)t * K + (i % K);
-                s_pos[i] = p.lb ? __ldcg(pp) : __ldg(pp);
-            }
-            set_sync(NSET);
-            if (warp == 0) {
-                if (lane == 0)
-                    for (int i = max(issued, w0); i < w0 + wn && !*abort_flag; ++i)
-                        if (!issue(i)) {
-                            atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                            *abort_flag = 1;
-                            break;
-                        }
-                __syncwarp();
-            } else {
-                const int grp = (tid - 32) / kGroupThreads, gtid = (tid - 32) - grp * kGroupThreads;
-                // unit i belongs to consumer group i % G
-                for (int i = w0 + ((grp - w0 % G) % G + G) % G; i < w0 + wn; i += G) {
-                    const int s = i % NS;
-                    // the warp decides together, so that no lane is left alone at a __syncwarp
-                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (i / NS) & 1, p.wait_limit_ns))) {
-                        if (lane == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                        *abort_flag = 1;
-                        break;
-                    }
-                    const int u = (int)blockIdx.x + i * GC, part = u % p.splits;
-                    if constexpr (FP8)
-                        quantise_unit(p, ring + (size_t)s * chunk, s_pos + (i - w0) * K, part, gtid, pol_out);
-                    else
-                        copy_unit<VB>(p, ring + (size_t)s * chunk, s_pos + (i - w0) * K, part, gtid, pol_out);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[s]);
-                }
-            }
-            set_sync(NSET);   // every unit of the window consumed
-        }
         if (*abort_flag && tid == 0) {
             // let every issued load land before the CTA's shared memory goes away
             for (int j = max(0, issued - NS); j < issued; ++j)
@@ -869,8 +798,9 @@ cudaError_t launch_dispatch_lb(const LbParams &p_in, bool fp8, int num_sms, cuda
                      ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
     const int VB = v32 ? 32 : 16;
     p.vec32 = (reinterpret_cast<uintptr_t>(p.recv) & 31) == 0;
-    // dynamic copy: each part's K destinations arrive by a bulk copy (16-byte multiple)
-    p.dyn = EP_LB_DYN && p.K % 4 == 0 && (reinterpret_cast<uintptr_t>(p.pos) & 15) == 0;
+    if (reinterpret_cast<uintptr_t>(p.pos) & 15) return cudaErrorInvalidValue;   // the handle's: 256-byte aligned
+    if ((int64_t)p.T * p.splits >= (int64_t(1) << 28)) return cudaErrorInvalidValue;   // stage tags hold 28 bits
+    p.dyn_batch = p.splits * (fp8 ? EP_LB_DYN_TOKENS_FP8 : EP_LB_DYN_TOKENS_BF16);
     if (!lb_unit_shape(p.H, fp8, VB, &p.splits, &p.chunk_bytes)) return cudaErrorInvalidValue;
     const size_t limit = smem_limit();
     const size_t fixed = carve(0, p.chunk_bytes, p.E).total;

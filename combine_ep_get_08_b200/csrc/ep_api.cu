@@ -153,8 +153,7 @@ EP_API int ep_handle_create(const ep_config *cfg, ep_handle **out) {
     h->G = h->plan.G;
     h->tokens_per_chunk = h->plan.tokens_per_chunk;
 
-    e = ep::dispatch_prepare();
-    if (e == cudaSuccess) e = ep::dispatch_lb_prepare();
+    e = ep::dispatch_lb_prepare();
     if (e != cudaSuccess) return fail(cuda_fail(e, "cudaFuncSetAttribute(dispatch)"));
     h->lb = ep::plan_lb(T, K, h->num_sms);
 
@@ -297,13 +296,6 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
     return EP_OK;
 }
 
-#ifndef EP_FP8_CHUNKED
-#define EP_FP8_CHUNKED 0   // 1: ep_dispatch_fp8 runs the chunked, staged kernel of dispatch_lb.cu
-#endif
-#ifndef EP_BF16_CHUNKED
-#define EP_BF16_CHUNKED 0  // 1: ep_dispatch does too
-#endif
-
 static ep::LbParams lb_params(const ep_handle *h, const void *x, void *recv, float *scales, int lb);
 
 static int dispatch_common(const ep_handle *h, const void *x, void *recv, float *scales, bool fp8,
@@ -334,7 +326,6 @@ static int dispatch_common(const ep_handle *h, const void *x, void *recv, float 
     p.status = h->status;
     p.wait_limit_ns = h->wait_limit_ns;
     p.splits = 1;
-    p.stages = 0;
     p.n_token_units = p.T * p.splits;
     p.n_zero_units = c.expert_alignment > 1
                          ? (int)((h->cap + ep::kZeroRowsPerUnit - 1) / ep::kZeroRowsPerUnit)
@@ -344,11 +335,15 @@ static int dispatch_common(const ep_handle *h, const void *x, void *recv, float 
     p.prefetch_x = (int64_t)c.num_tokens * c.hidden * 2 <= (int64_t)h->l2_bytes / 2;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
-    cudaError_t e;
-    if (fp8 ? EP_FP8_CHUNKED : EP_BF16_CHUNKED)
-        e = ep::launch_dispatch_lb(lb_params(h, x, recv, scales, 0), fp8, sms, s);
-    else
-        e = fp8 ? ep::launch_dispatch_fp8(p, sms, s) : ep::launch_dispatch_bf16(p, sms, s);
+    // Batches that fill the GPU (at least two tokens per SM) take the chunked
+    // kernel of dispatch_lb.cu with its dynamically claimed copy order (against
+    // the earlier staged bf16 / register FP8 kernels: dsv3 bf16 93.6 -> 90.8 us,
+    // large FP8 260.2 -> 218.2 us in one A/B run); smaller ones the register
+    // kernels of dispatch.cu.
+    const bool chunked = c.num_tokens >= 2 * sms && c.num_tokens < ep::kLbMaxTokens;
+    cudaError_t e = chunked ? ep::launch_dispatch_lb(lb_params(h, x, recv, scales, 0), fp8, sms, s)
+                    : fp8   ? ep::launch_dispatch_fp8(p, sms, s)
+                            : ep::launch_dispatch_bf16(p, sms, s);
     if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(dispatch_fp8)" : "launch(dispatch)");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return EP_OK;
@@ -413,6 +408,10 @@ static int layout_dispatch_common(ep_handle *h, const int64_t *topk_idx, const f
     if (rc != EP_OK) return rc;
     const ep_config &c = h->cfg;
     if (fp8 && c.hidden % 128 != 0) return EP_ERR_ARG;
+    if (c.num_tokens >= ep::kLbMaxTokens) {
+        ep::record_error("ep_layout_dispatch: at most 2^22 - 1 tokens per call");
+        return EP_ERR_UNSUPPORTED;
+    }
     if (c.num_tokens > 0 && (!topk_idx || !x || !recv || (fp8 && !scales))) return EP_ERR_ARG;
     if (!aligned(topk_idx, 8) || !aligned(topk_weights, 4) || !aligned(x, 16) || !aligned(recv, 16) ||
         !aligned(scales, 4) || !aligned(num_tokens_per_expert, 4) || !aligned(num_tokens_per_rank, 4) ||
@@ -479,7 +478,6 @@ static int combine_common(const ep_handle *h, const void *y, const float *topk_w
     p.status = h->status;
     p.wait_limit_ns = h->wait_limit_ns;
     p.splits = 1;
-    p.stages = 0;
     p.n_units = p.T * p.splits;
     const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
     cudaError_t e = ep::launch_combine(p, sms, reinterpret_cast<cudaStream_t>(stream));

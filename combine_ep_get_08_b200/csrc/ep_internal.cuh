@@ -65,8 +65,6 @@ struct DispatchParams {
     int splits;                  // column splits per token
     int n_token_units;           // T * splits
     int n_zero_units;            // ceil(cap / kZeroRowsPerUnit) when A > 1, else 0
-    int stages;                  // shared-memory ring depth (staged kernel)
-    int groups;                  // consumer groups (staged kernel)
     int scale_group_rows;        // column-major scales: rows per [H/128][scale_ld] group
     int prefetch_x;              // 1: each CTA prefetches its x rows into L2 before the dependency wait
     // low-latency static layout (ll_M > 0): destinations computed in-kernel
@@ -87,7 +85,6 @@ struct CombineParams {
     int T, K, H;
     int splits;
     int n_units;
-    int stages;                  // shared-memory ring depth (staged kernel)
 };
 
 // Expert GEMM with the combine fused into its epilogue.
@@ -119,6 +116,7 @@ cudaError_t launch_gemm_combine(const GemmCombineArgs &g, int num_sms, cudaStrea
 // ---------------------------------------------------------------------------
 constexpr int kLbSuper = 16;          // token chunks per super-chunk (one pre-pass CTA each)
 constexpr int kLbMaxPairs = 4096;     // (token, k) pairs per chunk at most
+constexpr int kLbMaxTokens = 1 << 22; // tokens per call of the chunked kernel, below this
 
 // Device-side control words of the fused path (in the handle's allocation,
 // zeroed at creation; each kernel leaves them as it found them).
@@ -169,6 +167,7 @@ struct LbParams {
     int prefetch_x;              // 1: the chunk's x rows are prefetched into L2 at its start
     int vec32;                   // FP8: 1 when recv is 32-byte aligned (32-byte code stores)
     int dyn;                     // 1: row parts are claimed in batches from ctl->units (K % 4 == 0)
+    int dyn_batch;               // row parts per claim
 };
 cudaError_t launch_layout_counts(const LbParams &p, cudaStream_t s);
 // The fused (lb = 1) or handle-driven (lb = 0) chunked dispatch, bf16 or FP8.
@@ -201,9 +200,6 @@ cudaError_t launch_dispatch_bf16(const DispatchParams &p, int num_sms, cudaStrea
 cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream_t s);
 // Low-latency static layout + copy in one launch (p.ll_M > 0).
 cudaError_t launch_ll_dispatch(const DispatchParams &p, bool fp8, int num_sms, cudaStream_t s);
-// Per device, before the first dispatch launch: kernel attributes (dynamic
-// shared memory of the staged kernel).
-cudaError_t dispatch_prepare();
 cudaError_t launch_combine(const CombineParams &p, int num_sms, cudaStream_t s);
 
 // Error text for ep_last_error and the library's launch counter (ep_api.cu).

@@ -102,9 +102,12 @@ SMALL = [
     dict(T=20000, H=64, E=64, R=8, K=8, A=4, router="topk", seed=27),        # beyond one cluster: cooperative
     dict(T=16384, H=64, E=256, R=64, K=8, A=2, router="group", seed=28),     # 131072 pairs: cooperative
     dict(T=8192, H=64, E=256, R=64, K=8, A=2, router="group", seed=30),      # 16-CTA cluster, 4096 pairs each
-    # staged bf16 dispatch whose CTAs walk more than one window of staged
-    # destinations (4096 / K = 64 units per window, ~82 units per CTA)
+    # K = 64: a token's destinations fill a whole stage slot (256 bytes)
     dict(T=12000, H=128, E=128, R=8, K=64, A=1, router="topk", seed=29),
+    # K % 4 != 0 on the chunked dispatch: destination spans start inside a
+    # 16-byte word (1 200 tokens fill the GPU: chunked, not the register kernel)
+    dict(T=1200, H=512, E=64, R=8, K=6, A=5, router="topk", seed=32),
+    dict(T=1201, H=256, E=32, R=4, K=3, A=2, router="uniform", seed=33),
 ]
 
 
@@ -271,9 +274,9 @@ def test_host_argument_errors():
 def test_sm_limit_parity(sms, fp8):
     """Dispatch and combine capped to a few SMs (ep_set_sm_limit, the num_sms
     budget of bowenzhou.top "deepep/01-overview" section 1.1) against the
-    oracle.  With one SM the staged bf16 dispatch runs all 1200 tokens in one
-    CTA, so it walks three windows of staged destinations (512 units each at
-    K = 8); the FP8 and combine grids shrink to the cap."""
+    oracle.  With one SM the chunked dispatch runs in one CTA, which claims
+    every row part of the 1200 tokens in turn and wraps its 16-stage ring
+    ~150 times; the combine grid shrinks to the cap."""
     wl = workloads.generate(None, T=1200, H=2048, E=64, R=8, K=8, A=4, router="topk", seed=61)
     run_full(wl, fp8, sm_limit=sms)
 
