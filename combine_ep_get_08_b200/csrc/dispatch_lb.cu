@@ -799,9 +799,10 @@ cudaError_t launch_dispatch_lb(const LbParams &p_in, bool fp8, int num_sms, cuda
     const int VB = v32 ? 32 : 16;
     p.vec32 = (reinterpret_cast<uintptr_t>(p.recv) & 31) == 0;
     if (reinterpret_cast<uintptr_t>(p.pos) & 15) return cudaErrorInvalidValue;   // the handle's: 256-byte aligned
+    if (!lb_unit_shape(p.H, fp8, VB, &p.splits, &p.chunk_bytes)) return cudaErrorInvalidValue;
     if ((int64_t)p.T * p.splits >= (int64_t(1) << 28)) return cudaErrorInvalidValue;   // stage tags hold 28 bits
     p.dyn_batch = p.splits * (fp8 ? EP_LB_DYN_TOKENS_FP8 : EP_LB_DYN_TOKENS_BF16);
-    if (!lb_unit_shape(p.H, fp8, VB, &p.splits, &p.chunk_bytes)) return cudaErrorInvalidValue;
+    if (p.dyn_batch < 1) return cudaErrorInvalidValue;
     const size_t limit = smem_limit();
     const size_t fixed = carve(0, p.chunk_bytes, p.E).total;
     int ns = (int)(EP_LB_RING_BYTES / p.chunk_bytes);
