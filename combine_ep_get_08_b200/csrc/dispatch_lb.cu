@@ -69,8 +69,8 @@ constexpr int kStageDst = kMaxTopk + 4;  // int32 per stage for a token's destin
 #define EP_LB_DYN_TOKENS_BF16 1     // tokens per claim of the dynamic copy, bf16 (dsv3: 1 -> 90.8 us,
 #endif                              // 2 -> 92.4 us, 4 -> 94.7 us)
 #ifndef EP_LB_DYN_TOKENS_FP8
-#define EP_LB_DYN_TOKENS_FP8 4      // tokens per claim, FP8
-#endif
+#define EP_LB_DYN_TOKENS_FP8 1      // tokens per claim, FP8 (skew: 1 -> 84.9 us, 2 -> 86.0, 4 -> 87.2,
+#endif                              // 8 -> 86.7; large: 212.0, 214.4, 217.5, 221.5)
 
 template <int G>
 struct Shape {

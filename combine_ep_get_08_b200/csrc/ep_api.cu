@@ -417,6 +417,15 @@ static int layout_dispatch_common(ep_handle *h, const int64_t *topk_idx, const f
         !aligned(scales, 4) || !aligned(num_tokens_per_expert, 4) || !aligned(num_tokens_per_rank, 4) ||
         !aligned(expert_offsets, 4) || !aligned(rank_offsets, 4))
         return EP_ERR_ARG;
+    const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
+    if (c.num_tokens > 0 && c.num_tokens < 2 * sms) {
+        // too few tokens to fill the GPU: the layout kernel, then the register
+        // dispatch (decode: 17.9 us for the two against 31.6 us fused)
+        rc = ep_get_layout(h, topk_idx, topk_weights, num_tokens_per_expert, num_tokens_per_rank,
+                           is_token_in_rank, expert_offsets, rank_offsets, stream);
+        if (rc != EP_OK) return rc;
+        return dispatch_common(h, x, recv, scales, fp8, stream);
+    }
     DeviceGuard g(h->device);
     if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
     ep::LbParams p = lb_params(h, x, recv, scales, 1);
@@ -433,7 +442,6 @@ static int layout_dispatch_common(ep_handle *h, const int64_t *topk_idx, const f
     g_launches.fetch_add(1, std::memory_order_relaxed);
     h->has_layout = true;
     if (c.num_tokens == 0) return EP_OK;
-    const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
     e = ep::launch_dispatch_lb(p, fp8, sms, s);
     if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(layout_dispatch_fp8)" : "launch(layout_dispatch)");
     g_launches.fetch_add(1, std::memory_order_relaxed);

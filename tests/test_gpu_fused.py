@@ -142,7 +142,10 @@ CASES = [
     dict(T=300, H=1024, E=8, R=2, K=8, A=300, router="topk", seed=26),       # A > T*K/E
     dict(T=20000, H=64, E=64, R=8, K=8, A=4, router="topk", seed=27),         # 148 chunks, 10 super-chunks
     dict(T=3000, H=128, E=128, R=8, K=64, A=1, router="topk", seed=29),       # 4096-pair chunks
+    dict(T=400, H=128, E=1024, R=128, K=64, A=2, router="topk", seed=34),     # max E and K in the fused kernel
 ]
+# Batches of fewer than two tokens per SM (tiny, T = 1, 33, 300 above) run as
+# ep_get_layout + ep_dispatch inside ep_layout_dispatch; the same checks apply.
 
 
 @pytest.mark.parametrize("spec", CASES, ids=lambda s: s.get("name") or f"T{s['T']}H{s['H']}E{s['E']}K{s['K']}A{s['A']}")
@@ -172,6 +175,14 @@ def test_fused_sm_limit(sms, fp8):
     ring stages and phases carry over from one chunk to the next."""
     wl = workloads.generate(None, T=1200, H=2048, E=64, R=8, K=8, A=4, router="topk", seed=61)
     run_fused(wl, fp8, sm_limit=sms)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_fused_kernel_small_batch(fp8):
+    """A 64-token batch under a one-SM cap takes the fused kernel (two tokens
+    per SM are enough): 64 one-token chunks, four super-chunks, one CTA."""
+    wl = workloads.generate("tiny")
+    run_fused(wl, fp8, sm_limit=1)
 
 
 def test_fused_masked_and_repeated():
