@@ -83,9 +83,9 @@ __host__ __device__ __forceinline__ size_t up(size_t v, size_t a) { return (v + 
 
 // Dynamic shared memory carve-up (same on host and device).
 struct Carve {
-    size_t ring, bars, zeros, e16, rk16, cnt, base, agg, unit, stpos, total;
+    size_t ring, bars, zeros, e16, rk16, cnt, base, agg, unit, stpos, peer, total;
 };
-__host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int E) {
+__host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int E, int peer_ranks = 0) {
     Carve c;
     size_t o = 0;
     c.ring = o;  o += up((size_t)stages * chunk_bytes, 128);
@@ -100,6 +100,8 @@ __host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int
     c.unit = o;  o += (size_t)kMaxStages * sizeof(int32_t);
     o = up(o, 128);                      // bulk-copy destinations: 16-byte aligned
     c.stpos = o; o += (size_t)kMaxStages * kStageDst * sizeof(int32_t);
+    o = up(o, 128);
+    c.peer = o;  o += peer_ranks ? 2 * sizeof(void *) * peer_ranks + sizeof(int32_t) * (2 * (size_t)peer_ranks + 1) : 0;
     c.total = up(o, 128);
     return c;
 }
@@ -143,6 +145,41 @@ __device__ __forceinline__ bool valid_id(int64_t e, int E) { return e >= 0 && e 
 
 __device__ __forceinline__ int64_t scale_at(const LbParams &p, int row, int b, int NB) {
     return p.scale_ld == 0 ? (int64_t)row * NB + b : (int64_t)b * p.scale_ld + row;
+}
+
+// Peer mode: where received row `row` of this rank lives -- rank r = the last
+// one with roff[r] <= row (empty segments share their start with the next),
+// row row0[r] + row - roff[r] of r's buffer.  The table is staged in shared
+// memory once per CTA.
+struct PeerTab {
+    uint8_t **base;    // [R] (null: not peer mode)
+    float **sbase;     // [R]
+    int32_t *row0;     // [R]
+    int32_t *roff;     // [R+1]
+    int R;
+};
+__device__ __forceinline__ int peer_rank(const PeerTab &t, int row) {
+    int lo = 0, hi = t.R - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (t.roff[mid] <= row)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+// Received row `row` (row_bytes each) of the local buffer, or of its destination rank's.
+__device__ __forceinline__ uint8_t *row_addr(const LbParams &p, const PeerTab &t, int row, int row_bytes) {
+    if (!t.base) return static_cast<uint8_t *>(p.recv) + (int64_t)row * row_bytes;
+    const int r = peer_rank(t, row);
+    return t.base[r] + (int64_t)(t.row0[r] + row - t.roff[r]) * row_bytes;
+}
+// Scale (row, b) of an FP8 row, local or at its destination rank (row-major there).
+__device__ __forceinline__ float *scale_addr(const LbParams &p, const PeerTab &t, int row, int b, int NB) {
+    if (!t.base) return p.recv_scale + scale_at(p, row, b, NB);
+    const int r = peer_rank(t, row);
+    return t.sbase[r] + (int64_t)(t.row0[r] + row - t.roff[r]) * NB + b;
 }
 
 // ---------------------------------------------------------------------------
@@ -262,7 +299,8 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_counts_kernel(LbPara
 // dependency wait, so it does not delay the latency-bound layout work).
 // ---------------------------------------------------------------------------
 template <bool FP8>
-__device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros, int lane, int n_cta, int chunk) {
+__device__ __forceinline__ void pad_rows(const LbParams &p, const PeerTab &tab, const uint8_t *zeros, int lane,
+                                         int n_cta, int chunk) {
     pdl_wait();   // offsets and counts come from the kernel before
     if (p.lb && p.prefetch_x && lane == 0) {
         const uint64_t pol_x = policy_evict_last();
@@ -278,6 +316,19 @@ __device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros
     const bool bulk_scales = FP8 && p.scale_ld == 0 && (NB * 4) % 16 == 0 &&
                              (reinterpret_cast<uintptr_t>(p.recv_scale) & 15) == 0;
     uint8_t *recv = static_cast<uint8_t *>(p.recv);
+    if (tab.base) {
+        // peer mode: plain 16-byte stores only, the warp's lanes across each row
+        for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
+            const int r0 = __ldcg(p.eoff + e) + __ldcg(p.cnt + e), r1 = __ldcg(p.eoff + e + 1);
+            for (int r = r0; r < r1; ++r) {
+                uint8_t *o = row_addr(p, tab, r, row_bytes);
+                for (int off = lane * 16; off < row_bytes; off += 32 * 16) st_v4(o + off, make_uint4(0, 0, 0, 0));
+                if (FP8)
+                    for (int b = lane; b < NB; b += 32) *scale_addr(p, tab, r, b, NB) = 0.0f;
+            }
+        }
+        return;
+    }
     for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
         const int r0 = __ldcg(p.eoff + e) + __ldcg(p.cnt + e), r1 = __ldcg(p.eoff + e + 1);
         for (int r = r0 + lane; r < r1; r += 32) {
@@ -303,10 +354,9 @@ __device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros
 
 // bf16 unit: copy the staged part of a token row to its K rows.
 template <int VB>
-__device__ __forceinline__ void copy_unit(const LbParams &p, const uint8_t *src, const int32_t *dsts, int part,
-                                          int gtid, uint64_t pol) {
+__device__ __forceinline__ void copy_unit(const LbParams &p, const PeerTab &tab, const uint8_t *src,
+                                          const int32_t *dsts, int part, int gtid, uint64_t pol) {
     const int row_bytes = 2 * p.H, chunk = p.chunk_bytes, nv = chunk / VB;
-    uint8_t *recv = static_cast<uint8_t *>(p.recv);
     for (int v = gtid; v < nv; v += kGroupThreads) {
         if constexpr (VB == 32) {
             const uint4 a = *reinterpret_cast<const uint4 *>(src + v * 32);
@@ -316,13 +366,13 @@ __device__ __forceinline__ void copy_unit(const LbParams &p, const uint8_t *src,
             val.v[4] = b.x; val.v[5] = b.y; val.v[6] = b.z; val.v[7] = b.w;
             for (int k = 0; k < p.K; ++k) {
                 const int dst = dsts[k];
-                if (dst >= 0) st_v8_policy(recv + (int64_t)dst * row_bytes + (int64_t)part * chunk + v * 32, val, pol);
+                if (dst >= 0) st_v8_policy(row_addr(p, tab, dst, row_bytes) + (int64_t)part * chunk + v * 32, val, pol);
             }
         } else {
             const uint4 val = *reinterpret_cast<const uint4 *>(src + v * 16);
             for (int k = 0; k < p.K; ++k) {
                 const int dst = dsts[k];
-                if (dst >= 0) st_v4_policy(recv + (int64_t)dst * row_bytes + (int64_t)part * chunk + v * 16, val, pol);
+                if (dst >= 0) st_v4_policy(row_addr(p, tab, dst, row_bytes) + (int64_t)part * chunk + v * 16, val, pol);
             }
         }
     }
@@ -331,8 +381,8 @@ __device__ __forceinline__ void copy_unit(const LbParams &p, const uint8_t *src,
 // FP8 unit: thread gtid quantises elements [gtid*32, gtid*32+32) of the
 // staged part (4 consecutive lanes per 1x128 block) and stores the 32 code
 // bytes to each of the K rows; the block's first lane stores its scale.
-__device__ __forceinline__ void quantise_unit(const LbParams &p, const uint8_t *src, const int32_t *dsts, int part,
-                                              int gtid, uint64_t pol) {
+__device__ __forceinline__ void quantise_unit(const LbParams &p, const PeerTab &tab, const uint8_t *src,
+                                              const int32_t *dsts, int part, int gtid, uint64_t pol) {
     constexpr int TPB = 128 / kFp8Ept, NW = kFp8Ept / 2;
     const int U = p.chunk_bytes / 2;           // elements per unit (a multiple of 128)
     const bool act = gtid * kFp8Ept < U;       // whole blocks of 4 lanes are active or idle
@@ -356,18 +406,17 @@ __device__ __forceinline__ void quantise_unit(const LbParams &p, const uint8_t *
     u32x8 v;
 #pragma unroll
     for (int i = 0; i < 8; ++i) v.v[i] = q[i];
-    uint8_t *recv = static_cast<uint8_t *>(p.recv);
     for (int k = 0; k < p.K; ++k) {
         const int dst = dsts[k];
         if (dst < 0) continue;
-        uint8_t *o = recv + (int64_t)dst * p.H + col;
+        uint8_t *o = row_addr(p, tab, dst, p.H) + col;
         if (p.vec32) {
             st_v8_policy(o, v, pol);
         } else {   // a 16-byte aligned buffer
             st_v4_policy(o, make_uint4(q[0], q[1], q[2], q[3]), pol);
             st_v4_policy(o + 16, make_uint4(q[4], q[5], q[6], q[7]), pol);
         }
-        if (lead) p.recv_scale[scale_at(p, dst, b, NB)] = scale;
+        if (lead) *scale_addr(p, tab, dst, b, NB) = scale;
     }
 }
 
@@ -376,7 +425,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     using S = Shape<G>;
     constexpr int NSET = S::kSetThreads;
     extern __shared__ __align__(128) uint8_t smem[];
-    const Carve cv = carve(p.stages, p.chunk_bytes, p.E);
+    const Carve cv = carve(p.stages, p.chunk_bytes, p.E, p.peer_base ? p.R : 0);
     uint8_t *ring = smem + cv.ring;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + cv.bars);
     uint64_t *empty = full + kMaxStages;
@@ -418,10 +467,36 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         // of that launch finished, and that launch completed before this one
         s_tag = (__ldcg(&p.ctl->epoch) % 0x7fffffffu) + 1u;
     }
+    // peer mode: the destination table, staged once (rank offsets come from the
+    // layout kernel before, so every thread waits for it first; the x prefetch
+    // is issued before that wait)
+    PeerTab tab{};
+    if (p.peer_base) {
+        if (tid == 0 && p.prefetch_x) {
+            const uint64_t pol_x = policy_evict_last();
+            for (int i = 0; i < n_cta; ++i) {
+                const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
+                bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
+            }
+        }
+        pdl_wait();
+        unsigned char *pm = smem + cv.peer;
+        tab.R = p.R;
+        tab.base = reinterpret_cast<uint8_t **>(pm);
+        tab.sbase = reinterpret_cast<float **>(pm + sizeof(void *) * p.R);
+        tab.row0 = reinterpret_cast<int32_t *>(pm + 2 * sizeof(void *) * p.R);
+        tab.roff = tab.row0 + p.R;
+        for (int i = tid; i < p.R; i += S::kThreads) {
+            tab.base[i] = p.peer_base[i];
+            tab.sbase[i] = p.peer_sbase ? p.peer_sbase[i] : nullptr;
+            tab.row0[i] = __ldcg(p.peer_row0 + i);
+        }
+        for (int i = tid; i <= p.R; i += S::kThreads) tab.roff[i] = __ldcg(p.roff + i);
+    }
     __syncthreads();
 
     if (warp == S::kPadWarp) {
-        pad_rows<FP8>(p, zeros, lane, n_cta, chunk);
+        pad_rows<FP8>(p, tab, zeros, lane, n_cta, chunk);
     } else {
         const uint64_t pol_out = policy_evict_first();
         const unsigned int tag = s_tag;
@@ -432,7 +507,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         // together all of x) goes into L2 now, overlapping the kernel before;
         // with lb = 1 the padding warp does that after the dependency wait,
         // where it cannot delay the latency-bound layout phases
-        if (tid == 0 && p.prefetch_x && !p.lb) {
+        if (tid == 0 && p.prefetch_x && !p.lb && !p.peer_base) {
             const uint64_t pol_x = policy_evict_last();
             for (int i = 0; i < n_cta; ++i) {
                 const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
@@ -657,9 +732,9 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
                     const int part = u % p.splits;
                     const int32_t *dsts = s_stpos + s * kStageDst + lead;
                     if constexpr (FP8)
-                        quantise_unit(p, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
+                        quantise_unit(p, tab, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
                     else
-                        copy_unit<VB>(p, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
+                        copy_unit<VB>(p, tab, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[s]);
                 }
@@ -794,23 +869,26 @@ cudaError_t launch_layout_counts(const LbParams &p, cudaStream_t s) {
 
 cudaError_t launch_dispatch_lb(const LbParams &p_in, bool fp8, int num_sms, cudaStream_t s) {
     LbParams p = p_in;
-    const bool v32 = !fp8 && p.H % 16 == 0 &&
+    // peer destinations are only known to be 16-byte aligned: 16-byte stores there
+    const bool v32 = !fp8 && !p.peer_base && p.H % 16 == 0 &&
                      ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
     const int VB = v32 ? 32 : 16;
-    p.vec32 = (reinterpret_cast<uintptr_t>(p.recv) & 31) == 0;
+    p.vec32 = !p.peer_base && (reinterpret_cast<uintptr_t>(p.recv) & 31) == 0;
+    if (p.peer_base && p.lb) return cudaErrorInvalidValue;   // peer mode takes a layout computed before
     if (reinterpret_cast<uintptr_t>(p.pos) & 15) return cudaErrorInvalidValue;   // the handle's: 256-byte aligned
     if (!lb_unit_shape(p.H, fp8, VB, &p.splits, &p.chunk_bytes)) return cudaErrorInvalidValue;
     if ((int64_t)p.T * p.splits >= (int64_t(1) << 28)) return cudaErrorInvalidValue;   // stage tags hold 28 bits
     p.dyn_batch = p.splits * (fp8 ? EP_LB_DYN_TOKENS_FP8 : EP_LB_DYN_TOKENS_BF16);
     if (p.dyn_batch < 1) return cudaErrorInvalidValue;
     const size_t limit = smem_limit();
-    const size_t fixed = carve(0, p.chunk_bytes, p.E).total;
+    const int pr = p.peer_base ? p.R : 0;
+    const size_t fixed = carve(0, p.chunk_bytes, p.E, pr).total;
     int ns = (int)(EP_LB_RING_BYTES / p.chunk_bytes);
-    while (ns > 0 && carve(ns, p.chunk_bytes, p.E).total > limit) --ns;
+    while (ns > 0 && carve(ns, p.chunk_bytes, p.E, pr).total > limit) --ns;
     ns = ns > kMaxStages ? kMaxStages : ns;
     if (ns < 2 || fixed > limit) return cudaErrorInvalidValue;
     p.stages = ns;
-    const size_t smem = carve(ns, p.chunk_bytes, p.E).total;
+    const size_t smem = carve(ns, p.chunk_bytes, p.E, pr).total;
     const int grid = p.nchunks < num_sms ? p.nchunks : num_sms;
     if (grid <= 0) return cudaSuccess;
     if (fp8)
