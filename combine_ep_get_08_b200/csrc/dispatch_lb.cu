@@ -65,6 +65,7 @@ constexpr int kMaxStages = 16;
 constexpr int kZeroBytes = 8192;        // zeroed shared memory the padding warp copies from
 constexpr int kFp8Ept = 32;             // FP8: bf16 elements per consumer thread
 constexpr int kStageDst = kMaxTopk + 4;  // int32 per stage for a token's destinations (+ alignment lead)
+constexpr int kMaxGroups = 2;            // consumer groups per CTA at most
 #ifndef EP_LB_DYN_TOKENS_BF16
 #define EP_LB_DYN_TOKENS_BF16 1     // tokens per claim of the dynamic copy, bf16 (dsv3: 1 -> 90.8 us,
 #endif                              // 2 -> 92.4 us, 4 -> 94.7 us)
@@ -83,7 +84,7 @@ __host__ __device__ __forceinline__ size_t up(size_t v, size_t a) { return (v + 
 
 // Dynamic shared memory carve-up (same on host and device).
 struct Carve {
-    size_t ring, bars, zeros, e16, rk16, cnt, base, agg, unit, stpos, peer, total;
+    size_t ring, bars, zeros, e16, rk16, cnt, base, agg, unit, stpos, peer, paddr, total;
 };
 __host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int E, int peer_ranks = 0) {
     Carve c;
@@ -102,6 +103,8 @@ __host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int
     c.stpos = o; o += (size_t)kMaxStages * kStageDst * sizeof(int32_t);
     o = up(o, 128);
     c.peer = o;  o += peer_ranks ? 2 * sizeof(void *) * peer_ranks + sizeof(int32_t) * (2 * (size_t)peer_ranks + 1) : 0;
+    o = up(o, 128);
+    c.paddr = o; o += peer_ranks ? (size_t)kMaxGroups * 2 * kMaxTopk * 2 * sizeof(void *) : 0;
     c.total = up(o, 128);
     return c;
 }
@@ -352,10 +355,23 @@ __device__ __forceinline__ void pad_rows(const LbParams &p, const PeerTab &tab, 
     bulk_wait_all();
 }
 
+// A unit's K destination rows: local rows by index, or (peer mode) addresses
+// the consumer group computed once for the unit (null: no row).
+struct UnitDst {
+    const int32_t *rows;          // local: received row indices (-1: none)
+    uint8_t *const *addr;         // peer: row addresses
+    float *const *saddr;          // peer FP8: scale row addresses
+    __device__ __forceinline__ uint8_t *row(const LbParams &p, int k, int row_bytes) const {
+        if (addr) return addr[k];
+        const int d = rows[k];
+        return d >= 0 ? static_cast<uint8_t *>(p.recv) + (int64_t)d * row_bytes : nullptr;
+    }
+};
+
 // bf16 unit: copy the staged part of a token row to its K rows.
 template <int VB>
-__device__ __forceinline__ void copy_unit(const LbParams &p, const PeerTab &tab, const uint8_t *src,
-                                          const int32_t *dsts, int part, int gtid, uint64_t pol) {
+__device__ __forceinline__ void copy_unit(const LbParams &p, const UnitDst &ud, const uint8_t *src, int part,
+                                          int gtid, uint64_t pol) {
     const int row_bytes = 2 * p.H, chunk = p.chunk_bytes, nv = chunk / VB;
     for (int v = gtid; v < nv; v += kGroupThreads) {
         if constexpr (VB == 32) {
@@ -365,14 +381,14 @@ __device__ __forceinline__ void copy_unit(const LbParams &p, const PeerTab &tab,
             val.v[0] = a.x; val.v[1] = a.y; val.v[2] = a.z; val.v[3] = a.w;
             val.v[4] = b.x; val.v[5] = b.y; val.v[6] = b.z; val.v[7] = b.w;
             for (int k = 0; k < p.K; ++k) {
-                const int dst = dsts[k];
-                if (dst >= 0) st_v8_policy(row_addr(p, tab, dst, row_bytes) + (int64_t)part * chunk + v * 32, val, pol);
+                uint8_t *o = ud.row(p, k, row_bytes);
+                if (o) st_v8_policy(o + (int64_t)part * chunk + v * 32, val, pol);
             }
         } else {
             const uint4 val = *reinterpret_cast<const uint4 *>(src + v * 16);
             for (int k = 0; k < p.K; ++k) {
-                const int dst = dsts[k];
-                if (dst >= 0) st_v4_policy(row_addr(p, tab, dst, row_bytes) + (int64_t)part * chunk + v * 16, val, pol);
+                uint8_t *o = ud.row(p, k, row_bytes);
+                if (o) st_v4_policy(o + (int64_t)part * chunk + v * 16, val, pol);
             }
         }
     }
@@ -381,8 +397,8 @@ __device__ __forceinline__ void copy_unit(const LbParams &p, const PeerTab &tab,
 // FP8 unit: thread gtid quantises elements [gtid*32, gtid*32+32) of the
 // staged part (4 consecutive lanes per 1x128 block) and stores the 32 code
 // bytes to each of the K rows; the block's first lane stores its scale.
-__device__ __forceinline__ void quantise_unit(const LbParams &p, const PeerTab &tab, const uint8_t *src,
-                                              const int32_t *dsts, int part, int gtid, uint64_t pol) {
+__device__ __forceinline__ void quantise_unit(const LbParams &p, const UnitDst &ud, const uint8_t *src, int part,
+                                              int gtid, uint64_t pol) {
     constexpr int TPB = 128 / kFp8Ept, NW = kFp8Ept / 2;
     const int U = p.chunk_bytes / 2;           // elements per unit (a multiple of 128)
     const bool act = gtid * kFp8Ept < U;       // whole blocks of 4 lanes are active or idle
@@ -407,21 +423,27 @@ __device__ __forceinline__ void quantise_unit(const LbParams &p, const PeerTab &
 #pragma unroll
     for (int i = 0; i < 8; ++i) v.v[i] = q[i];
     for (int k = 0; k < p.K; ++k) {
-        const int dst = dsts[k];
-        if (dst < 0) continue;
-        uint8_t *o = row_addr(p, tab, dst, p.H) + col;
+        uint8_t *o = ud.row(p, k, p.H);
+        if (!o) continue;
+        o += col;
         if (p.vec32) {
             st_v8_policy(o, v, pol);
         } else {   // a 16-byte aligned buffer
             st_v4_policy(o, make_uint4(q[0], q[1], q[2], q[3]), pol);
             st_v4_policy(o + 16, make_uint4(q[4], q[5], q[6], q[7]), pol);
         }
-        if (lead) *scale_addr(p, tab, dst, b, NB) = scale;
+        if (lead) {
+            if (ud.addr)
+                ud.saddr[k][b] = scale;
+            else
+                p.recv_scale[scale_at(p, ud.rows[k], b, NB)] = scale;
+        }
     }
 }
 
 template <int VB, bool FP8, int G>
 __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbParams p) {
+    static_assert(G <= kMaxGroups, "consumer groups");
     using S = Shape<G>;
     constexpr int NSET = S::kSetThreads;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -437,6 +459,8 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     int32_t *s_agg = reinterpret_cast<int32_t *>(smem + cv.agg);
     int32_t *s_unit = reinterpret_cast<int32_t *>(smem + cv.unit);     // [stages] row part | lead << 28 (-1: end)
     int32_t *s_stpos = reinterpret_cast<int32_t *>(smem + cv.stpos);   // [stages][kStageDst] its destinations
+    uint8_t **s_paddr = reinterpret_cast<uint8_t **>(smem + cv.paddr);  // peer: [group][2][K] row addresses
+    float **s_psaddr = reinterpret_cast<float **>(smem + cv.paddr) + kMaxGroups * 2 * kMaxTopk;   // and scale rows
     __shared__ int s_ticket;
     __shared__ int s_abort;
     __shared__ unsigned int s_tag;
@@ -721,20 +745,56 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
                 const int grp = (tid - 32) / kGroupThreads, gtid = (tid - 32) - grp * kGroupThreads;
                 for (int g = grp;; g += G) {
                     const int s = g % NS;
-                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (g / NS) & 1, p.wait_limit_ns))) {
-                        if (lane == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                        *abort_flag = 1;
-                        break;
+                    const bool got = mbar_wait_bounded(&full[s], (g / NS) & 1, p.wait_limit_ns);
+                    UnitDst ud{nullptr, nullptr, nullptr};
+                    int su = -1;
+                    if (tab.base) {
+                        // peer mode: the K destination addresses, once per unit, into this
+                        // group's slot (two slots in turn: a thread writes the next unit's
+                        // only after the whole group passed this unit's barrier).  The
+                        // group decides together whether the stage arrived: every thread
+                        // reaches the barrier, whatever its own wait gave.
+                        const int slot = (grp * 2 + ((g / G) & 1)) * kMaxTopk;
+                        if (got) {
+                            su = s_unit[s];
+                            if (su >= 0 && gtid < K) {
+                                const int d = s_stpos[s * kStageDst + (su >> 28) + gtid];
+                                s_paddr[slot + gtid] = d >= 0 ? row_addr(p, tab, d, FP8 ? p.H : 2 * p.H) : nullptr;
+                                if (FP8) s_psaddr[slot + gtid] = d >= 0 ? scale_addr(p, tab, d, 0, p.H / 128) : nullptr;
+                            }
+                        }
+                        int all_got;
+                        asm volatile(
+                            "{\n\t.reg .pred pi, po;\n\t"
+                            "setp.ne.u32 pi, %1, 0;\n\t"
+                            "bar.red.and.pred po, %2, %3, pi;\n\t"
+                            "selp.u32 %0, 1, 0, po;\n\t}"
+                            : "=r"(all_got)
+                            : "r"((unsigned)got), "r"(2 + grp), "r"(kGroupThreads)
+                            : "memory");
+                        if (!all_got) {
+                            if (gtid == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                            *abort_flag = 1;
+                            break;
+                        }
+                        ud.addr = s_paddr + slot;
+                        ud.saddr = s_psaddr + slot;
+                    } else {
+                        if (!__all_sync(0xffffffffu, got)) {
+                            if (lane == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                            *abort_flag = 1;
+                            break;
+                        }
+                        su = s_unit[s];
                     }
-                    const int su = s_unit[s];
                     if (su < 0) break;
                     const int u = su & 0x0fffffff, lead = su >> 28;
                     const int part = u % p.splits;
-                    const int32_t *dsts = s_stpos + s * kStageDst + lead;
+                    ud.rows = s_stpos + s * kStageDst + lead;
                     if constexpr (FP8)
-                        quantise_unit(p, tab, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
+                        quantise_unit(p, ud, ring + (size_t)s * chunk, part, gtid, pol_out);
                     else
-                        copy_unit<VB>(p, tab, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
+                        copy_unit<VB>(p, ud, ring + (size_t)s * chunk, part, gtid, pol_out);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[s]);
                 }
