@@ -319,19 +319,7 @@ __device__ __forceinline__ void pad_rows(const LbParams &p, const PeerTab &tab, 
     const bool bulk_scales = FP8 && p.scale_ld == 0 && (NB * 4) % 16 == 0 &&
                              (reinterpret_cast<uintptr_t>(p.recv_scale) & 15) == 0;
     uint8_t *recv = static_cast<uint8_t *>(p.recv);
-    if (tab.base) {
-        // peer mode: plain 16-byte stores only, the warp's lanes across each row
-        for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
-            const int r0 = __ldcg(p.eoff + e) + __ldcg(p.cnt + e), r1 = __ldcg(p.eoff + e + 1);
-            for (int r = r0; r < r1; ++r) {
-                uint8_t *o = row_addr(p, tab, r, row_bytes);
-                for (int off = lane * 16; off < row_bytes; off += 32 * 16) st_v4(o + off, make_uint4(0, 0, 0, 0));
-                if (FP8)
-                    for (int b = lane; b < NB; b += 32) *scale_addr(p, tab, r, b, NB) = 0.0f;
-            }
-        }
-        return;
-    }
+    if (tab.base) return;   // peer mode: the consumer groups write the padding rows after their copy
     for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
         const int r0 = __ldcg(p.eoff + e) + __ldcg(p.cnt + e), r1 = __ldcg(p.eoff + e + 1);
         for (int r = r0 + lane; r < r1; r += 32) {
@@ -461,6 +449,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     int32_t *s_stpos = reinterpret_cast<int32_t *>(smem + cv.stpos);   // [stages][kStageDst] its destinations
     uint8_t **s_paddr = reinterpret_cast<uint8_t **>(smem + cv.paddr);  // peer: [group][2][K] row addresses
     float **s_psaddr = reinterpret_cast<float **>(smem + cv.paddr) + kMaxGroups * 2 * kMaxTopk;   // and scale rows
+    __shared__ int s_pclaim[kMaxGroups * 2];   // peer mode: each group's expert claim (two slots in turn)
     __shared__ int s_ticket;
     __shared__ int s_abort;
     __shared__ unsigned int s_tag;
@@ -798,6 +787,27 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[s]);
                 }
+                // peer mode: padding rows (plain 16-byte stores into the peers), one
+                // expert per claim, the group's threads across each row
+                if (tab.base && p.A > 1) {
+                    const int row_bytes_q = FP8 ? p.H : 2 * p.H, NB = p.H / 128;
+                    for (int it = 0;; ++it) {
+                        // one thread claims (or, after an abort anywhere in the CTA, ends
+                        // the loop for the whole group); two slots in turn, as the addresses
+                        int *cl = s_pclaim + grp * 2 + (it & 1);
+                        if (gtid == 0) *cl = *abort_flag ? p.E : (int)atomicAdd(&p.ctl->pads, 1u);
+                        asm volatile("bar.sync %0, %1;" : : "r"(2 + grp), "r"(kGroupThreads) : "memory");
+                        const int e = *cl;
+                        if (e >= p.E) break;
+                        const int r0 = __ldcg(p.eoff + e) + __ldcg(p.cnt + e), r1 = __ldcg(p.eoff + e + 1);
+                        for (int r = r0; r < r1; ++r) {
+                            uint8_t *o = row_addr(p, tab, r, row_bytes_q);
+                            for (int off = gtid * 16; off < row_bytes_q; off += kGroupThreads * 16)
+                                st_v4(o + off, make_uint4(0, 0, 0, 0));
+                            if (FP8 && gtid < NB) *scale_addr(p, tab, r, gtid, NB) = 0.0f;
+                        }
+                    }
+                }
             }
         }
 
@@ -816,6 +826,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
             __threadfence();
             atomicExch(&p.ctl->ticket, 0u);
             atomicExch(&p.ctl->units, 0u);
+            atomicExch(&p.ctl->pads, 0u);
             atomicExch(&p.ctl->done, 0u);
             atomicExch(&p.ctl->epoch, s_tag);
         }
