@@ -160,6 +160,7 @@ struct PeerTab {
     int32_t *row0;     // [R]
     int32_t *roff;     // [R+1]
     int R;
+    bool v32;          // every base is 32-byte aligned: 32-byte stores
 };
 __device__ __forceinline__ int peer_rank(const PeerTab &t, int row) {
     int lo = 0, hi = t.R - 1;
@@ -349,6 +350,7 @@ struct UnitDst {
     const int32_t *rows;          // local: received row indices (-1: none)
     uint8_t *const *addr;         // peer: row addresses
     float *const *saddr;          // peer FP8: scale row addresses
+    bool v16;                     // peer buffers only 16-byte aligned: 32-byte vectors as two 16-byte stores
     __device__ __forceinline__ uint8_t *row(const LbParams &p, int k, int row_bytes) const {
         if (addr) return addr[k];
         const int d = rows[k];
@@ -370,7 +372,14 @@ __device__ __forceinline__ void copy_unit(const LbParams &p, const UnitDst &ud, 
             val.v[4] = b.x; val.v[5] = b.y; val.v[6] = b.z; val.v[7] = b.w;
             for (int k = 0; k < p.K; ++k) {
                 uint8_t *o = ud.row(p, k, row_bytes);
-                if (o) st_v8_policy(o + (int64_t)part * chunk + v * 32, val, pol);
+                if (!o) continue;
+                o += (int64_t)part * chunk + v * 32;
+                if (ud.v16) {
+                    st_v4_policy(o, a, pol);
+                    st_v4_policy(o + 16, b, pol);
+                } else {
+                    st_v8_policy(o, val, pol);
+                }
             }
         } else {
             const uint4 val = *reinterpret_cast<const uint4 *>(src + v * 16);
@@ -414,7 +423,7 @@ __device__ __forceinline__ void quantise_unit(const LbParams &p, const UnitDst &
         uint8_t *o = ud.row(p, k, p.H);
         if (!o) continue;
         o += col;
-        if (p.vec32) {
+        if (p.vec32 && !ud.v16) {
             st_v8_policy(o, v, pol);
         } else {   // a 16-byte aligned buffer
             st_v4_policy(o, make_uint4(q[0], q[1], q[2], q[3]), pol);
@@ -506,7 +515,11 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         }
         for (int i = tid; i <= p.R; i += S::kThreads) tab.roff[i] = __ldcg(p.roff + i);
     }
-    __syncthreads();
+    // peer mode: 32-byte stores only if every destination base allows them
+    int misaligned = 0;
+    if (p.peer_base)
+        for (int i = tid; i < p.R; i += S::kThreads) misaligned |= (reinterpret_cast<uintptr_t>(p.peer_base[i]) & 31) != 0;
+    tab.v32 = !__syncthreads_or(misaligned);
 
     if (warp == S::kPadWarp) {
         pad_rows<FP8>(p, tab, zeros, lane, n_cta, chunk);
@@ -735,7 +748,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
                 for (int g = grp;; g += G) {
                     const int s = g % NS;
                     const bool got = mbar_wait_bounded(&full[s], (g / NS) & 1, p.wait_limit_ns);
-                    UnitDst ud{nullptr, nullptr, nullptr};
+                    UnitDst ud{nullptr, nullptr, nullptr, tab.base && !tab.v32};
                     int su = -1;
                     if (tab.base) {
                         // peer mode: the K destination addresses, once per unit, into this
@@ -941,10 +954,11 @@ cudaError_t launch_layout_counts(const LbParams &p, cudaStream_t s) {
 cudaError_t launch_dispatch_lb(const LbParams &p_in, bool fp8, int num_sms, cudaStream_t s) {
     LbParams p = p_in;
     // peer destinations are only known to be 16-byte aligned: 16-byte stores there
-    const bool v32 = !fp8 && !p.peer_base && p.H % 16 == 0 &&
-                     ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
+    // peer destinations: the kernel checks their bases and falls back to 16-byte stores
+    const uintptr_t dst_bits = p.peer_base ? 0 : reinterpret_cast<uintptr_t>(p.recv);
+    const bool v32 = !fp8 && p.H % 16 == 0 && ((reinterpret_cast<uintptr_t>(p.x) | dst_bits) & 31) == 0;
     const int VB = v32 ? 32 : 16;
-    p.vec32 = !p.peer_base && (reinterpret_cast<uintptr_t>(p.recv) & 31) == 0;
+    p.vec32 = (dst_bits & 31) == 0;
     if (p.peer_base && p.lb) return cudaErrorInvalidValue;   // peer mode takes a layout computed before
     if (reinterpret_cast<uintptr_t>(p.pos) & 15) return cudaErrorInvalidValue;   // the handle's: 256-byte aligned
     if (!lb_unit_shape(p.H, fp8, VB, &p.splits, &p.chunk_bytes)) return cudaErrorInvalidValue;
