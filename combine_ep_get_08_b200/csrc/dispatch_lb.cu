@@ -65,7 +65,6 @@ constexpr int kMaxStages = 16;
 constexpr int kZeroBytes = 8192;        // zeroed shared memory the padding warp copies from
 constexpr int kFp8Ept = 32;             // FP8: bf16 elements per consumer thread
 constexpr int kStageDst = kMaxTopk + 4;  // int32 per stage for a token's destinations (+ alignment lead)
-constexpr int kMaxGroups = 2;            // consumer groups per CTA at most
 #ifndef EP_LB_DYN_TOKENS_BF16
 #define EP_LB_DYN_TOKENS_BF16 1     // tokens per claim of the dynamic copy, bf16 (dsv3: 1 -> 90.8 us,
 #endif                              // 2 -> 92.4 us, 4 -> 94.7 us)
@@ -84,9 +83,9 @@ __host__ __device__ __forceinline__ size_t up(size_t v, size_t a) { return (v + 
 
 // Dynamic shared memory carve-up (same on host and device).
 struct Carve {
-    size_t ring, bars, zeros, e16, rk16, cnt, base, agg, unit, stpos, peer, paddr, total;
+    size_t ring, bars, zeros, e16, rk16, cnt, base, agg, unit, stpos, total;
 };
-__host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int E, int peer_ranks = 0) {
+__host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int E) {
     Carve c;
     size_t o = 0;
     c.ring = o;  o += up((size_t)stages * chunk_bytes, 128);
@@ -101,10 +100,6 @@ __host__ __device__ __forceinline__ Carve carve(int stages, int chunk_bytes, int
     c.unit = o;  o += (size_t)kMaxStages * sizeof(int32_t);
     o = up(o, 128);                      // bulk-copy destinations: 16-byte aligned
     c.stpos = o; o += (size_t)kMaxStages * kStageDst * sizeof(int32_t);
-    o = up(o, 128);
-    c.peer = o;  o += peer_ranks ? 2 * sizeof(void *) * peer_ranks + sizeof(int32_t) * (2 * (size_t)peer_ranks + 1) : 0;
-    o = up(o, 128);
-    c.paddr = o; o += peer_ranks ? (size_t)kMaxGroups * 2 * kMaxTopk * 2 * sizeof(void *) : 0;
     c.total = up(o, 128);
     return c;
 }
@@ -148,42 +143,6 @@ __device__ __forceinline__ bool valid_id(int64_t e, int E) { return e >= 0 && e 
 
 __device__ __forceinline__ int64_t scale_at(const LbParams &p, int row, int b, int NB) {
     return p.scale_ld == 0 ? (int64_t)row * NB + b : (int64_t)b * p.scale_ld + row;
-}
-
-// Peer mode: where received row `row` of this rank lives -- rank r = the last
-// one with roff[r] <= row (empty segments share their start with the next),
-// row row0[r] + row - roff[r] of r's buffer.  The table is staged in shared
-// memory once per CTA.
-struct PeerTab {
-    uint8_t **base;    // [R] (null: not peer mode)
-    float **sbase;     // [R]
-    int32_t *row0;     // [R]
-    int32_t *roff;     // [R+1]
-    int R;
-    bool v32;          // every base is 32-byte aligned: 32-byte stores
-};
-__device__ __forceinline__ int peer_rank(const PeerTab &t, int row) {
-    int lo = 0, hi = t.R - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (t.roff[mid] <= row)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    return lo;
-}
-// Received row `row` (row_bytes each) of the local buffer, or of its destination rank's.
-__device__ __forceinline__ uint8_t *row_addr(const LbParams &p, const PeerTab &t, int row, int row_bytes) {
-    if (!t.base) return static_cast<uint8_t *>(p.recv) + (int64_t)row * row_bytes;
-    const int r = peer_rank(t, row);
-    return t.base[r] + (int64_t)(t.row0[r] + row - t.roff[r]) * row_bytes;
-}
-// Scale (row, b) of an FP8 row, local or at its destination rank (row-major there).
-__device__ __forceinline__ float *scale_addr(const LbParams &p, const PeerTab &t, int row, int b, int NB) {
-    if (!t.base) return p.recv_scale + scale_at(p, row, b, NB);
-    const int r = peer_rank(t, row);
-    return t.sbase[r] + (int64_t)(t.row0[r] + row - t.roff[r]) * NB + b;
 }
 
 // ---------------------------------------------------------------------------
@@ -303,8 +262,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_counts_kernel(LbPara
 // dependency wait, so it does not delay the latency-bound layout work).
 // ---------------------------------------------------------------------------
 template <bool FP8>
-__device__ __forceinline__ void pad_rows(const LbParams &p, const PeerTab &tab, const uint8_t *zeros, int lane,
-                                         int n_cta, int chunk) {
+__device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros, int lane, int n_cta, int chunk) {
     pdl_wait();   // offsets and counts come from the kernel before
     if (p.lb && p.prefetch_x && lane == 0) {
         const uint64_t pol_x = policy_evict_last();
@@ -320,7 +278,6 @@ __device__ __forceinline__ void pad_rows(const LbParams &p, const PeerTab &tab, 
     const bool bulk_scales = FP8 && p.scale_ld == 0 && (NB * 4) % 16 == 0 &&
                              (reinterpret_cast<uintptr_t>(p.recv_scale) & 15) == 0;
     uint8_t *recv = static_cast<uint8_t *>(p.recv);
-    if (tab.base) return;   // peer mode: the consumer groups write the padding rows after their copy
     for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
         const int r0 = __ldcg(p.eoff + e) + __ldcg(p.cnt + e), r1 = __ldcg(p.eoff + e + 1);
         for (int r = r0 + lane; r < r1; r += 32) {
@@ -344,25 +301,12 @@ __device__ __forceinline__ void pad_rows(const LbParams &p, const PeerTab &tab, 
     bulk_wait_all();
 }
 
-// A unit's K destination rows: local rows by index, or (peer mode) addresses
-// the consumer group computed once for the unit (null: no row).
-struct UnitDst {
-    const int32_t *rows;          // local: received row indices (-1: none)
-    uint8_t *const *addr;         // peer: row addresses
-    float *const *saddr;          // peer FP8: scale row addresses
-    bool v16;                     // peer buffers only 16-byte aligned: 32-byte vectors as two 16-byte stores
-    __device__ __forceinline__ uint8_t *row(const LbParams &p, int k, int row_bytes) const {
-        if (addr) return addr[k];
-        const int d = rows[k];
-        return d >= 0 ? static_cast<uint8_t *>(p.recv) + (int64_t)d * row_bytes : nullptr;
-    }
-};
-
 // bf16 unit: copy the staged part of a token row to its K rows.
 template <int VB>
-__device__ __forceinline__ void copy_unit(const LbParams &p, const UnitDst &ud, const uint8_t *src, int part,
+__device__ __forceinline__ void copy_unit(const LbParams &p, const uint8_t *src, const int32_t *dsts, int part,
                                           int gtid, uint64_t pol) {
     const int row_bytes = 2 * p.H, chunk = p.chunk_bytes, nv = chunk / VB;
+    uint8_t *recv = static_cast<uint8_t *>(p.recv);
     for (int v = gtid; v < nv; v += kGroupThreads) {
         if constexpr (VB == 32) {
             const uint4 a = *reinterpret_cast<const uint4 *>(src + v * 32);
@@ -371,21 +315,14 @@ __device__ __forceinline__ void copy_unit(const LbParams &p, const UnitDst &ud, 
             val.v[0] = a.x; val.v[1] = a.y; val.v[2] = a.z; val.v[3] = a.w;
             val.v[4] = b.x; val.v[5] = b.y; val.v[6] = b.z; val.v[7] = b.w;
             for (int k = 0; k < p.K; ++k) {
-                uint8_t *o = ud.row(p, k, row_bytes);
-                if (!o) continue;
-                o += (int64_t)part * chunk + v * 32;
-                if (ud.v16) {
-                    st_v4_policy(o, a, pol);
-                    st_v4_policy(o + 16, b, pol);
-                } else {
-                    st_v8_policy(o, val, pol);
-                }
+                const int dst = dsts[k];
+                if (dst >= 0) st_v8_policy(recv + (int64_t)dst * row_bytes + (int64_t)part * chunk + v * 32, val, pol);
             }
         } else {
             const uint4 val = *reinterpret_cast<const uint4 *>(src + v * 16);
             for (int k = 0; k < p.K; ++k) {
-                uint8_t *o = ud.row(p, k, row_bytes);
-                if (o) st_v4_policy(o + (int64_t)part * chunk + v * 16, val, pol);
+                const int dst = dsts[k];
+                if (dst >= 0) st_v4_policy(recv + (int64_t)dst * row_bytes + (int64_t)part * chunk + v * 16, val, pol);
             }
         }
     }
@@ -394,7 +331,7 @@ __device__ __forceinline__ void copy_unit(const LbParams &p, const UnitDst &ud, 
 // FP8 unit: thread gtid quantises elements [gtid*32, gtid*32+32) of the
 // staged part (4 consecutive lanes per 1x128 block) and stores the 32 code
 // bytes to each of the K rows; the block's first lane stores its scale.
-__device__ __forceinline__ void quantise_unit(const LbParams &p, const UnitDst &ud, const uint8_t *src, int part,
+__device__ __forceinline__ void quantise_unit(const LbParams &p, const uint8_t *src, const int32_t *dsts, int part,
                                               int gtid, uint64_t pol) {
     constexpr int TPB = 128 / kFp8Ept, NW = kFp8Ept / 2;
     const int U = p.chunk_bytes / 2;           // elements per unit (a multiple of 128)
@@ -419,32 +356,27 @@ __device__ __forceinline__ void quantise_unit(const LbParams &p, const UnitDst &
     u32x8 v;
 #pragma unroll
     for (int i = 0; i < 8; ++i) v.v[i] = q[i];
+    uint8_t *recv = static_cast<uint8_t *>(p.recv);
     for (int k = 0; k < p.K; ++k) {
-        uint8_t *o = ud.row(p, k, p.H);
-        if (!o) continue;
-        o += col;
-        if (p.vec32 && !ud.v16) {
+        const int dst = dsts[k];
+        if (dst < 0) continue;
+        uint8_t *o = recv + (int64_t)dst * p.H + col;
+        if (p.vec32) {
             st_v8_policy(o, v, pol);
         } else {   // a 16-byte aligned buffer
             st_v4_policy(o, make_uint4(q[0], q[1], q[2], q[3]), pol);
             st_v4_policy(o + 16, make_uint4(q[4], q[5], q[6], q[7]), pol);
         }
-        if (lead) {
-            if (ud.addr)
-                ud.saddr[k][b] = scale;
-            else
-                p.recv_scale[scale_at(p, ud.rows[k], b, NB)] = scale;
-        }
+        if (lead) p.recv_scale[scale_at(p, dst, b, NB)] = scale;
     }
 }
 
 template <int VB, bool FP8, int G>
 __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbParams p) {
-    static_assert(G <= kMaxGroups, "consumer groups");
     using S = Shape<G>;
     constexpr int NSET = S::kSetThreads;
     extern __shared__ __align__(128) uint8_t smem[];
-    const Carve cv = carve(p.stages, p.chunk_bytes, p.E, p.peer_base ? p.R : 0);
+    const Carve cv = carve(p.stages, p.chunk_bytes, p.E);
     uint8_t *ring = smem + cv.ring;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + cv.bars);
     uint64_t *empty = full + kMaxStages;
@@ -456,9 +388,6 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     int32_t *s_agg = reinterpret_cast<int32_t *>(smem + cv.agg);
     int32_t *s_unit = reinterpret_cast<int32_t *>(smem + cv.unit);     // [stages] row part | lead << 28 (-1: end)
     int32_t *s_stpos = reinterpret_cast<int32_t *>(smem + cv.stpos);   // [stages][kStageDst] its destinations
-    uint8_t **s_paddr = reinterpret_cast<uint8_t **>(smem + cv.paddr);  // peer: [group][2][K] row addresses
-    float **s_psaddr = reinterpret_cast<float **>(smem + cv.paddr) + kMaxGroups * 2 * kMaxTopk;   // and scale rows
-    __shared__ int s_pclaim[kMaxGroups * 2];   // peer mode: each group's expert claim (two slots in turn)
     __shared__ int s_ticket;
     __shared__ int s_abort;
     __shared__ unsigned int s_tag;
@@ -489,40 +418,10 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         // of that launch finished, and that launch completed before this one
         s_tag = (__ldcg(&p.ctl->epoch) % 0x7fffffffu) + 1u;
     }
-    // peer mode: the destination table, staged once (rank offsets come from the
-    // layout kernel before, so every thread waits for it first; the x prefetch
-    // is issued before that wait)
-    PeerTab tab{};
-    if (p.peer_base) {
-        if (tid == 0 && p.prefetch_x) {
-            const uint64_t pol_x = policy_evict_last();
-            for (int i = 0; i < n_cta; ++i) {
-                const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
-                bulk_prefetch_l2(x + (int64_t)t * row_bytes + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
-            }
-        }
-        pdl_wait();
-        unsigned char *pm = smem + cv.peer;
-        tab.R = p.R;
-        tab.base = reinterpret_cast<uint8_t **>(pm);
-        tab.sbase = reinterpret_cast<float **>(pm + sizeof(void *) * p.R);
-        tab.row0 = reinterpret_cast<int32_t *>(pm + 2 * sizeof(void *) * p.R);
-        tab.roff = tab.row0 + p.R;
-        for (int i = tid; i < p.R; i += S::kThreads) {
-            tab.base[i] = p.peer_base[i];
-            tab.sbase[i] = p.peer_sbase ? p.peer_sbase[i] : nullptr;
-            tab.row0[i] = __ldcg(p.peer_row0 + i);
-        }
-        for (int i = tid; i <= p.R; i += S::kThreads) tab.roff[i] = __ldcg(p.roff + i);
-    }
-    // peer mode: 32-byte stores only if every destination base allows them
-    int misaligned = 0;
-    if (p.peer_base)
-        for (int i = tid; i < p.R; i += S::kThreads) misaligned |= (reinterpret_cast<uintptr_t>(p.peer_base[i]) & 31) != 0;
-    tab.v32 = !__syncthreads_or(misaligned);
+    __syncthreads();
 
     if (warp == S::kPadWarp) {
-        pad_rows<FP8>(p, tab, zeros, lane, n_cta, chunk);
+        pad_rows<FP8>(p, zeros, lane, n_cta, chunk);
     } else {
         const uint64_t pol_out = policy_evict_first();
         const unsigned int tag = s_tag;
@@ -533,7 +432,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         // together all of x) goes into L2 now, overlapping the kernel before;
         // with lb = 1 the padding warp does that after the dependency wait,
         // where it cannot delay the latency-bound layout phases
-        if (tid == 0 && p.prefetch_x && !p.lb && !p.peer_base) {
+        if (tid == 0 && p.prefetch_x && !p.lb) {
             const uint64_t pol_x = policy_evict_last();
             for (int i = 0; i < n_cta; ++i) {
                 const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
@@ -747,79 +646,22 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
                 const int grp = (tid - 32) / kGroupThreads, gtid = (tid - 32) - grp * kGroupThreads;
                 for (int g = grp;; g += G) {
                     const int s = g % NS;
-                    const bool got = mbar_wait_bounded(&full[s], (g / NS) & 1, p.wait_limit_ns);
-                    UnitDst ud{nullptr, nullptr, nullptr, tab.base && !tab.v32};
-                    int su = -1;
-                    if (tab.base) {
-                        // peer mode: the K destination addresses, once per unit, into this
-                        // group's slot (two slots in turn: a thread writes the next unit's
-                        // only after the whole group passed this unit's barrier).  The
-                        // group decides together whether the stage arrived: every thread
-                        // reaches the barrier, whatever its own wait gave.
-                        const int slot = (grp * 2 + ((g / G) & 1)) * kMaxTopk;
-                        if (got) {
-                            su = s_unit[s];
-                            if (su >= 0 && gtid < K) {
-                                const int d = s_stpos[s * kStageDst + (su >> 28) + gtid];
-                                s_paddr[slot + gtid] = d >= 0 ? row_addr(p, tab, d, FP8 ? p.H : 2 * p.H) : nullptr;
-                                if (FP8) s_psaddr[slot + gtid] = d >= 0 ? scale_addr(p, tab, d, 0, p.H / 128) : nullptr;
-                            }
-                        }
-                        int all_got;
-                        asm volatile(
-                            "{\n\t.reg .pred pi, po;\n\t"
-                            "setp.ne.u32 pi, %1, 0;\n\t"
-                            "bar.red.and.pred po, %2, %3, pi;\n\t"
-                            "selp.u32 %0, 1, 0, po;\n\t}"
-                            : "=r"(all_got)
-                            : "r"((unsigned)got), "r"(2 + grp), "r"(kGroupThreads)
-                            : "memory");
-                        if (!all_got) {
-                            if (gtid == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                            *abort_flag = 1;
-                            break;
-                        }
-                        ud.addr = s_paddr + slot;
-                        ud.saddr = s_psaddr + slot;
-                    } else {
-                        if (!__all_sync(0xffffffffu, got)) {
-                            if (lane == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                            *abort_flag = 1;
-                            break;
-                        }
-                        su = s_unit[s];
+                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (g / NS) & 1, p.wait_limit_ns))) {
+                        if (lane == 0) atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *abort_flag = 1;
+                        break;
                     }
+                    const int su = s_unit[s];
                     if (su < 0) break;
                     const int u = su & 0x0fffffff, lead = su >> 28;
                     const int part = u % p.splits;
-                    ud.rows = s_stpos + s * kStageDst + lead;
+                    const int32_t *dsts = s_stpos + s * kStageDst + lead;
                     if constexpr (FP8)
-                        quantise_unit(p, ud, ring + (size_t)s * chunk, part, gtid, pol_out);
+                        quantise_unit(p, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
                     else
-                        copy_unit<VB>(p, ud, ring + (size_t)s * chunk, part, gtid, pol_out);
+                        copy_unit<VB>(p, ring + (size_t)s * chunk, dsts, part, gtid, pol_out);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[s]);
-                }
-                // peer mode: padding rows (plain 16-byte stores into the peers), one
-                // expert per claim, the group's threads across each row
-                if (tab.base && p.A > 1) {
-                    const int row_bytes_q = FP8 ? p.H : 2 * p.H, NB = p.H / 128;
-                    for (int it = 0;; ++it) {
-                        // one thread claims (or, after an abort anywhere in the CTA, ends
-                        // the loop for the whole group); two slots in turn, as the addresses
-                        int *cl = s_pclaim + grp * 2 + (it & 1);
-                        if (gtid == 0) *cl = *abort_flag ? p.E : (int)atomicAdd(&p.ctl->pads, 1u);
-                        asm volatile("bar.sync %0, %1;" : : "r"(2 + grp), "r"(kGroupThreads) : "memory");
-                        const int e = *cl;
-                        if (e >= p.E) break;
-                        const int r0 = __ldcg(p.eoff + e) + __ldcg(p.cnt + e), r1 = __ldcg(p.eoff + e + 1);
-                        for (int r = r0; r < r1; ++r) {
-                            uint8_t *o = row_addr(p, tab, r, row_bytes_q);
-                            for (int off = gtid * 16; off < row_bytes_q; off += kGroupThreads * 16)
-                                st_v4(o + off, make_uint4(0, 0, 0, 0));
-                            if (FP8 && gtid < NB) *scale_addr(p, tab, r, gtid, NB) = 0.0f;
-                        }
-                    }
                 }
             }
         }
@@ -839,7 +681,6 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
             __threadfence();
             atomicExch(&p.ctl->ticket, 0u);
             atomicExch(&p.ctl->units, 0u);
-            atomicExch(&p.ctl->pads, 0u);
             atomicExch(&p.ctl->done, 0u);
             atomicExch(&p.ctl->epoch, s_tag);
         }
@@ -953,27 +794,23 @@ cudaError_t launch_layout_counts(const LbParams &p, cudaStream_t s) {
 
 cudaError_t launch_dispatch_lb(const LbParams &p_in, bool fp8, int num_sms, cudaStream_t s) {
     LbParams p = p_in;
-    // peer destinations are only known to be 16-byte aligned: 16-byte stores there
-    // peer destinations: the kernel checks their bases and falls back to 16-byte stores
-    const uintptr_t dst_bits = p.peer_base ? 0 : reinterpret_cast<uintptr_t>(p.recv);
-    const bool v32 = !fp8 && p.H % 16 == 0 && ((reinterpret_cast<uintptr_t>(p.x) | dst_bits) & 31) == 0;
+    const bool v32 = !fp8 && p.H % 16 == 0 &&
+                     ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0;
     const int VB = v32 ? 32 : 16;
-    p.vec32 = (dst_bits & 31) == 0;
-    if (p.peer_base && p.lb) return cudaErrorInvalidValue;   // peer mode takes a layout computed before
+    p.vec32 = (reinterpret_cast<uintptr_t>(p.recv) & 31) == 0;
     if (reinterpret_cast<uintptr_t>(p.pos) & 15) return cudaErrorInvalidValue;   // the handle's: 256-byte aligned
     if (!lb_unit_shape(p.H, fp8, VB, &p.splits, &p.chunk_bytes)) return cudaErrorInvalidValue;
     if ((int64_t)p.T * p.splits >= (int64_t(1) << 28)) return cudaErrorInvalidValue;   // stage tags hold 28 bits
     p.dyn_batch = p.splits * (fp8 ? EP_LB_DYN_TOKENS_FP8 : EP_LB_DYN_TOKENS_BF16);
     if (p.dyn_batch < 1) return cudaErrorInvalidValue;
     const size_t limit = smem_limit();
-    const int pr = p.peer_base ? p.R : 0;
-    const size_t fixed = carve(0, p.chunk_bytes, p.E, pr).total;
+    const size_t fixed = carve(0, p.chunk_bytes, p.E).total;
     int ns = (int)(EP_LB_RING_BYTES / p.chunk_bytes);
-    while (ns > 0 && carve(ns, p.chunk_bytes, p.E, pr).total > limit) --ns;
+    while (ns > 0 && carve(ns, p.chunk_bytes, p.E).total > limit) --ns;
     ns = ns > kMaxStages ? kMaxStages : ns;
     if (ns < 2 || fixed > limit) return cudaErrorInvalidValue;
     p.stages = ns;
-    const size_t smem = carve(ns, p.chunk_bytes, p.E, pr).total;
+    const size_t smem = carve(ns, p.chunk_bytes, p.E).total;
     const int grid = p.nchunks < num_sms ? p.nchunks : num_sms;
     if (grid <= 0) return cudaSuccess;
     if (fp8)

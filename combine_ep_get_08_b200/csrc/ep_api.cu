@@ -584,19 +584,6 @@ static int peer_common(const ep_handle *h, PeerOp op, const void *x, const void 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
     const char *what;
-    if (op != PeerOp::kCombine && c.num_tokens >= 2 * sms && c.num_tokens < ep::kLbMaxTokens) {
-        // a batch that fills the GPU: the chunked dispatch kernel in peer mode
-        // (dynamically claimed row parts, staged x; plain stores to the peers)
-        ep::LbParams p = lb_params(h, x, nullptr, nullptr, 0);
-        p.peer_base = reinterpret_cast<uint8_t *const *>(const_cast<void *const *>(bases));
-        p.peer_sbase = scale_bases;
-        p.peer_row0 = row0;
-        const bool fp8 = op == PeerOp::kDispatchFp8;
-        e = ep::launch_dispatch_lb(p, fp8, sms, s);
-        if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(dispatch_fp8_peer)" : "launch(dispatch_peer)");
-        g_launches.fetch_add(1, std::memory_order_relaxed);
-        return EP_OK;
-    }
     switch (op) {
         case PeerOp::kDispatch: e = ep::launch_dispatch_peer(l, sms, s); what = "launch(dispatch_peer)"; break;
         case PeerOp::kDispatchFp8:

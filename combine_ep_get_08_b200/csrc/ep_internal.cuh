@@ -125,7 +125,6 @@ struct LbControl {
     unsigned int ticket;         // next chunk to take (reset by the last dispatch CTA)
     unsigned int done;           // dispatch CTAs finished (reset by the last)
     unsigned int units;          // next batch of row parts to copy (dynamic copy; reset by the last)
-    unsigned int pads;           // next expert whose padding rows to write (peer mode; reset by the last)
     unsigned int epoch;          // tag of the last completed dispatch launch (look-back flags)
 };
 
@@ -167,13 +166,8 @@ struct LbParams {
     int stages;                  // ring depth
     int prefetch_x;              // 1: the chunk's x rows are prefetched into L2 at its start
     int vec32;                   // FP8: 1 when recv is 32-byte aligned (32-byte code stores)
+    int dyn;                     // 1: row parts are claimed in batches from ctl->units (K % 4 == 0)
     int dyn_batch;               // row parts per claim
-    // peer mode (lb = 0): the rows bound for rank r go to peer_base[r] at row
-    // peer_row0[r] + (row - rank_offsets[r]) (FP8 scales to peer_sbase[r],
-    // row-major); null peer_base: the local recv buffer
-    uint8_t *const *peer_base;   // device array [R]
-    float *const *peer_sbase;    // device array [R] (FP8)
-    const int32_t *peer_row0;    // device array [R]
 };
 cudaError_t launch_layout_counts(const LbParams &p, cudaStream_t s);
 // The fused (lb = 1) or handle-driven (lb = 0) chunked dispatch, bf16 or FP8.
