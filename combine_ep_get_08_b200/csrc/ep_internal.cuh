@@ -125,6 +125,7 @@ struct LbControl {
     unsigned int ticket;         // next chunk to take (reset by the last dispatch CTA)
     unsigned int done;           // dispatch CTAs finished (reset by the last)
     unsigned int units;          // next batch of row parts to copy (dynamic copy; reset by the last)
+    unsigned int pads;           // next expert whose padding rows to write (reset by the last)
     unsigned int epoch;          // tag of the last completed dispatch launch (look-back flags)
 };
 
