@@ -50,6 +50,9 @@
 #ifndef EP_LB_FP8_GROUPS
 #define EP_LB_FP8_GROUPS 2          // FP8 consumer groups per CTA (quantisation needs more warps)
 #endif
+#ifndef EP_LB_FUSED_PREFETCH
+#define EP_LB_FUSED_PREFETCH 1      // fused path, x into L2: 0 never, 1 after the dependency wait, 2 after
+#endif                              // this CTA's layout phase
 #ifndef EP_LB_RING_BYTES
 #define EP_LB_RING_BYTES (112 * 1024)
 #endif
@@ -262,9 +265,17 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_counts_kernel(LbPara
 // dependency wait, so it does not delay the latency-bound layout work).
 // ---------------------------------------------------------------------------
 template <bool FP8>
-__device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros, int lane, int n_cta, int chunk) {
+__device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros, int lane, int n_cta, int chunk,
+                                         volatile int *rows_done) {
     pdl_wait();   // offsets and counts come from the kernel before
-    if (p.lb && p.prefetch_x && lane == 0) {
+    if (EP_LB_FUSED_PREFETCH == 2 && p.lb && p.prefetch_x && lane == 0) {
+        // after this CTA's layout phase has published its rows (the flag is set
+        // on an abort too; bounded all the same)
+        const unsigned long long t0 = globaltimer_ns();
+        while (!*rows_done && globaltimer_ns() - t0 < p.wait_limit_ns) {
+        }
+    }
+    if (EP_LB_FUSED_PREFETCH && p.lb && p.prefetch_x && lane == 0) {
         const uint64_t pol_x = policy_evict_last();
         const uint8_t *x = static_cast<const uint8_t *>(p.x);
         for (int i = 0; i < n_cta; ++i) {
@@ -397,6 +408,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     int32_t *s_stpos = reinterpret_cast<int32_t *>(smem + cv.stpos);   // [stages][kStageDst] its destinations
     __shared__ int s_ticket;
     __shared__ int s_abort;
+    __shared__ int s_rows_done;   // this CTA's layout phase is over (its rows published, or aborted)
     __shared__ unsigned int s_tag;
     volatile int *abort_flag = &s_abort;
 
@@ -421,6 +433,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         }
         fence_async_smem();
         s_abort = 0;
+        s_rows_done = 0;
         // the previous launch's tag is stable: it changes only after every CTA
         // of that launch finished, and that launch completed before this one
         s_tag = (__ldcg(&p.ctl->epoch) % 0x7fffffffu) + 1u;
@@ -428,7 +441,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
     __syncthreads();
 
     if (warp == S::kPadWarp) {
-        pad_rows<FP8>(p, zeros, lane, n_cta, chunk);
+        pad_rows<FP8>(p, zeros, lane, n_cta, chunk, &s_rows_done);
     } else {
         const uint64_t pol_out = policy_evict_first();
         const unsigned int tag = s_tag;
@@ -584,6 +597,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
             if (tid == 0) st_release_u32(p.ready + c, tag);
         }
         pdl_wait();            // (a no-op after the first wait) the layout before is complete and visible
+        if (tid == 0) *static_cast<volatile int *>(&s_rows_done) = 1;
 
         // ---- phase 2: the copy; row parts claimed in batches of dyn_batch ----
         // The producer claims a batch from ctl->units (the next claim is
