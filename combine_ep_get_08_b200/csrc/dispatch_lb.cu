@@ -50,9 +50,16 @@
 #ifndef EP_LB_FP8_GROUPS
 #define EP_LB_FP8_GROUPS 2          // FP8 consumer groups per CTA (quantisation needs more warps)
 #endif
-#ifndef EP_LB_FUSED_PREFETCH
-#define EP_LB_FUSED_PREFETCH 1      // fused path, x into L2: 0 never, 1 after the dependency wait, 2 after
-#endif                              // this CTA's layout phase
+// Fused path, x into L2: 0 never, 1 after the dependency wait, 2 after this
+// CTA's layout phase.  Layout then dispatch span (two runs each): dsv3 bf16
+// 102.4 / 103.3 / 98.9 us for 0 / 1 / 2; skew FP8 90.7 / 93.7 / 95.8 us;
+// large FP8 229.3 / 229.3 / 229.1 us.
+#ifndef EP_LB_FUSED_PREFETCH_BF16
+#define EP_LB_FUSED_PREFETCH_BF16 2
+#endif
+#ifndef EP_LB_FUSED_PREFETCH_FP8
+#define EP_LB_FUSED_PREFETCH_FP8 0
+#endif
 #ifndef EP_LB_RING_BYTES
 #define EP_LB_RING_BYTES (112 * 1024)
 #endif
@@ -260,22 +267,24 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_counts_kernel(LbPara
 // eoff[e+1]); every row is written with bulk
 // shared->global copies of a zeroed block: a zero bf16 row, or zero codes and
 // (row-major, when 16-byte sized) zero scales; with lb = 1 also its routing
-// (row_src = row_slot = -1, row_weight = 0).  Before that, with lb = 1 and
-// prefetch_x, lane 0 pulls this CTA's x chunks into L2 (issued here, after the
-// dependency wait, so it does not delay the latency-bound layout work).
+// (row_src = row_slot = -1, row_weight = 0).  Before that, in the fused path
+// (lb = 1) with prefetch_x, lane 0 may pull this CTA's share of x into L2,
+// issued late enough not to delay the latency-bound layout work (bf16: once
+// this CTA's layout phase is over; FP8: not at all, which measured faster).
 // ---------------------------------------------------------------------------
 template <bool FP8>
 __device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros, int lane, int n_cta, int chunk,
                                          volatile int *rows_done) {
     pdl_wait();   // offsets and counts come from the kernel before
-    if (EP_LB_FUSED_PREFETCH == 2 && p.lb && p.prefetch_x && lane == 0) {
+    constexpr int kPrefetch = FP8 ? EP_LB_FUSED_PREFETCH_FP8 : EP_LB_FUSED_PREFETCH_BF16;
+    if (kPrefetch == 2 && p.lb && p.prefetch_x && lane == 0) {
         // after this CTA's layout phase has published its rows (the flag is set
         // on an abort too; bounded all the same)
         const unsigned long long t0 = globaltimer_ns();
         while (!*rows_done && globaltimer_ns() - t0 < p.wait_limit_ns) {
         }
     }
-    if (EP_LB_FUSED_PREFETCH && p.lb && p.prefetch_x && lane == 0) {
+    if (kPrefetch && p.lb && p.prefetch_x && lane == 0) {
         const uint64_t pol_x = policy_evict_last();
         const uint8_t *x = static_cast<const uint8_t *>(p.x);
         for (int i = 0; i < n_cta; ++i) {
