@@ -136,11 +136,12 @@ def test_kernel_figures_writeback_arithmetic():
     wl = workloads.generate("dsv3", with_x=False)
     ms = lambda v: [v * 1e-3] * 3  # noqa: E731  (µs -> ms samples)
     split = {"layout": ms(13.0), "dispatch": ms(90.0), "combine": ms(80.0),
-             "flush_after_dispatch": ms(50.0), "flush_after_combine": ms(42.0), "flush_clean": ms(40.0)}
+             "flush_after_dispatch": ms(50.0), "flush_after_combine": ms(42.0), "flush_clean": ms(40.0),
+             "dispatch_reuse": ms(88.0)}
     f = bench.kernel_figures(wl, 32768, split, False, 6500.0)
     b = 528482304
     assert f["bytes_per_call"] == {"dispatch": b, "combine": b}
-    assert f["us_per_call"] == {"layout": 13.0, "dispatch": 90.0, "combine": 80.0}
+    assert f["us_per_call"] == {"layout": 13.0, "dispatch": 90.0, "combine": 80.0, "dispatch_on_reused_layout": 88.0}
     wb = f["with_writeback"]
     assert wb["dispatch_us"] == 100.0 and wb["combine_us"] == 82.0
     assert abs(wb["dispatch_gbs"] - b / 100e-6 / 1e9) < 0.1
