@@ -60,6 +60,14 @@
 #ifndef EP_LB_FUSED_PREFETCH_FP8
 #define EP_LB_FUSED_PREFETCH_FP8 0
 #endif
+// Positions from the handle (lb = 0), x into L2: 0 never, 1 before the
+// dependency wait (overlapping the layout kernel), 2 after it (padding warp).
+#ifndef EP_LB_NORMAL_PREFETCH_BF16
+#define EP_LB_NORMAL_PREFETCH_BF16 1
+#endif
+#ifndef EP_LB_NORMAL_PREFETCH_FP8
+#define EP_LB_NORMAL_PREFETCH_FP8 1
+#endif
 #ifndef EP_LB_RING_BYTES
 #define EP_LB_RING_BYTES (112 * 1024)
 #endif
@@ -277,6 +285,15 @@ __device__ __forceinline__ void pad_rows(const LbParams &p, const uint8_t *zeros
                                          volatile int *rows_done) {
     pdl_wait();   // offsets and counts come from the kernel before
     constexpr int kPrefetch = FP8 ? EP_LB_FUSED_PREFETCH_FP8 : EP_LB_FUSED_PREFETCH_BF16;
+    constexpr int kPrefetchNormal = FP8 ? EP_LB_NORMAL_PREFETCH_FP8 : EP_LB_NORMAL_PREFETCH_BF16;
+    if (kPrefetchNormal == 2 && !p.lb && p.prefetch_x && lane == 0) {
+        const uint64_t pol_x = policy_evict_last();
+        const uint8_t *x = static_cast<const uint8_t *>(p.x);
+        for (int i = 0; i < n_cta; ++i) {
+            const int u = (int)blockIdx.x + i * (int)gridDim.x, t = u / p.splits, part = u - t * p.splits;
+            bulk_prefetch_l2(x + (int64_t)t * 2 * p.H + (int64_t)part * chunk, (uint32_t)chunk, pol_x);
+        }
+    }
     if (kPrefetch == 2 && p.lb && p.prefetch_x && lane == 0) {
         // after this CTA's layout phase has published its rows (the flag is set
         // on an abort too; bounded all the same)
@@ -461,7 +478,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         // together all of x) goes into L2 now, overlapping the kernel before;
         // with lb = 1 the padding warp does that after the dependency wait,
         // where it cannot delay the latency-bound layout phases
-        if (tid == 0 && p.prefetch_x && !p.lb) {
+        if (tid == 0 && p.prefetch_x && !p.lb && (FP8 ? EP_LB_NORMAL_PREFETCH_FP8 : EP_LB_NORMAL_PREFETCH_BF16) == 1) {
             const uint64_t pol_x = policy_evict_last();
             for (int i = 0; i < n_cta; ++i) {
                 const int u = (int)blockIdx.x + i * GC, t = u / p.splits, part = u - t * p.splits;
