@@ -71,6 +71,9 @@
 #ifndef EP_LB_NORMAL_PREFETCH_FP8
 #define EP_LB_NORMAL_PREFETCH_FP8 1
 #endif
+#ifndef EP_LB_PREISSUE
+#define EP_LB_PREISSUE 1            // lb = 0: claim and load the first parts' x before the dependency wait
+#endif
 #ifndef EP_LB_RING_BYTES
 #define EP_LB_RING_BYTES (112 * 1024)
 #endif
@@ -625,6 +628,59 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
             set_sync(NSET);
             if (tid == 0) st_release_u32(p.ready + c, tag);
         }
+        // The producer's row parts: claimed in batches of dyn_batch from
+        // ctl->units, one claim ahead (next_part() returns -1 when none is left).
+        unsigned int claim_cur = 0, claim_next = 0;
+        int part_u = 0, part_end = 0;
+        auto next_part = [&]() -> int {
+            for (;;) {
+                if (part_u < part_end) return part_u++;
+                if ((int64_t)claim_cur * p.dyn_batch >= total_units) return -1;
+                claim_cur = claim_next;
+                claim_next = atomicAdd(&p.ctl->units, 1u);
+                part_u = (int)claim_cur * p.dyn_batch;
+                part_end = min(total_units, part_u + p.dyn_batch);
+                if (part_u >= total_units) return -1;
+            }
+        };
+        // the destinations of part u: the 16-byte aligned span of pos that
+        // holds its token's K entries (pos is followed by other arrays of the
+        // handle's allocation, so the span never leaves it); the consumers skip
+        // `lead` entries
+        auto dst_span = [&](int u, int64_t *a0, int *lead, uint32_t *span) {
+            const int64_t b0 = (int64_t)(u / p.splits) * K * 4;
+            *a0 = b0 & ~(int64_t)15;
+            *lead = (int)(b0 - *a0) / 4;
+            *span = (uint32_t)((b0 + K * 4 - *a0 + 15) & ~(int64_t)15);
+        };
+        // x is an input and the claim counter belongs to the dispatch: with
+        // positions from the handle (lb = 0) the producer claims its first
+        // parts and fills the ring with their x bytes before the dependency
+        // wait, overlapping the layout kernel; their destinations follow after it
+        int pre = 0;
+        if (tid == 0) {
+            claim_cur = atomicAdd(&p.ctl->units, 1u);
+            claim_next = atomicAdd(&p.ctl->units, 1u);
+            part_u = (int)claim_cur * p.dyn_batch;
+            part_end = min(total_units, part_u + p.dyn_batch);
+            if (!p.lb && EP_LB_PREISSUE) {
+                for (; pre < NS; ++pre) {
+                    const int u = next_part();
+                    if (u < 0) break;
+                    int64_t a0;
+                    int lead;
+                    uint32_t span;
+                    dst_span(u, &a0, &lead, &span);
+                    const int t = u / p.splits, part = u - t * p.splits;
+                    s_unit[pre] = u | (lead << 28);
+                    mbar_arrive_expect_tx(&full[pre], (uint32_t)chunk + span);
+                    bulk_g2s(ring + (size_t)pre * chunk, x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk,
+                             &full[pre]);
+                    ++issued;
+                }
+            }
+        }
+        __syncwarp();
         pdl_wait();            // (a no-op after the first wait) the layout before is complete and visible
         if (tid == 0) *static_cast<volatile int *>(&s_rows_done) = 1;
 
@@ -640,44 +696,46 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
         {
             if (warp == 0) {
                 if (lane == 0) {
-                    int g = 0;
-                    unsigned int claim = atomicAdd(&p.ctl->units, 1u);
-                    while (!*abort_flag) {
-                        const int u0 = (int)claim * p.dyn_batch;
-                        if (u0 >= total_units) break;
-                        const unsigned int next = atomicAdd(&p.ctl->units, 1u);
-                        for (int u = u0; u < min(total_units, u0 + p.dyn_batch) && !*abort_flag; ++u, ++g) {
-                            const int s = g % NS;
-                            bool ok = g < NS || mbar_wait_bounded(&empty[s], ((g / NS) - 1) & 1, p.wait_limit_ns);
-                            const int t = u / p.splits, part = u - t * p.splits;
-                            if (ok && p.lb) {   // the chunk's rows are written (released by its CTA)
-                                const unsigned int *rf = p.ready + t / p.tpc;
-                                if (ld_acquire_u32(rf) != tag) {
-                                    const unsigned long long tw0 = globaltimer_ns();
-                                    while (ok && ld_acquire_u32(rf) != tag) ok = globaltimer_ns() - tw0 <= p.wait_limit_ns;
-                                }
-                                fence_proxy_async_global();   // those generic writes, before the bulk read below
+                    // the destinations of the parts issued before the wait
+                    for (int g = 0; g < pre; ++g) {
+                        const int u = s_unit[g] & 0x0fffffff;
+                        int64_t a0;
+                        int lead;
+                        uint32_t span;
+                        dst_span(u, &a0, &lead, &span);
+                        bulk_g2s(s_stpos + g * kStageDst, reinterpret_cast<const uint8_t *>(p.pos) + a0, span, &full[g]);
+                    }
+                    int g = pre;
+                    for (;; ++g) {
+                        if (*abort_flag) break;
+                        const int u = next_part();
+                        if (u < 0) break;
+                        const int s = g % NS;
+                        bool ok = g < NS || mbar_wait_bounded(&empty[s], ((g / NS) - 1) & 1, p.wait_limit_ns);
+                        const int t = u / p.splits, part = u - t * p.splits;
+                        if (ok && p.lb) {   // the chunk's rows are written (released by its CTA)
+                            const unsigned int *rf = p.ready + t / p.tpc;
+                            if (ld_acquire_u32(rf) != tag) {
+                                const unsigned long long tw0 = globaltimer_ns();
+                                while (ok && ld_acquire_u32(rf) != tag) ok = globaltimer_ns() - tw0 <= p.wait_limit_ns;
                             }
-                            if (!ok) {
-                                atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                                *abort_flag = 1;
-                                break;
-                            }
-                            // the token's K destinations: the 16-byte aligned span that holds
-                            // them (pos is followed by other arrays of the handle's allocation,
-                            // so the span never leaves it); the consumers skip `lead` entries
-                            const int64_t b0 = (int64_t)t * K * 4, a0 = b0 & ~(int64_t)15;
-                            const int lead = (int)(b0 - a0) / 4;
-                            const uint32_t span = (uint32_t)((b0 + K * 4 - a0 + 15) & ~(int64_t)15);
-                            s_unit[s] = u | (lead << 28);
-                            mbar_arrive_expect_tx(&full[s], (uint32_t)chunk + span);
-                            bulk_g2s(ring + (size_t)s * chunk, x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk,
-                                     &full[s]);
-                            bulk_g2s(s_stpos + s * kStageDst, reinterpret_cast<const uint8_t *>(p.pos) + a0, span,
-                                     &full[s]);
-                            ++issued;
+                            fence_proxy_async_global();   // those generic writes, before the bulk read below
                         }
-                        claim = next;
+                        if (!ok) {
+                            atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                            *abort_flag = 1;
+                            break;
+                        }
+                        int64_t a0;
+                        int lead;
+                        uint32_t span;
+                        dst_span(u, &a0, &lead, &span);
+                        s_unit[s] = u | (lead << 28);
+                        mbar_arrive_expect_tx(&full[s], (uint32_t)chunk + span);
+                        bulk_g2s(ring + (size_t)s * chunk, x + (int64_t)t * row_bytes + (int64_t)part * chunk, chunk,
+                                 &full[s]);
+                        bulk_g2s(s_stpos + s * kStageDst, reinterpret_cast<const uint8_t *>(p.pos) + a0, span, &full[s]);
+                        ++issued;
                     }
                     // one end marker per consumer group
                     for (int k = 0; k < G && !*abort_flag; ++k, ++g) {
