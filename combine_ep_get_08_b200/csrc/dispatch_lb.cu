@@ -71,8 +71,15 @@
 #ifndef EP_LB_NORMAL_PREFETCH_FP8
 #define EP_LB_NORMAL_PREFETCH_FP8 1
 #endif
-#ifndef EP_LB_PREISSUE
-#define EP_LB_PREISSUE 1            // lb = 0: claim and load the first parts' x before the dependency wait
+// lb = 0: claim the first row parts and load their x before the dependency
+// wait.  Two runs each, dispatch alone / layout-then-dispatch span: skew FP8
+// 81.0 / 95.9 us with, 82.8 / 97.7 us without; dsv3 bf16 96.7 / 100.6 us with,
+// 93.0 / 98.9 us without.
+#ifndef EP_LB_PREISSUE_BF16
+#define EP_LB_PREISSUE_BF16 0
+#endif
+#ifndef EP_LB_PREISSUE_FP8
+#define EP_LB_PREISSUE_FP8 1
 #endif
 #ifndef EP_LB_RING_BYTES
 #define EP_LB_RING_BYTES (112 * 1024)
@@ -663,7 +670,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1) dispatch_lb_kernel(LbPa
             claim_next = atomicAdd(&p.ctl->units, 1u);
             part_u = (int)claim_cur * p.dyn_batch;
             part_end = min(total_units, part_u + p.dyn_batch);
-            if (!p.lb && EP_LB_PREISSUE) {
+            if (!p.lb && (FP8 ? EP_LB_PREISSUE_FP8 : EP_LB_PREISSUE_BF16)) {
                 for (; pre < NS; ++pre) {
                     const int u = next_part();
                     if (u < 0) break;
