@@ -66,6 +66,10 @@ def _bind(lib):
     lib.oracle_expert_combine.restype = ctypes.c_int
     lib.oracle_combine.argtypes = [i32, i32, i32, i32, P, P, P, i32, P, P]
     lib.oracle_combine.restype = ctypes.c_int
+    lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_value.restype = ctypes.c_double
+    lib.oracle_expert_combine_fp8.argtypes = [i32] * 6 + [P] * 4 + [i64] + [P] * 3 + [i32, P, P]
+    lib.oracle_expert_combine_fp8.restype = ctypes.c_int
     return lib
 
 
@@ -263,5 +267,42 @@ def expert_combine(act_bits, w_bits, topk_idx, pos, topk_weights, sel_tokens=Non
                                        n, _ptr(sel), _ptr(out))
     if rc != OK:
         raise ValueError(f"oracle_expert_combine failed ({rc})")
+    return out
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one OCP E4M3 code (see ep_oracle.c)."""
+    return float(_load().oracle_e4m3_value(int(code) & 0xFF))
+
+
+def expert_combine_fp8(act_q, act_scale, w_q, w_scale, topk_idx, pos, topk_weights, scale_ld: int = 0,
+                       sel_tokens=None) -> np.ndarray:
+    """fp64 out[t] = sum_k w[t,k] * A[pos[t,k]] @ W_e^T with A and W_e restored from E4M3 codes and
+    their block scales (1x128 for the rows, 128x128 for the expert matrices; see ep_oracle.c).
+    act_scale is row-major [rows, I/128] when scale_ld == 0, else column-major with that leading
+    dimension."""
+    a = _c(act_q, np.uint8)
+    rows, I = a.shape
+    sa = _c(act_scale, np.float32)
+    if scale_ld == 0:
+        assert sa.shape == (rows, I // 128)
+    else:
+        assert sa.size >= (I // 128) * scale_ld and scale_ld >= rows
+    w = _c(w_q, np.uint8)
+    E, N, I2 = w.shape
+    assert I2 == I
+    sw = _c(w_scale, np.float32)
+    assert sw.shape == (E, N // 128, I // 128)
+    idx = _c(topk_idx, np.int64)
+    p = _c(pos, np.int32)
+    T, K = p.shape
+    tw = _c(topk_weights, np.float32)
+    sel = None if sel_tokens is None else _c(sel_tokens, np.int32)
+    n = T if sel is None else sel.shape[0]
+    out = np.empty((n, N), np.float64)
+    rc = _load().oracle_expert_combine_fp8(T, K, I, N, E, rows, _ptr(idx), _ptr(p), _ptr(a), _ptr(sa),
+                                           int(scale_ld), _ptr(w), _ptr(sw), _ptr(tw), n, _ptr(sel), _ptr(out))
+    if rc != OK:
+        raise ValueError(f"oracle_expert_combine_fp8 failed ({rc})")
     return out
 

@@ -381,3 +381,79 @@ int oracle_expert_combine(int32_t T, int32_t K, int32_t I, int32_t N, int32_t E,
     return ORACLE_OK;
 }
 
+
+/*
+ * Value of an OCP E4M3 code (sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits; exponent 0 is subnormal with step 2^-9; S.1111.111 is NaN; there is
+ * no infinity).  Exact in double.
+ */
+static double e4m3_value(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 0xF, m = c & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(8.0 + (double)m, e - 10);   /* (1 + m/8) * 2^(e-7) */
+    return s ? -v : v;
+}
+
+double oracle_e4m3_value(uint8_t c) { return e4m3_value(c); }
+
+/*
+ * The expert GEMM followed by combine, with FP8 operands: the expert inputs
+ * are the E4M3 codes and 1x128 dequantisation scales that the FP8 dispatch
+ * writes (a received row restores as q * scale, "2kiu.com/news/5702702"
+ * section 2.3), and each expert matrix is E4M3 with one fp32 scale per
+ * 128 x 128 block -- the per-block scaling of "m.nlpx.cn/news/135159"
+ * section 4.1, consumed by a grouped FP8 GEMM as in "lesson14_deepep"
+ * section 3.
+ *
+ * act_q [rows, I] codes; act_scale: row-major [rows, I/128] when
+ * scale_ld == 0, else column-major, scale of (r, b) at act_scale[b * scale_ld + r];
+ * w_q [E, N, I] codes; w_scale [E, N/128, I/128].  For each selected token t:
+ *   out[t, n] = sum_k topk_w[t,k] * sum_i A[pos[t,k], i] * W_e[n, i],
+ *   A[r, i] = q[r, i] * act_scale(r, i/128),
+ *   W_e[n, i] = w_q[e, n, i] * w_scale[e, n/128, i/128],
+ * e = topk_idx[t,k], in fp64 (every product and partial sum of the tests'
+ * inputs is exact there); masked pairs add nothing.
+ */
+int oracle_expert_combine_fp8(int32_t T, int32_t K, int32_t I, int32_t N, int32_t E, int32_t rows,
+                              const int64_t *topk_idx, const int32_t *pos, const uint8_t *act_q,
+                              const float *act_scale, int64_t scale_ld, const uint8_t *w_q,
+                              const float *w_scale, const float *topk_w, int32_t n_sel,
+                              const int32_t *sel_tokens, double *out)
+{
+    if (T < 0 || K <= 0 || I <= 0 || N <= 0 || E <= 0 || rows < 0) return ORACLE_BAD_ARG;
+    if (I % 128 != 0 || N % 128 != 0 || scale_ld < 0 || (scale_ld > 0 && scale_ld < rows)) return ORACLE_BAD_ARG;
+    const int32_t IB = I / 128, NB = N / 128;
+    for (int32_t j = 0; j < n_sel; ++j) {
+        int32_t t = sel_tokens ? sel_tokens[j] : j;
+        if (t < 0 || t >= T) return ORACLE_BAD_ARG;
+        double *o = out + (int64_t)j * N;
+        for (int32_t n = 0; n < N; ++n) o[n] = 0.0;
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t e = topk_idx[(int64_t)t * K + k];
+            int32_t r = pos[(int64_t)t * K + k];
+            if (e == -1 || r == -1) continue;
+            if (e < 0 || e >= E || r < 0 || r >= rows) return ORACLE_BAD_ARG;
+            const uint8_t *a = act_q + (int64_t)r * I;
+            const uint8_t *we = w_q + (int64_t)e * N * I;
+            const float *se = w_scale + (int64_t)e * NB * IB;
+            double wk = (double)topk_w[(int64_t)t * K + k];
+            for (int32_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int32_t i = 0; i < I; ++i) {
+                    int32_t b = i / 128;
+                    double sa = scale_ld > 0 ? (double)act_scale[(int64_t)b * scale_ld + r]
+                                             : (double)act_scale[(int64_t)r * IB + b];
+                    double sw = (double)se[(int64_t)(n / 128) * IB + b];
+                    acc += (e4m3_value(a[i]) * sa) * (e4m3_value(we[(int64_t)n * I + i]) * sw);
+                }
+                o[n] += wk * acc;
+            }
+        }
+    }
+    return ORACLE_OK;
+}

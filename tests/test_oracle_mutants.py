@@ -14,6 +14,7 @@ import pytest
 import oracle
 import test_oracle_dispatch_combine as tdc
 import test_oracle_expert_combine as tec
+import test_oracle_expert_combine_fp8 as tef
 import test_oracle_fp8 as tf8
 import test_oracle_layout as tlay
 import test_oracle_ll as tll
@@ -60,10 +61,37 @@ MUTANTS = {
         "if (e < 0) { pos[i] = -1; recv_count[0] += 1; continue; }"),
     "expert matrix transposed": ("* (double)bf16_bits_to_float(we[(int64_t)n * I + i]);",
                                  "* (double)bf16_bits_to_float(we[(int64_t)i * N + n]);"),
-    "expert taken from k = 0": ("int64_t e = topk_idx[(int64_t)t * K + k];\n            int32_t r = pos[",
-                                "int64_t e = topk_idx[(int64_t)t * K];\n            int32_t r = pos["),
-    "gemm weight of the wrong slot": ("double wk = (double)topk_w[(int64_t)t * K + k];\n            for (int32_t n",
-                                      "double wk = (double)topk_w[(int64_t)t * K + (K - 1 - k)];\n            for (int32_t n"),
+    "expert taken from k = 0": (
+        "int64_t e = topk_idx[(int64_t)t * K + k];\n            int32_t r = pos[(int64_t)t * K + k];\n"
+        "            if (e == -1 || r == -1) continue;\n"
+        "            if (e < 0 || e >= E || r < 0 || r >= rows) return ORACLE_BAD_ARG;\n"
+        "            const uint16_t *a",
+        "int64_t e = topk_idx[(int64_t)t * K];\n            int32_t r = pos[(int64_t)t * K + k];\n"
+        "            if (e == -1 || r == -1) continue;\n"
+        "            if (e < 0 || e >= E || r < 0 || r >= rows) return ORACLE_BAD_ARG;\n"
+        "            const uint16_t *a"),
+    "gemm weight of the wrong slot": (
+        "double wk = (double)topk_w[(int64_t)t * K + k];\n            for (int32_t n = 0; n < N; ++n) {\n"
+        "                double acc = 0.0;\n                for (int32_t i = 0; i < I; ++i)\n",
+        "double wk = (double)topk_w[(int64_t)t * K + (K - 1 - k)];\n            for (int32_t n = 0; n < N; ++n) {\n"
+        "                double acc = 0.0;\n                for (int32_t i = 0; i < I; ++i)\n"),
+    "fp8 gemm: expert taken from k = 0": (
+        "            const uint8_t *we = w_q + (int64_t)e * N * I;",
+        "            const uint8_t *we = w_q + (int64_t)topk_idx[(int64_t)t * K] * N * I;"),
+    "fp8 gemm: weight of the wrong slot": (
+        "double wk = (double)topk_w[(int64_t)t * K + k];\n            for (int32_t n = 0; n < N; ++n) {\n"
+        "                double acc = 0.0;\n                for (int32_t i = 0; i < I; ++i) {\n",
+        "double wk = (double)topk_w[(int64_t)t * K + (K - 1 - k)];\n            for (int32_t n = 0; n < N; ++n) {\n"
+        "                double acc = 0.0;\n                for (int32_t i = 0; i < I; ++i) {\n"),
+    "e4m3 value: exponent bias off by one": ("ldexp(8.0 + (double)m, e - 10)", "ldexp(8.0 + (double)m, e - 9)"),
+    "e4m3 value: subnormal step 2^-8": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -8);"),
+    "fp8 gemm: row scale of block 0": ("(double)act_scale[(int64_t)r * IB + b];", "(double)act_scale[(int64_t)r * IB];"),
+    "fp8 gemm: column-major scale read row-major": (
+        "(double)act_scale[(int64_t)b * scale_ld + r]", "(double)act_scale[(int64_t)r * IB + b]"),
+    "fp8 gemm: expert block scale transposed": (
+        "se[(int64_t)(n / 128) * IB + b]", "se[(int64_t)b * NB + n / 128]"),
+    "fp8 gemm: expert block scale dropped": (
+        "(e4m3_value(we[(int64_t)n * I + i]) * sw)", "(e4m3_value(we[(int64_t)n * I + i]) + 0.0 * sw)"),
     "padding row not zeroed": (
         "            memset(dst, 0, sizeof(uint16_t) * (size_t)H);\n",
         "            memset(dst, 0, sizeof(uint16_t) * (size_t)(H / 2));\n"),
@@ -104,6 +132,11 @@ PINS = [
     ("gemm scaled identity", lambda lib: tec.test_scaled_identity_experts(lib)),
     ("gemm rank one", lambda lib: tec.test_rank_one_experts(lib)),
     ("gemm masked", lambda lib: tec.test_masked_slots_and_selection(lib)),
+    ("fp8 gemm decoder", lambda lib: tef.test_e4m3_decoder_all_codes(lib)),
+    ("fp8 gemm unit scales", lambda lib: tef.test_unit_scales_reduce_to_bf16_gemm(lib)),
+    ("fp8 gemm block scales", lambda lib: tef.test_block_scales_closed_form(lib)),
+    ("fp8 gemm column-major", lambda lib: tef.test_column_major_scales(lib)),
+    ("fp8 gemm masked", lambda lib: tef.test_masked_slots_and_selection_fp8(lib)),
     ("ll worked example", lambda lib: tll.test_ll_worked_example(lib)),
     ("ll brute force", lambda lib: tll.test_ll_bruteforce_tiny(lib)),
     ("ll round trip", lambda lib: tll.test_ll_round_trip(lib)),
