@@ -898,6 +898,8 @@ EGEMM = dict(T=4096, H=7168, E=32, R=8, K=8, A=128, router="topk", seed=5, I=204
 EGEMM_DESC = ("one expert-parallel rank of a DeepSeek-V3 layer: 32 local experts receiving 4096 tokens x "
               "top-8 (32768 rows, 1024 per expert, align 128); expert down projection 2048 -> 7168 bf16 "
               "with the top-k weighted combine in the epilogue")
+EGEMM_DESC_FP8 = EGEMM_DESC.replace("2048 -> 7168 bf16", "2048 -> 7168 E4M3 (1x128 row scales, 128x128 "
+                                     "expert-matrix scales)")
 
 
 def run_peer(args, world, rank, local):
@@ -1025,6 +1027,97 @@ def run_peer(args, world, rank, local):
     return 0
 
 
+def expert_gemm_inputs(dev, fp8: bool, rank: int = 0):
+    """Handle, layout and synthetic operands of the expert GEMM workload (EGEMM).
+    bf16: act ~ N(0,1), W_e ~ N(0,1)/sqrt(I).  E4M3: codes of 32*N(0,1) (saturating
+    cast), row scales U(1/64, 1/16) per 128 columns, expert scales
+    U(0.5, 1.5)/(32*sqrt(I)) per 128 x 128 block."""
+    import torch
+
+    import combine_ep_get_08_b200 as ep
+    import workloads
+
+    c = dict(EGEMM)
+    I = c.pop("I")
+    seed = c.pop("seed") + 1000 * rank
+    wl = workloads.generate(None, seed=seed, with_x=False, **c)
+    N = wl.H
+    cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
+    h = ep.ep_handle_create(cfg)
+    idx, tw = wl.topk_idx.to(dev), wl.topk_weights.to(dev)
+    ep.ep_get_layout(h, idx, tw)
+    rows = ep.ep_get_num_rows(h)
+    cap = ep.ep_capacity_rows(cfg)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    ops = {"wl": wl, "h": h, "I": I, "N": N, "rows": rows, "cap": cap, "tw": tw, "fp8": fp8,
+           "acc": torch.empty((wl.T, N), dtype=torch.float32, device=dev),
+           "out": torch.empty((wl.T, N), dtype=torch.bfloat16, device=dev)}
+    if fp8:
+        def e4m3(shape):
+            v = torch.randn(shape, generator=gen, device=dev) * 32.0
+            return v.clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+        ops["act"] = e4m3((cap, I))
+        ops["sa"] = torch.rand((cap, I // 128), generator=gen, device=dev) * (3.0 / 64.0) + 1.0 / 64.0
+        ops["w"] = e4m3((wl.E, N, I))
+        ops["sw"] = (torch.rand((wl.E, N // 128, I // 128), generator=gen, device=dev) + 0.5) / (32.0 * I ** 0.5)
+    else:
+        ops["act"] = torch.randn((cap, I), generator=gen, device=dev).to(torch.bfloat16)
+        ops["w"] = (torch.randn((wl.E, N, I), generator=gen, device=dev) / I ** 0.5).to(torch.bfloat16)
+    return ops
+
+
+def expert_gemm_call(o, stream):
+    import combine_ep_get_08_b200 as ep
+    if o["fp8"]:
+        ep.ep_expert_combine_fp8(o["h"], o["act"], o["sa"], o["I"], o["w"], o["sw"], o["N"], o["tw"], o["acc"],
+                                 o["out"], stream=stream.cuda_stream)
+    else:
+        ep.ep_expert_combine(o["h"], o["act"], o["I"], o["w"], o["N"], o["tw"], o["acc"], o["out"],
+                             stream=stream.cuda_stream)
+
+
+def gemm_peak(fp8: bool):
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16 = float(json.load(f)["bf16_tflops"])
+        src = "measured burst (MEASURED_PEAKS.json bf16_tflops)"
+    except Exception:  # noqa: BLE001
+        bf16, src = 1590.0, "fallback 1.59 PFLOP/s"
+    if fp8:
+        return 2.0 * bf16, src + " x 2 (nominal dense FP8 / bf16 ratio, 4.5 / 2.25 PFLOP/s)"
+    return bf16, src
+
+
+def time_expert_gemm(o, steps, warmup, flush, stream):
+    """Per-call CUDA-event times (ms) of the expert GEMM, L2 flushed before each call."""
+    import torch
+    for _ in range(warmup):
+        expert_gemm_call(o, stream)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in evs:
+        flush.sum()
+        e0.record(stream)
+        expert_gemm_call(o, stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def expert_gemm_summary(o, ms):
+    """Per-config entry of the default bench line for one expert GEMM dtype."""
+    wl = o["wl"]
+    pairs = int((wl.topk_idx >= 0).sum())
+    flops_call = 2.0 * pairs * o["N"] * o["I"]
+    peak, src = gemm_peak(o["fp8"])
+    mean_ms = statistics.mean(ms)
+    tf = flops_call / (mean_ms * 1e-3) / 1e12
+    return {"workload": EGEMM_DESC if not o["fp8"] else EGEMM_DESC_FP8, "steps": len(ms),
+            "us_per_call": round(mean_ms * 1e3, 2), "tflops": round(tf, 1), "peak": peak, "peak_source": src,
+            "frac": round(tf / peak, 4), "dtype": "e4m3" if o["fp8"] else "bf16"}
+
+
 def run_expert_gemm(args, world, rank, local):
     import numpy as np
     import torch
@@ -1039,67 +1132,46 @@ def run_expert_gemm(args, world, rank, local):
     if rank == 0:
         build_lib.build()
     barrier(world)
-    c = dict(EGEMM)
-    I = c.pop("I")
-    seed = c.pop("seed") + 1000 * rank
-    wl = workloads.generate(None, seed=seed, with_x=False, **c)
-    N = wl.H
-    cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
-    h = ep.ep_handle_create(cfg)
+    fp8 = args.gemm_dtype == "e4m3"
+    o = expert_gemm_inputs(dev, fp8, rank)
+    wl, h, I, N, rows = o["wl"], o["h"], o["I"], o["N"], o["rows"]
     if args.sm_limit:
         ep.ep_set_sm_limit(h, args.sm_limit)
-    idx, tw = wl.topk_idx.to(dev), wl.topk_weights.to(dev)
-    ep.ep_get_layout(h, idx, tw)
-    rows = ep.ep_get_num_rows(h)
-    cap = ep.ep_capacity_rows(cfg)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(seed)
-    act = torch.randn((cap, I), generator=gen, device=dev).to(torch.bfloat16)
-    w = (torch.randn((wl.E, N, I), generator=gen, device=dev) / I ** 0.5).to(torch.bfloat16)
-    acc = torch.empty((wl.T, N), dtype=torch.float32, device=dev)
-    out = torch.empty((wl.T, N), dtype=torch.bfloat16, device=dev)
     flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
-        ep.ep_expert_combine(h, act, I, w, N, tw, acc, out, stream=stream.cuda_stream)
+        expert_gemm_call(o, stream)
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     launches0 = ep.ep_launch_count()
     sampler = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
     with sampler:
-        for e0, e1 in evs:
-            flush.sum()
-            e0.record(stream)
-            ep.ep_expert_combine(h, act, I, w, N, tw, acc, out, stream=stream.cuda_stream)
-            e1.record(stream)
-        torch.cuda.synchronize()
+        ms = time_expert_gemm(o, args.steps, 0, flush, stream)
     barrier(world)
     launches = ep.ep_launch_count() - launches0
-    ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = max_over_ranks(sum(ms), world, dev)
     pairs = int((wl.topk_idx >= 0).sum())
     flops_call = 2.0 * pairs * N * I               # algorithmic: real rows only
     all_flops = sum_over_ranks(flops_call * args.steps, world, dev)
     tflops = all_flops / (total_ms * 1e-3) / 1e12
     status = ep.ep_get_status(h)
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peak, peak_src = float(json.load(f)["bf16_tflops"]), "measured burst (MEASURED_PEAKS.json bf16_tflops)"
-    except Exception:  # noqa: BLE001
-        peak, peak_src = 1590.0, "fallback 1.59 PFLOP/s"
+    peak, peak_src = gemm_peak(fp8)
     mean_ms = statistics.mean(ms)
+    kernel = "gemm_combine_fp8_kernel" if fp8 else "gemm_combine_kernel"
     if rank == 0:
         line = {
-            "metric": "expert GEMM + fused combine TFLOP/s", "value": round(tflops, 1), "unit": "TFLOP/s",
+            "metric": ("expert GEMM (E4M3) + fused combine TFLOP/s" if fp8
+                       else "expert GEMM + fused combine TFLOP/s"),
+            "value": round(tflops, 1), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": EGEMM_DESC, "rows": rows, "padded_rows_computed": rows, "pairs": pairs,
+            "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
+            "config": {"workload": EGEMM_DESC_FP8 if fp8 else EGEMM_DESC, "rows": rows,
+                       "padded_rows_computed": rows, "pairs": pairs,
                        "inner": I, "n_out": N, "sm_limit": args.sm_limit or None,
                        "l2": "flushed (256 MiB read, outside the timed events) before each call"},
-            "roofline": {"bound": "tensor", "kernel": "gemm_combine_kernel (+ memset and bf16 rounding)",
+            "roofline": {"bound": "tensor", "kernel": kernel + " (+ memset and bf16 rounding)",
                          "achieved": round(flops_call / (mean_ms * 1e-3) / 1e12, 1), "peak": peak,
                          "peak_source": peak_src, "unit": "TFLOP/s",
                          "frac": round(flops_call / (mean_ms * 1e-3) / 1e12 / peak, 4), "traffic": None},
@@ -1108,13 +1180,21 @@ def run_expert_gemm(args, world, rank, local):
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             oracle.build()
-            o = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A)
-            act_b = workloads.bf16_bits(act[:rows])
-            w_b = workloads.bf16_bits(w)
+            ol = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A)
+            if fp8:
+                a_h, sa_h = o["act"][:rows].cpu().numpy(), o["sa"][:rows].cpu().numpy()
+                w_h, sw_h = o["w"].cpu().numpy(), o["sw"].cpu().numpy()
+                one = lambda t: oracle.expert_combine_fp8(  # noqa: E731
+                    a_h, sa_h, w_h, sw_h, wl.topk_idx.numpy(), ol.pos, wl.topk_weights.numpy(),
+                    sel_tokens=np.array([t], np.int32))
+            else:
+                act_b = workloads.bf16_bits(o["act"][:rows])
+                w_b = workloads.bf16_bits(o["w"])
+                one = lambda t: oracle.expert_combine(  # noqa: E731
+                    act_b, w_b, wl.topk_idx.numpy(), ol.pos, wl.topk_weights.numpy(), np.array([t], np.int32))
             n_tok, t0 = 0, time.perf_counter()
             while time.perf_counter() - t0 < args.cpu_budget:
-                oracle.expert_combine(act_b, w_b, wl.topk_idx.numpy(), o.pos, wl.topk_weights.numpy(),
-                                      np.array([n_tok % wl.T], np.int32))
+                one(n_tok % wl.T)
                 n_tok += 1
             el = time.perf_counter() - t0
             line["cpu_baseline"] = {
@@ -1206,6 +1286,8 @@ def main(argv=None):
     ap.add_argument("--ncu-ingest", metavar="REP", help="record DRAM traffic from an ncu report and exit")
     ap.add_argument("--peer", action="store_true",
                     help="time ep_dispatch_peer + ep_combine_peer (R destination buffers on this GPU)")
+    ap.add_argument("--gemm-dtype", choices=["bf16", "e4m3"], default="bf16",
+                    help="operand type of --expert-gemm")
     ap.add_argument("--expert-gemm", action="store_true",
                     help="time ep_expert_combine (expert GEMM + fused combine) instead of the step")
     args = ap.parse_args(argv)

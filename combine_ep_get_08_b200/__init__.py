@@ -85,6 +85,7 @@ def _load():
             "ep_set_wait_limit": ([P, U64, I32], ctypes.c_int),
             "ep_set_sm_limit": ([P, I32], ctypes.c_int),
             "ep_expert_combine": ([P, P, I32, P, I32, P, P, P, P], ctypes.c_int),
+            "ep_expert_combine_fp8": ([P, P, P, I32, P, P, I32, P, P, P, P], ctypes.c_int),
             "ep_ll_capacity_rows": ([CFG, I32], I64),
             "ep_ll_scale_buffer_floats": ([CFG, I32, I32], I64),
             "ep_ll_handle_create": ([CFG, I32, ctypes.POINTER(P)], ctypes.c_int),
@@ -318,6 +319,13 @@ def ep_set_wait_limit(h: int, limit_ns: int, extra_arrivals: int = 0) -> None:
 def ep_expert_combine(h: int, act, inner: int, w, n_out: int, topk_weights, out_acc, out, stream=None) -> None:
     _check("ep_expert_combine", _load().ep_expert_combine(
         h, _ptr(act), inner, _ptr(w), n_out, _ptr(topk_weights), _ptr(out_acc), _ptr(out), _stream(stream)))
+
+
+def ep_expert_combine_fp8(h: int, act_q, act_scales, inner: int, w_q, w_scales, n_out: int, topk_weights, out_acc,
+                          out, stream=None) -> None:
+    _check("ep_expert_combine_fp8", _load().ep_expert_combine_fp8(
+        h, _ptr(act_q), _ptr(act_scales), inner, _ptr(w_q), _ptr(w_scales), n_out, _ptr(topk_weights),
+        _ptr(out_acc), _ptr(out), _stream(stream)))
 
 
 def ep_ll_capacity_rows(cfg: ep_config, num_max_dispatch_tokens: int) -> int:

@@ -504,16 +504,19 @@ EP_API int ep_ll_combine(const ep_handle *h, const void *y, const float *topk_we
     return combine_common(h, y, topk_weights, out, true, stream);
 }
 
-EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner, const void *w, int32_t n_out,
-                             const float *topk_weights, float *out_acc, void *out, ep_stream_t stream) {
+static int expert_combine_common(const ep_handle *h, const void *act, const float *act_scales, int32_t inner,
+                                 const void *w, const float *w_scales, int32_t n_out, const float *topk_weights,
+                                 float *out_acc, void *out, bool fp8, ep_stream_t stream) {
     int rc = check_mode(h, false, true);
     if (rc != EP_OK) return rc;
     const ep_config &c = h->cfg;
-    if (c.expert_alignment % 128 != 0 || inner <= 0 || inner % 64 != 0 || n_out <= 0 || n_out % 256 != 0)
+    if (c.expert_alignment % 128 != 0 || inner <= 0 || inner % (fp8 ? 128 : 64) != 0 || n_out <= 0 ||
+        n_out % 256 != 0)
         return EP_ERR_ARG;
     if ((int64_t)c.num_experts * n_out > INT32_MAX || h->cap > INT32_MAX) return EP_ERR_UNSUPPORTED;
     if (c.num_tokens == 0) return EP_OK;
     if (!act || !w || !topk_weights || !out_acc || !out) return EP_ERR_ARG;
+    if (fp8 && (!act_scales || !w_scales || !aligned(act_scales, 4) || !aligned(w_scales, 4))) return EP_ERR_ARG;
     if (!aligned(act, 16) || !aligned(w, 16) || !aligned(out_acc, 16) || !aligned(out, 16) ||
         !aligned(topk_weights, 4))
         return EP_ERR_ARG;
@@ -531,6 +534,10 @@ EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner,
     a.p.K = c.num_topk;
     a.p.N = n_out;
     a.p.I = inner;
+    a.p.act_scale = act_scales;
+    a.p.w_scale = w_scales;
+    a.p.scale_ld = h->scale_layout == EP_SCALES_COL_MAJOR_TMA ? (int)((h->cap + 3) / 4 * 4) : 0;
+    a.fp8 = fp8;
     a.act = act;
     a.w = w;
     a.out = out;
@@ -538,9 +545,22 @@ EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner,
     a.T = c.num_tokens;
     const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
     cudaError_t e = ep::launch_gemm_combine(a, sms, reinterpret_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "launch(expert_combine)");
+    if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(expert_combine_fp8)" : "launch(expert_combine)");
     g_launches.fetch_add(2, std::memory_order_relaxed);
     return EP_OK;
+}
+
+EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner, const void *w, int32_t n_out,
+                             const float *topk_weights, float *out_acc, void *out, ep_stream_t stream) {
+    return expert_combine_common(h, act, nullptr, inner, w, nullptr, n_out, topk_weights, out_acc, out, false,
+                                 stream);
+}
+
+EP_API int ep_expert_combine_fp8(const ep_handle *h, const uint8_t *act_q, const float *act_scales, int32_t inner,
+                                 const uint8_t *w_q, const float *w_scales, int32_t n_out,
+                                 const float *topk_weights, float *out_acc, void *out, ep_stream_t stream) {
+    return expert_combine_common(h, act_q, act_scales, inner, w_q, w_scales, n_out, topk_weights, out_acc, out,
+                                 true, stream);
 }
 
 // ---- peer-memory exchange (one process per GPU) ----

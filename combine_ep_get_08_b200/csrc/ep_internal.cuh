@@ -97,14 +97,19 @@ struct GemmCombineParams {
     unsigned int *status;
     unsigned long long wait_limit_ns;
     int E, K, N, I;              // N output features, I inner features
+    // FP8 form only
+    const float *act_scale;      // row-major [cap, I/128], or [I/128][scale_ld] when scale_ld > 0
+    const float *w_scale;        // [E, N/128, I/128]: one scale per 128 x 128 block of W_e
+    int scale_ld;
 };
 struct GemmCombineArgs {
     GemmCombineParams p;
-    const void *act;             // [cap, I] bf16, received-row layout
-    const void *w;               // [E, N, I] bf16
+    const void *act;             // [cap, I] bf16 (or E4M3 codes when fp8), received-row layout
+    const void *w;               // [E, N, I] bf16 (or E4M3 codes when fp8)
     void *out;                   // [T, N] bf16
     int64_t cap;
     int T;
+    bool fp8;
 };
 // memset of the accumulator, the GEMM (one CTA per SM, num_sms CTAs) and the bf16 rounding
 cudaError_t launch_gemm_combine(const GemmCombineArgs &g, int num_sms, cudaStream_t s);

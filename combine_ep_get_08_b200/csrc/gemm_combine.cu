@@ -304,6 +304,240 @@ __global__ void __launch_bounds__(kGThreads, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" : : "r"(tmem), "r"(kGTmemCols) : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// FP8 form: E4M3 rows with one fp32 scale per row and 128 inner elements (what
+// the FP8 dispatch writes) times E4M3 expert matrices with one fp32 scale per
+// 128 x 128 block ("m.nlpx.cn/news/135159" section 4.1, per-block scaling;
+// the grouped FP8 expert GEMM of "lesson14_deepep" section 3):
+//   out[t, :] = bf16_rn( sum_k w[t,k] * sum_b sa[r, b] * sw[e, :/128, b] * (q[r, b] . Wq_e[:, b]) ).
+// The scales change every 128 inner elements, so they cannot ride inside one
+// tensor-core accumulation: each 128-deep k-block is its own tcgen05.mma
+// (kind::f8f6f4, M=128, N=256, K=32, four per k-block) into one of two TMEM
+// partial buffers, and the epilogue warps fold each partial into fp32
+// registers with its two scales (sa of the row, sw of the 128-column half)
+// while the tensor cores fill the other buffer.  Eight epilogue warps: warp w
+// reads TMEM lanes 32*(w%4).. and one 128-column half of the tile, so a thread
+// keeps 128 running sums.  After the tile's last k-block the sums are scaled by
+// the pair's top-k weight and added into the token's fp32 row as in the bf16
+// kernel.  Same persistent tile order, producer and bounded waits.
+// ---------------------------------------------------------------------------
+constexpr int kFK = 128;                              // inner elements per stage: one 128-byte row = one scale block
+constexpr int kFStages = 4;
+constexpr uint32_t kFABytes = kGM * kFK;              // 16 KB
+constexpr uint32_t kFBBytes = kGN * kFK;              // 32 KB
+constexpr int kFEpiWarps = 8;                         // 4 lane quarters x 2 column halves
+constexpr int kFThreads = 64 + 32 * kFEpiWarps;
+constexpr int kFHalf = kGN / 2;                       // columns per epilogue thread
+constexpr uint32_t kFTmemCols = 2 * kGN;              // two partial buffers
+constexpr size_t kFSmem = 1024 + kFStages * (size_t)(kFABytes + kFBBytes) + kFEpiWarps * kGStageT + 256;
+
+// Instruction descriptor of tcgen05.mma kind::f8f6f4: fp32 accumulator (bits
+// 4-5 = 1), E4M3 A and B (format code 0 at bits 7-9 and 10-12), both K-major,
+// N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kFIdesc = (1u << 4) | ((uint32_t)(kGN >> 3) << 17) | ((uint32_t)(kGM >> 4) << 24);
+
+__device__ __forceinline__ void umma_e4m3(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n"
+        :
+        : "r"(tmem_d), "l"(a), "l"(b), "r"(kFIdesc), "r"(accumulate));
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : : : "memory");
+}
+
+__global__ void __launch_bounds__(kFThreads, 1)
+    gemm_combine_fp8_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                            GemmCombineParams p) {
+    extern __shared__ uint8_t g_smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(g_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;
+    uint8_t *sB = base + kFStages * kFABytes;
+    float *sT = reinterpret_cast<float *>(sB + kFStages * kFBBytes);   // [epilogue warps][32 rows][32 cols], swizzled
+    uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sT) + kFEpiWarps * kGStageT);
+    uint64_t *empty = full + kFStages;
+    uint64_t *part_full = empty + kFStages;   // [2] a k-block's partial product is in TMEM buffer j
+    uint64_t *part_empty = part_full + 2;     // [2] every epilogue warp has folded buffer j
+    uint64_t *drain = part_empty + 2;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows = __ldg(&p.eoff[p.E]);
+    const int n_blocks = p.N / kGN;
+    const int tiles = (rows / kGM) * n_blocks;
+    const int k_blocks = p.I / kFK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kFStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&part_full[j], 1);
+            mbar_init(&part_empty[j], kFEpiWarps);   // lane 0 of each epilogue warp
+        }
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_async_smem();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :
+                     : "r"(smem_u32(s_tmem)), "r"(kFTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" : : : "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 0) {
+        // ---- TMA producer ----
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
+                const GemmTile g = tile_coords(p.eoff, p.E, n_blocks, tile);
+                for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+                    const int s = it % kFStages, use = it / kFStages;
+                    if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1, p.wait_limit_ns)) {
+                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *s_abort = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], kFABytes + kFBBytes);
+                    tma_load_2d(sA + s * kFABytes, &map_a, kb * kFK, g.m * kGM, &full[s]);
+                    tma_load_2d(sB + s * kFBBytes, &map_b, kb * kFK, g.e * p.N + g.n * kGN, &full[s]);
+                }
+            }
+            if (*s_abort)
+                for (int j = max(0, it - kFStages); j < it; ++j)
+                    mbar_wait_bounded(&full[j % kFStages], (j / kFStages) & 1, p.wait_limit_ns);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer: one partial product per k-block, alternating TMEM buffers ----
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
+                bool ok = true;
+                for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+                    const int j = it & 1, juse = it >> 1, s = it % kFStages;
+                    if (juse > 0 && !mbar_wait_bounded(&part_empty[j], (juse - 1) & 1, p.wait_limit_ns)) {
+                        ok = false;
+                    } else if (!mbar_wait_bounded(&full[s], (it / kFStages) & 1, p.wait_limit_ns)) {
+                        ok = false;
+                    }
+                    if (!ok) {
+                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *s_abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d = tmem + (uint32_t)(j * kGN);
+                    const uint64_t a = umma_desc_k_sw128(smem_u32(sA + s * kFABytes));
+                    const uint64_t b = umma_desc_k_sw128(smem_u32(sB + s * kFBBytes));
+#pragma unroll
+                    for (int kk = 0; kk < kFK / 32; ++kk)   // 32 E4M3 = 32 bytes = 2 descriptor units
+                        umma_e4m3(d, a + 2 * kk, b + 2 * kk, kk != 0);
+                    umma_commit(&empty[s]);
+                    umma_commit(&part_full[j]);
+                }
+                if (!ok) break;
+            }
+            umma_commit(drain);
+            mbar_wait_bounded(drain, 0, p.wait_limit_ns);
+        }
+    } else {
+        // ---- epilogue: fold the scaled partials, then combine ----
+        const int ew = warp - 2;
+        const int q = warp & 3;                    // TMEM lanes 32q .. 32q+31
+        const int h = ew >> 2;                     // column half of the tile
+        const int IB = p.I / kFK, NB = p.N / 128;
+        float4 *tile4 = reinterpret_cast<float4 *>(sT + ew * (kGStageT / 4));
+        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * kFHalf);
+        int it = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            const GemmTile g = tile_coords(p.eoff, p.E, n_blocks, tile);
+            const int r = g.m * kGM + q * 32 + lane;
+            const int src = __ldg(&p.row_src[r]);
+            float wt = 0.0f;
+            if (src >= 0) wt = __ldg(&p.topk_w[(int64_t)src * p.K + __ldg(&p.row_slot[r])]);
+            const float *sa_row = p.scale_ld > 0 ? p.act_scale + r : p.act_scale + (int64_t)r * IB;
+            const int64_t sa_step = p.scale_ld > 0 ? p.scale_ld : 1;
+            const float *sw_blk = p.w_scale + ((int64_t)g.e * NB + 2 * g.n + h) * IB;
+            float acc[kFHalf];
+#pragma unroll
+            for (int c = 0; c < kFHalf; ++c) acc[c] = 0.0f;
+            float sa_next = __ldg(sa_row), sw_next = __ldg(sw_blk);
+            bool ok = true;
+            for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+                const float sc = sa_next * sw_next;
+                if (kb + 1 < k_blocks) {
+                    sa_next = __ldg(sa_row + (kb + 1) * sa_step);
+                    sw_next = __ldg(sw_blk + kb + 1);
+                }
+                const int j = it & 1;
+                if (*s_abort || !mbar_wait_bounded(&part_full[j], (it >> 1) & 1, p.wait_limit_ns)) {
+                    if (!*s_abort) {
+                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                        *s_abort = 1;
+                    }
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < kFHalf / 16; ++c) {
+                    uint32_t v[16];
+                    tmem_ld16(lane_base + (uint32_t)(j * kGN + c * 16), v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[c * 16 + i] = fmaf(sc, __uint_as_float(v[i]), acc[c * 16 + i]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&part_empty[j]);
+            }
+            if (!ok) break;
+            // combine: a thread holds one row of 128 columns; each 32-column chunk is
+            // transposed through shared memory so eight lanes cover 128 contiguous bytes
+            const int sub = lane >> 3, k4 = lane & 7;
+#pragma unroll
+            for (int c = 0; c < kFHalf / 32; ++c) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    tile4[lane * 8 + (k ^ (lane & 7))] =
+                        make_float4(wt * acc[c * 32 + 4 * k], wt * acc[c * 32 + 4 * k + 1],
+                                    wt * acc[c * 32 + 4 * k + 2], wt * acc[c * 32 + 4 * k + 3]);
+                __syncwarp();
+                float *ocol = p.out_acc + (int64_t)g.n * kGN + h * kFHalf + c * 32 + k4 * 4;
+#pragma unroll
+                for (int i0 = 0; i0 < 32; i0 += 4) {
+                    const int i = i0 + sub;
+                    const int t = __shfl_sync(0xffffffffu, src, i);
+                    const float4 val = tile4[i * 8 + (k4 ^ (i & 7))];
+                    if (t >= 0) atomicAdd(reinterpret_cast<float4 *>(ocol + (int64_t)t * p.N), val);
+                }
+                __syncwarp();
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" : : "r"(tmem), "r"(kFTmemCols) : "memory");
+}
+
 __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
@@ -336,15 +570,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// A [rows_total, inner] bf16 row-major matrix read in (box_rows x 64) tiles with 128-byte swizzle.
-bool make_map(CUtensorMap *map, const void *ptr, int64_t rows_total, int inner, int box_rows) {
+// A [rows_total, inner] row-major matrix (bf16, or one byte per element when fp8) read in
+// (box_rows x 128 bytes) tiles with 128-byte swizzle.
+bool make_map(CUtensorMap *map, const void *ptr, int64_t rows_total, int inner, int box_rows, bool fp8) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const int esize = fp8 ? 1 : 2;
     const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows_total};
-    const cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kGK, (cuuint32_t)box_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)inner * esize};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / esize), (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+    return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr),
+              dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -352,24 +589,31 @@ bool make_map(CUtensorMap *map, const void *ptr, int64_t rows_total, int inner, 
 }  // namespace
 
 cudaError_t launch_gemm_combine(const GemmCombineArgs &g, int num_sms, cudaStream_t s) {
-    // the kernel attribute belongs to each device's context: set it once per device
-    static int ready[64];
+    // the kernel attributes belong to each device's context: set them once per device
+    static int ready[kMaxDevices];
     int dev = 0;
     cudaError_t e0 = cudaGetDevice(&dev);
     if (e0 != cudaSuccess) return e0;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     if (!__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE)) {
-        const cudaError_t e = cudaFuncSetAttribute(gemm_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)kGSmem);
+        cudaError_t e = cudaFuncSetAttribute(gemm_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kGSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemm_combine_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kFSmem);
         if (e != cudaSuccess) return e;
         __atomic_store_n(&ready[dev], 1, __ATOMIC_RELEASE);
     }
     CUtensorMap map_a, map_b;
-    if (!make_map(&map_a, g.act, g.cap, g.p.I, kGM) || !make_map(&map_b, g.w, (int64_t)g.p.E * g.p.N, g.p.I, kGN))
+    if (!make_map(&map_a, g.act, g.cap, g.p.I, kGM, g.fp8) ||
+        !make_map(&map_b, g.w, (int64_t)g.p.E * g.p.N, g.p.I, kGN, g.fp8))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaMemsetAsync(g.p.out_acc, 0, sizeof(float) * (size_t)g.T * g.p.N, s);
     if (e != cudaSuccess) return e;
-    gemm_combine_kernel<<<num_sms, kGThreads, kGSmem, s>>>(map_a, map_b, g.p);
+    if (g.fp8)
+        gemm_combine_fp8_kernel<<<num_sms, kFThreads, kFSmem, s>>>(map_a, map_b, g.p);
+    else
+        gemm_combine_kernel<<<num_sms, kGThreads, kGSmem, s>>>(map_a, map_b, g.p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t n8 = (int64_t)g.T * g.p.N / 8;

@@ -418,6 +418,33 @@ EP_API int ep_expert_combine(const ep_handle *h, const void *act, int32_t inner,
                              const float *topk_weights, float *out_acc, void *out, ep_stream_t stream);
 
 /*
+ * The same expert GEMM and fused combine with FP8 operands: the rows are the
+ * E4M3 codes and fp32 dequantisation scales that ep_dispatch_fp8 writes
+ * (a row restores as code * scale per 128 columns, "2kiu.com/news/5702702"
+ * section 2.3), and each expert matrix is E4M3 with one fp32 scale per
+ * 128 x 128 block (per-block scaling, "m.nlpx.cn/news/135159" section 4.1;
+ * the grouped FP8 expert GEMM that consumes the dispatch in "lesson14_deepep"
+ * section 3).
+ *   out[t, n] = bf16_rn( sum_k topk_weights[t,k] * sum_i A[r,i] * W_e[n,i] ),
+ *   r = pos[t,k], e = topk_idx[t,k],
+ *   A[r,i] = act_q[r,i] * scale(r, i/128),  W_e[n,i] = w_q[e,n,i] * w_scales[e, n/128, i/128].
+ * act_q [capacity, inner] E4M3 in h's received-row layout; act_scales in h's
+ * scale layout (ep_set_scale_layout: row-major [capacity, inner/128], or
+ * column-major with the TMA-aligned leading dimension), as ep_dispatch_fp8
+ * writes them for hidden == inner; w_q [E, n_out, inner] E4M3; w_scales
+ * [E, n_out/128, inner/128] fp32; topk_weights, out_acc and out as in
+ * ep_expert_combine.  The tensor cores multiply E4M3 (tcgen05 kind::f8f6f4)
+ * one 128-deep block at a time; each block's fp32 product is scaled by its
+ * two scales and summed in fp32.  Needs expert_alignment % 128 == 0,
+ * inner % 128 == 0, n_out % 256 == 0, 16-byte aligned act_q, w_q, out_acc and
+ * out, 4-byte aligned scales; else EP_ERR_ARG.  Same ordering caveat and
+ * launches as ep_expert_combine.
+ */
+EP_API int ep_expert_combine_fp8(const ep_handle *h, const uint8_t *act_q, const float *act_scales, int32_t inner,
+                                 const uint8_t *w_q, const float *w_scales, int32_t n_out,
+                                 const float *topk_weights, float *out_acc, void *out, ep_stream_t stream);
+
+/*
  * Peer-memory exchange between the GPUs of a node.  One process per GPU, R =
  * the number of GPUs, rank r owning experts [r*L, (r+1)*L).  This is the
  * exchange step of DeepEP's normal mode done inside the kernels: tokens

@@ -428,6 +428,8 @@ int oracle_expert_combine_fp8(int32_t T, int32_t K, int32_t I, int32_t N, int32_
     if (T < 0 || K <= 0 || I <= 0 || N <= 0 || E <= 0 || rows < 0) return ORACLE_BAD_ARG;
     if (I % 128 != 0 || N % 128 != 0 || scale_ld < 0 || (scale_ld > 0 && scale_ld < rows)) return ORACLE_BAD_ARG;
     const int32_t IB = I / 128, NB = N / 128;
+    double value[256];                    /* e4m3_value of every code, looked up below */
+    for (int c = 0; c < 256; ++c) value[c] = e4m3_value((uint8_t)c);
     for (int32_t j = 0; j < n_sel; ++j) {
         int32_t t = sel_tokens ? sel_tokens[j] : j;
         if (t < 0 || t >= T) return ORACLE_BAD_ARG;
@@ -449,7 +451,7 @@ int oracle_expert_combine_fp8(int32_t T, int32_t K, int32_t I, int32_t N, int32_
                     double sa = scale_ld > 0 ? (double)act_scale[(int64_t)b * scale_ld + r]
                                              : (double)act_scale[(int64_t)r * IB + b];
                     double sw = (double)se[(int64_t)(n / 128) * IB + b];
-                    acc += (e4m3_value(a[i]) * sa) * (e4m3_value(we[(int64_t)n * I + i]) * sw);
+                    acc += (value[a[i]] * sa) * (value[we[(int64_t)n * I + i]] * sw);
                 }
                 o[n] += wk * acc;
             }

@@ -91,7 +91,7 @@ MUTANTS = {
     "fp8 gemm: expert block scale transposed": (
         "se[(int64_t)(n / 128) * IB + b]", "se[(int64_t)b * NB + n / 128]"),
     "fp8 gemm: expert block scale dropped": (
-        "(e4m3_value(we[(int64_t)n * I + i]) * sw)", "(e4m3_value(we[(int64_t)n * I + i]) + 0.0 * sw)"),
+        "(value[we[(int64_t)n * I + i]] * sw)", "(value[we[(int64_t)n * I + i]] + 0.0 * sw)"),
     "padding row not zeroed": (
         "            memset(dst, 0, sizeof(uint16_t) * (size_t)H);\n",
         "            memset(dst, 0, sizeof(uint16_t) * (size_t)(H / 2));\n"),
