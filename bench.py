@@ -673,6 +673,18 @@ def run_cuda(args, world, rank, local):
         for name, mode in PER_CONFIG:
             per_config[name + ("" if mode == "normal" else "_" + mode)] = config_summary(
                 name, mode, args, dev, rank, stream, peak, n, args.warmup)
+        # the expert GEMM with the fused combine, both operand types (tensor-bound)
+        flush_g = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        for fp8 in (False, True):
+            o = expert_gemm_inputs(dev, fp8, rank)
+            ms = time_expert_gemm(o, n, args.warmup, flush_g, stream)
+            entry = expert_gemm_summary(o, ms)
+            entry["device_status"] = int(ep.ep_get_status(o["h"]))
+            per_config["expert_gemm_" + ("e4m3" if fp8 else "bf16")] = entry
+            ep.ep_handle_destroy(o["h"])
+            del o
+        del flush_g
+        torch.cuda.empty_cache()
 
     if rank == 0:
         line = {

@@ -326,7 +326,14 @@ constexpr int kFStages = 4;
 constexpr uint32_t kFABytes = kGM * kFK;              // 16 KB
 constexpr uint32_t kFBBytes = kGN * kFK;              // 32 KB
 constexpr int kFEpiWarps = 8;                         // 4 lane quarters x 2 column halves
-constexpr int kFThreads = 64 + 32 * kFEpiWarps;
+constexpr int kFEpiWarp0 = 4;                         // epilogue warps are the 2nd and 3rd warpgroups
+constexpr int kFThreads = 32 * (kFEpiWarp0 + kFEpiWarps);
+// Register split (setmaxnreg, per warpgroup): the launch gives 384 threads x 168;
+// the producer warpgroup drops to 40 and the two epilogue warpgroups rise to 232
+// (128 x 40 + 256 x 232 = 384 x 168), room for 128 running sums and 64 loaded columns.
+constexpr int kFRegsLaunch = 168, kFRegsLow = 40, kFRegsHigh = 232;
+static_assert(128 * kFRegsLow + 256 * kFRegsHigh <= kFThreads * kFRegsLaunch, "register split exceeds the launch");
+constexpr int kFLdBatch = 4;                          // 16-column TMEM loads in flight per wait
 constexpr int kFHalf = kGN / 2;                       // columns per epilogue thread
 constexpr uint32_t kFTmemCols = 2 * kGN;              // two partial buffers
 constexpr size_t kFSmem = 1024 + kFStages * (size_t)(kFABytes + kFBBytes) + kFEpiWarps * kGStageT + 256;
@@ -353,6 +360,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
           "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" : : : "memory");
+}
+
+// 16 columns of this lane, no wait: the caller waits with tmem_wait_ld and
+// then passes the registers through tmem_fence_regs before using them.
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t *v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" : : : "memory"); }
+// Orders every use of the 16 registers after the preceding (volatile) wait.
+__device__ __forceinline__ void tmem_fence_regs(uint32_t *v) {
+    asm volatile(""
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                   "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                   "+r"(v[15]));
 }
 
 __global__ void __launch_bounds__(kFThreads, 1)
@@ -401,65 +427,68 @@ __global__ void __launch_bounds__(kFThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-
-    if (warp == 0) {
-        // ---- TMA producer ----
-        if (lane == 0) {
-            int it = 0;
-            for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
-                const GemmTile g = tile_coords(p.eoff, p.E, n_blocks, tile);
-                for (int kb = 0; kb < k_blocks; ++kb, ++it) {
-                    const int s = it % kFStages, use = it / kFStages;
-                    if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1, p.wait_limit_ns)) {
-                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                        *s_abort = 1;
-                        break;
+    if (warp < kFEpiWarp0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" : : "n"(kFRegsLow));
+        if (warp == 0) {
+            // ---- TMA producer ----
+            if (lane == 0) {
+                int it = 0;
+                for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
+                    const GemmTile g = tile_coords(p.eoff, p.E, n_blocks, tile);
+                    for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+                        const int s = it % kFStages, use = it / kFStages;
+                        if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1, p.wait_limit_ns)) {
+                            atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                            *s_abort = 1;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[s], kFABytes + kFBBytes);
+                        tma_load_2d(sA + s * kFABytes, &map_a, kb * kFK, g.m * kGM, &full[s]);
+                        tma_load_2d(sB + s * kFBBytes, &map_b, kb * kFK, g.e * p.N + g.n * kGN, &full[s]);
                     }
-                    mbar_arrive_expect_tx(&full[s], kFABytes + kFBBytes);
-                    tma_load_2d(sA + s * kFABytes, &map_a, kb * kFK, g.m * kGM, &full[s]);
-                    tma_load_2d(sB + s * kFBBytes, &map_b, kb * kFK, g.e * p.N + g.n * kGN, &full[s]);
                 }
+                if (*s_abort)
+                    for (int j = max(0, it - kFStages); j < it; ++j)
+                        mbar_wait_bounded(&full[j % kFStages], (j / kFStages) & 1, p.wait_limit_ns);
             }
-            if (*s_abort)
-                for (int j = max(0, it - kFStages); j < it; ++j)
-                    mbar_wait_bounded(&full[j % kFStages], (j / kFStages) & 1, p.wait_limit_ns);
-        }
-    } else if (warp == 1) {
-        // ---- MMA issuer: one partial product per k-block, alternating TMEM buffers ----
-        if (lane == 0) {
-            int it = 0;
-            for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
-                bool ok = true;
-                for (int kb = 0; kb < k_blocks; ++kb, ++it) {
-                    const int j = it & 1, juse = it >> 1, s = it % kFStages;
-                    if (juse > 0 && !mbar_wait_bounded(&part_empty[j], (juse - 1) & 1, p.wait_limit_ns)) {
-                        ok = false;
-                    } else if (!mbar_wait_bounded(&full[s], (it / kFStages) & 1, p.wait_limit_ns)) {
-                        ok = false;
+        } else if (warp == 1) {
+            // ---- MMA issuer: one partial product per k-block, alternating TMEM buffers ----
+            if (lane == 0) {
+                int it = 0;
+                for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
+                    bool ok = true;
+                    for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+                        const int j = it & 1, juse = it >> 1, s = it % kFStages;
+                        if (juse > 0 && !mbar_wait_bounded(&part_empty[j], (juse - 1) & 1, p.wait_limit_ns)) {
+                            ok = false;
+                        } else if (!mbar_wait_bounded(&full[s], (it / kFStages) & 1, p.wait_limit_ns)) {
+                            ok = false;
+                        }
+                        if (!ok) {
+                            atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
+                            *s_abort = 1;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d = tmem + (uint32_t)(j * kGN);
+                        const uint64_t a = umma_desc_k_sw128(smem_u32(sA + s * kFABytes));
+                        const uint64_t b = umma_desc_k_sw128(smem_u32(sB + s * kFBBytes));
+    #pragma unroll
+                        for (int kk = 0; kk < kFK / 32; ++kk)   // 32 E4M3 = 32 bytes = 2 descriptor units
+                            umma_e4m3(d, a + 2 * kk, b + 2 * kk, kk != 0);
+                        umma_commit(&empty[s]);
+                        umma_commit(&part_full[j]);
                     }
-                    if (!ok) {
-                        atomicOr(p.status, EP_DEV_WAIT_TIMEOUT);
-                        *s_abort = 1;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t d = tmem + (uint32_t)(j * kGN);
-                    const uint64_t a = umma_desc_k_sw128(smem_u32(sA + s * kFABytes));
-                    const uint64_t b = umma_desc_k_sw128(smem_u32(sB + s * kFBBytes));
-#pragma unroll
-                    for (int kk = 0; kk < kFK / 32; ++kk)   // 32 E4M3 = 32 bytes = 2 descriptor units
-                        umma_e4m3(d, a + 2 * kk, b + 2 * kk, kk != 0);
-                    umma_commit(&empty[s]);
-                    umma_commit(&part_full[j]);
+                    if (!ok) break;
                 }
-                if (!ok) break;
+                umma_commit(drain);
+                mbar_wait_bounded(drain, 0, p.wait_limit_ns);
             }
-            umma_commit(drain);
-            mbar_wait_bounded(drain, 0, p.wait_limit_ns);
         }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" : : "n"(kFRegsHigh));
         // ---- epilogue: fold the scaled partials, then combine ----
-        const int ew = warp - 2;
+        const int ew = warp - kFEpiWarp0;
         const int q = warp & 3;                    // TMEM lanes 32q .. 32q+31
         const int h = ew >> 2;                     // column half of the tile
         const int IB = p.I / kFK, NB = p.N / 128;
@@ -497,11 +526,19 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 }
                 tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < kFHalf / 16; ++c) {
-                    uint32_t v[16];
-                    tmem_ld16(lane_base + (uint32_t)(j * kGN + c * 16), v);
+                for (int c0 = 0; c0 < kFHalf / 16; c0 += kFLdBatch) {
+                    uint32_t v[kFLdBatch][16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[c * 16 + i] = fmaf(sc, __uint_as_float(v[i]), acc[c * 16 + i]);
+                    for (int c = 0; c < kFLdBatch; ++c)
+                        tmem_ld16_async(lane_base + (uint32_t)(j * kGN + (c0 + c) * 16), v[c]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < kFLdBatch; ++c) {
+                        tmem_fence_regs(v[c]);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            acc[(c0 + c) * 16 + i] = fmaf(sc, __uint_as_float(v[c][i]), acc[(c0 + c) * 16 + i]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
