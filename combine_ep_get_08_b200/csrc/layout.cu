@@ -542,8 +542,10 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
         const int e = tid / P, part = tid % P, rows = kLayoutWarps / P;
         const bool act = e < E;
         int local = 0;
-        if (act)
+        if (act) {
+#pragma unroll 8
             for (int w = part * rows; w < (part + 1) * rows; ++w) local += s_cnt[w * ES + e];
+        }
         int incl = local;
         for (int o = 1; o < P; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, o, P);
@@ -562,10 +564,17 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
     // distinct tokens per rank and is_token_in_rank rows, from the staged ids
     if (R <= 64 && K <= 32 && (K & (K - 1)) == 0) {
         // a token's K pairs are K consecutive lanes of one warp: each lane
-        // contributes its pair's rank bit and a shuffle OR gives the token's mask
+        // contributes its pair's rank bit and a shuffle OR gives the token's
+        // mask.  Lane j of a token's group then writes words j, j+K, ... of
+        // its is_token_in_rank row and counts ranks j, j+K, ... : the counts
+        // of the warp's tokens are summed by shuffles and added to the
+        // histogram by the group's first K lanes, one address per lane.
         const int span = (npairs + 31) / 32 * 32;
+        const int j = lane & (K - 1);
+        const bool row_words = p.u_in_rank && (R & 3) == 0 && (reinterpret_cast<uintptr_t>(p.u_in_rank) & 3) == 0;
         for (int i = tid; i < span; i += kLayoutThreads) {
-            const int e = i < npairs ? s_ep[i] : -1;
+            const bool tok = i < npairs;
+            const int e = tok ? s_ep[i] : -1;
             const int r = e >= 0 ? s_rk[e] : -1;
             unsigned int lo = (r >= 0 && r < 32) ? 1u << r : 0u;
             unsigned int hi = r >= 32 ? 1u << (r - 32) : 0u;
@@ -573,12 +582,24 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) layout_cluster_kernel(Layou
                 lo |= __shfl_xor_sync(0xffffffffu, lo, o);
                 hi |= __shfl_xor_sync(0xffffffffu, hi, o);
             }
-            if (i < npairs && i % K == 0) {
-                const int t = t_begin + i / K;
-                const unsigned long long mask = ((unsigned long long)hi << 32) | lo;
-                for (unsigned long long m = mask; m; m &= m - 1)
-                    atomicAdd(&s_hist[E + __ffsll((long long)m) - 1], 1);
-                if (p.u_in_rank) write_in_rank_row(p.u_in_rank + (int64_t)t * R, R, mask);
+            const unsigned long long mask = ((unsigned long long)hi << 32) | lo;
+            for (int rb = 0; rb < R; rb += K) {
+                const int rr = rb + j;
+                int c = (tok && rr < R) ? (int)((mask >> rr) & 1ull) : 0;
+                for (int o = K; o < 32; o <<= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+                if (lane < K && rr < R && c) atomicAdd(&s_hist[E + rr], c);
+            }
+            if (tok && p.u_in_rank) {
+                uint8_t *row = p.u_in_rank + (int64_t)(t_begin + i / K) * R;
+                if (row_words) {
+                    for (int w = j; w < R / 4; w += K) {
+                        const unsigned int bits = (unsigned int)(mask >> (4 * w)) & 0xfu;
+                        reinterpret_cast<unsigned int *>(row)[w] = (bits & 1u) | ((bits >> 1) & 1u) << 8 |
+                                                                  ((bits >> 2) & 1u) << 16 | ((bits >> 3) & 1u) << 24;
+                    }
+                } else {
+                    for (int q = j; q < R; q += K) row[q] = (uint8_t)((mask >> q) & 1ull);
+                }
             }
         }
     } else {
