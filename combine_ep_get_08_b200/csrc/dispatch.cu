@@ -374,6 +374,259 @@ __global__ void __launch_bounds__(kThreads, EP_FP8_MINB) dispatch_fp8_kernel(Dis
     }
 }
 
+// ---------------------------------------------------------------------------
+// Layout and dispatch in one launch, for batches too small to fill the GPU
+// (ep_layout_dispatch with fewer than two tokens per SM).  The padded layout
+// of a small batch is cheap enough to compute in every CTA: each CTA reads
+// all T*K ids (an L2 hit after the first), counts every expert and the pairs
+// of the tokens before its own, and scans the padded counts into the expert
+// offsets.  A pair's row is then its expert's offset + the pairs of that
+// expert in earlier tokens + the earlier slots of its own token with the same
+// expert: the (token, k) order of the lesson14_deepep practice task's queues.
+// CTA c handles tokens c, c + G, ...: it writes their routing entries, their
+// is_token_in_rank rows and their copies (the first row is loaded before the
+// counting, so the two overlap); the padding rows of experts c, c + G, ...
+// are written as well; CTA 0 writes the counts and offsets, the last CTA the
+// distinct tokens per rank.  No CTA waits on another.
+// ---------------------------------------------------------------------------
+template <bool FP8, int W>   // W: bf16 elements per thread (FP8) or vector bytes (bf16)
+__global__ void __launch_bounds__(kThreads, 1) layout_dispatch_small_kernel(DispatchParams p, LayoutParams lp) {
+    __shared__ int32_t s_tot[kMaxExperts + 1];   // pairs per expert (later: tokens per rank, CTA 0)
+    __shared__ int32_t s_before[kMaxExperts];    // pairs per expert among tokens [0, upto)
+    __shared__ int32_t s_eoff[kMaxExperts + 1];  // padded expert offsets
+    __shared__ int32_t s_dst[kMaxTopk];
+    __shared__ int32_t s_id[kMaxTopk];          // the current token's ids (-1: none or invalid)
+    __shared__ int16_t s_rk[kMaxExperts];        // rank of expert e (e / L)
+    __shared__ int32_t s_warp[kThreads / 32 + 1];
+    constexpr int EPT = W, TPB = 128 / (FP8 ? W : 128), NW = W / 2;
+    const int E = lp.E, K = lp.K, T = lp.T, R = lp.R, L = lp.L, A = lp.A, H = p.H;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, G = gridDim.x;
+    const int64_t *idx = lp.topk_idx;
+    const uint8_t *x = static_cast<const uint8_t *>(p.x);
+    uint8_t *recv = static_cast<uint8_t *>(p.recv);
+    const int row_bytes = FP8 ? H : H * 2;
+
+    // the first token's row is requested before the counting
+    unsigned int w8[FP8 ? NW : 1];
+    typename Vec<FP8 ? 16 : W>::T v0;
+    const int nthr_row = FP8 ? H / EPT : row_bytes / W;
+    if (blockIdx.x < T && tid < nthr_row) {
+        if constexpr (FP8)
+            Fp8Io<EPT>::load(x + (int64_t)blockIdx.x * H * 2 + (int64_t)tid * EPT * 2, w8);
+        else
+            v0 = Vec<W>::load(x + (int64_t)blockIdx.x * row_bytes + (int64_t)tid * W);
+    }
+
+    for (int e = tid; e < E; e += kThreads) {
+        s_tot[e] = 0;
+        s_before[e] = 0;
+        s_rk[e] = (int16_t)(e / L);
+    }
+    __syncthreads();
+    const int64_t npairs = (int64_t)T * K, nbefore = (int64_t)blockIdx.x * K;
+    bool bad = false;
+    for (int64_t i = tid; i < npairs; i += kThreads) {
+        const int64_t e = __ldg(idx + i);
+        if (e >= 0 && e < E) {
+            atomicAdd(&s_tot[e], 1);
+            if (i < nbefore) atomicAdd(&s_before[e], 1);
+        } else if (e != -1) {
+            bad = true;
+        }
+    }
+    if (bad && blockIdx.x == 0) atomicOr(lp.status, EP_DEV_BAD_EXPERT);
+    __syncthreads();
+    // padded exclusive offsets: per = E / kThreads consecutive experts per thread
+    {
+        const int per = (E + kThreads - 1) / kThreads;
+        const int lo = min(E, tid * per), hi = min(E, lo + per);
+        int sum = 0;
+        for (int e = lo; e < hi; ++e) sum += (s_tot[e] + A - 1) / A * A;
+        int inc = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        if (lane == 31) s_warp[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            const int wv = lane < kThreads / 32 ? s_warp[lane] : 0;
+            int wi = wv;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += v;
+            }
+            if (lane < kThreads / 32) s_warp[lane] = wi - wv;
+            if (lane == kThreads / 32 - 1) s_warp[kThreads / 32] = wi;
+        }
+        __syncthreads();
+        int run = s_warp[warp] + inc - sum;
+        for (int e = lo; e < hi; ++e) {
+            s_eoff[e] = run;
+            run += (s_tot[e] + A - 1) / A * A;
+        }
+        if (tid == 0) s_eoff[E] = s_warp[kThreads / 32];
+    }
+    __syncthreads();
+
+    const int NB = H / 128;
+    int upto = blockIdx.x;
+    for (int t = blockIdx.x; t < T; t += G) {
+        if (t > upto) {   // pairs of the tokens between this CTA's previous token and t
+            for (int64_t i = (int64_t)upto * K + tid; i < (int64_t)t * K; i += kThreads) {
+                const int64_t e = __ldg(idx + i);
+                if (e >= 0 && e < E) atomicAdd(&s_before[e], 1);
+            }
+            upto = t;
+            __syncthreads();
+            if (tid < nthr_row) {   // this token's row (the first one was loaded before the counting)
+                if constexpr (FP8)
+                    Fp8Io<EPT>::load(x + (int64_t)t * H * 2 + (int64_t)tid * EPT * 2, w8);
+                else
+                    v0 = Vec<W>::load(x + (int64_t)t * row_bytes + (int64_t)tid * W);
+            }
+        }
+        const int64_t *row = idx + (int64_t)t * K;
+        if (tid < K) {
+            const int64_t e = __ldg(row + tid);
+            s_id[tid] = (e >= 0 && e < E) ? (int)e : -1;
+        }
+        __syncthreads();
+        if (tid < K) {
+            const int e = s_id[tid];
+            int dst = -1;
+            if (e >= 0) {
+                int same = 0;
+                for (int k2 = 0; k2 < tid; ++k2) same += s_id[k2] == e;
+                dst = s_eoff[e] + s_before[e] + same;
+                lp.row_src[dst] = t;
+                lp.row_slot[dst] = tid;
+                if (lp.topk_weights) lp.row_weight[dst] = __ldg(lp.topk_weights + (int64_t)t * K + tid);
+            }
+            lp.pos[(int64_t)t * K + tid] = dst;
+            s_dst[tid] = dst;
+        }
+        if (lp.u_in_rank) {
+            for (int r = tid; r < R; r += kThreads) {
+                uint8_t in = 0;
+                for (int k = 0; k < K; ++k) {
+                    const int e = s_id[k];
+                    if (e >= 0 && s_rk[e] == r) in = 1;
+                }
+                lp.u_in_rank[(int64_t)t * R + r] = in;
+            }
+        }
+        __syncthreads();
+        if constexpr (FP8) {
+            const uint8_t *xr = x + (int64_t)t * H * 2;
+            for (int g0 = 0; g0 < nthr_row; g0 += kThreads) {
+                const int g = g0 + tid;
+                const bool act = g < nthr_row;
+                if (g0 > 0) {
+                    if (act) {
+                        Fp8Io<EPT>::load(xr + (int64_t)g * EPT * 2, w8);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < NW; ++i) w8[i] = 0;
+                    }
+                } else if (!act) {
+#pragma unroll
+                    for (int i = 0; i < NW; ++i) w8[i] = 0;
+                }
+                unsigned int q[8];
+                const float scale = quantize_block<TPB, NW>(w8, q);
+                if (act) {
+                    const int b = g / TPB;
+                    const bool lead = (g % TPB) == 0;
+                    for (int k = 0; k < K; ++k) {
+                        const int dst = s_dst[k];
+                        if (dst < 0) continue;
+                        Fp8Io<EPT>::store(recv + (int64_t)dst * H + (int64_t)g * EPT, q);
+                        if (lead) p.recv_scale[scale_index(p, dst, b, NB)] = scale;
+                    }
+                }
+            }
+        } else {
+            const uint8_t *xr = x + (int64_t)t * row_bytes;
+            for (int v = tid; v < nthr_row; v += kThreads) {
+                const typename Vec<W>::T val = v == tid ? v0 : Vec<W>::load(xr + (int64_t)v * W);
+                for (int k = 0; k < K; ++k) {
+                    const int dst = s_dst[k];
+                    if (dst >= 0) Vec<W>::store(recv + (int64_t)dst * row_bytes + (int64_t)v * W, val);
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // padding rows of experts blockIdx.x, blockIdx.x + G, ...
+    for (int e = blockIdx.x; e < E; e += G) {
+        const int r0 = s_eoff[e] + s_tot[e], r1 = s_eoff[e + 1];
+        for (int r = r0 + tid; r < r1; r += kThreads) {
+            lp.row_src[r] = -1;
+            lp.row_slot[r] = -1;
+            if (lp.topk_weights) lp.row_weight[r] = 0.0f;
+        }
+        for (int r = r0; r < r1; ++r) {
+            uint8_t *o = recv + (int64_t)r * row_bytes;
+            for (int v = tid; v < row_bytes / 16; v += kThreads) st_v4(o + v * 16, make_uint4(0, 0, 0, 0));
+            if constexpr (FP8)
+                for (int b = tid; b < NB; b += kThreads) p.recv_scale[scale_index(p, r, b, NB)] = 0.0f;
+        }
+    }
+
+    if (blockIdx.x == 0) {
+        for (int e = tid; e < E; e += kThreads) {
+            lp.cnt[e] = s_tot[e];
+            if (lp.u_cnt) lp.u_cnt[e] = s_tot[e];
+        }
+        for (int e = tid; e <= E; e += kThreads) {
+            lp.eoff[e] = s_eoff[e];
+            if (lp.u_eoff) lp.u_eoff[e] = s_eoff[e];
+        }
+        for (int r = tid; r <= R; r += kThreads) {
+            lp.roff[r] = s_eoff[r * L];
+            if (lp.u_roff) lp.u_roff[r] = s_eoff[r * L];
+        }
+    }
+    if (blockIdx.x == G - 1) {
+        // distinct tokens per rank, by the last CTA (s_tot is free now)
+        __syncthreads();
+        for (int r = tid; r < R; r += kThreads) s_tot[r] = 0;
+        __syncthreads();
+        for (int t = tid; t < T; t += kThreads) {
+            const int64_t *row = idx + (int64_t)t * K;
+            if (R <= 64) {
+                unsigned long long mask = 0;
+                for (int k = 0; k < K; ++k) {
+                    const int64_t e = __ldg(row + k);
+                    if (e >= 0 && e < E) mask |= 1ull << s_rk[e];
+                }
+                for (unsigned long long m = mask; m; m &= m - 1) atomicAdd(&s_tot[__ffsll((long long)m) - 1], 1);
+            } else {
+                for (int k = 0; k < K; ++k) {
+                    const int64_t e = __ldg(row + k);
+                    if (e < 0 || e >= E) continue;
+                    const int r = s_rk[e];
+                    bool dup = false;
+                    for (int k2 = 0; k2 < k; ++k2) {
+                        const int64_t e2 = __ldg(row + k2);
+                        if (e2 >= 0 && e2 < E && s_rk[e2] == r) dup = true;
+                    }
+                    if (!dup) atomicAdd(&s_tot[r], 1);
+                }
+            }
+        }
+        __syncthreads();
+        for (int r = tid; r < R; r += kThreads) {
+            lp.rank_tok[r] = s_tot[r];
+            if (lp.u_rank_tok) lp.u_rank_tok[r] = s_tot[r];
+        }
+    }
+}
+
 }  // namespace
 
 // Launch that may start while the previous kernel on the stream finishes
@@ -474,6 +727,25 @@ cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream
         const int grid = persistent_grid(units, blocks_per_sm(k, kThreads, 0, &occ16), num_sms);
         return launch_pdl(dispatch_fp8_kernel<16, false>, grid, kThreads, 0, s, p);
     }
+}
+
+// The single-launch layout + dispatch of a small batch (one CTA per token).
+cudaError_t launch_layout_dispatch_small(const DispatchParams &p, const LayoutParams &lp, bool fp8, cudaStream_t s) {
+    const int grid = lp.T;
+    const bool v32 = ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0 &&
+                     (fp8 || p.H % 16 == 0);
+    if (fp8) {
+        if (v32)
+            layout_dispatch_small_kernel<true, 32><<<grid, kThreads, 0, s>>>(p, lp);
+        else
+            layout_dispatch_small_kernel<true, 16><<<grid, kThreads, 0, s>>>(p, lp);
+    } else {
+        if (v32)
+            layout_dispatch_small_kernel<false, 32><<<grid, kThreads, 0, s>>>(p, lp);
+        else
+            layout_dispatch_small_kernel<false, 16><<<grid, kThreads, 0, s>>>(p, lp);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace ep

@@ -418,16 +418,53 @@ static int layout_dispatch_common(ep_handle *h, const int64_t *topk_idx, const f
         !aligned(expert_offsets, 4) || !aligned(rank_offsets, 4))
         return EP_ERR_ARG;
     const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
-    if (c.num_tokens > 0 && c.num_tokens < 2 * sms) {
-        // too few tokens to fill the GPU: the layout kernel, then the register
-        // dispatch (decode: 17.9 us for the two against 31.6 us fused)
-        rc = ep_get_layout(h, topk_idx, topk_weights, num_tokens_per_expert, num_tokens_per_rank,
-                           is_token_in_rank, expert_offsets, rank_offsets, stream);
-        if (rc != EP_OK) return rc;
-        return dispatch_common(h, x, recv, scales, fp8, stream);
-    }
     DeviceGuard g(h->device);
     if (g.err != cudaSuccess) return cuda_fail(g.err, "cudaSetDevice");
+    if (c.num_tokens > 0 && c.num_tokens < 2 * sms) {
+        // too few tokens to fill the GPU: one launch, one CTA per token, each
+        // counting all pairs itself (decode: 17.9 us for the layout kernel and
+        // the register dispatch, 31.6 us for the chunked kernel with look-back)
+        ep::LayoutParams lp{};
+        lp.topk_idx = topk_idx;
+        lp.topk_weights = topk_weights;
+        lp.T = c.num_tokens;
+        lp.K = c.num_topk;
+        lp.E = c.num_experts;
+        lp.R = c.num_ranks;
+        lp.L = c.num_experts / c.num_ranks;
+        lp.A = c.expert_alignment;
+        lp.pos = h->pos;
+        lp.row_src = h->row_src;
+        lp.row_slot = h->row_slot;
+        lp.row_weight = h->row_weight;
+        lp.cnt = h->cnt;
+        lp.rank_tok = h->rank_tok;
+        lp.eoff = h->eoff;
+        lp.roff = h->roff;
+        lp.u_cnt = num_tokens_per_expert;
+        lp.u_rank_tok = num_tokens_per_rank;
+        lp.u_eoff = expert_offsets;
+        lp.u_roff = rank_offsets;
+        lp.u_in_rank = is_token_in_rank;
+        lp.status = h->status;
+        lp.wait_limit_ns = h->wait_limit_ns;
+        ep::DispatchParams p{};
+        p.x = x;
+        p.recv = recv;
+        p.recv_scale = scales;
+        p.scale_ld = h->scale_layout == EP_SCALES_COL_MAJOR_TMA ? (int)((h->cap + 3) / 4 * 4) : 0;
+        p.scale_group_rows = (int)h->cap;
+        p.H = c.hidden;
+        p.T = c.num_tokens;
+        p.K = c.num_topk;
+        p.E = c.num_experts;
+        p.status = h->status;
+        cudaError_t e = ep::launch_layout_dispatch_small(p, lp, fp8, reinterpret_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(layout_dispatch_fp8)" : "launch(layout_dispatch)");
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        h->has_layout = true;
+        return EP_OK;
+    }
     ep::LbParams p = lb_params(h, x, recv, scales, 1);
     p.topk_idx = topk_idx;
     p.topk_weights = topk_weights;

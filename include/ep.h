@@ -236,9 +236,10 @@ EP_API int ep_dispatch_fp8(const ep_handle *h, const void *x, void *recv_q, floa
  * set by ep_set_wait_limit, the first chunk never publishes its counts: a
  * test hook that makes the waits of the chunks after it run out.
  * A batch too small to fill the GPU (fewer than two tokens per SM, within
- * the ep_set_sm_limit cap) runs as ep_get_layout followed by ep_dispatch
- * instead, which is faster at that size.  T must be below 2^22 (else
- * EP_ERR_UNSUPPORTED).
+ * the ep_set_sm_limit cap) takes one launch instead: one CTA per token, each
+ * counting all T*K pairs itself (an L2 hit after the first CTA) and scanning
+ * the padded counts, so no CTA waits on another; the same outputs.  T must be
+ * below 2^22 (else EP_ERR_UNSUPPORTED).
  * Defined by: the same passages as ep_get_layout and ep_dispatch (the
  * queue order of the "lesson14_deepep" moe_dispatch loop; do_expand,
  * expert_alignment and do_zero_padding of bowenzhou.top "deepep/01-overview"

@@ -143,9 +143,11 @@ CASES = [
     dict(T=20000, H=64, E=64, R=8, K=8, A=4, router="topk", seed=27),         # 148 chunks, 10 super-chunks
     dict(T=3000, H=128, E=128, R=8, K=64, A=1, router="topk", seed=29),       # 4096-pair chunks
     dict(T=400, H=128, E=1024, R=128, K=64, A=2, router="topk", seed=34),     # max E and K in the fused kernel
+    dict(T=100, H=512, E=64, R=8, K=8, A=16, router="zipf", seed=35),        # small batch, padding rows
+    dict(T=295, H=7168, E=256, R=32, K=8, A=1, router="topk", seed=36),       # largest small batch on 148 SMs
 ]
-# Batches of fewer than two tokens per SM (tiny, T = 1, 33, 300 above) run as
-# ep_get_layout + ep_dispatch inside ep_layout_dispatch; the same checks apply.
+# Batches of fewer than two tokens per SM (tiny, T = 1, 33, 100, 295 above)
+# take the single-launch small-batch kernel; the same checks apply.
 
 
 @pytest.mark.parametrize("spec", CASES, ids=lambda s: s.get("name") or f"T{s['T']}H{s['H']}E{s['E']}K{s['K']}A{s['A']}")
@@ -195,6 +197,63 @@ def test_fused_masked_and_repeated():
     wl.topk_idx = idx
     run_fused(wl, False)
     run_fused(wl, True)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_small_batch_masked_and_repeated(fp8):
+    """The single-launch small-batch kernel with -1 slots, a token with no
+    expert and repeated experts inside tokens."""
+    wl = workloads.generate(None, T=120, H=1024, E=64, R=8, K=8, A=4, router="topk", seed=72)
+    idx = wl.topk_idx.clone()
+    g = torch.Generator().manual_seed(6)
+    idx[torch.rand(idx.shape, generator=g) < 0.25] = -1
+    idx[3, :] = -1
+    idx[10:20, 1] = idx[10:20, 0]
+    wl.topk_idx = idx
+    run_fused(wl, fp8)
+
+
+def test_small_batch_column_major_scales():
+    """Column-major (TMA-aligned) scales from the small-batch kernel."""
+    dev = torch.device("cuda")
+    wl = workloads.generate(None, T=90, H=1024, E=32, R=4, K=4, A=8, router="topk", seed=73)
+    idx, w = wl.topk_idx.numpy(), wl.topk_weights.numpy()
+    o = oracle.layout(idx, wl.E, wl.R, wl.A, topk_weights=w)
+    cfg = ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A)
+    h = ep.ep_handle_create(cfg)
+    try:
+        ep.ep_set_scale_layout(h, ep.EP_SCALES_COL_MAJOR_TMA)
+        cap = ep.ep_capacity_rows(cfg)
+        ld = (cap + 3) // 4 * 4
+        q = torch.full((cap, wl.H), 0x5A, dtype=torch.uint8, device=dev)
+        s = torch.full((ep.ep_scale_buffer_floats(cfg, ep.EP_SCALES_COL_MAJOR_TMA),), -3.0, dtype=torch.float32,
+                       device=dev)
+        ep.ep_layout_dispatch_fp8(h, wl.topk_idx.to(dev), wl.topk_weights.to(dev), wl.x.to(dev), q, s)
+        assert ep.ep_get_status(h) == 0
+        oq, osc = oracle.dispatch_fp8(workloads.bf16_bits(wl.x), o.row_src)
+        np.testing.assert_array_equal(q[:o.rows].cpu().numpy(), oq)
+        got = s.cpu().numpy().reshape(wl.H // 128, ld)[:, :o.rows].T
+        np.testing.assert_array_equal(got.view(np.uint32), osc.view(np.uint32))
+    finally:
+        ep.ep_handle_destroy(h)
+
+
+def test_small_batch_invalid_id_sets_status():
+    """An id outside [0, E) other than -1 sets EP_DEV_BAD_EXPERT in the
+    small-batch kernel too, and its pair gets no row."""
+    dev = torch.device("cuda")
+    wl = workloads.generate(None, T=50, H=256, E=16, R=4, K=2, A=1, router="uniform", seed=4)
+    idx = wl.topk_idx.clone()
+    idx[7, 1] = 16
+    h = ep.ep_handle_create(ep.make_config(wl.T, wl.H, wl.E, wl.R, wl.K, wl.A))
+    try:
+        fused(h, wl, False, idx_d=idx.to(dev))
+        assert ep.ep_get_status(h) & ep.EP_DEV_BAD_EXPERT
+        pos = torch.empty((wl.T, wl.K), dtype=torch.int32, device=dev)
+        ep.ep_copy_routing(h, pos)
+        assert int(pos[7, 1]) == -1
+    finally:
+        ep.ep_handle_destroy(h)
 
 
 def test_fused_invalid_id_sets_status():
