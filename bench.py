@@ -1241,7 +1241,8 @@ def ncu_ingest(rep: str, workload: str) -> int:
     per_role = {}
     for r in rows[2:]:
         name = r[col["Kernel Name"]]
-        role = ("layout" if "layout" in name else "dispatch" if "dispatch" in name
+        # a kernel that dispatches (the layout fused in or not) is the dispatch
+        role = ("dispatch" if "dispatch" in name else "layout" if "layout" in name
                 else "combine" if "combine" in name else None)
         if role is None:
             continue

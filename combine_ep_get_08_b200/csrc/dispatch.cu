@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, EP_FP8_MINB) dispatch_fp8_kernel(Dis
 // distinct tokens per rank.  No CTA waits on another.
 // ---------------------------------------------------------------------------
 template <bool FP8, int W>   // W: bf16 elements per thread (FP8) or vector bytes (bf16)
-__global__ void __launch_bounds__(kThreads, 1) layout_dispatch_small_kernel(DispatchParams p, LayoutParams lp) {
+__device__ __forceinline__ void small_layout_dispatch(const DispatchParams &p, const LayoutParams &lp) {
     __shared__ int32_t s_tot[kMaxExperts + 1];   // pairs per expert (later: tokens per rank, CTA 0)
     __shared__ int32_t s_before[kMaxExperts];    // pairs per expert among tokens [0, upto)
     __shared__ int32_t s_eoff[kMaxExperts + 1];  // padded expert offsets
@@ -405,12 +405,14 @@ __global__ void __launch_bounds__(kThreads, 1) layout_dispatch_small_kernel(Disp
     const uint8_t *x = static_cast<const uint8_t *>(p.x);
     uint8_t *recv = static_cast<uint8_t *>(p.recv);
     const int row_bytes = FP8 ? H : H * 2;
+    const bool copy = x != nullptr;   // false: the layout alone (ep_get_layout of a small batch)
+    pdl_launch_dependents();          // a kernel launched next may start its set-up now
 
     // the first token's row is requested before the counting
     unsigned int w8[FP8 ? NW : 1];
     typename Vec<FP8 ? 16 : W>::T v0;
     const int nthr_row = FP8 ? H / EPT : row_bytes / W;
-    if (blockIdx.x < T && tid < nthr_row) {
+    if (copy && blockIdx.x < T && tid < nthr_row) {
         if constexpr (FP8)
             Fp8Io<EPT>::load(x + (int64_t)blockIdx.x * H * 2 + (int64_t)tid * EPT * 2, w8);
         else
@@ -481,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) layout_dispatch_small_kernel(Disp
             }
             upto = t;
             __syncthreads();
-            if (tid < nthr_row) {   // this token's row (the first one was loaded before the counting)
+            if (copy && tid < nthr_row) {   // this token's row (the first one was loaded before the counting)
                 if constexpr (FP8)
                     Fp8Io<EPT>::load(x + (int64_t)t * H * 2 + (int64_t)tid * EPT * 2, w8);
                 else
@@ -519,6 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) layout_dispatch_small_kernel(Disp
             }
         }
         __syncthreads();
+        if (!copy) continue;
         if constexpr (FP8) {
             const uint8_t *xr = x + (int64_t)t * H * 2;
             for (int g0 = 0; g0 < nthr_row; g0 += kThreads) {
@@ -569,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) layout_dispatch_small_kernel(Disp
             lp.row_slot[r] = -1;
             if (lp.topk_weights) lp.row_weight[r] = 0.0f;
         }
-        for (int r = r0; r < r1; ++r) {
+        for (int r = r0; r < r1 && copy; ++r) {
             uint8_t *o = recv + (int64_t)r * row_bytes;
             for (int v = tid; v < row_bytes / 16; v += kThreads) st_v4(o + v * 16, make_uint4(0, 0, 0, 0));
             if constexpr (FP8)
@@ -625,6 +628,16 @@ __global__ void __launch_bounds__(kThreads, 1) layout_dispatch_small_kernel(Disp
             if (lp.u_rank_tok) lp.u_rank_tok[r] = s_tot[r];
         }
     }
+}
+
+template <bool FP8, int W>
+__global__ void __launch_bounds__(kThreads, 1) layout_dispatch_small_kernel(DispatchParams p, LayoutParams lp) {
+    small_layout_dispatch<FP8, W>(p, lp);
+}
+
+// The same without the copy (p.x == nullptr): ep_get_layout of a small batch.
+__global__ void __launch_bounds__(kThreads, 1) layout_small_kernel(DispatchParams p, LayoutParams lp) {
+    small_layout_dispatch<false, 16>(p, lp);
 }
 
 }  // namespace
@@ -729,9 +742,15 @@ cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream
     }
 }
 
-// The single-launch layout + dispatch of a small batch (one CTA per token).
-cudaError_t launch_layout_dispatch_small(const DispatchParams &p, const LayoutParams &lp, bool fp8, cudaStream_t s) {
-    const int grid = lp.T;
+// The single-launch layout + dispatch of a small batch (one CTA per token, at
+// most num_sms CTAs); with p.x == nullptr the layout alone.
+cudaError_t launch_layout_dispatch_small(const DispatchParams &p, const LayoutParams &lp, bool fp8, int num_sms,
+                                         cudaStream_t s) {
+    const int grid = lp.T < num_sms ? lp.T : num_sms;
+    if (p.x == nullptr) {
+        layout_small_kernel<<<grid, kThreads, 0, s>>>(p, lp);
+        return cudaGetLastError();
+    }
     const bool v32 = ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31) == 0 &&
                      (fp8 || p.H % 16 == 0);
     if (fp8) {

@@ -289,7 +289,21 @@ EP_API int ep_get_layout(ep_handle *h, const int64_t *topk_idx, const float *top
     p.status = h->status;
     p.wait_limit_ns = h->wait_limit_ns;
     p.barrier_extra = h->barrier_extra;
-    cudaError_t e = ep::launch_layout(p, h->plan, reinterpret_cast<cudaStream_t>(stream));
+    const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
+    cudaError_t e;
+    if (c.num_tokens > 0 && c.num_tokens < 2 * sms) {
+        // fewer than two tokens per SM: one CTA per token, each counting all
+        // pairs itself (the small-batch kernel without its copy)
+        ep::DispatchParams d{};
+        d.H = c.hidden;
+        d.T = c.num_tokens;
+        d.K = c.num_topk;
+        d.E = c.num_experts;
+        d.status = h->status;
+        e = ep::launch_layout_dispatch_small(d, p, false, sms, reinterpret_cast<cudaStream_t>(stream));
+    } else {
+        e = ep::launch_layout(p, h->plan, reinterpret_cast<cudaStream_t>(stream));
+    }
     if (e != cudaSuccess) return cuda_fail(e, "launch(layout)");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     h->has_layout = true;
@@ -459,7 +473,7 @@ static int layout_dispatch_common(ep_handle *h, const int64_t *topk_idx, const f
         p.K = c.num_topk;
         p.E = c.num_experts;
         p.status = h->status;
-        cudaError_t e = ep::launch_layout_dispatch_small(p, lp, fp8, reinterpret_cast<cudaStream_t>(stream));
+        cudaError_t e = ep::launch_layout_dispatch_small(p, lp, fp8, sms, reinterpret_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return cuda_fail(e, fp8 ? "launch(layout_dispatch_fp8)" : "launch(layout_dispatch)");
         g_launches.fetch_add(1, std::memory_order_relaxed);
         h->has_layout = true;

@@ -205,8 +205,10 @@ const void *layout_kernel_ptr();
 cudaError_t launch_dispatch_bf16(const DispatchParams &p, int num_sms, cudaStream_t s);
 cudaError_t launch_dispatch_fp8(const DispatchParams &p, int num_sms, cudaStream_t s);
 // Layout and dispatch in one launch for batches of fewer than two tokens per
-// SM: one CTA per token, each counting all pairs itself (dispatch.cu).
-cudaError_t launch_layout_dispatch_small(const DispatchParams &p, const LayoutParams &lp, bool fp8, cudaStream_t s);
+// SM: one CTA per token (at most num_sms), each counting all pairs itself
+// (dispatch.cu); p.x == nullptr: the layout alone.
+cudaError_t launch_layout_dispatch_small(const DispatchParams &p, const LayoutParams &lp, bool fp8, int num_sms,
+                                         cudaStream_t s);
 // Low-latency static layout + copy in one launch (p.ll_M > 0).
 cudaError_t launch_ll_dispatch(const DispatchParams &p, bool fp8, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams &p, int num_sms, cudaStream_t s);

@@ -213,6 +213,15 @@ def test_small_batch_masked_and_repeated(fp8):
     run_fused(wl, fp8)
 
 
+@pytest.mark.parametrize("fp8", [False, True])
+def test_small_batch_fewer_ctas_than_tokens(fp8):
+    """Under a 7-SM cap a 13-token batch still takes the small-batch kernel
+    (fewer than two tokens per SM) with 7 CTAs: six of them handle two tokens
+    each and carry their counts of earlier pairs from one token to the next."""
+    wl = workloads.generate(None, T=13, H=512, E=16, R=4, K=4, A=4, router="topk", seed=74)
+    run_fused(wl, fp8, sm_limit=7)
+
+
 def test_small_batch_column_major_scales():
     """Column-major (TMA-aligned) scales from the small-batch kernel."""
     dev = torch.device("cuda")

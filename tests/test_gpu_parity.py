@@ -11,7 +11,7 @@ import torch
 import combine_ep_get_08_b200 as ep
 import oracle
 import workloads
-from ep_harness import ROW_CHUNK, TOKEN_CHUNK, assert_layout_equal, chunks as _chunks, combine_close, gpu_layout
+from ep_harness import ROW_CHUNK, TOKEN_CHUNK, assert_layout_equal, chunks as _chunks, combine_close, config_of, gpu_layout
 
 pytestmark = pytest.mark.gpu
 
@@ -320,3 +320,22 @@ def test_col_major_tma_scales():
         np.testing.assert_array_equal(s_c[:, :g.rows].t().cpu().numpy().view(np.uint32), osc.view(np.uint32))
     finally:
         ep.ep_handle_destroy(g.handle)
+
+
+@pytest.mark.parametrize("T", [1, 13, 64, 295])
+def test_small_batch_layout(T):
+    """ep_get_layout of a batch with fewer than two tokens per SM runs the
+    small-batch kernel without its copy (one CTA per token, each counting all
+    pairs); under a 5-SM cap (T = 13) five CTAs handle 2-3 tokens each."""
+    wl = workloads.generate(None, T=T, H=256, E=64, R=8, K=8, A=4, router="topk", seed=300 + T)
+    h = ep.ep_handle_create(config_of(wl))
+    if T == 13:
+        ep.ep_set_sm_limit(h, 5)
+    g = gpu_layout(wl, handle=h)
+    try:
+        assert g.status == 0
+        o = oracle.layout(wl.topk_idx.numpy(), wl.E, wl.R, wl.A, topk_weights=wl.topk_weights.numpy())
+        assert_layout_equal(g, o)
+    finally:
+        ep.ep_handle_destroy(h)
+
