@@ -157,10 +157,11 @@ EP_API int ep_handle_get_view(const ep_handle *h, ep_handle_view *out);
  *   is_token_in_rank [T, R] uint8 (0/1), expert_offsets [E+1] int32,
  *   rank_offsets [R+1] int32.
  * topk_idx/topk_weights need 8/4-byte alignment only.  One kernel launch:
- * a thread-block cluster of up to 16 CTAs (at most 4096 pairs each) that
- * exchanges its histograms in distributed shared memory, or, for larger
- * batches, a cooperative grid whose one grid-wide wait is bounded
- * (EP_DEV_WAIT_TIMEOUT).
+ * for fewer than two tokens per SM (within the ep_set_sm_limit cap), one CTA
+ * per token that counts all pairs itself; else a thread-block cluster of up
+ * to 16 CTAs (at most 4096 pairs each) that exchanges its histograms in
+ * distributed shared memory, or, for larger batches, a cooperative grid
+ * whose one grid-wide wait is bounded (EP_DEV_WAIT_TIMEOUT).
  * Defined by: the V1 layout tensors num_tokens_per_rank, is_token_in_rank
  * and num_tokens_per_expert of bowenzhou.top "deepep/01-overview" section
  * 1.4; the per-expert queue order (tokens in order, then k) of the
