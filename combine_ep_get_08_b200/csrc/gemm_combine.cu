@@ -315,11 +315,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
 // (kind::f8f6f4, M=128, N=256, K=32, four per k-block) into one of two TMEM
 // partial buffers, and the epilogue warps fold each partial into fp32
 // registers with its two scales (sa of the row, sw of the 128-column half)
-// while the tensor cores fill the other buffer.  Eight epilogue warps: warp w
-// reads TMEM lanes 32*(w%4).. and one 128-column half of the tile, so a thread
-// keeps 128 running sums.  After the tile's last k-block the sums are scaled by
-// the pair's top-k weight and added into the token's fp32 row as in the bf16
-// kernel.  Same persistent tile order, producer and bounded waits.
+// while the tensor cores fill the other buffer.  Twelve warps: warpgroup 0
+// holds the TMA producer (warp 0) and the MMA issuer (warp 1); warpgroups 1-2
+// are eight epilogue warps, warp w reading TMEM lanes 32*(w%4).. and one
+// 128-column half of the tile, so a thread keeps 128 running sums (setmaxnreg
+// moves registers from warpgroup 0 to them).  After the tile's last k-block
+// the sums are scaled by the pair's top-k weight and added into the token's
+// fp32 row as in the bf16 kernel.  Same persistent tile order, producer and
+// bounded waits.
 // ---------------------------------------------------------------------------
 constexpr int kFK = 128;                              // inner elements per stage: one 128-byte row = one scale block
 constexpr int kFStages = 4;
