@@ -3,9 +3,10 @@
 One capture of ep_get_layout + ep_dispatch + ep_combine (static buffers, the
 inputs rewritten in place between replays) must give the oracle's layout and
 the identity-expert round trip on every replay -- for a batch that takes the
-cluster layout kernel and for one that takes the cooperative kernel, whose
+cluster layout kernel, for one that takes the cooperative kernel, whose
 grid-wide wait takes its target from the device (a replayed launch carries the
-parameters of the captured one).
+parameters of the captured one), and for a small batch (fewer than two tokens
+per SM) that takes the small-batch layout kernel.
 """
 import numpy as np
 import pytest
@@ -31,10 +32,11 @@ def _built():
 SHAPES = [
     dict(T=2048, H=256, E=64, R=8, K=8, A=4, router="topk"),     # cluster layout (8 CTAs)
     dict(T=20000, H=64, E=64, R=8, K=8, A=2, router="topk"),     # cooperative layout (160 000 pairs)
+    dict(T=128, H=512, E=256, R=32, K=8, A=2, router="topk"),    # small-batch layout (one CTA per token)
 ]
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=["cluster", "cooperative"])
+@pytest.mark.parametrize("shape", SHAPES, ids=["cluster", "cooperative", "small"])
 def test_normal_path_graph_replay(shape):
     dev = torch.device("cuda")
     wls = [workloads.generate(None, seed=70 + i, **shape) for i in range(3)]
