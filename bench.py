@@ -191,11 +191,17 @@ STEP_KERNEL_SOURCES = ("combine.cu", "dispatch.cu", "dispatch_lb.cu", "ep_intern
 
 
 def kernel_source_digest() -> str:
+    """Digest of the step kernels' code: comments and blank lines are left out,
+    so that a comment edit does not invalidate the recorded DRAM traffic."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "combine_ep_get_08_b200", "csrc")
     for name in STEP_KERNEL_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+        h.update(name.encode() + "\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()[:16]
 
 

@@ -387,11 +387,12 @@ __global__ void __launch_bounds__(kThreads, EP_FP8_MINB) dispatch_fp8_kernel(Dis
 // is_token_in_rank rows and their copies (the first row is loaded before the
 // counting, so the two overlap); the padding rows of experts c, c + G, ...
 // are written as well; CTA 0 writes the counts and offsets, the last CTA the
-// distinct tokens per rank.  No CTA waits on another.
+// distinct tokens per rank.  No CTA waits on another.  With p.x == nullptr
+// the same kernel computes the layout alone (ep_get_layout of a small batch).
 // ---------------------------------------------------------------------------
 template <bool FP8, int W>   // W: bf16 elements per thread (FP8) or vector bytes (bf16)
 __device__ __forceinline__ void small_layout_dispatch(const DispatchParams &p, const LayoutParams &lp) {
-    __shared__ int32_t s_tot[kMaxExperts + 1];   // pairs per expert (later: tokens per rank, CTA 0)
+    __shared__ int32_t s_tot[kMaxExperts + 1];   // pairs per expert (later: tokens per rank, last CTA)
     __shared__ int32_t s_before[kMaxExperts];    // pairs per expert among tokens [0, upto)
     __shared__ int32_t s_eoff[kMaxExperts + 1];  // padded expert offsets
     __shared__ int32_t s_dst[kMaxTopk];

@@ -150,3 +150,21 @@ def test_kernel_figures_writeback_arithmetic():
     # a flush that ran faster than the clean one charges nothing
     split["flush_after_combine"] = ms(39.0)
     assert bench.kernel_figures(wl, 32768, split, True, 6500.0)["with_writeback"]["combine_us"] == 80.0
+
+
+def test_kernel_digest_ignores_comments_only(tmp_path, monkeypatch):
+    """The digest that stamps the recorded DRAM traffic changes with the step
+    kernels' code, not with their comments."""
+    import shutil
+    csrc = tmp_path / "combine_ep_get_08_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in bench.STEP_KERNEL_SOURCES:
+        shutil.copy(os.path.join(ROOT, "combine_ep_get_08_b200", "csrc", name), csrc / name)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    d0 = bench.kernel_source_digest()
+    f = csrc / "combine.cu"
+    text = f.read_text()
+    f.write_text("// a new comment line\n" + text.replace("namespace ep {", "namespace ep {  /* note */", 1) + "\n\n")
+    assert bench.kernel_source_digest() == d0
+    f.write_text(text.replace("kLoadsInFlight = 8", "kLoadsInFlight = 4", 1))
+    assert bench.kernel_source_digest() != d0
