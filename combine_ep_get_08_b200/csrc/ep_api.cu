@@ -651,6 +651,7 @@ static int peer_common(const ep_handle *h, PeerOp op, const void *x, const void 
     l.H = c.hidden;
     l.cap = h->cap;
     l.zero_rows = c.expert_alignment > 1;
+    l.prefetch_x = (int64_t)c.num_tokens * c.hidden * 2 <= (int64_t)h->l2_bytes / 2;
     const int sms = h->sm_limit > 0 && h->sm_limit < h->num_sms ? h->sm_limit : h->num_sms;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;

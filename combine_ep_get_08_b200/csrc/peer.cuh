@@ -18,6 +18,7 @@ struct PeerLaunch {
     int T, K, R, H;
     int64_t cap;
     bool zero_rows;           // expert_alignment > 1: padding rows are written as zeros
+    bool prefetch_x;          // dispatch: x fits in half the L2; each CTA pulls its rows in first
 };
 
 cudaError_t launch_dispatch_peer(const PeerLaunch &l, int num_sms, cudaStream_t s);
