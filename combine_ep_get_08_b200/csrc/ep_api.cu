@@ -929,7 +929,7 @@ EP_API const char *ep_status_string(int code) {
         case EP_OK: return "ok";
         case EP_ERR_ARG: return "invalid argument (null pointer, size, alignment or E % R != 0)";
         case EP_ERR_CUDA: return "CUDA runtime error (see ep_last_error)";
-        case EP_ERR_UNSUPPORTED: return "sizes beyond this build's limits";
+        case EP_ERR_UNSUPPORTED: return "sizes beyond the library's limits";
         case EP_ERR_STATE: return "handle has no layout yet, or is of the other layout mode";
         case EP_ERR_DEVICE: return "device reported an error (bad expert id, wait timeout or slot overflow)";
         default: return "unknown status";

@@ -68,7 +68,7 @@ enum ep_error {
     EP_OK = 0,
     EP_ERR_ARG = -1,         /* null pointer, bad size, misalignment, E % R != 0 ... */
     EP_ERR_CUDA = -2,        /* a CUDA runtime call failed (see ep_last_error) */
-    EP_ERR_UNSUPPORTED = -3, /* sizes beyond this build's limits (see ep_config) */
+    EP_ERR_UNSUPPORTED = -3, /* sizes beyond the library's limits (see ep_config) */
     EP_ERR_STATE = -4,       /* handle used before ep_get_layout, or on another device */
     EP_ERR_DEVICE = -5       /* ep_get_status found device-side error bits */
 };
