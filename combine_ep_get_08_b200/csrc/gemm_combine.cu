@@ -359,17 +359,6 @@ __device__ __forceinline__ void umma_e4m3(uint32_t tmem_d, uint64_t a, uint64_t 
         : "r"(tmem_d), "l"(a), "l"(b), "r"(kFIdesc), "r"(accumulate));
 }
 
-// 16 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15}, [%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" : : : "memory");
-}
-
 // 16 columns of this lane, no wait: the caller waits with tmem_wait_ld and
 // then passes the registers through tmem_fence_regs before using them.
 __device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t *v) {
