@@ -168,3 +168,28 @@ def test_kernel_digest_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.kernel_source_digest() == d0
     f.write_text(text.replace("kLoadsInFlight = 8", "kLoadsInFlight = 4", 1))
     assert bench.kernel_source_digest() != d0
+
+
+def test_expert_gemm_summary_arithmetic(monkeypatch, tmp_path):
+    """TFLOP/s of the expert GEMM entries: 2 x (non-masked pairs) x N x I per
+    call over the mean event time; the E4M3 peak is twice the measured bf16
+    burst (the nominal dense FP8 / bf16 ratio)."""
+    import types
+
+    import numpy as np
+    import torch
+    peaks = tmp_path / "MEASURED_PEAKS.json"
+    peaks.write_text(json.dumps({"bf16_tflops": 1600.0, "hbm_gbs": 6500.0}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.gemm_peak(False)[0] == 1600.0 and bench.gemm_peak(True)[0] == 3200.0
+    idx = torch.from_numpy(np.array([[0, 1], [2, -1]], np.int64))    # 3 real pairs
+    wl = types.SimpleNamespace(topk_idx=idx)
+    for fp8, peak in ((False, 1600.0), (True, 3200.0)):
+        o = {"wl": wl, "N": 1024, "I": 512, "fp8": fp8}
+        e = bench.expert_gemm_summary(o, [0.002, 0.004])                # mean 3 us
+        want = 2.0 * 3 * 1024 * 512 / 3e-6 / 1e12
+        assert abs(e["tflops"] - round(want, 1)) < 1e-9
+        assert e["peak"] == peak and abs(e["frac"] - round(want / peak, 4)) < 1e-12
+        assert e["dtype"] == ("e4m3" if fp8 else "bf16") and e["us_per_call"] == 3.0
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path / "none"))
+    assert bench.gemm_peak(False)[0] == 1590.0                         # the fallback without the file
